@@ -1,0 +1,56 @@
+"""CPU oracle for the BitLinear hot path.  TEST INFRASTRUCTURE ONLY.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and ``bench.py`` (its CPU-baseline
+and reference legs) may import this package.  The product path never calls it:
+the CUDA library has no CPU fallback.  The oracle shares no code with the CUDA
+path; the two meet only in the seeded inputs of ``workloads``.
+
+What it computes, and where the method is stated (page title, then section):
+
+* ``absmean_beta`` and ``ternarize`` -- "ultragraph -- when the graph is the
+  1-bit LLM, part 2", section "the bytes": beta = (1/n) sum_i |W_i| + eps,
+  W_q = clip(round(W / beta), -1, 1).  One beta per weight tensor ("global beta"
+  in section "autograd on a byte-graph, and the straight-through lie").
+* ``act_quant`` -- same page, section "the bytes" and the per-token fix in
+  section "attention, as graph ops": s = max_i |x_i| / 127 + eps per row,
+  x_q = clip(round(x / s), -127, 127), the symmetric range [-127, 127].
+* ``contract`` and ``dequant`` -- same page, section "autograd on a byte-graph",
+  deployed-path equation y = (x_q W_q^T)(s beta) + b: an integer matmul, then
+  one rescale by the row scale times beta.
+* ``pack5`` / ``unpack5`` -- "ultragraph-1bit 0.12.0" (PyPI), sections "A whole
+  ternary GPT" and "Layout" (5 ternary values per byte, ~1.6 bits/weight), and
+  "a 1-bit llm, from scratch", tl;dr (1.6 bits each).  Byte = sum_k (t_k+1) 3^k.
+
+Readings where the pages leave a step open (each is also listed in the design doc):
+
+1. Precision.  The pages' arrays are numpy float32, so every quantizer step is
+   IEEE-754 float32 with round-to-nearest-even, in the order written.
+2. The mean in beta is the exact real sum of |W| rounded once to float64
+   (``math.fsum`` is correctly rounded), divided by n in float64, rounded to
+   float32; eps is then added in float32.  A float32 running sum would make
+   beta depend on summation order, which no two implementations share.
+3. "round" is round-half-to-even (numpy's ``rint``/``round``).
+4. eps is the same value in both quantizers (1e-5 unless a caller passes
+   another) and is added after the mean / after max/127.
+5. Dequantization multiplies s by beta first (the page's grouping "(s beta)"),
+   then the float32 accumulator by that product, then adds b separately.
+6. Packing runs along K in order: trit 5j+k of a row is digit k (little-endian)
+   of byte j; trits past K are 0 (digit 1), so an all-padding byte is 121; the
+   row stride ``ldp`` is ceil(K/5) rounded up to 16 bytes.
+
+Every function here is pinned by ``tests/test_oracle_pins.py`` against hand-
+worked values, closed forms, invariants or brute force; none is unpinned.
+"""
+from .layer import (  # noqa: F401
+    ACT_QMAX,
+    absmean_beta,
+    act_quant,
+    bitlinear,
+    contract,
+    contract_entries,
+    dequant,
+    pack5,
+    pack5_ldp,
+    ternarize,
+    unpack5,
+)

@@ -1,0 +1,97 @@
+"""Plausible mistakes planted in the oracle (on the CPU) must fail a pin.
+
+Each mutation is a wrong variant of one oracle step; the check is that at
+least one of the pins in test_oracle_pins.py rejects it.  Nothing here runs on
+the GPU.
+"""
+import math
+
+import numpy as np
+import pytest
+
+import oracle
+import oracle.layer as ob
+
+F32 = np.float32
+
+
+def _run_pins():
+    return pytest.main(["-q", "-x", "-p", "no:cacheprovider",
+                        __file__.replace("test_oracle_mutations.py", "test_oracle_pins.py")])
+
+
+def _beta_f32_running_sum(W, eps):
+    a = np.abs(np.asarray(W, F32)).ravel()
+    tot = F32(0)
+    for v in a:
+        tot = F32(tot + v)
+    return F32(F32(tot / F32(a.size)) + F32(eps))
+
+
+def _ternarize_half_away(W, beta):
+    q = np.trunc(np.asarray(W, F32) / F32(beta) + np.copysign(F32(0.5), W))
+    return np.clip(q, -1, 1).astype(np.int8)
+
+
+def _act_quant_half_away(X, eps):
+    X = np.asarray(X, F32)
+    s = np.max(np.abs(X), axis=1) / F32(127) + F32(eps)
+    r = X / s[:, None]
+    q = np.trunc(r + np.copysign(F32(0.5), r))
+    return np.clip(q, -127, 127).astype(np.int8), s.astype(F32)
+
+
+def _act_quant_per_tensor(X, eps):
+    X = np.asarray(X, F32)
+    s = np.full(X.shape[0], np.max(np.abs(X)) / F32(127) + F32(eps), F32)
+    return np.clip(np.rint(X / s[:, None]), -127, 127).astype(np.int8), s
+
+
+def _act_quant_128(X, eps):
+    X = np.asarray(X, F32)
+    s = np.max(np.abs(X), axis=1) / F32(128) + F32(eps)
+    return np.clip(np.rint(X / s[:, None]), -128, 127).astype(np.int8), s.astype(F32)
+
+
+def _pack_big_endian(Wq, ldp=None):
+    Wq = np.asarray(Wq)
+    N, K = Wq.shape
+    ldp = ldp or ob.pack5_ldp(K)
+    t = np.zeros((N, ldp * 5), np.int64)
+    t[:, :K] = Wq
+    d = (t + 1).reshape(N, ldp, 5)
+    return sum(d[:, :, k] * 3 ** (4 - k) for k in range(5)).astype(np.uint8)
+
+
+def _contract_transposed_w(Xq, Wq):
+    Wq = np.asarray(Wq)
+    if Wq.shape[0] == Wq.shape[1]:
+        Wq = Wq.T
+    return (np.asarray(Xq).astype(np.int64) @ Wq.astype(np.int64).T).astype(np.int32)
+
+
+def _dequant_acc_times_s_first(acc, s, beta, bias=None):
+    y = (np.asarray(acc).astype(F32) * np.asarray(s, F32).reshape(-1, 1)) * F32(beta)
+    return y if bias is None else y + np.asarray(bias, F32)
+
+
+def _beta_no_eps(W, eps):
+    return ob.absmean_beta(W, 0.0)
+
+
+MUTANTS = {
+    "absmean_beta": [_beta_f32_running_sum, _beta_no_eps],
+    "ternarize": [_ternarize_half_away],
+    "act_quant": [_act_quant_half_away, _act_quant_per_tensor, _act_quant_128],
+    "pack5": [_pack_big_endian],
+    "contract": [_contract_transposed_w],
+    "dequant": [_dequant_acc_times_s_first],
+}
+
+
+@pytest.mark.parametrize("name,mutant", [(n, f) for n, fs in MUTANTS.items() for f in fs],
+                         ids=lambda v: getattr(v, "__name__", v))
+def test_pins_reject_mutant(name, mutant, monkeypatch):
+    monkeypatch.setattr(ob, name, mutant)
+    monkeypatch.setattr(oracle, name, mutant)
+    assert _run_pins() != 0, f"pins did not catch {mutant.__name__}"
