@@ -1,0 +1,540 @@
+#!/usr/bin/env python
+"""BitLinear benchmark: one JSON line on rank 0.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload 2] [--impl ours|reference]
+
+A step is one pass of the whole BitLinear hot path over one batch of the
+workload: for every weight tensor, absmean beta (a1) and ternarize + pack
+(a2, a3); for every call, per-row int8 quantization of X, the ternary x int8
+contraction and the fused dequant (a4-a6).  The default workload is batch-1
+decode: (K,N) = (2560,6912) and (6912,2560) with packed trits, M = 1.
+
+Timing: inputs are resident in HBM; R replicas of every buffer rotate so each
+rotation touches >= 4x the L2 size (no step reuses the previous step's data
+from L2).  Each replica's step is captured once as a CUDA graph; W warm-up
+replays, then exactly K timed replays bracketed by barrier + synchronize, timed
+with CUDA events on the launching stream; the max over ranks is reported.
+Per-call durations come from external events inside the same graphs (the last
+R timed replays).  SM clocks and throttle reasons are sampled through NVML
+during the timed region.  `e2e` repeats the step through the public Python API
+with the step's inputs copied from pinned host memory and Y copied back.
+
+Under torchrun each rank runs its own independently seeded batch (weak
+scaling, no data-path collective); only the timing reduction crosses ranks.
+`--impl reference` times the CPU oracle instead (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads  # noqa: E402
+
+METRIC = "BitLinear GMAC/s and weight-stream GB/s (% of HBM/int8 peak), M=1..4096"
+UNIT = "GMAC/s"
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=50)
+    ap.add_argument("--workload", type=int, default=2)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--cpu-seconds", type=float, default=12.0,
+                    help="target CPU time of the oracle baseline sample")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--path", type=int, default=0, help="pin the linear kernel path (BL_PATH_*)")
+    return ap.parse_args()
+
+
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    return int(os.environ.get("RANK", "0")), ws, int(os.environ.get("LOCAL_RANK", "0"))
+
+
+# ----------------------------------------------------------------- clocks ---
+class ClockSampler:
+    """Polls NVML for SM clock and throttle reasons while the timed region runs."""
+
+    REASONS = {
+        "gpu_idle": 0x1, "applications_clocks_setting": 0x2, "sw_power_cap": 0x4,
+        "hw_slowdown": 0x8, "sync_boost": 0x10, "sw_thermal_slowdown": 0x20,
+        "hw_thermal_slowdown": 0x40, "hw_power_brake_slowdown": 0x80,
+        "display_clock_setting": 0x100,
+    }
+
+    def __init__(self, device_index_uuid):
+        self.samples, self.reasons, self.max_mhz, self.ok = [], set(), None, False
+        try:
+            import pynvml as nv
+            nv.nvmlInit()
+            self.nv = nv
+            self.h = nv.nvmlDeviceGetHandleByUUID(device_index_uuid)
+            self.max_mhz = nv.nvmlDeviceGetMaxClockInfo(self.h, nv.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as e:  # pragma: no cover - depends on the box
+            self.err = repr(e)
+        self._stop = threading.Event()
+
+    def _poll(self):
+        nv = self.nv
+        while not self._stop.is_set():
+            self._sample_once()
+            time.sleep(0.0005)
+
+    def _sample_once(self):
+        nv = self.nv
+        try:
+            self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+            r = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+            for k, bit in self.REASONS.items():
+                if r & bit and k != "gpu_idle":
+                    self.reasons.add(k)
+        except Exception:
+            pass
+
+    def __enter__(self):
+        if self.ok:
+            self._sample_once()
+            self.t = threading.Thread(target=self._poll, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self.ok:
+            self._stop.set()
+            self.t.join()
+            self._sample_once()
+
+    def summary(self):
+        if not self.ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0}
+        return {"sm_mhz": float(np.median(self.samples)), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+# ------------------------------------------------------------ peaks/traffic --
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as fh:
+            d = json.load(fh)
+        return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]),
+                "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "source": "fallback"}
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    d = os.path.join(ROOT, "int8_row_absmax_b200", "csrc")
+    for f in sorted(os.listdir(d)):
+        if f.endswith((".cu", ".cuh")):
+            with open(os.path.join(d, f), "rb") as fh:
+                h.update(f.encode() + fh.read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(kernel: str, workload: int):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on
+    the current kernel sources (else None)."""
+    p = os.path.join(ROOT, "profiles", "dram_traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as fh:
+        d = json.load(fh)
+    rec = d.get(f"{kernel}@{workload}")
+    if not rec or rec.get("source_hash") != kernel_source_hash():
+        return None
+    return rec.get("dram_bytes_per_launch")
+
+
+# ------------------------------------------------------------- the step ----
+class Step:
+    """Device buffers and API calls for one replica of the workload's step."""
+
+    def __init__(self, bl, torch, probs, dev, fmt):
+        self.bl, self.torch, self.fmt = bl, torch, fmt
+        self.tensors = []          # weight tensors: (W, beta, Wout, absmean ws)
+        self.calls = []            # linear calls: (X, tensor index, Y, lin ws, M, K, N)
+        seen = {}
+        for p in probs:
+            key = id(p.W)
+            if key not in seen:
+                W = torch.from_numpy(p.W).to(dev)
+                beta = torch.zeros(1, dtype=torch.float32, device=dev)
+                if fmt == bl.PACK5:
+                    Wout = torch.empty((p.N, bl.pack5_ldp(p.K)), dtype=torch.uint8, device=dev)
+                else:
+                    Wout = torch.empty((p.N, p.K), dtype=torch.int8, device=dev)
+                ws = bl.workspace(4096, dev)
+                seen[key] = len(self.tensors)
+                self.tensors.append((W, beta, Wout, ws, p.N, p.K))
+            X = torch.from_numpy(np.ascontiguousarray(p.X)).to(dev)
+            Y = torch.empty((p.M, p.N), dtype=torch.float32, device=dev)
+            lws = bl.workspace(bl.linear_workspace_size(p.M, p.N, p.K, fmt), dev)
+            self.calls.append((X, seen[key], Y, lws, p.M, p.K, p.N, p.eps))
+
+    def nbytes(self):
+        n = 0
+        for W, beta, Wout, ws, N, K in self.tensors:
+            n += W.numel() * 4 + Wout.numel()
+        for X, ti, Y, lws, M, K, N, eps in self.calls:
+            n += X.numel() * 4 + Y.numel() * 4 + lws.numel()
+        return n
+
+    def run(self, events=None, path=0):
+        """Issue the whole step on the current stream; events[i] mark call boundaries."""
+        bl = self.bl
+        k = 0
+
+        def mark():
+            nonlocal k
+            if events is not None:
+                events[k].record()
+            k += 1
+        mark()
+        for W, beta, Wout, ws, N, K in self.tensors:
+            bl.absmean(W, 1e-5, ws=ws, beta=beta)
+            mark()
+            if self.fmt == bl.PACK5:
+                bl.ternarize_pack5(W, beta, out=Wout)
+            else:
+                bl.ternarize(W, beta, out=Wout)
+            mark()
+        for X, ti, Y, lws, M, K, N, eps in self.calls:
+            W, beta, Wout, ws, _, _ = self.tensors[ti]
+            bl.linear(X, Wout, self.fmt, N, K, beta, eps=eps, ws=lws, out=Y, path=path)
+            mark()
+
+    def labels(self):
+        out = []
+        for i, (W, beta, Wout, ws, N, K) in enumerate(self.tensors):
+            out += [("absmean", i), ("ternarize_pack5" if self.fmt == self.bl.PACK5 else "ternarize", i)]
+        for j, c in enumerate(self.calls):
+            out.append(("linear", j))
+        return out
+
+
+def algorithmic_bytes(kind, N, K, M, fmt):
+    """Bytes each kind of call must move at minimum (inputs read + outputs written)."""
+    wbytes = N * math.ceil(K / 5) if fmt == 1 else N * K
+    if kind == "absmean":
+        return 4 * N * K
+    if kind.startswith("ternarize"):
+        return 4 * N * K + wbytes
+    if kind == "linear":
+        return wbytes + 4 * M * K + 4 * M * N
+    raise ValueError(kind)
+
+
+# ------------------------------------------------------------ our arm ------
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+    rank, world, local = dist_env()
+    if world > 1:
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=120))
+    dev = torch.device("cuda", local if world > 1 else 0)
+    torch.cuda.set_device(dev)
+    import int8_row_absmax_b200 as bl
+    bl.load()
+
+    wl = workloads.WORKLOADS[args.workload]
+    fmt = bl.PACK5 if wl.fmt == workloads.FMT_PACK5 else bl.I8
+    probs = list(workloads.problems(args.workload, rank=rank))
+    macs_per_step = sum(p.M * p.N * p.K for p in probs)
+
+    props = torch.cuda.get_device_properties(dev)
+    l2 = int(getattr(props, "L2_cache_size", 126 * 2 ** 20))
+    first = Step(bl, torch, probs, dev, fmt)
+    R = max(2, math.ceil(4 * l2 / first.nbytes()))
+    steps = [first] + [Step(bl, torch, probs, dev, fmt) for _ in range(R - 1)]
+    torch.cuda.synchronize()
+
+    # one eager step per replica: launches must succeed and the device stay clean
+    for s in steps:
+        s.run(path=args.path)
+    if bl.sync_status(dev) != "BL_OK":
+        raise RuntimeError("device status not clean after the eager step")
+
+    labels = first.labels()
+    n_ev = len(labels) + 1
+    stream = torch.cuda.Stream(device=dev)
+    graphs, evsets = [], []
+    with torch.cuda.stream(stream):
+        for s in steps:
+            evs = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(n_ev)]
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                s.run(events=evs, path=args.path)
+            graphs.append(g)
+            evsets.append(evs)
+    torch.cuda.synchronize()
+
+    K, Wm = args.steps, args.warmup
+    with torch.cuda.stream(stream):
+        for i in range(Wm):
+            graphs[i % R].replay()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    clk = ClockSampler(str(props.uuid) if str(props.uuid).startswith("GPU-") else "GPU-" + str(props.uuid))
+    torch.cuda.synchronize()
+    with clk:
+        with torch.cuda.stream(stream):
+            t0.record(stream)
+            for i in range(K):
+                graphs[(Wm + i) % R].replay()
+            t1.record(stream)
+        torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    ms = t0.elapsed_time(t1)
+    t = torch.tensor([ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms_max = float(t.item())
+    if bl.sync_status(dev) != "BL_OK":
+        raise RuntimeError("device status not clean after the timed region")
+
+    # per-call durations from the external events (the last replay of each replica)
+    per_call = {}
+    for evs in evsets:
+        for i, lab in enumerate(labels):
+            per_call.setdefault(lab, []).append(evs[i].elapsed_time(evs[i + 1]))
+    shapes = {}
+    for i, (W, beta, Wout, ws, N, Kd) in enumerate(first.tensors):
+        shapes[("absmean", i)] = (N, Kd, 0)
+        shapes[(labels[2 * i + 1][0], i)] = (N, Kd, 0)
+    for j, (X, ti, Y, lws, M, Kd, N, eps) in enumerate(first.calls):
+        shapes[("linear", j)] = (N, Kd, M)
+    kinds = {}
+    for lab, v in per_call.items():
+        kind = lab[0]
+        N, Kd, M = shapes[lab]
+        d = kinds.setdefault(kind, {"ms": 0.0, "bytes": 0, "launches": 0})
+        d["ms"] += float(np.mean(v))
+        d["bytes"] += algorithmic_bytes(kind, N, Kd, M, fmt)
+        d["launches"] += 1 if kind != "linear" else bl.linear_plan(M, N, Kd, fmt, args.path)[1]
+    peaks = measured_peaks()
+    kern_names = {"absmean": "absmean_kernel", "ternarize_pack5": "ternarize_pack5_kernel",
+                  "ternarize": "ternarize_i8_kernel", "linear": "linear"}
+    kernels = {}
+    for kind, d in kinds.items():
+        gbs = d["bytes"] / (d["ms"] * 1e-3) / 1e9
+        kernels[kind] = {"ms_per_step": round(d["ms"], 5), "algorithmic_bytes": d["bytes"],
+                         "launches": d["launches"], "achieved_gbs": round(gbs, 1),
+                         "frac_hbm": round(gbs / peaks["hbm_gbs"], 4)}
+    # the dominant single-kernel call (linear may be two launches: act quant + contraction)
+    single = [k for k in kinds if k != "linear" or kinds[k]["launches"] == len(first.calls)]
+    dom = max(single, key=lambda k: kinds[k]["ms"])
+    dkind = kinds[dom]
+    achieved = dkind["bytes"] / (dkind["ms"] * 1e-3) / 1e9
+    roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"],
+                "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
+                "traffic": ncu_traffic(kern_names[dom], args.workload),
+                "kernel": kern_names[dom], "peak_source": peaks["source"] + " (MEASURED_PEAKS.json hbm_gbs)"
+                if peaks["source"] == "measured" else "fallback 6.65 TB/s"}
+
+    launches_per_step = sum(d["launches"] for d in kinds.values())
+    value = macs_per_step * K * world / (ms_max * 1e-3) / 1e9
+    lin = kinds.get("linear")
+    line = {
+        "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world,
+        "steps": K, "warmup": Wm, "ms_per_step": round(ms_max / K, 6),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "i8xtrit->i32,f32",
+        "data": "synthetic",
+        "config": {"workload": f"{wl.id}:{wl.name}", "shapes_MKN": [list(s) for s in wl.shapes],
+                   "weight_format": wl.fmt, "parallelism": f"dp{world} (independent batches)",
+                   "l2_defeat": f"{R} rotating replicas, {R * first.nbytes() / 2**20:.0f} MiB >= 4x L2 "
+                                f"({l2 / 2**20:.0f} MiB)",
+                   "step": "absmean + ternarize/pack per weight tensor, then quantize_act + "
+                           "contraction + dequant per call", "timing": "CUDA graph per replica, CUDA events"},
+        "macs_per_step": macs_per_step,
+        "linear_only": None if lin is None else {
+            "gmacs": round(macs_per_step / (lin["ms"] * 1e-3) / 1e9, 1),
+            "weight_stream_gbs": round(sum(
+                (p.N * math.ceil(p.K / 5) if fmt == bl.PACK5 else p.N * p.K) for p in probs)
+                / (lin["ms"] * 1e-3) / 1e9, 1),
+            "ms_per_step": round(lin["ms"], 5)},
+        "kernels": kernels,
+        "roofline": roofline,
+        "clocks": clk.summary(),
+        "gpu_launches": launches_per_step * K,
+        "gpu": torch.cuda.get_device_name(dev),
+    }
+    if line["linear_only"] is not None:
+        line["linear_only"]["frac_hbm"] = round(line["linear_only"]["weight_stream_gbs"] / peaks["hbm_gbs"], 4)
+
+    # ---- end to end through the public API, host buffers -------------------
+    line["e2e"] = e2e(bl, torch, probs, dev, fmt, args.e2e_steps, world)
+    for g in graphs:
+        del g
+    graphs.clear()
+
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(args.workload, args.cpu_seconds)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def e2e(bl, torch, probs, dev, fmt, steps, world):
+    """The step through the public API with pinned host inputs copied in and Y copied out."""
+    host_W, host_X, seen = [], [], {}
+    for p in probs:
+        if id(p.W) not in seen:
+            seen[id(p.W)] = len(host_W)
+            host_W.append(torch.from_numpy(p.W).pin_memory())
+        host_X.append(torch.from_numpy(np.ascontiguousarray(p.X)).pin_memory())
+    dW = [torch.empty_like(h, device=dev) for h in host_W]
+    dX = [torch.empty_like(h, device=dev) for h in host_X]
+    hY = [torch.empty((p.M, p.N), dtype=torch.float32).pin_memory() for p in probs]
+    ws = [bl.workspace(4096, dev) for _ in host_W]
+    h2d = sum(h.numel() * 4 for h in host_W) + sum(h.numel() * 4 for h in host_X)
+    d2h = sum(h.numel() * 4 for h in hY)
+
+    def one():
+        for h, d in zip(host_W, dW):
+            d.copy_(h, non_blocking=True)
+        for h, d in zip(host_X, dX):
+            d.copy_(h, non_blocking=True)
+        packed = []
+        for i, W in enumerate(dW):
+            if fmt == bl.PACK5:
+                packed.append(bl.quantize_weights_pack5(W, 1e-5, ws=ws[i]))
+            else:
+                packed.append(bl.quantize_weights(W, 1e-5, ws=ws[i]))
+        for j, p in enumerate(probs):
+            Wd, beta = packed[seen[id(p.W)]]
+            Y = bl.linear(dX[j], Wd, fmt, p.N, p.K, beta, eps=p.eps)
+            hY[j].copy_(Y, non_blocking=True)
+
+    one()
+    torch.cuda.synchronize()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record()
+    for _ in range(steps):
+        one()
+    t1.record()
+    torch.cuda.synchronize()
+    ms = t0.elapsed_time(t1)
+    t = torch.tensor([ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        import torch.distributed as dist
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms = float(t.item())
+    macs = sum(p.M * p.N * p.K for p in probs)
+    return {"value": round(macs * steps * world / (ms * 1e-3) / 1e9, 2), "unit": UNIT,
+            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+            "steps": steps, "ms_per_step": round(ms / steps, 4)}
+
+
+# ------------------------------------------------------------ CPU oracle ----
+def oracle_step(probs, rows_frac=1.0):
+    """The oracle on (a row slice of) the step's problems; returns MACs done."""
+    import oracle
+    macs, done = 0, {}
+    for p in probs:
+        n = max(1, int(round(p.N * rows_frac)))
+        W = p.W[:n]
+        key = id(p.W)
+        if key not in done:
+            beta = oracle.absmean_beta(W, p.eps)
+            Wq = oracle.ternarize(W, beta)
+            if p.fmt == workloads.FMT_PACK5:
+                oracle.unpack5(oracle.pack5(Wq), p.K)
+            done[key] = (beta, Wq)
+        beta, Wq = done[key]
+        Xq, s = oracle.act_quant(p.X, p.eps)
+        oracle.dequant(oracle.contract(Xq, Wq), s, beta)
+        macs += p.M * n * p.K
+    return macs
+
+
+def cpu_sample_fraction(wid, seconds):
+    """Row fraction of the step the oracle finishes in about `seconds`."""
+    probs = list(workloads.problems(wid))
+    frac = 1.0 / 64
+    t = time.perf_counter()
+    oracle_step(probs, frac)
+    dt = time.perf_counter() - t
+    return probs, min(1.0, frac * seconds / max(dt, 1e-3))
+
+
+def cpu_baseline(wid, seconds):
+    """The oracle as committed, single-threaded numpy, on a bounded sample of the
+    step: a row slice of every weight when a whole step is too long, else whole
+    steps repeated until about `seconds` of CPU time."""
+    probs, frac = cpu_sample_fraction(wid, seconds)
+    t = time.perf_counter()
+    macs, reps = 0, 0
+    while True:
+        macs += oracle_step(probs, frac)
+        reps += 1
+        if frac < 1.0 or time.perf_counter() - t >= seconds:
+            break
+    dt = time.perf_counter() - t
+    what = (f"{reps} whole step(s)" if frac >= 1.0 else
+            f"the step on the first {frac:.4f} of each weight's rows (beta over that slice)")
+    return {"value": round(macs / dt / 1e9, 4), "unit": UNIT, "cores": 1, "kind": "oracle",
+            "sample": f"{what}, numpy oracle as committed, {dt:.1f} s"}
+
+
+def run_reference(args):
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return
+    wl = workloads.WORKLOADS[args.workload]
+    # each reference step: the oracle's whole step on a row slice sized so the run stays short
+    probs, frac = cpu_sample_fraction(args.workload, max(0.05, 60.0 / max(1, args.steps + args.warmup)))
+    for _ in range(args.warmup):
+        oracle_step(probs, frac)
+    t = time.perf_counter()
+    macs = 0
+    for _ in range(args.steps):
+        macs += oracle_step(probs, frac)
+    dt = time.perf_counter() - t
+    value = macs / dt / 1e9
+    line = {"impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": UNIT,
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(dt / max(1, args.steps) * 1e3, 3), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "i8xtrit->i64,f32", "data": "synthetic",
+            "config": {"workload": f"{wl.id}:{wl.name}", "shapes_MKN": [list(s) for s in wl.shapes],
+                       "weight_format": wl.fmt, "parallelism": "cpu oracle, rank 0"},
+            "cpu_baseline": {"value": round(value, 4), "unit": UNIT, "cores": 1, "kind": "oracle",
+                             "sample": f"each step: the whole step on the first {frac:.4f} of each "
+                                       f"weight's rows"},
+            "e2e": {"value": round(value, 4), "unit": UNIT, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

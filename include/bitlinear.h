@@ -1,0 +1,191 @@
+/*
+ * bitlinear.h -- C ABI of a B200 (sm_100a) BitLinear library: ternary weights
+ * times per-row absmax int8 activations, accumulated exactly in int32.
+ *
+ * The operation follows "ultragraph -- when the graph is the 1-bit LLM, part 2":
+ *   section "the bytes":
+ *     beta = (1/n) sum_i |W_i| + eps,   W_q = clip(round(W / beta), -1, 1)
+ *     s    = max_i |x_i| / 127 + eps,   x_q = clip(round(x / s), -127, 127)
+ *   section "autograd on a byte-graph, and the straight-through lie":
+ *     y = (x_q W_q^T)(s beta) + b        (the deployed forward path)
+ * and the dense trit format of "ultragraph-1bit 0.12.0" (PyPI), sections
+ * "A whole ternary GPT" and "Layout": five ternary values per byte.
+ *
+ * Conventions shared by every entry point
+ *   - Matrices are row-major.  W is [N, K] (out x in), X is [M, K], Y is [M, N].
+ *   - Every pointer argument is a DEVICE pointer owned by the caller; the library
+ *     allocates no memory.  Scratch memory is passed in as `ws` (device, 256-byte
+ *     aligned) with a size from the matching *_workspace_size function.
+ *   - Calls are asynchronous on `stream` (NULL = the legacy default stream).  A
+ *     validation error returns at once and launches nothing.  A failed launch
+ *     returns BL_ERR_CUDA.  Conditions found on the device (non-finite inputs,
+ *     a bounded wait that gave up) are recorded in a per-device status word and
+ *     reported by bl_sync_status().
+ *   - Arithmetic is IEEE-754 float32, round-to-nearest-even, in the order the
+ *     formulas are written; no step is contracted into an FMA.  "round" is
+ *     round-half-to-even.  Trit codes, int8 codes, scales, beta and int32
+ *     accumulators are exact; Y is the float32 product acc * (s * beta) [+ b].
+ *   - The mean in beta is the exact real sum of |W|, rounded once to float64,
+ *     divided by n in float64, rounded to float32; eps is added in float32.
+ *   - Inputs must be finite; eps must be finite and > 0; 1 <= K <= 131072 so
+ *     that every accumulator (|acc| <= 127 K < 2^24) is exact in float32.
+ *   - No C++ exception crosses this boundary.
+ */
+#ifndef BITLINEAR_H_
+#define BITLINEAR_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#include <cuda_runtime_api.h> /* cudaStream_t */
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  BL_OK = 0,
+  BL_ERR_INVALID_ARG = 1,    /* null pointer, bad size, eps <= 0, K out of range */
+  BL_ERR_ALIGNMENT = 2,      /* a pointer or stride breaks the stated alignment */
+  BL_ERR_UNSUPPORTED = 3,    /* a forced kernel path cannot take this shape */
+  BL_ERR_WORKSPACE = 4,      /* ws NULL, too small, unaligned, or (device) not cleared */
+  BL_ERR_CUDA = 5,           /* a CUDA runtime call or launch failed */
+  BL_ERR_DEVICE_TIMEOUT = 6, /* a bounded device-side wait gave up */
+  BL_ERR_NONFINITE = 7       /* a kernel met a NaN or Inf input */
+} bl_status;
+
+/* Weight storage formats. */
+typedef enum {
+  /* One trit per byte, int8 in {-1,0,+1}, [N, ldw] with ldw >= K: the pages'
+   * "1 edge = 1 byte" layout ("the bytes"). */
+  BL_W_I8 = 0,
+  /* Five trits per byte, uint8 [N, ldw], ldw = bl_pack5_ldp(K) or any larger
+   * multiple of 16.  Byte j of row n is sum_{k<5} (W_q[n,5j+k] + 1) * 3^k, trits
+   * past K count as 0, so whole padding bytes are 121 ("A whole ternary GPT"). */
+  BL_W_PACK5 = 1
+} bl_wfmt;
+
+/* Kernel selection for the *_ex entry points (tests and benchmarks pin a path). */
+typedef enum {
+  BL_PATH_AUTO = 0, /* dispatch on M, K, N and the format */
+  BL_PATH_SIMT = 1, /* dp4a tile kernel: any shape, any format */
+  BL_PATH_GEMV = 2, /* packed-trit decode GEMV on CUDA cores: BL_W_PACK5, M <= 4 */
+  BL_PATH_TC = 3    /* tcgen05 kind::i8 tensor-core GEMM with fused dequant */
+} bl_path;
+
+/* Packed row stride in bytes: ceil(K/5) rounded up to a multiple of 16. */
+int64_t bl_pack5_ldp(int64_t K);
+
+/* Bytes of `ws` that bl_absmean and bl_quantize_weights* need (4096). */
+size_t bl_quantize_weights_workspace_size(int64_t N, int64_t K);
+
+/* Step 1 of the weight quantization: beta = (1/n) sum |W| + eps ("the bytes",
+ * absmean equation), one scalar for the whole tensor ("global beta", section
+ * "autograd on a byte-graph").
+ *   W        [N, K] float32, contiguous, 4-byte aligned (16 bytes for full speed).
+ *   eps      finite, > 0.
+ *   beta_dev one float32 on the device: receives beta.
+ *   ws       >= bl_quantize_weights_workspace_size(N, K) bytes (4 KB), 256-byte
+ *            aligned, ZERO-FILLED before its first use (e.g. cudaMemsetAsync);
+ *            every call leaves it zero-filled again, so a workspace is cleared
+ *            once and reused.  Calls sharing one workspace must not overlap on
+ *            the GPU (issue them on one stream).  A workspace found not cleared
+ *            is reported as BL_ERR_WORKSPACE by bl_sync_status.
+ * A non-finite weight sets BL_ERR_NONFINITE in the status word. */
+bl_status bl_absmean(const float* W, int64_t N, int64_t K, float eps, float* beta_dev, void* ws,
+                     size_t ws_bytes, cudaStream_t stream);
+
+/* Step 2: W_q = clip(round(W / beta), -1, 1) with beta read from beta_dev
+ * ("the bytes").  W [N, K] float32 contiguous -> Wq [N, K] int8 contiguous. */
+bl_status bl_ternarize(const float* W, int64_t N, int64_t K, const float* beta_dev, int8_t* Wq,
+                       cudaStream_t stream);
+
+/* Steps 2 and 3 fused: the codes of bl_ternarize written straight into the
+ * packed format, Wp [N, ldp] uint8 (ldp % 16 == 0, ldp >= ceil(K/5), Wp 16-byte
+ * aligned).  Equals bl_ternarize followed by bl_pack. */
+bl_status bl_ternarize_pack5(const float* W, int64_t N, int64_t K, const float* beta_dev,
+                             uint8_t* Wp, int64_t ldp, cudaStream_t stream);
+
+/* bl_absmean then bl_ternarize: the whole absmean ternarization, one trit per
+ * byte.  Wq [N, K] int8 contiguous; beta_dev receives beta (no host sync).
+ * Errors: BL_ERR_INVALID_ARG, BL_ERR_WORKSPACE, BL_ERR_CUDA; a non-finite
+ * weight sets BL_ERR_NONFINITE in the status word (codes are then unspecified). */
+bl_status bl_quantize_weights(const float* W, int64_t N, int64_t K, float eps, int8_t* Wq,
+                              float* beta_dev, void* ws, size_t ws_bytes, cudaStream_t stream);
+
+/* bl_absmean then bl_ternarize_pack5: the same codes, packed five per byte,
+ * without the int8 round trip. */
+bl_status bl_quantize_weights_pack5(const float* W, int64_t N, int64_t K, float eps,
+                                    uint8_t* Wp, int64_t ldp, float* beta_dev, void* ws,
+                                    size_t ws_bytes, cudaStream_t stream);
+
+/* int8 trits [N, K] (contiguous) -> packed [N, ldp] (format BL_W_PACK5).
+ * Codes outside {-1,0,1} are a caller error (the byte is then unspecified). */
+bl_status bl_pack(const int8_t* Wq, int64_t N, int64_t K, uint8_t* Wp, int64_t ldp,
+                  cudaStream_t stream);
+
+/* packed [N, ldp] -> int8 trits [N, K] (contiguous); the inverse of bl_pack. */
+bl_status bl_unpack(const uint8_t* Wp, int64_t N, int64_t K, int64_t ldp, int8_t* Wq,
+                    cudaStream_t stream);
+
+/* Per-row absmax int8 quantization ("the bytes"; per-token scales, section
+ * "attention, as graph ops").
+ *   X  [M, K] float32, contiguous.   Xq [M, K] int8, contiguous.   s [M] float32.
+ * Rows are independent: row m's outputs depend on row m of X only. */
+bl_status bl_quantize_act(const float* X, int64_t M, int64_t K, float eps, int8_t* Xq,
+                          float* s, cudaStream_t stream);
+
+/* Bytes of `ws` that bl_linear needs for this shape and format. */
+size_t bl_linear_workspace_size(int64_t M, int64_t N, int64_t K, bl_wfmt f);
+
+/* The BitLinear forward: Y = (X_q W_q^T)(s beta) [+ bias], X_q and s computed
+ * from X inside the call (deployed-path equation).
+ *   X        [M, K] float32 contiguous.  M may be 0 (nothing is launched).
+ *   W        weights in format f, [N, ldw] (BL_W_I8: ldw >= K; BL_W_PACK5:
+ *            ldw % 16 == 0, ldw >= ceil(K/5), W 16-byte aligned).
+ *   beta_dev the tensor's beta on the device (from bl_quantize_weights*).
+ *   bias     [N] float32 or NULL.
+ *   Y        [M, N] float32 contiguous output.
+ *   ws       >= bl_linear_workspace_size(M, N, K, f) bytes, 256-byte aligned. */
+bl_status bl_linear(const float* X, int64_t M, int64_t K, const void* W, bl_wfmt f, int64_t N,
+                    int64_t ldw, const float* beta_dev, const float* bias, float eps, float* Y,
+                    void* ws, size_t ws_bytes, cudaStream_t stream);
+
+/* bl_linear with the kernel path pinned (BL_PATH_*); BL_ERR_UNSUPPORTED when the
+ * pinned path cannot take the shape.  Results are identical across paths. */
+bl_status bl_linear_ex(const float* X, int64_t M, int64_t K, const void* W, bl_wfmt f,
+                       int64_t N, int64_t ldw, const float* beta_dev, const float* bias,
+                       float eps, float* Y, void* ws, size_t ws_bytes, int path,
+                       cudaStream_t stream);
+
+/* The kernel path bl_linear_ex(..., path) would run for this shape (BL_PATH_*),
+ * or -1 if that path cannot take it; *launches (if not NULL) receives the number
+ * of kernel launches the call makes.  Host-only, no CUDA call. */
+int bl_linear_plan(int64_t M, int64_t N, int64_t K, bl_wfmt f, int path, int* launches);
+
+/* The contraction alone: acc[m,n] = sum_k Xq[m,k] * W_q[n,k] in int32, from
+ * pre-quantized activations Xq [M, K] int8 contiguous; acc [M, N] int32.
+ * (The integer product x_q W_q^T of the deployed-path equation.) */
+bl_status bl_linear_acc(const int8_t* Xq, int64_t M, int64_t K, const void* W, bl_wfmt f,
+                        int64_t N, int64_t ldw, int32_t* acc, cudaStream_t stream);
+
+/* bl_linear_acc with the kernel path pinned; ws as for bl_linear (may be NULL
+ * when bl_linear_acc_workspace_size returns 0). */
+size_t bl_linear_acc_workspace_size(int64_t M, int64_t N, int64_t K, bl_wfmt f, int path);
+bl_status bl_linear_acc_ex(const int8_t* Xq, int64_t M, int64_t K, const void* W, bl_wfmt f,
+                           int64_t N, int64_t ldw, int32_t* acc, void* ws, size_t ws_bytes,
+                           int path, cudaStream_t stream);
+
+/* Synchronizes `stream`, then reads and clears this device's status word:
+ * BL_ERR_DEVICE_TIMEOUT or BL_ERR_NONFINITE if a kernel recorded one, BL_ERR_CUDA
+ * if the stream reports an error, else BL_OK. */
+bl_status bl_sync_status(cudaStream_t stream);
+
+/* A static, human-readable name for a status code. */
+const char* bl_status_string(bl_status s);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* BITLINEAR_H_ */

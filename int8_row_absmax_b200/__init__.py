@@ -1,0 +1,259 @@
+"""Python binding of the B200 BitLinear library (ctypes over libbitlinear.so).
+
+Argument marshalling only: every step of the computation runs in the CUDA
+kernels behind the C ABI (include/bitlinear.h).  PyTorch supplies device
+memory and the current stream.  There is no CPU fallback: if the library was
+not built, or no GPU is visible, every call raises.
+
+    import int8_row_absmax_b200 as bl
+    Wp, beta = bl.quantize_weights_pack5(W)          # W [N,K] float32 on cuda
+    Y = bl.linear(X, Wp, bl.PACK5, N=W.shape[0], K=W.shape[1], beta=beta)
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Tuple
+
+PKG_DIR = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(PKG_DIR, "libbitlinear.so")
+
+I8, PACK5 = 0, 1                       # bl_wfmt
+PATH_AUTO, PATH_SIMT, PATH_GEMV, PATH_TC = 0, 1, 2, 3   # bl_path
+
+STATUS = {0: "BL_OK", 1: "BL_ERR_INVALID_ARG", 2: "BL_ERR_ALIGNMENT", 3: "BL_ERR_UNSUPPORTED",
+          4: "BL_ERR_WORKSPACE", 5: "BL_ERR_CUDA", 6: "BL_ERR_DEVICE_TIMEOUT",
+          7: "BL_ERR_NONFINITE"}
+
+# Every symbol the header declares, with (restype, argtypes).
+_P, _I64, _SZ, _F, _I = ctypes.c_void_p, ctypes.c_int64, ctypes.c_size_t, ctypes.c_float, ctypes.c_int
+SIGNATURES = {
+    "bl_pack5_ldp": (_I64, [_I64]),
+    "bl_quantize_weights_workspace_size": (_SZ, [_I64, _I64]),
+    "bl_absmean": (_I, [_P, _I64, _I64, _F, _P, _P, _SZ, _P]),
+    "bl_ternarize": (_I, [_P, _I64, _I64, _P, _P, _P]),
+    "bl_ternarize_pack5": (_I, [_P, _I64, _I64, _P, _P, _I64, _P]),
+    "bl_quantize_weights": (_I, [_P, _I64, _I64, _F, _P, _P, _P, _SZ, _P]),
+    "bl_quantize_weights_pack5": (_I, [_P, _I64, _I64, _F, _P, _I64, _P, _P, _SZ, _P]),
+    "bl_pack": (_I, [_P, _I64, _I64, _P, _I64, _P]),
+    "bl_unpack": (_I, [_P, _I64, _I64, _I64, _P, _P]),
+    "bl_quantize_act": (_I, [_P, _I64, _I64, _F, _P, _P, _P]),
+    "bl_linear_workspace_size": (_SZ, [_I64, _I64, _I64, _I]),
+    "bl_linear": (_I, [_P, _I64, _I64, _P, _I, _I64, _I64, _P, _P, _F, _P, _P, _SZ, _P]),
+    "bl_linear_ex": (_I, [_P, _I64, _I64, _P, _I, _I64, _I64, _P, _P, _F, _P, _P, _SZ, _I, _P]),
+    "bl_linear_plan": (_I, [_I64, _I64, _I64, _I, _I, ctypes.POINTER(ctypes.c_int)]),
+    "bl_linear_acc": (_I, [_P, _I64, _I64, _P, _I, _I64, _I64, _P, _P]),
+    "bl_linear_acc_workspace_size": (_SZ, [_I64, _I64, _I64, _I, _I]),
+    "bl_linear_acc_ex": (_I, [_P, _I64, _I64, _P, _I, _I64, _I64, _P, _P, _SZ, _I, _P]),
+    "bl_sync_status": (_I, [_P]),
+    "bl_status_string": (ctypes.c_char_p, [_I]),
+}
+
+_lib = None
+
+
+class BitLinearError(RuntimeError):
+    def __init__(self, fn: str, code: int):
+        super().__init__(f"{fn} returned {STATUS.get(code, code)}")
+        self.code = code
+        self.status = STATUS.get(code, str(code))
+
+
+def load(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Load the in-tree library (raises if it has not been built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise RuntimeError(f"{path} is missing: build it with python -m int8_row_absmax_b200.build")
+    lib = ctypes.CDLL(path)
+    for name, (res, args) in SIGNATURES.items():
+        fn = getattr(lib, name)
+        fn.restype, fn.argtypes = res, args
+    _lib = lib
+    return lib
+
+
+def _torch():
+    import torch
+    if not torch.cuda.is_available():
+        raise RuntimeError("BitLinear runs on the GPU only: no CUDA device is visible")
+    return torch
+
+
+def _ptr(t) -> Optional[int]:
+    return None if t is None else t.data_ptr()
+
+
+def _stream(torch, t):
+    return ctypes.c_void_p(torch.cuda.current_stream(t.device).cuda_stream)
+
+
+def _check(fn: str, code: int):
+    if code != 0:
+        raise BitLinearError(fn, code)
+
+
+def _dev(t, dtype=None):
+    if not t.is_cuda:
+        raise ValueError("tensor must be on a CUDA device")
+    if not t.is_contiguous():
+        raise ValueError("tensor must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"expected {dtype}, got {t.dtype}")
+    return t
+
+
+def pack5_ldp(K: int) -> int:
+    return int(load().bl_pack5_ldp(K))
+
+
+def workspace(nbytes: int, device):
+    """A zero-filled, 256-byte aligned device byte buffer (torch allocations are
+    512-byte aligned).  The weight-quantization calls need it zero on first use
+    and leave it zero, so one workspace can be reused across calls."""
+    torch = _torch()
+    return torch.zeros(max(int(nbytes), 256), dtype=torch.uint8, device=device)
+
+
+def quantize_weights(W, eps: float = 1e-5, ws=None):
+    """W [N,K] float32 -> (Wq int8 [N,K], beta float32 [1] on the device)."""
+    torch, lib = _torch(), load()
+    _dev(W, torch.float32)
+    N, K = W.shape
+    Wq = torch.empty((N, K), dtype=torch.int8, device=W.device)
+    beta = torch.empty(1, dtype=torch.float32, device=W.device)
+    need = lib.bl_quantize_weights_workspace_size(N, K)
+    ws = workspace(need, W.device) if ws is None else ws
+    _check("bl_quantize_weights", lib.bl_quantize_weights(
+        _ptr(W), N, K, eps, _ptr(Wq), _ptr(beta), _ptr(ws), ws.numel(), _stream(torch, W)))
+    return Wq, beta
+
+
+def quantize_weights_pack5(W, eps: float = 1e-5, ws=None, out=None, beta=None):
+    """W [N,K] float32 -> (Wp uint8 [N, ldp], beta float32 [1] on the device)."""
+    torch, lib = _torch(), load()
+    _dev(W, torch.float32)
+    N, K = W.shape
+    ldp = pack5_ldp(K)
+    Wp = torch.empty((N, ldp), dtype=torch.uint8, device=W.device) if out is None else out
+    beta = torch.empty(1, dtype=torch.float32, device=W.device) if beta is None else beta
+    need = lib.bl_quantize_weights_workspace_size(N, K)
+    ws = workspace(need, W.device) if ws is None else ws
+    _check("bl_quantize_weights_pack5", lib.bl_quantize_weights_pack5(
+        _ptr(W), N, K, eps, _ptr(Wp), Wp.shape[1], _ptr(beta), _ptr(ws), ws.numel(),
+        _stream(torch, W)))
+    return Wp, beta
+
+
+def absmean(W, eps: float = 1e-5, ws=None, beta=None):
+    """beta = mean|W| + eps as a float32 [1] device tensor."""
+    torch, lib = _torch(), load()
+    _dev(W, torch.float32)
+    N, K = W.shape
+    beta = torch.empty(1, dtype=torch.float32, device=W.device) if beta is None else beta
+    ws = workspace(lib.bl_quantize_weights_workspace_size(N, K), W.device) if ws is None else ws
+    _check("bl_absmean", lib.bl_absmean(_ptr(W), N, K, eps, _ptr(beta), _ptr(ws), ws.numel(),
+                                        _stream(torch, W)))
+    return beta
+
+
+def ternarize(W, beta, out=None):
+    torch, lib = _torch(), load()
+    _dev(W, torch.float32)
+    N, K = W.shape
+    Wq = torch.empty((N, K), dtype=torch.int8, device=W.device) if out is None else out
+    _check("bl_ternarize", lib.bl_ternarize(_ptr(W), N, K, _ptr(beta), _ptr(Wq), _stream(torch, W)))
+    return Wq
+
+
+def ternarize_pack5(W, beta, out=None):
+    torch, lib = _torch(), load()
+    _dev(W, torch.float32)
+    N, K = W.shape
+    Wp = torch.empty((N, pack5_ldp(K)), dtype=torch.uint8, device=W.device) if out is None else out
+    _check("bl_ternarize_pack5", lib.bl_ternarize_pack5(_ptr(W), N, K, _ptr(beta), _ptr(Wp),
+                                                        Wp.shape[1], _stream(torch, W)))
+    return Wp
+
+
+def pack(Wq, ldp: Optional[int] = None):
+    torch, lib = _torch(), load()
+    _dev(Wq, torch.int8)
+    N, K = Wq.shape
+    ldp = pack5_ldp(K) if ldp is None else ldp
+    Wp = torch.empty((N, ldp), dtype=torch.uint8, device=Wq.device)
+    _check("bl_pack", lib.bl_pack(_ptr(Wq), N, K, _ptr(Wp), ldp, _stream(torch, Wq)))
+    return Wp
+
+
+def unpack(Wp, K: int):
+    torch, lib = _torch(), load()
+    _dev(Wp, torch.uint8)
+    N, ldp = Wp.shape
+    Wq = torch.empty((N, K), dtype=torch.int8, device=Wp.device)
+    _check("bl_unpack", lib.bl_unpack(_ptr(Wp), N, K, ldp, _ptr(Wq), _stream(torch, Wp)))
+    return Wq
+
+
+def quantize_act(X, eps: float = 1e-5) -> Tuple:
+    """X [M,K] float32 -> (Xq int8 [M,K], s float32 [M])."""
+    torch, lib = _torch(), load()
+    _dev(X, torch.float32)
+    M, K = X.shape
+    Xq = torch.empty((M, K), dtype=torch.int8, device=X.device)
+    s = torch.empty((M,), dtype=torch.float32, device=X.device)
+    _check("bl_quantize_act", lib.bl_quantize_act(_ptr(X), M, K, eps, _ptr(Xq), _ptr(s),
+                                                  _stream(torch, X)))
+    return Xq, s
+
+
+def linear_plan(M: int, N: int, K: int, fmt: int, path: int = PATH_AUTO):
+    """(resolved path, kernel launches) that bl_linear_ex would use; path -1 = unsupported."""
+    n = ctypes.c_int(0)
+    p = load().bl_linear_plan(M, N, K, fmt, path, ctypes.byref(n))
+    return int(p), int(n.value)
+
+
+def linear_workspace_size(M: int, N: int, K: int, fmt: int) -> int:
+    return int(load().bl_linear_workspace_size(M, N, K, fmt))
+
+
+def linear(X, W, fmt: int, N: int, K: int, beta, bias=None, eps: float = 1e-5,
+           path: int = PATH_AUTO, ws=None, out=None):
+    """Y = (X_q W_q^T)(s beta) + bias for X [M,K] float32 and W in format fmt."""
+    torch, lib = _torch(), load()
+    _dev(X, torch.float32)
+    M = X.shape[0]
+    if X.shape[1] != K or W.shape[0] != N:
+        raise ValueError("shape mismatch")
+    Y = torch.empty((M, N), dtype=torch.float32, device=X.device) if out is None else out
+    need = lib.bl_linear_workspace_size(M, N, K, fmt)
+    ws = workspace(need, X.device) if ws is None else ws
+    _check("bl_linear_ex", lib.bl_linear_ex(
+        _ptr(X), M, K, _ptr(W), fmt, N, W.shape[1], _ptr(beta), _ptr(bias), eps, _ptr(Y),
+        _ptr(ws), ws.numel(), path, _stream(torch, X)))
+    return Y
+
+
+def linear_acc(Xq, W, fmt: int, N: int, K: int, path: int = PATH_AUTO, ws=None):
+    """acc = X_q W_q^T in int32 from pre-quantized Xq [M,K] int8."""
+    torch, lib = _torch(), load()
+    _dev(Xq, torch.int8)
+    M = Xq.shape[0]
+    acc = torch.empty((M, N), dtype=torch.int32, device=Xq.device)
+    need = lib.bl_linear_acc_workspace_size(M, N, K, fmt, path)
+    if ws is None and need:
+        ws = workspace(need, Xq.device)
+    _check("bl_linear_acc_ex", lib.bl_linear_acc_ex(
+        _ptr(Xq), M, K, _ptr(W), fmt, N, W.shape[1], _ptr(acc), _ptr(ws),
+        0 if ws is None else ws.numel(), path, _stream(torch, Xq)))
+    return acc
+
+
+def sync_status(device=None) -> str:
+    """Synchronize the current stream and return the device status ("BL_OK" ...)."""
+    torch, lib = _torch(), load()
+    dev = torch.device("cuda") if device is None else device
+    code = lib.bl_sync_status(ctypes.c_void_p(torch.cuda.current_stream(dev).cuda_stream))
+    return STATUS.get(code, str(code))

@@ -1,0 +1,78 @@
+// Per-row (per-token) absmax int8 quantization of activations.
+//
+// "ultragraph -- when the graph is the 1-bit LLM, part 2", section "the bytes",
+// and the per-token fix in section "attention, as graph ops":
+//   s = max_i |x_i| / 127 + eps,   x_q = clip(round(x / s), -127, 127).
+// One scale per row, so no row's codes depend on another row.  All float32,
+// IEEE division, round half to even (rintf), in the written order.
+#pragma once
+
+#include "common.cuh"
+
+namespace bl {
+
+constexpr int kActThreads = 256;
+
+__device__ __forceinline__ int8_t act_code(float x, float s) {
+  float q = rintf(__fdiv_rn(x, s));
+  q = fminf(fmaxf(q, -float(kActQmax)), float(kActQmax));
+  return int8_t(int(q));
+}
+
+// One CTA per row: pass 1 finds max|x| (warp shuffles, then across warps), pass
+// 2 re-reads the row (an L1/L2 hit) and writes the codes.  Row stride of X is K;
+// Xq has stride ldq >= K and its bytes [K, ldq) are written as 0.
+__global__ void __launch_bounds__(kActThreads)
+act_quant_kernel(const float* __restrict__ X, int64_t K, float eps, int8_t* __restrict__ Xq,
+                 int64_t ldq, float* __restrict__ s_out) {
+  __shared__ float s_red[kActThreads / 32];
+  __shared__ float s_scale;
+  const int64_t m = blockIdx.x;
+  const float* xr = X + m * K;
+  int8_t* qr = Xq + m * ldq;
+  const bool vec = aligned(xr, 16) && aligned(qr, 4);
+  const int64_t K4 = vec ? (K >> 2) : 0;
+
+  float amax = 0.f;
+  bool bad = false;
+  for (int64_t i = threadIdx.x; i < K4; i += kActThreads) {
+    const float4 v = reinterpret_cast<const float4*>(xr)[i];
+    const float a = fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w)));
+    bad |= !(fabsf(v.x) <= 3.402823466e38f) | !(fabsf(v.y) <= 3.402823466e38f) |
+           !(fabsf(v.z) <= 3.402823466e38f) | !(fabsf(v.w) <= 3.402823466e38f);
+    amax = fmaxf(amax, a);
+  }
+  for (int64_t i = (K4 << 2) + threadIdx.x; i < K; i += kActThreads) {
+    const float a = fabsf(xr[i]);
+    bad |= !(a <= 3.402823466e38f);
+    amax = fmaxf(amax, a);
+  }
+  amax = warp_max(amax);
+  if ((threadIdx.x & 31) == 0) s_red[threadIdx.x >> 5] = amax;
+  if (__syncthreads_or(bad) && threadIdx.x == 0) raise_status(kDevNonFinite);
+  if (threadIdx.x < 32) {
+    float v = threadIdx.x < kActThreads / 32 ? s_red[threadIdx.x] : 0.f;
+    v = warp_max(v);
+    if (threadIdx.x == 0) {
+      const float s = __fadd_rn(__fdiv_rn(v, float(kActQmax)), eps);
+      s_scale = s;
+      s_out[m] = s;
+    }
+  }
+  __syncthreads();
+  const float s = s_scale;
+
+  for (int64_t i = threadIdx.x; i < K4; i += kActThreads) {
+    const float4 v = reinterpret_cast<const float4*>(xr)[i];
+    char4 q;
+    q.x = act_code(v.x, s);
+    q.y = act_code(v.y, s);
+    q.z = act_code(v.z, s);
+    q.w = act_code(v.w, s);
+    reinterpret_cast<char4*>(qr)[i] = q;
+  }
+  for (int64_t i = (K4 << 2) + threadIdx.x; i < K; i += kActThreads) qr[i] = act_code(xr[i], s);
+  for (int64_t i = K + threadIdx.x; i < ldq; i += kActThreads) qr[i] = 0;
+}
+
+}  // namespace bl

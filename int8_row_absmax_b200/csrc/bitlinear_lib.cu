@@ -1,0 +1,321 @@
+// C ABI of the BitLinear library (declared in include/bitlinear.h).
+//
+// Host-side argument checks, workspace carving and kernel dispatch.  Every
+// step of the computation runs in the kernels included below; there is no CPU
+// fallback.  One translation unit, so the per-device status word is a single
+// symbol without relocatable device code.
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+
+#include <cuda_runtime.h>
+
+#include "bitlinear.h"
+#include "common.cuh"
+#include "weight_quant.cuh"
+#include "pack.cuh"
+#include "act_quant.cuh"
+#include "linear_simt.cuh"
+
+namespace bl {
+namespace {
+
+constexpr size_t kWsAlign = 256;
+
+size_t align_up(size_t v) { return (v + kWsAlign - 1) / kWsAlign * kWsAlign; }
+
+bool eps_ok(float eps) { return std::isfinite(eps) && eps > 0.f; }
+
+bool is_aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+int num_sms() {
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  return sms > 0 ? sms : 148;
+}
+
+unsigned grid_for(int64_t work, int per_block, int max_blocks_per_sm = 8) {
+  int64_t g = ceil_div(work, per_block);
+  const int64_t cap = int64_t(num_sms()) * max_blocks_per_sm;
+  if (g > cap) g = cap;
+  return unsigned(g < 1 ? 1 : g);
+}
+
+bl_status launch_status() {
+  const cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? BL_OK : BL_ERR_CUDA;
+}
+
+bl_status check_weights_args(const float* W, int64_t N, int64_t K, const void* out) {
+  if (!W || !out || N < 1 || K < 1) return BL_ERR_INVALID_ARG;
+  if (N > (int64_t(1) << 40) / K) return BL_ERR_INVALID_ARG;
+  if (!is_aligned(W, 4)) return BL_ERR_ALIGNMENT;
+  return BL_OK;
+}
+
+// a1: beta of a weight tensor into beta_dev, one launch.
+bl_status launch_absmean(const float* W, int64_t n, float eps, float* beta_dev, void* ws,
+                         cudaStream_t st) {
+  auto* acc = static_cast<AbsAccum*>(ws);
+  absmean_kernel<<<grid_for(ceil_div(n, 16), kAbsThreads, 2), kAbsThreads, 0, st>>>(W, n, eps, acc, beta_dev);
+  return launch_status();
+}
+
+bl_status check_ws(const void* ws, size_t ws_bytes, size_t need) {
+  if (!ws || !is_aligned(ws, kWsAlign) || ws_bytes < need) return BL_ERR_WORKSPACE;
+  return BL_OK;
+}
+
+// ---- linear --------------------------------------------------------------
+struct LinWs {
+  int64_t ldx;
+  size_t xq_off, s_off, total;
+};
+LinWs lin_layout(int64_t M, int64_t K) {
+  LinWs l;
+  l.ldx = round_up(K, 16);
+  l.xq_off = 0;
+  l.s_off = align_up(size_t(M) * size_t(l.ldx));
+  l.total = l.s_off + align_up(size_t(M) * 4 + 4);
+  return l;
+}
+
+bl_status check_w(const void* W, bl_wfmt f, int64_t K, int64_t ldw) {
+  if (!W) return BL_ERR_INVALID_ARG;
+  if (f == BL_W_I8) {
+    if (ldw < K) return BL_ERR_INVALID_ARG;
+  } else if (f == BL_W_PACK5) {
+    if (ldw < ceil_div(K, 5)) return BL_ERR_INVALID_ARG;
+    if (ldw % 16 != 0 || !is_aligned(W, 16)) return BL_ERR_ALIGNMENT;
+  } else {
+    return BL_ERR_INVALID_ARG;
+  }
+  return BL_OK;
+}
+
+bl_status check_shape(int64_t M, int64_t K, int64_t N) {
+  if (M < 0 || N < 1 || K < 1 || K > kMaxK) return BL_ERR_INVALID_ARG;
+  if (M > (int64_t(1) << 31) - 1 || N > (int64_t(1) << 31) - 1) return BL_ERR_INVALID_ARG;
+  return BL_OK;
+}
+
+// Resolve the kernel path for a linear call; -1 when the pinned path cannot run it.
+int resolve_path(int64_t M, int64_t N, int64_t K, bl_wfmt f, int path, int* launches) {
+  (void)N;
+  (void)K;
+  (void)f;
+  int p = path;
+  if (p == BL_PATH_AUTO) p = BL_PATH_SIMT;
+  if (p != BL_PATH_SIMT) return -1;
+  if (launches) *launches = M == 0 ? 0 : 2;  // act_quant + contraction
+  return p;
+}
+
+bl_status run_simt(const int8_t* Xq, int64_t ldx, int64_t M, int64_t K, const void* W,
+                   bl_wfmt f, int64_t ldw, int64_t N, const float* s, const float* beta,
+                   const float* bias, float* Y, int32_t* acc, cudaStream_t st) {
+  const dim3 grid(unsigned(ceil_div(N, kSimtBN)), unsigned(ceil_div(M, kSimtBM)));
+  if (grid.y > 65535u) return BL_ERR_UNSUPPORTED;
+  const bool packed = f == BL_W_PACK5;
+  if (Y) {
+    if (packed) linear_simt_kernel<true, true><<<grid, 256, 0, st>>>(Xq, ldx, M, K, W, ldw, N, s, beta, bias, Y, nullptr);
+    else linear_simt_kernel<false, true><<<grid, 256, 0, st>>>(Xq, ldx, M, K, W, ldw, N, s, beta, bias, Y, nullptr);
+  } else {
+    if (packed) linear_simt_kernel<true, false><<<grid, 256, 0, st>>>(Xq, ldx, M, K, W, ldw, N, nullptr, nullptr, nullptr, nullptr, acc);
+    else linear_simt_kernel<false, false><<<grid, 256, 0, st>>>(Xq, ldx, M, K, W, ldw, N, nullptr, nullptr, nullptr, nullptr, acc);
+  }
+  return launch_status();
+}
+
+}  // namespace
+}  // namespace bl
+
+using namespace bl;
+
+extern "C" {
+
+int64_t bl_pack5_ldp(int64_t K) { return K < 1 ? 0 : round_up(ceil_div(K, 5), 16); }
+
+size_t bl_quantize_weights_workspace_size(int64_t N, int64_t K) {
+  if (N < 1 || K < 1) return 0;
+  return kAbsWsBytes;
+}
+
+bl_status bl_absmean(const float* W, int64_t N, int64_t K, float eps, float* beta_dev, void* ws,
+                     size_t ws_bytes, cudaStream_t stream) {
+  bl_status st = check_weights_args(W, N, K, beta_dev);
+  if (st != BL_OK) return st;
+  if (!eps_ok(eps)) return BL_ERR_INVALID_ARG;
+  if (!is_aligned(beta_dev, 4)) return BL_ERR_ALIGNMENT;
+  if ((st = check_ws(ws, ws_bytes, kAbsWsBytes)) != BL_OK) return st;
+  return launch_absmean(W, N * K, eps, beta_dev, ws, stream);
+}
+
+bl_status bl_ternarize(const float* W, int64_t N, int64_t K, const float* beta_dev, int8_t* Wq,
+                       cudaStream_t stream) {
+  bl_status st = check_weights_args(W, N, K, Wq);
+  if (st != BL_OK) return st;
+  if (!beta_dev) return BL_ERR_INVALID_ARG;
+  if (!is_aligned(beta_dev, 4)) return BL_ERR_ALIGNMENT;
+  const int64_t n = N * K;
+  ternarize_i8_kernel<<<grid_for(ceil_div(n, 4), 256), 256, 0, stream>>>(W, n, beta_dev, Wq);
+  return launch_status();
+}
+
+bl_status bl_ternarize_pack5(const float* W, int64_t N, int64_t K, const float* beta_dev,
+                             uint8_t* Wp, int64_t ldp, cudaStream_t stream) {
+  bl_status st = check_weights_args(W, N, K, Wp);
+  if (st != BL_OK) return st;
+  if (!beta_dev || ldp < ceil_div(K, 5)) return BL_ERR_INVALID_ARG;
+  if (ldp % 16 != 0 || !is_aligned(Wp, 16) || !is_aligned(beta_dev, 4)) return BL_ERR_ALIGNMENT;
+  ternarize_pack5_kernel<<<grid_for(N * (ldp / 4), 256), 256, 0, stream>>>(W, N, K, beta_dev, Wp, ldp);
+  return launch_status();
+}
+
+bl_status bl_quantize_weights(const float* W, int64_t N, int64_t K, float eps, int8_t* Wq,
+                              float* beta_dev, void* ws, size_t ws_bytes, cudaStream_t stream) {
+  bl_status st = check_weights_args(W, N, K, Wq);
+  if (st != BL_OK) return st;
+  st = bl_absmean(W, N, K, eps, beta_dev, ws, ws_bytes, stream);
+  if (st != BL_OK) return st;
+  return bl_ternarize(W, N, K, beta_dev, Wq, stream);
+}
+
+bl_status bl_quantize_weights_pack5(const float* W, int64_t N, int64_t K, float eps,
+                                    uint8_t* Wp, int64_t ldp, float* beta_dev, void* ws,
+                                    size_t ws_bytes, cudaStream_t stream) {
+  bl_status st = check_weights_args(W, N, K, Wp);
+  if (st != BL_OK) return st;
+  if (ldp < ceil_div(K, 5)) return BL_ERR_INVALID_ARG;
+  if (ldp % 16 != 0 || !is_aligned(Wp, 16)) return BL_ERR_ALIGNMENT;
+  st = bl_absmean(W, N, K, eps, beta_dev, ws, ws_bytes, stream);
+  if (st != BL_OK) return st;
+  return bl_ternarize_pack5(W, N, K, beta_dev, Wp, ldp, stream);
+}
+
+bl_status bl_pack(const int8_t* Wq, int64_t N, int64_t K, uint8_t* Wp, int64_t ldp,
+                  cudaStream_t stream) {
+  if (!Wq || !Wp || N < 1 || K < 1 || ldp < ceil_div(K, 5)) return BL_ERR_INVALID_ARG;
+  if (ldp % 16 != 0 || !is_aligned(Wp, 16)) return BL_ERR_ALIGNMENT;
+  pack5_kernel<<<grid_for(N * (ldp / 4), 256), 256, 0, stream>>>(Wq, N, K, Wp, ldp);
+  return launch_status();
+}
+
+bl_status bl_unpack(const uint8_t* Wp, int64_t N, int64_t K, int64_t ldp, int8_t* Wq,
+                    cudaStream_t stream) {
+  if (!Wq || !Wp || N < 1 || K < 1 || ldp < ceil_div(K, 5)) return BL_ERR_INVALID_ARG;
+  unpack5_kernel<<<grid_for(N * ceil_div(K, 5), 256), 256, 0, stream>>>(Wp, N, K, ldp, Wq, K);
+  return launch_status();
+}
+
+bl_status bl_quantize_act(const float* X, int64_t M, int64_t K, float eps, int8_t* Xq,
+                          float* s, cudaStream_t stream) {
+  if (M < 0 || K < 1 || !eps_ok(eps)) return BL_ERR_INVALID_ARG;
+  if (M == 0) return BL_OK;
+  if (!X || !Xq || !s || M > (int64_t(1) << 31) - 1) return BL_ERR_INVALID_ARG;
+  if (!is_aligned(X, 4) || !is_aligned(s, 4)) return BL_ERR_ALIGNMENT;
+  act_quant_kernel<<<unsigned(M), kActThreads, 0, stream>>>(X, K, eps, Xq, K, s);
+  return launch_status();
+}
+
+size_t bl_linear_workspace_size(int64_t M, int64_t N, int64_t K, bl_wfmt f) {
+  (void)N;
+  (void)f;
+  if (M < 0 || K < 1) return 0;
+  return lin_layout(M, K).total;
+}
+
+bl_status bl_linear_ex(const float* X, int64_t M, int64_t K, const void* W, bl_wfmt f,
+                       int64_t N, int64_t ldw, const float* beta_dev, const float* bias,
+                       float eps, float* Y, void* ws, size_t ws_bytes, int path,
+                       cudaStream_t stream) {
+  bl_status st = check_shape(M, K, N);
+  if (st != BL_OK) return st;
+  if (!eps_ok(eps)) return BL_ERR_INVALID_ARG;
+  st = check_w(W, f, K, ldw);
+  if (st != BL_OK) return st;
+  if (path < BL_PATH_AUTO || path > BL_PATH_TC) return BL_ERR_INVALID_ARG;
+  if (M == 0) return BL_OK;
+  if (!X || !Y || !beta_dev) return BL_ERR_INVALID_ARG;
+  if (!is_aligned(X, 4) || !is_aligned(Y, 4) || (bias && !is_aligned(bias, 4))) return BL_ERR_ALIGNMENT;
+  const LinWs l = lin_layout(M, K);
+  if (!ws || !is_aligned(ws, kWsAlign) || ws_bytes < l.total) return BL_ERR_WORKSPACE;
+  if (resolve_path(M, N, K, f, path, nullptr) < 0) return BL_ERR_UNSUPPORTED;
+  int8_t* Xq = reinterpret_cast<int8_t*>(static_cast<char*>(ws) + l.xq_off);
+  float* s = reinterpret_cast<float*>(static_cast<char*>(ws) + l.s_off);
+  act_quant_kernel<<<unsigned(M), kActThreads, 0, stream>>>(X, K, eps, Xq, l.ldx, s);
+  st = launch_status();
+  if (st != BL_OK) return st;
+  return run_simt(Xq, l.ldx, M, K, W, f, ldw, N, s, beta_dev, bias, Y, nullptr, stream);
+}
+
+int bl_linear_plan(int64_t M, int64_t N, int64_t K, bl_wfmt f, int path, int* launches) {
+  if (check_shape(M, K, N) != BL_OK || (f != BL_W_I8 && f != BL_W_PACK5)) return -1;
+  if (path < BL_PATH_AUTO || path > BL_PATH_TC) return -1;
+  return resolve_path(M, N, K, f, path, launches);
+}
+
+bl_status bl_linear(const float* X, int64_t M, int64_t K, const void* W, bl_wfmt f, int64_t N,
+                    int64_t ldw, const float* beta_dev, const float* bias, float eps, float* Y,
+                    void* ws, size_t ws_bytes, cudaStream_t stream) {
+  return bl_linear_ex(X, M, K, W, f, N, ldw, beta_dev, bias, eps, Y, ws, ws_bytes,
+                      BL_PATH_AUTO, stream);
+}
+
+size_t bl_linear_acc_workspace_size(int64_t M, int64_t N, int64_t K, bl_wfmt f, int path) {
+  (void)M;
+  (void)N;
+  (void)K;
+  (void)f;
+  (void)path;
+  return 0;
+}
+
+bl_status bl_linear_acc_ex(const int8_t* Xq, int64_t M, int64_t K, const void* W, bl_wfmt f,
+                           int64_t N, int64_t ldw, int32_t* acc, void* ws, size_t ws_bytes,
+                           int path, cudaStream_t stream) {
+  (void)ws;
+  (void)ws_bytes;
+  bl_status st = check_shape(M, K, N);
+  if (st != BL_OK) return st;
+  st = check_w(W, f, K, ldw);
+  if (st != BL_OK) return st;
+  if (path < BL_PATH_AUTO || path > BL_PATH_TC) return BL_ERR_INVALID_ARG;
+  if (M == 0) return BL_OK;
+  if (!Xq || !acc) return BL_ERR_INVALID_ARG;
+  if (!is_aligned(acc, 4)) return BL_ERR_ALIGNMENT;
+  if (path == BL_PATH_GEMV || path == BL_PATH_TC) return BL_ERR_UNSUPPORTED;
+  return run_simt(Xq, K, M, K, W, f, ldw, N, nullptr, nullptr, nullptr, nullptr, acc, stream);
+}
+
+bl_status bl_linear_acc(const int8_t* Xq, int64_t M, int64_t K, const void* W, bl_wfmt f,
+                        int64_t N, int64_t ldw, int32_t* acc, cudaStream_t stream) {
+  return bl_linear_acc_ex(Xq, M, K, W, f, N, ldw, acc, nullptr, 0, BL_PATH_AUTO, stream);
+}
+
+bl_status bl_sync_status(cudaStream_t stream) {
+  if (cudaStreamSynchronize(stream) != cudaSuccess) return BL_ERR_CUDA;
+  unsigned int word = 0u, zero = 0u;
+  if (cudaMemcpyFromSymbol(&word, g_status, sizeof(word)) != cudaSuccess) return BL_ERR_CUDA;
+  if (word && cudaMemcpyToSymbol(g_status, &zero, sizeof(zero)) != cudaSuccess) return BL_ERR_CUDA;
+  if (word & kDevTimeout) return BL_ERR_DEVICE_TIMEOUT;
+  if (word & kDevBadWorkspace) return BL_ERR_WORKSPACE;
+  if (word & kDevNonFinite) return BL_ERR_NONFINITE;
+  return launch_status();
+}
+
+const char* bl_status_string(bl_status s) {
+  switch (s) {
+    case BL_OK: return "BL_OK";
+    case BL_ERR_INVALID_ARG: return "BL_ERR_INVALID_ARG";
+    case BL_ERR_ALIGNMENT: return "BL_ERR_ALIGNMENT";
+    case BL_ERR_UNSUPPORTED: return "BL_ERR_UNSUPPORTED";
+    case BL_ERR_WORKSPACE: return "BL_ERR_WORKSPACE";
+    case BL_ERR_CUDA: return "BL_ERR_CUDA";
+    case BL_ERR_DEVICE_TIMEOUT: return "BL_ERR_DEVICE_TIMEOUT";
+    case BL_ERR_NONFINITE: return "BL_ERR_NONFINITE";
+  }
+  return "BL_ERR_UNKNOWN";
+}
+
+}  // extern "C"

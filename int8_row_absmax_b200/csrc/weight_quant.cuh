@@ -1,0 +1,275 @@
+// Absmean ternarization of a weight tensor.
+//
+// "ultragraph -- when the graph is the 1-bit LLM, part 2", section "the bytes":
+//   beta = (1/n) sum_i |W_i| + eps,   W_q = clip(round(W / beta), -1, 1).
+//
+// beta needs the exact sum of n float32 magnitudes: any float32 or float64 running
+// sum depends on the reduction order, and a one-ulp change in beta flips codes
+// that sit on a rounding boundary.  Every finite float32 |w| is m * 2^(e-150)
+// (m < 2^24, e the biased exponent), so the sum is an integer in units of 2^-149.
+//
+//   absmean (one launch):
+//     1. each thread adds magnitudes with exponents in a fast window [110, 140]
+//        into a 96-bit fixed-point accumulator (unit 2^-40); any other magnitude
+//        goes to per-exponent 64-bit bins in shared memory;
+//     2. each CTA adds its three 32-bit limb sums and its non-zero bins into the
+//        workspace accumulator block with 64-bit atomics (integer adds are exact,
+//        so the total does not depend on the schedule), then takes a ticket;
+//     3. the CTA that takes the last ticket places every bin and limb at its bit
+//        offset in a 512-bit integer (word-parallel, then one carry pass), rounds
+//        it once to float64 (nearest-even), divides by n in float64 (IEEE),
+//        rounds to float32, adds eps in float32, and clears the block again.
+//     The block must therefore be zero before the first call on a workspace;
+//     every call leaves it zero.  A magic word that must read 0 catches most
+//     workspaces that were never cleared (reported as BL_ERR_WORKSPACE).
+//   ternarize*:       round(w/beta) != 0 exactly when float32(|w|/beta) > 0.5,
+//                     i.e. (ties go to the even 0.5) when the real quotient exceeds
+//                     0.5 + 2^-25.  So the code is nonzero iff |w| > beta (0.5 +
+//                     2^-25); that product is exact in float64, and T = the least
+//                     float32 above it turns the test into one float compare per
+//                     weight, with the same codes as the IEEE division.
+#pragma once
+
+#include "common.cuh"
+
+namespace bl {
+
+constexpr int kAbsThreads = 256;
+constexpr uint32_t kFastLo = 110;  // exponent whose mantissa LSB is 2^-40
+constexpr uint32_t kFastHi = 140;  // m << 30 < 2^54: 2^42 adds fit in 96 bits
+
+// Accumulator block at the start of the weight-quantization workspace.
+struct AbsAccum {
+  unsigned long long limb[4];   // sums of the 32-bit limbs of the fast accumulators
+  unsigned long long bins[256]; // sum of m per biased exponent outside the window
+  unsigned int ticket;          // CTAs done so far in the current call
+  unsigned int magic;           // must be 0: a never-cleared workspace reads non-zero
+};
+constexpr size_t kAbsWsBytes = 4096;
+static_assert(sizeof(AbsAccum) <= kAbsWsBytes, "accumulator block");
+
+__device__ __forceinline__ void absmean_add(float w, unsigned long long& lo, uint32_t& hi,
+                                            unsigned long long* s_bins, bool& bad) {
+  const uint32_t u = __float_as_uint(w) & 0x7FFFFFFFu;
+  const uint32_t e = u >> 23;
+  const uint32_t sh = e - kFastLo;  // wraps for e < kFastLo
+  if (sh <= kFastHi - kFastLo) {
+    const unsigned long long v = (unsigned long long)((u & 0x7FFFFFu) | 0x800000u) << sh;
+    lo += v;
+    hi += (lo < v) ? 1u : 0u;
+  } else if (e == 255u) {
+    bad = true;
+  } else {
+    const uint32_t m = (u & 0x7FFFFFu) | (e ? 0x800000u : 0u);
+    if (m) atomicAdd(&s_bins[e], (unsigned long long)m);
+  }
+}
+
+// Ternary threshold T from beta: the least float32 strictly above beta*(0.5+2^-25).
+__device__ __forceinline__ float ternary_threshold(float beta) {
+  const double tm = __dmul_rn(double(beta), 0.5000000298023223876953125);  // exact
+  float T = __double2float_ru(tm);
+  if (double(T) == tm) T = __uint_as_float(__float_as_uint(T) + 1u);
+  return T;
+}
+
+constexpr int kBigWords = 16;  // 512 bits; the sum is below 2^330 units of 2^-149
+
+// Step 3, run by the last CTA: the exact sum as an integer, rounded once.
+__device__ void absmean_finalize(AbsAccum* acc, int64_t n, float eps, float* beta_out,
+                                 unsigned long long* s_word, uint32_t* s_big) {
+  const int t = threadIdx.x;
+  for (int i = t; i < kBigWords + 3; i += blockDim.x) s_word[i] = 0ull;
+  __syncthreads();
+  for (int j = t; j < 258; j += blockDim.x) {
+    unsigned long long v;
+    int shift;
+    if (j < 255) {
+      v = __ldcg(&acc->bins[j]);
+      shift = (j > 0 ? j : 1) - 1;                // m * 2^(max(e,1)-150) in units of 2^-149
+    } else {
+      v = __ldcg(&acc->limb[j - 255]);
+      shift = 32 * (j - 255) + int(kFastLo) - 1;  // limb i weighs 2^(32 i) * 2^(kFastLo-150)
+    }
+    if (v) {
+      const int w = shift >> 5, b = shift & 31;
+      const unsigned long long lo64 = v << b, hi64 = b ? (v >> (64 - b)) : 0ull;
+      atomicAdd(&s_word[w], lo64 & 0xFFFFFFFFull);
+      atomicAdd(&s_word[w + 1], lo64 >> 32);
+      atomicAdd(&s_word[w + 2], hi64);
+    }
+  }
+  __syncthreads();
+  // leave the block zero for the next call
+  for (int j = t; j < 256; j += blockDim.x) acc->bins[j] = 0ull;
+  if (t < 4) acc->limb[t] = 0ull;
+  if (t == 0) {
+    if (__ldcg(&acc->magic) != 0u) raise_status(kDevBadWorkspace);
+    acc->ticket = 0u;
+  }
+  if (t != 0) return;
+  unsigned long long carry = 0ull;
+  for (int i = 0; i < kBigWords; ++i) {
+    const unsigned long long sw = s_word[i] + carry;
+    s_big[i] = uint32_t(sw);
+    carry = sw >> 32;
+  }
+  int top = -1;
+  for (int i = kBigWords - 1; i >= 0; --i)
+    if (s_big[i]) { top = i * 32 + 31 - __clz(s_big[i]); break; }
+  double D = 0.0;
+  if (top >= 0) {
+    const int lsb = top - 52 > 0 ? top - 52 : 0;   // lowest bit kept in the mantissa
+    const int w0 = lsb >> 5, b0 = lsb & 31;
+    unsigned long long mant = ((unsigned long long)s_big[w0] |
+                               (w0 + 1 < kBigWords ? (unsigned long long)s_big[w0 + 1] << 32 : 0ull)) >> b0;
+    if (b0 && w0 + 2 < kBigWords) mant |= (unsigned long long)s_big[w0 + 2] << (64 - b0);
+    mant &= (1ull << (top - lsb + 1)) - 1ull;      // the bits [lsb, top]
+    if (lsb > 0) {                                 // round to nearest, ties to even
+      const int rpos = lsb - 1;
+      const int rnd = int((s_big[rpos >> 5] >> (rpos & 31)) & 1u);
+      bool sticky = (s_big[rpos >> 5] & ((1u << (rpos & 31)) - 1u)) != 0u;
+      for (int i = (rpos >> 5) - 1; i >= 0 && !sticky; --i) sticky = s_big[i] != 0u;
+      if (rnd && (sticky || (mant & 1ull))) mant += 1ull;  // 2^53 stays exact
+    }
+    D = ldexp(double(mant), lsb - 149);
+  }
+  const double d = __ddiv_rn(D, double(n));
+  *beta_out = __fadd_rn(__double2float_rn(d), eps);
+}
+
+__global__ void __launch_bounds__(kAbsThreads)
+absmean_kernel(const float* __restrict__ W, int64_t n, float eps, AbsAccum* __restrict__ acc,
+               float* __restrict__ beta_out) {
+  __shared__ unsigned long long s_bins[256];
+  __shared__ unsigned long long s_limb[3];
+  __shared__ unsigned long long s_word[kBigWords + 3];
+  __shared__ uint32_t s_big[kBigWords];
+  __shared__ bool s_last;
+  for (int i = threadIdx.x; i < 256; i += blockDim.x) s_bins[i] = 0ull;
+  if (threadIdx.x < 3) s_limb[threadIdx.x] = 0ull;
+  __syncthreads();
+
+  unsigned long long lo = 0ull;
+  uint32_t hi = 0u;
+  bool bad = false;
+  const int64_t tid = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
+  const int64_t nthr = int64_t(gridDim.x) * blockDim.x;
+  if (aligned(W, 16)) {
+    const int64_t n4 = n >> 2;
+    const float4* W4 = reinterpret_cast<const float4*>(W);
+    int64_t i = tid;
+    for (; i + 3 * nthr < n4; i += 4 * nthr) {
+      float4 v[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) v[u] = ld_stream_f4(W4 + i + u * nthr);
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        absmean_add(v[u].x, lo, hi, s_bins, bad);
+        absmean_add(v[u].y, lo, hi, s_bins, bad);
+        absmean_add(v[u].z, lo, hi, s_bins, bad);
+        absmean_add(v[u].w, lo, hi, s_bins, bad);
+      }
+    }
+    for (; i < n4; i += nthr) {
+      const float4 v = ld_stream_f4(W4 + i);
+      absmean_add(v.x, lo, hi, s_bins, bad);
+      absmean_add(v.y, lo, hi, s_bins, bad);
+      absmean_add(v.z, lo, hi, s_bins, bad);
+      absmean_add(v.w, lo, hi, s_bins, bad);
+    }
+    for (int64_t j = (n4 << 2) + tid; j < n; j += nthr) absmean_add(W[j], lo, hi, s_bins, bad);
+  } else {
+    for (int64_t j = tid; j < n; j += nthr) absmean_add(W[j], lo, hi, s_bins, bad);
+  }
+
+  // Exact CTA reduction of the 96-bit accumulators as three 32-bit limbs
+  // (each limb sum stays below 2^40).
+  const unsigned long long l0 = warp_sum_u64(lo & 0xFFFFFFFFull);
+  const unsigned long long l1 = warp_sum_u64(lo >> 32);
+  const unsigned long long l2 = warp_sum_u64((unsigned long long)hi);
+  if ((threadIdx.x & 31) == 0) {
+    atomicAdd(&s_limb[0], l0);
+    atomicAdd(&s_limb[1], l1);
+    atomicAdd(&s_limb[2], l2);
+  }
+  if (__syncthreads_or(bad) && threadIdx.x == 0) raise_status(kDevNonFinite);
+  for (int i = threadIdx.x; i < 256; i += blockDim.x)
+    if (s_bins[i]) atomicAdd(&acc->bins[i], s_bins[i]);
+  if (threadIdx.x < 3 && s_limb[threadIdx.x]) atomicAdd(&acc->limb[threadIdx.x], s_limb[threadIdx.x]);
+
+  // Last-CTA-done: the CTA whose ticket completes the grid finalizes.
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    const unsigned int ticket = atomicAdd(&acc->ticket, 1u);
+    if (ticket >= gridDim.x) raise_status(kDevBadWorkspace);
+    s_last = (ticket == gridDim.x - 1);
+  }
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  absmean_finalize(acc, n, eps, beta_out, s_word, s_big);
+}
+
+// W [N,K] float32 -> Wq [N,K] int8 codes.
+__global__ void __launch_bounds__(256)
+ternarize_i8_kernel(const float* __restrict__ W, int64_t n, const float* __restrict__ beta,
+                    int8_t* __restrict__ Wq) {
+  const float T = ternary_threshold(*beta);
+  const int64_t tid = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
+  const int64_t nthr = int64_t(gridDim.x) * blockDim.x;
+  if (aligned(W, 16) && aligned(Wq, 4)) {
+    const int64_t n4 = n >> 2;
+    for (int64_t i = tid; i < n4; i += nthr) {
+      const float4 v = ld_stream_f4(reinterpret_cast<const float4*>(W) + i);
+      char4 q;
+      q.x = char(trit_code(v.x, T));
+      q.y = char(trit_code(v.y, T));
+      q.z = char(trit_code(v.z, T));
+      q.w = char(trit_code(v.w, T));
+      reinterpret_cast<char4*>(Wq)[i] = q;
+    }
+    for (int64_t j = (n4 << 2) + tid; j < n; j += nthr) Wq[j] = int8_t(trit_code(W[j], T));
+  } else {
+    for (int64_t j = tid; j < n; j += nthr) Wq[j] = int8_t(trit_code(W[j], T));
+  }
+}
+
+// W [N,K] float32 -> Wp [N,ldp] packed bytes.  One thread per 4 output bytes
+// (20 weights): a 32-bit store, and five 128-bit loads when the group is whole.
+__global__ void __launch_bounds__(256)
+ternarize_pack5_kernel(const float* __restrict__ W, int64_t N, int64_t K,
+                       const float* __restrict__ beta, uint8_t* __restrict__ Wp, int64_t ldp) {
+  const float T = ternary_threshold(*beta);
+  const int64_t words = ldp >> 2;
+  const int64_t total = N * words;
+  const bool vec = aligned(W, 16) && (K & 3) == 0;
+  for (int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
+       i += int64_t(gridDim.x) * blockDim.x) {
+    const int64_t row = i / words, g = i - row * words;
+    const int64_t k0 = g * 20;
+    const float* wr = W + row * K;
+    uint32_t d[20];
+    if (vec && k0 + 20 <= K) {
+#pragma unroll
+      for (int v = 0; v < 5; ++v) {
+        const float4 f = ld_stream_f4(reinterpret_cast<const float4*>(wr + k0) + v);
+        d[4 * v + 0] = trit_digit(f.x, T);
+        d[4 * v + 1] = trit_digit(f.y, T);
+        d[4 * v + 2] = trit_digit(f.z, T);
+        d[4 * v + 3] = trit_digit(f.w, T);
+      }
+    } else {
+#pragma unroll
+      for (int k = 0; k < 20; ++k) d[k] = (k0 + k < K) ? trit_digit(wr[k0 + k], T) : 1u;
+    }
+    uint32_t word = 0u;
+#pragma unroll
+    for (int b = 0; b < 4; ++b)
+      word |= pack5_digits(d[5 * b], d[5 * b + 1], d[5 * b + 2], d[5 * b + 3], d[5 * b + 4]) << (8 * b);
+    *reinterpret_cast<uint32_t*>(Wp + row * ldp + 4 * g) = word;
+  }
+}
+
+}  // namespace bl

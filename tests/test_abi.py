@@ -1,0 +1,105 @@
+"""The C-ABI library without a GPU: it builds, loads, exports every symbol the
+header declares, and its host-side checks reject bad arguments before any CUDA
+call is made (no compute runs here)."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+import int8_row_absmax_b200 as pkg
+from int8_row_absmax_b200 import build as blbuild
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "bitlinear.h")
+
+
+def header_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(bl_\w+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    blbuild.build()
+    return pkg.load()
+
+
+def test_header_matches_binding_table():
+    assert header_functions() == sorted(pkg.SIGNATURES)
+
+
+def test_every_declared_symbol_is_exported(lib):
+    out = subprocess.run(["nm", "-D", "--defined-only", pkg.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = set(re.findall(r"\bT (bl_\w+)$", out, flags=re.M))
+    assert set(header_functions()) == exported
+    for name in header_functions():
+        assert getattr(lib, name) is not None
+
+
+def test_pack5_ldp(lib):
+    assert [lib.bl_pack5_ldp(k) for k in (1, 5, 80, 81, 128, 2560, 6912, 8192, 11008)] == \
+        [16, 16, 16, 32, 32, 512, 1392, 1648, 2208]
+    assert lib.bl_pack5_ldp(0) == 0
+
+
+def test_status_strings(lib):
+    for code, name in pkg.STATUS.items():
+        assert lib.bl_status_string(code).decode() == name
+
+
+def test_workspace_sizes(lib):
+    assert lib.bl_quantize_weights_workspace_size(0, 5) == 0
+    assert lib.bl_quantize_weights_workspace_size(4, 4) == 4096
+    assert lib.bl_quantize_weights_workspace_size(8192, 8192) == 4096
+    assert lib.bl_linear_workspace_size(16, 64, 100, 1) >= 16 * 112 + 16 * 4
+
+
+NULL = None
+
+
+@pytest.mark.parametrize("case,expect", [
+    # null weights / bad sizes / eps
+    (lambda L: L.bl_linear(1, 1, 8, NULL, 0, 4, 8, 1, NULL, 1e-5, 1, 1, 1 << 20, NULL), 1),
+    (lambda L: L.bl_linear(1, 1, 0, 16, 0, 4, 8, 1, NULL, 1e-5, 1, 1, 1 << 20, NULL), 1),
+    (lambda L: L.bl_linear(1, 1, 8, 16, 0, 4, 8, 1, NULL, 0.0, 1, 1, 1 << 20, NULL), 1),
+    (lambda L: L.bl_linear(1, 1, 8, 16, 0, 4, 8, 1, NULL, float("nan"), 1, 1, 1 << 20, NULL), 1),
+    (lambda L: L.bl_linear(1, 1, 200000, 16, 0, 4, 200000, 1, NULL, 1e-5, 1, 1, 1 << 20, NULL), 1),
+    (lambda L: L.bl_linear(1, -1, 8, 16, 0, 4, 8, 1, NULL, 1e-5, 1, 1, 1 << 20, NULL), 1),
+    # I8 weights with ldw < K
+    (lambda L: L.bl_linear(1, 1, 8, 16, 0, 4, 7, 1, NULL, 1e-5, 1, 1, 1 << 20, NULL), 1),
+    # packed weights: unaligned pointer, bad stride
+    (lambda L: L.bl_linear(16, 1, 8, 17, 1, 4, 16, 16, NULL, 1e-5, 16, 256, 1 << 20, NULL), 2),
+    (lambda L: L.bl_linear(16, 1, 8, 16, 1, 4, 8, 16, NULL, 1e-5, 16, 256, 1 << 20, NULL), 2),
+    # unknown format / path
+    (lambda L: L.bl_linear(16, 1, 8, 16, 7, 4, 16, 16, NULL, 1e-5, 16, 256, 1 << 20, NULL), 1),
+    (lambda L: L.bl_linear_ex(16, 1, 8, 16, 1, 4, 16, 16, NULL, 1e-5, 16, 256, 1 << 20, 9, NULL), 1),
+    # workspace missing / too small / unaligned
+    (lambda L: L.bl_linear(16, 4, 8, 16, 1, 4, 16, 16, NULL, 1e-5, 16, NULL, 0, NULL), 4),
+    (lambda L: L.bl_linear(16, 4, 8, 16, 1, 4, 16, 16, NULL, 1e-5, 16, 256, 8, NULL), 4),
+    (lambda L: L.bl_linear(16, 4, 8, 16, 1, 4, 16, 16, NULL, 1e-5, 16, 257, 1 << 20, NULL), 4),
+    # M == 0 is a no-op success, nothing launched
+    (lambda L: L.bl_linear(NULL, 0, 8, 16, 1, 4, 16, 16, NULL, 1e-5, NULL, NULL, 0, NULL), 0),
+    (lambda L: L.bl_quantize_act(NULL, 0, 8, 1e-5, NULL, NULL, NULL), 0),
+    # weight quantization argument checks
+    (lambda L: L.bl_quantize_weights(NULL, 4, 4, 1e-5, 16, 16, 256, 1 << 20, NULL), 1),
+    (lambda L: L.bl_quantize_weights(16, 4, 4, -1.0, 16, 16, 256, 1 << 20, NULL), 1),
+    (lambda L: L.bl_quantize_weights(16, 4, 4, 1e-5, 16, 16, 256, 4, NULL), 4),
+    (lambda L: L.bl_quantize_weights(18, 4, 4, 1e-5, 16, 16, 256, 1 << 20, NULL), 2),
+    (lambda L: L.bl_absmean(16, 4, 4, 1e-5, 16, 255, 4096, NULL), 4),
+    (lambda L: L.bl_absmean(16, 4, 4, 1e-5, 18, 256, 4096, NULL), 2),
+    (lambda L: L.bl_absmean(16, 0, 4, 1e-5, 16, 256, 4096, NULL), 1),
+    (lambda L: L.bl_ternarize(16, 4, 4, NULL, 16, NULL), 1),
+    (lambda L: L.bl_ternarize_pack5(16, 4, 4, 16, 16, 8, NULL), 2),
+    (lambda L: L.bl_quantize_weights_pack5(16, 4, 40, 1e-5, 16, 4, 16, 256, 1 << 20, NULL), 1),
+    (lambda L: L.bl_quantize_weights_pack5(16, 4, 40, 1e-5, 16, 24, 16, 256, 1 << 20, NULL), 2),
+    (lambda L: L.bl_pack(16, 4, 40, 16, 4, NULL), 1),
+    (lambda L: L.bl_pack(16, 4, 40, 17, 16, NULL), 2),
+    (lambda L: L.bl_unpack(NULL, 4, 40, 16, 16, NULL), 1),
+    (lambda L: L.bl_linear_acc(NULL, 2, 8, 16, 1, 4, 16, 16, NULL), 1),
+])
+def test_host_validation(lib, case, expect):
+    assert case(lib) == expect

@@ -1,0 +1,342 @@
+"""CUDA path vs the CPU oracle, element by element, through the C ABI.
+
+Integer outputs (trit codes, packed bytes, int8 codes, int32 accumulators) and
+the float32 scales and beta must be bit-exact.  Y must be within 1e-6 relative
+error of the oracle (the stated tolerance); since every float step is the same
+IEEE operation in the same order, it is also checked to be bit-identical.
+"""
+import numpy as np
+import pytest
+
+import oracle
+from workloads import problems, random_problem
+
+pytestmark = pytest.mark.gpu
+F32 = np.float32
+
+
+def dev(a):
+    import torch
+    return torch.from_numpy(np.ascontiguousarray(a)).cuda()
+
+
+def host(t):
+    return t.cpu().numpy()
+
+
+def assert_y_close(y, ref):
+    y, ref = np.asarray(y, np.float64), np.asarray(ref, np.float64)
+    rel = np.abs(y - ref) / np.maximum(np.abs(ref), 1e-30)
+    assert rel.size == 0 or float(rel.max()) <= 1e-6, f"max rel err {rel.max():.3e}"
+    np.testing.assert_array_equal(y, ref)
+
+
+def check_ok(bl):
+    assert bl.sync_status() == "BL_OK"
+
+
+# ------------------------------------------------------------ weights -------
+@pytest.mark.parametrize("N,K", [(256, 128), (7, 3), (1, 1), (33, 81), (300, 2560), (64, 1001)])
+def test_quantize_weights_int8(bl, N, K):
+    p = random_problem(N * 7 + K, 1, K, N)
+    Wq, beta = bl.quantize_weights(dev(p.W), 1e-5)
+    rb = oracle.absmean_beta(p.W, 1e-5)
+    check_ok(bl)
+    assert host(beta)[0] == rb
+    np.testing.assert_array_equal(host(Wq), oracle.ternarize(p.W, rb))
+
+
+@pytest.mark.parametrize("N,K", [(256, 128), (5, 7), (3, 4), (17, 99), (40, 2560), (11, 6912)])
+def test_quantize_weights_pack5(bl, N, K):
+    p = random_problem(N * 13 + K, 1, K, N)
+    Wp, beta = bl.quantize_weights_pack5(dev(p.W), 1e-5)
+    rb = oracle.absmean_beta(p.W, 1e-5)
+    check_ok(bl)
+    assert host(beta)[0] == rb
+    np.testing.assert_array_equal(host(Wp), oracle.pack5(oracle.ternarize(p.W, rb)))
+
+
+def test_beta_wide_dynamic_range(bl):
+    """Magnitudes outside the fast accumulator window take the exponent bins."""
+    rng = np.random.default_rng(5)
+    W = (rng.standard_normal((97, 131)) * 0.02).astype(F32)
+    W.ravel()[::7] *= F32(2.0 ** 30)
+    W.ravel()[3::11] *= F32(2.0 ** -40)
+    W.ravel()[5::13] = F32(1e-42)            # subnormal
+    W.ravel()[2::17] = F32(0.0)
+    Wq, beta = bl.quantize_weights(dev(W), 1e-5)
+    rb = oracle.absmean_beta(W, 1e-5)
+    check_ok(bl)
+    assert host(beta)[0] == rb
+    np.testing.assert_array_equal(host(Wq), oracle.ternarize(W, rb))
+
+
+def test_beta_constant_tensor_large(bl):
+    W = np.full((3001, 1001), F32(0.02), F32)
+    _, beta = bl.quantize_weights(dev(W), 1e-5)
+    check_ok(bl)
+    assert host(beta)[0] == F32(F32(0.02) + F32(1e-5))
+
+
+def test_ternary_rounding_boundary(bl):
+    """Weights placed exactly on, and one float below and above, the place
+    where float32(w / beta) crosses 0.5; beta is held fixed by the bulk."""
+    rng = np.random.default_rng(6)
+    W = (rng.standard_normal((64, 257)) * 0.02).astype(F32)
+    for _ in range(3):   # the edits move beta by far less than an ulp; settle it
+        b = oracle.absmean_beta(W, 1e-5)
+        half = F32(b * F32(0.5))                      # w/beta rounds to 0.5 here
+        cand = [half, np.nextafter(half, F32(1)), np.nextafter(half, F32(0)),
+                np.nextafter(np.nextafter(half, F32(1)), F32(1))]
+        t = F32(b * F32(1.5))
+        cand += [t, np.nextafter(t, F32(0)), np.nextafter(t, F32(9))]
+        flat = W.ravel()
+        for i, c in enumerate(cand):
+            flat[10 * i] = c
+            flat[10 * i + 1] = -c
+    rb = oracle.absmean_beta(W, 1e-5)
+    Wq, beta = bl.quantize_weights(dev(W), 1e-5)
+    check_ok(bl)
+    assert host(beta)[0] == rb
+    ref = oracle.ternarize(W, rb)
+    np.testing.assert_array_equal(host(Wq), ref)
+    assert len(set(ref.ravel()[:80:10].tolist())) > 1   # the boundary really splits
+
+
+def test_nonfinite_weight_is_reported(bl):
+    W = np.ones((4, 8), F32)
+    W[2, 3] = np.inf
+    bl.quantize_weights(dev(W), 1e-5)
+    assert bl.sync_status() == "BL_ERR_NONFINITE"
+    check_ok(bl)
+
+
+# ------------------------------------------------------------ packing -------
+@pytest.mark.parametrize("N,K", [(1, 1), (3, 5), (7, 23), (64, 2560), (9, 6913)])
+def test_pack_unpack(bl, N, K):
+    rng = np.random.default_rng(K)
+    Wq = rng.integers(-1, 2, (N, K)).astype(np.int8)
+    Wp = bl.pack(dev(Wq))
+    np.testing.assert_array_equal(host(Wp), oracle.pack5(Wq))
+    np.testing.assert_array_equal(host(bl.unpack(Wp, K)), Wq)
+    check_ok(bl)
+
+
+def test_pack_all_patterns(bl):
+    import itertools
+    pats = np.array(list(itertools.product((-1, 0, 1), repeat=5)), np.int8).reshape(1, -1)
+    Wp = bl.pack(dev(pats))
+    np.testing.assert_array_equal(host(Wp), oracle.pack5(pats))
+
+
+# ------------------------------------------------------------ activations ---
+@pytest.mark.parametrize("M,K", [(8, 128), (1, 2560), (3, 7), (5, 1), (17, 6912), (2, 11008), (70, 333)])
+def test_quantize_act(bl, M, K):
+    p = random_problem(M * 3 + K, M, K, 1)
+    X = p.X * np.linspace(0.01, 100, M, dtype=F32)[:, None]
+    Xq, s = bl.quantize_act(dev(X), 1e-5)
+    rq, rs = oracle.act_quant(X, 1e-5)
+    check_ok(bl)
+    np.testing.assert_array_equal(host(s), rs)
+    np.testing.assert_array_equal(host(Xq), rq)
+
+
+def test_quantize_act_ties_and_zero_rows(bl):
+    X = np.zeros((4, 9), F32)
+    X[0] = [127, 0.5, 1.5, 2.5, -0.5, -1.5, -2.5, 126.5, -127]
+    X[2] = [-127, 63.5, 0, 1, 2, 3, 4, 5, 6]
+    for eps in (2.0 ** -30, 1e-5, 2.0 ** -10):
+        Xq, s = bl.quantize_act(dev(X), eps)
+        rq, rs = oracle.act_quant(X, eps)
+        np.testing.assert_array_equal(host(s), rs)
+        np.testing.assert_array_equal(host(Xq), rq)
+    check_ok(bl)
+
+
+def test_nonfinite_activation_is_reported(bl):
+    X = np.ones((3, 10), F32)
+    X[1, 4] = np.nan
+    bl.quantize_act(dev(X), 1e-5)
+    assert bl.sync_status() == "BL_ERR_NONFINITE"
+    check_ok(bl)
+
+
+# ------------------------------------------------------------ linear --------
+def _layer(bl, p, fmt, path, bias=None):
+    if fmt == bl.PACK5:
+        Wd, beta = bl.quantize_weights_pack5(dev(p.W), p.eps)
+    else:
+        Wd, beta = bl.quantize_weights(dev(p.W), p.eps)
+    Y = bl.linear(dev(p.X), Wd, fmt, p.N, p.K, beta, None if bias is None else dev(bias),
+                  p.eps, path=path)
+    return host(Y), Wd, beta
+
+
+PATHS = ["simt", "auto"]
+
+
+def _path(bl, name):
+    return {"simt": bl.PATH_SIMT, "auto": bl.PATH_AUTO, "gemv": bl.PATH_GEMV,
+            "tc": bl.PATH_TC}[name]
+
+
+@pytest.mark.parametrize("path", PATHS)
+@pytest.mark.parametrize("fmt", ["i8", "pack5"])
+@pytest.mark.parametrize("M,K,N", [(8, 128, 256), (1, 2560, 96), (3, 7, 5), (65, 161, 130),
+                                   (130, 1001, 67), (2, 6912, 40), (1, 1, 1)])
+def test_linear_small(bl, path, fmt, M, K, N):
+    p = random_problem(M + 10 * K + 100 * N, M, K, N)
+    f = bl.PACK5 if fmt == "pack5" else bl.I8
+    Y, _, _ = _layer(bl, p, f, _path(bl, path))
+    check_ok(bl)
+    assert_y_close(Y, oracle.bitlinear(p.X, p.W, p.eps)["Y"])
+
+
+def test_linear_bias(bl):
+    p = random_problem(77, 5, 300, 45)
+    b = np.random.default_rng(1).standard_normal(45).astype(F32)
+    Y, _, _ = _layer(bl, p, bl.PACK5, bl.PATH_AUTO, bias=b)
+    check_ok(bl)
+    assert_y_close(Y, oracle.bitlinear(p.X, p.W, p.eps, bias=b)["Y"])
+
+
+@pytest.mark.parametrize("path", PATHS)
+def test_linear_acc_exact(bl, path):
+    rng = np.random.default_rng(3)
+    M, K, N = 37, 517, 71
+    Xq = rng.integers(-127, 128, (M, K)).astype(np.int8)
+    Wq = rng.integers(-1, 2, (N, K)).astype(np.int8)
+    ref = oracle.contract(Xq, Wq)
+    acc_i8 = bl.linear_acc(dev(Xq), dev(Wq), bl.I8, N, K, path=_path(bl, path))
+    acc_p5 = bl.linear_acc(dev(Xq), bl.pack(dev(Wq)), bl.PACK5, N, K, path=_path(bl, path))
+    check_ok(bl)
+    np.testing.assert_array_equal(host(acc_i8), ref)
+    np.testing.assert_array_equal(host(acc_p5), ref)
+
+
+def test_linear_extreme_accumulators(bl):
+    K = 8192
+    Xq = np.full((2, K), 127, np.int8)
+    Xq[1] = -127
+    Wq = np.ones((3, K), np.int8)
+    Wq[1] = -1
+    Wq[2, ::2] = 0
+    acc = bl.linear_acc(dev(Xq), bl.pack(dev(Wq)), bl.PACK5, 3, K)
+    check_ok(bl)
+    np.testing.assert_array_equal(host(acc), oracle.contract(Xq, Wq))
+
+
+def test_workload_tiny(bl):
+    p = next(problems(1))
+    Y, Wd, beta = _layer(bl, p, bl.I8, bl.PATH_AUTO)
+    r = oracle.bitlinear(p.X, p.W, p.eps)
+    check_ok(bl)
+    assert host(beta)[0] == r["beta"]
+    np.testing.assert_array_equal(host(Wd), r["Wq"])
+    assert_y_close(Y, r["Y"])
+
+
+def test_workload_gpt_layers(bl):
+    """All 24 BitLinears of the d_model-128, 4-layer ternary GPT at M = 2048."""
+    for p in problems(3):
+        Y, _, _ = _layer(bl, p, bl.I8, bl.PATH_AUTO)
+        assert_y_close(Y, oracle.bitlinear(p.X, p.W, p.eps)["Y"])
+    check_ok(bl)
+
+
+def test_row_independence_and_batching(bl):
+    """Per-token scales: a row's output is the same alone or in a batch, and
+    does not move when another row changes ("attention, as graph ops")."""
+    p = random_problem(9, 12, 700, 50)
+    Wp, beta = bl.quantize_weights_pack5(dev(p.W), p.eps)
+    Y = host(bl.linear(dev(p.X), Wp, bl.PACK5, p.N, p.K, beta))
+    for m in (0, 5, 11):
+        one = host(bl.linear(dev(p.X[m:m + 1]), Wp, bl.PACK5, p.N, p.K, beta))
+        np.testing.assert_array_equal(one[0], Y[m])
+    X2 = p.X.copy()
+    X2[3] *= F32(1e4)
+    Y2 = host(bl.linear(dev(X2), Wp, bl.PACK5, p.N, p.K, beta))
+    keep = [r for r in range(12) if r != 3]
+    np.testing.assert_array_equal(Y2[keep], Y[keep])
+    check_ok(bl)
+
+
+def test_repeatable(bl):
+    p = random_problem(10, 33, 999, 77)
+    a, _, _ = _layer(bl, p, bl.PACK5, bl.PATH_AUTO)
+    b, _, _ = _layer(bl, p, bl.PACK5, bl.PATH_AUTO)
+    np.testing.assert_array_equal(a, b)
+
+
+# ------------------------------------------------ full sizes, sampled ------
+_PROBLEM_CACHE = {}
+_BETA_CACHE = {}
+
+
+def _problem(wid, idx):
+    key = (wid, idx)
+    if key not in _PROBLEM_CACHE:
+        if wid == 5 and _PROBLEM_CACHE:       # keep one shared 8192^2 weight, not ten
+            for k in [k for k in _PROBLEM_CACHE if k[0] != 5]:
+                del _PROBLEM_CACHE[k]
+        if wid == 5:
+            for i, p in enumerate(problems(5)):
+                _PROBLEM_CACHE[(5, i)] = p
+        else:
+            _PROBLEM_CACHE.clear()
+            _PROBLEM_CACHE[key] = next(problems(wid, only=[idx]))
+    return _PROBLEM_CACHE[key]
+
+
+def _oracle_beta(p):
+    key = (p.workload, id(p.W))
+    if key not in _BETA_CACHE:
+        _BETA_CACHE.clear()
+        _BETA_CACHE[key] = oracle.absmean_beta(p.W, p.eps)
+    return _BETA_CACHE[key]
+
+
+def _sampled_check(bl, p, fmt, n_samples=512, seed=0):
+    """Full-size call on the GPU; the oracle computes sampled outputs one by one
+    (beta over the whole tensor, row quantization for the sampled rows only)."""
+    import torch
+    Wd_fn = bl.quantize_weights_pack5 if fmt == bl.PACK5 else bl.quantize_weights
+    Wd, beta = Wd_fn(dev(p.W), p.eps)
+    Y = bl.linear(dev(p.X), Wd, fmt, p.N, p.K, beta, eps=p.eps)
+    torch.cuda.synchronize()
+    check_ok(bl)
+    rb = _oracle_beta(p)
+    assert host(beta)[0] == rb
+    rng = np.random.default_rng(seed)
+    ms = rng.integers(0, p.M, n_samples)
+    ns = rng.integers(0, p.N, n_samples)
+    ms[:2], ns[:2] = [0, p.M - 1], [p.N - 1, 0]
+    Xq, s = oracle.act_quant(p.X[ms], p.eps)
+    Wq = oracle.ternarize(p.W[ns], rb)
+    acc = oracle.contract_entries(Xq, Wq)
+    ref = oracle.dequant(acc, s, rb)
+    got = host(Y)[ms, ns]
+    assert_y_close(got, ref)
+    rows = np.unique(ns)[:64]
+    if fmt == bl.PACK5:
+        np.testing.assert_array_equal(host(Wd)[rows], oracle.pack5(oracle.ternarize(p.W[rows], rb)))
+    else:
+        np.testing.assert_array_equal(host(Wd)[rows], oracle.ternarize(p.W[rows], rb))
+
+
+@pytest.mark.parametrize("idx", [0, 1])
+def test_workload_decode_full(bl, idx):
+    p = _problem(2, idx)
+    _sampled_check(bl, p, bl.PACK5, n_samples=p.N)   # M = 1: every output
+
+
+@pytest.mark.parametrize("idx", [0, 1])
+def test_workload_prefill_full_sampled(bl, idx):
+    p = _problem(4, idx)
+    _sampled_check(bl, p, bl.PACK5, n_samples=512, seed=idx)
+
+
+@pytest.mark.parametrize("idx", range(10))
+def test_workload_sweep_full_sampled(bl, idx):
+    p = _problem(5, idx)
+    _sampled_check(bl, p, bl.PACK5, n_samples=256, seed=idx)
