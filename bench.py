@@ -240,6 +240,22 @@ def algorithmic_bytes(kind, N, K, M, fmt):
     raise ValueError(kind)
 
 
+# ------------------------------------------------------- rank arithmetic ---
+def max_over_ranks(ms: float, dist=None, device=None) -> float:
+    """The timed region's duration as the max over ranks (the slowest rank)."""
+    if dist is None or not dist.is_initialized() or dist.get_world_size() == 1:
+        return float(ms)
+    import torch
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_gmacs(macs_per_step_per_rank: int, steps: int, world: int, ms: float) -> float:
+    """Weak scaling: every rank does its own step; value = all ranks' MACs / slowest time."""
+    return macs_per_step_per_rank * steps * world / (ms * 1e-3) / 1e9
+
+
 # ------------------------------------------------------------ our arm ------
 def run_ours(args):
     import torch
@@ -305,11 +321,7 @@ def run_ours(args):
         torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
-    ms = t0.elapsed_time(t1)
-    t = torch.tensor([ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    ms_max = float(t.item())
+    ms_max = max_over_ranks(t0.elapsed_time(t1), dist, dev)
     if bl.sync_status(dev) != "BL_OK":
         raise RuntimeError("device status not clean after the timed region")
 
@@ -353,7 +365,7 @@ def run_ours(args):
                 if peaks["source"] == "measured" else "fallback 6.65 TB/s"}
 
     launches_per_step = sum(d["launches"] for d in kinds.values())
-    value = macs_per_step * K * world / (ms_max * 1e-3) / 1e9
+    value = whole_job_gmacs(macs_per_step, K, world, ms_max)
     lin = kinds.get("linear")
     line = {
         "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world,
@@ -436,14 +448,10 @@ def e2e(bl, torch, probs, dev, fmt, steps, world):
         one()
     t1.record()
     torch.cuda.synchronize()
-    ms = t0.elapsed_time(t1)
-    t = torch.tensor([ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        import torch.distributed as dist
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    ms = float(t.item())
+    import torch.distributed as dist
+    ms = max_over_ranks(t0.elapsed_time(t1), dist, dev)
     macs = sum(p.M * p.N * p.K for p in probs)
-    return {"value": round(macs * steps * world / (ms * 1e-3) / 1e9, 2), "unit": UNIT,
+    return {"value": round(whole_job_gmacs(macs, steps, world, ms), 2), "unit": UNIT,
             "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
             "steps": steps, "ms_per_step": round(ms / steps, 4)}
 
