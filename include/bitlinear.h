@@ -176,6 +176,35 @@ bl_status bl_linear_acc_ex(const int8_t* Xq, int64_t M, int64_t K, const void* W
                            int64_t N, int64_t ldw, int32_t* acc, void* ws, size_t ws_bytes,
                            int path, cudaStream_t stream);
 
+/* Size of the scratch array built into the library for bl_linear_noalloc. */
+#define BL_LINEAR_NOALLOC_SCRATCH_BYTES ((size_t)16 << 20)
+
+/* bl_linear for callers that cannot allocate device memory at all: a plugin or
+ * custom-op interface that hands the library only its input and output buffers
+ * and owns every allocation under a fixed memory plan, or a latency-critical
+ * loop where cudaMalloc (which may synchronize the whole device) is not allowed.
+ * The paper has no counterpart to this entry point: it is a deployment
+ * convenience of this library.
+ *
+ * Same arguments and results as bl_linear, minus the workspace.  The scratch
+ * (quantized activations and row scales) is a static device array of
+ * BL_LINEAR_NOALLOC_SCRATCH_BYTES that every GPU loading the library holds until
+ * the process exits.  Nothing is allocated: no cudaMalloc, cudaFree or
+ * allocating library routine is called.
+ *   - Shapes whose bl_linear_workspace_size(M, N, K, f) exceeds the array are
+ *     rejected with BL_ERR_WORKSPACE before anything is launched.
+ *   - The first call on each device looks up the array's device address with
+ *     cudaGetSymbolAddress (with that device current); make that first call
+ *     before any stream capture.
+ *   - All calls on a device share the one array and it keeps the last call's
+ *     contents: calls that overlap on the GPU (other streams, other host
+ *     threads) race on it, so issue them in order on one stream.  Every scratch
+ *     byte a call reads is written earlier in the same call, so nothing needs
+ *     clearing between calls. */
+bl_status bl_linear_noalloc(const float* X, int64_t M, int64_t K, const void* W, bl_wfmt f,
+                            int64_t N, int64_t ldw, const float* beta_dev, const float* bias,
+                            float eps, float* Y, cudaStream_t stream);
+
 /* Synchronizes `stream`, then reads and clears this device's status word:
  * BL_ERR_DEVICE_TIMEOUT or BL_ERR_NONFINITE if a kernel recorded one, BL_ERR_CUDA
  * if the stream reports an error, else BL_OK. */

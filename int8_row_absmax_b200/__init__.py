@@ -41,6 +41,7 @@ SIGNATURES = {
     "bl_linear_workspace_size": (_SZ, [_I64, _I64, _I64, _I]),
     "bl_linear": (_I, [_P, _I64, _I64, _P, _I, _I64, _I64, _P, _P, _F, _P, _P, _SZ, _P]),
     "bl_linear_ex": (_I, [_P, _I64, _I64, _P, _I, _I64, _I64, _P, _P, _F, _P, _P, _SZ, _I, _P]),
+    "bl_linear_noalloc": (_I, [_P, _I64, _I64, _P, _I, _I64, _I64, _P, _P, _F, _P, _P]),
     "bl_linear_plan": (_I, [_I64, _I64, _I64, _I, _I, ctypes.POINTER(ctypes.c_int)]),
     "bl_linear_acc": (_I, [_P, _I64, _I64, _P, _I, _I64, _I64, _P, _P]),
     "bl_linear_acc_workspace_size": (_SZ, [_I64, _I64, _I64, _I, _I]),
@@ -234,6 +235,21 @@ def linear(X, W, fmt: int, N: int, K: int, beta, bias=None, eps: float = 1e-5,
         _ptr(X), M, K, _ptr(W), fmt, N, W.shape[1], _ptr(beta), _ptr(bias), eps, _ptr(Y),
         _ptr(ws), ws.numel(), path, _stream(torch, X)))
     return Y
+
+
+NOALLOC_SCRATCH_BYTES = 16 << 20
+
+
+def linear_noalloc(X, W, fmt: int, N: int, K: int, beta, out, bias=None, eps: float = 1e-5):
+    """bl_linear_noalloc: Y written into the caller's `out`; the library's static
+    scratch array replaces the workspace, so no device memory is allocated."""
+    torch, lib = _torch(), load()
+    _dev(X, torch.float32)
+    _dev(out, torch.float32)
+    _check("bl_linear_noalloc", lib.bl_linear_noalloc(
+        _ptr(X), X.shape[0], K, _ptr(W), fmt, N, W.shape[1], _ptr(beta), _ptr(bias), eps,
+        _ptr(out), _stream(torch, X)))
+    return out
 
 
 def linear_acc(Xq, W, fmt: int, N: int, K: int, path: int = PATH_AUTO, ws=None):

@@ -7,6 +7,7 @@
 #include <cmath>
 #include <cstdint>
 #include <cstring>
+#include <mutex>
 
 #include <cuda_runtime.h>
 
@@ -125,6 +126,29 @@ bl_status run_simt(const int8_t* Xq, int64_t ldx, int64_t M, int64_t K, const vo
     else linear_simt_kernel<false, false><<<grid, 256, 0, st>>>(Xq, ldx, M, K, W, ldw, N, nullptr, nullptr, nullptr, nullptr, acc);
   }
   return launch_status();
+}
+
+// ---- scratch for bl_linear_noalloc -------------------------------------------
+// A file-scope device array: every GPU that loads the library holds it until the
+// process exits.  Its name in host code is only a host-side stand-in, so the
+// device address is looked up once per device with cudaGetSymbolAddress.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[BL_LINEAR_NOALLOC_SCRATCH_BYTES];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[kMaxDevices] = {};
+
+// Device address of the scratch array on the current device (nullptr on error).
+void* noalloc_scratch_ptr() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess) return nullptr;
+    g_noalloc_ptr[dev] = p;
+  }
+  return g_noalloc_ptr[dev];
 }
 
 }  // namespace
@@ -260,6 +284,22 @@ bl_status bl_linear(const float* X, int64_t M, int64_t K, const void* W, bl_wfmt
                     void* ws, size_t ws_bytes, cudaStream_t stream) {
   return bl_linear_ex(X, M, K, W, f, N, ldw, beta_dev, bias, eps, Y, ws, ws_bytes,
                       BL_PATH_AUTO, stream);
+}
+
+bl_status bl_linear_noalloc(const float* X, int64_t M, int64_t K, const void* W, bl_wfmt f,
+                            int64_t N, int64_t ldw, const float* beta_dev, const float* bias,
+                            float eps, float* Y, cudaStream_t stream) {
+  bl_status st = check_shape(M, K, N);
+  if (st != BL_OK) return st;
+  if (!eps_ok(eps)) return BL_ERR_INVALID_ARG;
+  if ((st = check_w(W, f, K, ldw)) != BL_OK) return st;
+  if (M == 0) return BL_OK;
+  const size_t need = bl_linear_workspace_size(M, N, K, f);
+  if (need > BL_LINEAR_NOALLOC_SCRATCH_BYTES) return BL_ERR_WORKSPACE;
+  void* scratch = noalloc_scratch_ptr();
+  if (!scratch) return BL_ERR_CUDA;
+  return bl_linear_ex(X, M, K, W, f, N, ldw, beta_dev, bias, eps, Y, scratch,
+                      BL_LINEAR_NOALLOC_SCRATCH_BYTES, BL_PATH_AUTO, stream);
 }
 
 size_t bl_linear_acc_workspace_size(int64_t M, int64_t N, int64_t K, bl_wfmt f, int path) {
