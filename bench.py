@@ -14,9 +14,11 @@ rotation touches >= 4x the L2 size (no step reuses the previous step's data
 from L2).  Each replica's step is captured once as a CUDA graph; W warm-up
 replays, then exactly K timed replays bracketed by barrier + synchronize, timed
 with CUDA events on the launching stream; the max over ranks is reported.
-Per-call durations come from external events inside the same graphs (the last
-R timed replays).  SM clocks and throttle reasons are sampled through NVML
-during the timed region.  `e2e` repeats the step through the public Python API
+Per-call durations (the roofline's kernel times) come right after the timed
+region from CUDA events around graphs that repeat one call of the step over the
+same rotating replicas (event nodes inside a graph cost microseconds each, so
+none sit inside the timed step graphs).  SM clocks and throttle reasons are
+sampled through NVML during the timed region.  `e2e` repeats the step through the public Python API
 with the step's inputs copied from pinned host memory and Y copied back.
 
 Under torchrun each rank runs its own independently seeded batch (weak
@@ -195,29 +197,26 @@ class Step:
             n += X.numel() * 4 + Y.numel() * 4 + lws.numel()
         return n
 
-    def run(self, events=None, path=0):
-        """Issue the whole step on the current stream; events[i] mark call boundaries."""
+    def run(self, only=None, path=0):
+        """Issue the step on the current stream: every call, or only call `only`
+        (an index into labels())."""
         bl = self.bl
-        k = 0
-
-        def mark():
-            nonlocal k
-            if events is not None:
-                events[k].record()
-            k += 1
-        mark()
+        k = -1
         for W, beta, Wout, ws, N, K in self.tensors:
-            bl.absmean(W, 1e-5, ws=ws, beta=beta)
-            mark()
-            if self.fmt == bl.PACK5:
-                bl.ternarize_pack5(W, beta, out=Wout)
-            else:
-                bl.ternarize(W, beta, out=Wout)
-            mark()
+            k += 1
+            if only is None or only == k:
+                bl.absmean(W, 1e-5, ws=ws, beta=beta)
+            k += 1
+            if only is None or only == k:
+                if self.fmt == bl.PACK5:
+                    bl.ternarize_pack5(W, beta, out=Wout)
+                else:
+                    bl.ternarize(W, beta, out=Wout)
         for X, ti, Y, lws, M, K, N, eps in self.calls:
-            W, beta, Wout, ws, _, _ = self.tensors[ti]
-            bl.linear(X, Wout, self.fmt, N, K, beta, eps=eps, ws=lws, out=Y, path=path)
-            mark()
+            k += 1
+            if only is None or only == k:
+                W, beta, Wout, ws, _, _ = self.tensors[ti]
+                bl.linear(X, Wout, self.fmt, N, K, beta, eps=eps, ws=lws, out=Y, path=path)
 
     def labels(self):
         out = []
@@ -288,17 +287,14 @@ def run_ours(args):
         raise RuntimeError("device status not clean after the eager step")
 
     labels = first.labels()
-    n_ev = len(labels) + 1
     stream = torch.cuda.Stream(device=dev)
-    graphs, evsets = [], []
+    graphs = []
     with torch.cuda.stream(stream):
         for s in steps:
-            evs = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(n_ev)]
             g = torch.cuda.CUDAGraph()
             with torch.cuda.graph(g, stream=stream):
-                s.run(events=evs, path=args.path)
+                s.run(path=args.path)
             graphs.append(g)
-            evsets.append(evs)
     torch.cuda.synchronize()
 
     K, Wm = args.steps, args.warmup
@@ -325,11 +321,27 @@ def run_ours(args):
     if bl.sync_status(dev) != "BL_OK":
         raise RuntimeError("device status not clean after the timed region")
 
-    # per-call durations from the external events (the last replay of each replica)
+    # per-call durations: for each call of the step, one graph that issues that
+    # call for every replica in turn, repeated; CUDA events around its replays
     per_call = {}
-    for evs in evsets:
+    reps = max(1, 64 // R)
+    with torch.cuda.stream(stream):
         for i, lab in enumerate(labels):
-            per_call.setdefault(lab, []).append(evs[i].elapsed_time(evs[i + 1]))
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                for _ in range(reps):
+                    for s in steps:
+                        s.run(only=i, path=args.path)
+            g.replay()
+            c0 = torch.cuda.Event(enable_timing=True)
+            c1 = torch.cuda.Event(enable_timing=True)
+            c0.record(stream)
+            for _ in range(4):
+                g.replay()
+            c1.record(stream)
+            torch.cuda.synchronize()
+            per_call[lab] = [c0.elapsed_time(c1) / (4 * reps * R)]
+            del g
     shapes = {}
     for i, (W, beta, Wout, ws, N, Kd) in enumerate(first.tensors):
         shapes[("absmean", i)] = (N, Kd, 0)

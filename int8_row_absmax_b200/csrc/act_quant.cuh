@@ -19,6 +19,30 @@ __device__ __forceinline__ int8_t act_code(float x, float s) {
   return int8_t(int(q));
 }
 
+// act_code kept out of line: the rare near-tie path of act_code_fast.
+__device__ __noinline__ int act_code_slow(float x, float s) { return act_code(x, s); }
+
+// Reciprocal of the row scale for act_code_fast, or 0 when the fast path is not
+// safe for this scale (s not a normal float, or 1/s not a normal float).
+__device__ __forceinline__ float act_recip(float s) {
+  const float r = __frcp_rn(s);
+  return (s >= 1.17549435e-38f && r >= 1.17549435e-38f && r <= 1.0e37f) ? r : 0.f;
+}
+
+// The same code as act_code, with one multiply instead of the IEEE division in
+// all but near-tie cases.  For |x| <= 127 s, y' = x * RN(1/s) differs from the
+// real quotient y = x / s by at most 1.5 ulp(y) <= 1.5 * 2^-17 < 2^-16, and
+// float32(y) is within 2^-18 of y.  So unless y' lies within 2^-15 of a
+// half-integer, y, float32(y) and y' all round to the same integer; the rare
+// near-tie values take the exact division.
+__device__ __forceinline__ int8_t act_code_fast(float x, float s, float r) {
+  const float y = __fmul_rn(x, r);
+  const float q = rintf(y);
+  if (r == 0.f || fabsf(fabsf(__fsub_rn(y, q)) - 0.5f) < 3.0517578125e-05f)
+    return int8_t(act_code_slow(x, s));
+  return int8_t(int(fminf(fmaxf(q, -float(kActQmax)), float(kActQmax))));
+}
+
 // One CTA per row: pass 1 finds max|x| (warp shuffles, then across warps), pass
 // 2 re-reads the row (an L1/L2 hit) and writes the codes.  Row stride of X is K;
 // Xq has stride ldq >= K and its bytes [K, ldq) are written as 0.
@@ -61,17 +85,18 @@ act_quant_kernel(const float* __restrict__ X, int64_t K, float eps, int8_t* __re
   }
   __syncthreads();
   const float s = s_scale;
+  const float r = act_recip(s);
 
   for (int64_t i = threadIdx.x; i < K4; i += kActThreads) {
     const float4 v = reinterpret_cast<const float4*>(xr)[i];
     char4 q;
-    q.x = act_code(v.x, s);
-    q.y = act_code(v.y, s);
-    q.z = act_code(v.z, s);
-    q.w = act_code(v.w, s);
+    q.x = act_code_fast(v.x, s, r);
+    q.y = act_code_fast(v.y, s, r);
+    q.z = act_code_fast(v.z, s, r);
+    q.w = act_code_fast(v.w, s, r);
     reinterpret_cast<char4*>(qr)[i] = q;
   }
-  for (int64_t i = (K4 << 2) + threadIdx.x; i < K; i += kActThreads) qr[i] = act_code(xr[i], s);
+  for (int64_t i = (K4 << 2) + threadIdx.x; i < K; i += kActThreads) qr[i] = act_code_fast(xr[i], s, r);
   for (int64_t i = K + threadIdx.x; i < ldq; i += kActThreads) qr[i] = 0;
 }
 

@@ -17,6 +17,7 @@
 #include "pack.cuh"
 #include "act_quant.cuh"
 #include "linear_simt.cuh"
+#include "gemv_pack5.cuh"
 
 namespace bl {
 namespace {
@@ -58,7 +59,7 @@ bl_status check_weights_args(const float* W, int64_t N, int64_t K, const void* o
 bl_status launch_absmean(const float* W, int64_t n, float eps, float* beta_dev, void* ws,
                          cudaStream_t st) {
   auto* acc = static_cast<AbsAccum*>(ws);
-  absmean_kernel<<<grid_for(ceil_div(n, 16), kAbsThreads, 2), kAbsThreads, 0, st>>>(W, n, eps, acc, beta_dev);
+  absmean_kernel<<<grid_for(ceil_div(n, 64), kAbsThreads, 4), kAbsThreads, 0, st>>>(W, n, eps, acc, beta_dev);
   return launch_status();
 }
 
@@ -101,15 +102,83 @@ bl_status check_shape(int64_t M, int64_t K, int64_t N) {
 }
 
 // Resolve the kernel path for a linear call; -1 when the pinned path cannot run it.
-int resolve_path(int64_t M, int64_t N, int64_t K, bl_wfmt f, int path, int* launches) {
-  (void)N;
-  (void)K;
-  (void)f;
+// `fused_quant`: bl_linear (X in float32) rather than bl_linear_acc (X_q given).
+int resolve_path(int64_t M, int64_t N, int64_t K, bl_wfmt f, int path, int* launches,
+                 bool fused_quant = true) {
+  const int64_t ldp = round_up(ceil_div(K, 5), 16);
+  const bool gemv_ok = f == BL_W_PACK5 && M >= 1 && gemv_feasible(M, N, K, ldp);
   int p = path;
-  if (p == BL_PATH_AUTO) p = BL_PATH_SIMT;
-  if (p != BL_PATH_SIMT) return -1;
-  if (launches) *launches = M == 0 ? 0 : 2;  // act_quant + contraction
+  if (p == BL_PATH_AUTO) p = gemv_ok ? BL_PATH_GEMV : BL_PATH_SIMT;
+  int n = 0;
+  if (p == BL_PATH_SIMT) {
+    n = fused_quant ? 2 : 1;  // act_quant + contraction
+  } else if (p == BL_PATH_GEMV) {
+    if (!gemv_ok) return -1;
+    n = 1;                    // quantization fused into the GEMV
+  } else {
+    return -1;
+  }
+  if (launches) *launches = M == 0 ? 0 : n;
   return p;
+}
+
+template <int M, int CH, bool F, bool D>
+bl_status launch_gemv_inst(const GemvPlan& P, const GemvArgs& a, cudaStream_t st) {
+  auto kern = gemv_pack5_kernel<M, CH, F, D>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kGemvMaxSmem) != cudaSuccess)
+    return BL_ERR_CUDA;
+  kern<<<P.grid, P.nwarps * 32, P.smem, st>>>(a);
+  return launch_status();
+}
+
+template <bool F, bool D>
+bl_status launch_gemv_fd(const GemvPlan& P, const GemvArgs& a, cudaStream_t st) {
+  switch (P.M * 8 + P.CH) {
+    case 1 * 8 + 1: return launch_gemv_inst<1, 1, F, D>(P, a, st);
+    case 1 * 8 + 2: return launch_gemv_inst<1, 2, F, D>(P, a, st);
+    case 1 * 8 + 3: return launch_gemv_inst<1, 3, F, D>(P, a, st);
+    case 1 * 8 + 4: return launch_gemv_inst<1, 4, F, D>(P, a, st);
+    case 2 * 8 + 1: return launch_gemv_inst<2, 1, F, D>(P, a, st);
+    case 2 * 8 + 2: return launch_gemv_inst<2, 2, F, D>(P, a, st);
+    case 3 * 8 + 1: return launch_gemv_inst<3, 1, F, D>(P, a, st);
+    case 4 * 8 + 1: return launch_gemv_inst<4, 1, F, D>(P, a, st);
+  }
+  return BL_ERR_UNSUPPORTED;
+}
+
+// The packed-trit GEMV: Y from float32 X (fused quantization) or acc from X_q.
+bl_status run_gemv(const float* X, const int8_t* Xq, int64_t ldxq, int64_t M, int64_t K,
+                   const void* W, int64_t ldw, int64_t N, const float* beta, const float* bias,
+                   float eps, float* Y, int32_t* acc, cudaStream_t st) {
+  GemvPlan P;
+  const bool x_copyable = X && is_aligned(X, 16) && (K % 4) == 0;
+  if (!gemv_make_plan(M, N, K, ldw, num_sms(), P, x_copyable)) return BL_ERR_UNSUPPORTED;
+  GemvArgs a;
+  a.X = X;
+  a.Xq = Xq;
+  a.ldxq = ldxq;
+  a.Wp = static_cast<const uint8_t*>(W);
+  a.N = N;
+  a.K = K;
+  a.ldp = ldw;
+  a.beta = beta;
+  a.bias = bias;
+  a.eps = eps;
+  a.Y = Y;
+  a.acc = acc;
+  a.S = P.S;
+  a.slice = P.slice;
+  a.G = P.G;
+  a.RS = P.RS;
+  a.nstage = P.nstage;
+  a.rows_per_cta = P.rows_per_cta;
+  a.xstage_off = P.xstage_off;
+  a.part_off = P.part_off;
+  a.bar_off = P.bar_off;
+  a.stage_off = P.stage_off;
+  a.xf_off = P.xf_off;
+  a.xf_bytes = P.xf_bytes;
+  return Y ? launch_gemv_fd<true, true>(P, a, st) : launch_gemv_fd<false, false>(P, a, st);
 }
 
 bl_status run_simt(const int8_t* Xq, int64_t ldx, int64_t M, int64_t K, const void* W,
@@ -264,7 +333,10 @@ bl_status bl_linear_ex(const float* X, int64_t M, int64_t K, const void* W, bl_w
   if (!is_aligned(X, 4) || !is_aligned(Y, 4) || (bias && !is_aligned(bias, 4))) return BL_ERR_ALIGNMENT;
   const LinWs l = lin_layout(M, K);
   if (!ws || !is_aligned(ws, kWsAlign) || ws_bytes < l.total) return BL_ERR_WORKSPACE;
-  if (resolve_path(M, N, K, f, path, nullptr) < 0) return BL_ERR_UNSUPPORTED;
+  const int p = resolve_path(M, N, K, f, path, nullptr);
+  if (p < 0) return BL_ERR_UNSUPPORTED;
+  if (p == BL_PATH_GEMV)
+    return run_gemv(X, nullptr, 0, M, K, W, ldw, N, beta_dev, bias, eps, Y, nullptr, stream);
   int8_t* Xq = reinterpret_cast<int8_t*>(static_cast<char*>(ws) + l.xq_off);
   float* s = reinterpret_cast<float*>(static_cast<char*>(ws) + l.s_off);
   act_quant_kernel<<<unsigned(M), kActThreads, 0, stream>>>(X, K, eps, Xq, l.ldx, s);
@@ -324,7 +396,10 @@ bl_status bl_linear_acc_ex(const int8_t* Xq, int64_t M, int64_t K, const void* W
   if (M == 0) return BL_OK;
   if (!Xq || !acc) return BL_ERR_INVALID_ARG;
   if (!is_aligned(acc, 4)) return BL_ERR_ALIGNMENT;
-  if (path == BL_PATH_GEMV || path == BL_PATH_TC) return BL_ERR_UNSUPPORTED;
+  const int p = resolve_path(M, N, K, f, path, nullptr, false);
+  if (p < 0) return BL_ERR_UNSUPPORTED;
+  if (p == BL_PATH_GEMV)
+    return run_gemv(nullptr, Xq, K, M, K, W, ldw, N, nullptr, nullptr, 0.f, nullptr, acc, stream);
   return run_simt(Xq, K, M, K, W, f, ldw, N, nullptr, nullptr, nullptr, nullptr, acc, stream);
 }
 

@@ -9,9 +9,12 @@
 // (m < 2^24, e the biased exponent), so the sum is an integer in units of 2^-149.
 //
 //   absmean (one launch):
-//     1. each thread adds magnitudes with exponents in a fast window [110, 140]
-//        into a 96-bit fixed-point accumulator (unit 2^-40); any other magnitude
-//        goes to per-exponent 64-bit bins in shared memory;
+//     1. each thread adds magnitudes with exponents in a fast window [110, 141]
+//        into a 96-bit fixed-point accumulator (unit 2^-40): one mad.wide.u32 per
+//        weight adds m * 2^(e-110), where shl.b32 turns any shift outside the
+//        window into a zero factor; a warp-uniform slow path (taken only for a
+//        batch that holds such a weight) puts those magnitudes into
+//        per-exponent 64-bit bins in shared memory;
 //     2. each CTA adds its three 32-bit limb sums and its non-zero bins into the
 //        workspace accumulator block with 64-bit atomics (integer adds are exact,
 //        so the total does not depend on the schedule), then takes a ticket;
@@ -36,7 +39,7 @@ namespace bl {
 
 constexpr int kAbsThreads = 256;
 constexpr uint32_t kFastLo = 110;  // exponent whose mantissa LSB is 2^-40
-constexpr uint32_t kFastHi = 140;  // m << 30 < 2^54: 2^42 adds fit in 96 bits
+constexpr uint32_t kFastHi = 141;  // m * 2^31 < 2^55: a batch of 16 stays below 2^59
 
 // Accumulator block at the start of the weight-quantization workspace.
 struct AbsAccum {
@@ -48,21 +51,51 @@ struct AbsAccum {
 constexpr size_t kAbsWsBytes = 4096;
 static_assert(sizeof(AbsAccum) <= kAbsWsBytes, "accumulator block");
 
-__device__ __forceinline__ void absmean_add(float w, unsigned long long& lo, uint32_t& hi,
-                                            unsigned long long* s_bins, bool& bad) {
+// 1 << s for s < 32, and 0 for any larger (unsigned) s: PTX clamps the shift.
+__device__ __forceinline__ uint32_t shl_clamp(uint32_t x, uint32_t sft) {
+  uint32_t r;
+  asm("shl.b32 %0, %1, %2;" : "=r"(r) : "r"(x), "r"(sft));
+  return r;
+}
+
+__device__ __forceinline__ unsigned long long mad_wide_u32(uint32_t a, uint32_t b,
+                                                           unsigned long long c) {
+  unsigned long long d;
+  asm("mad.wide.u32 %0, %1, %2, %3;" : "=l"(d) : "r"(a), "r"(b), "l"(c));
+  return d;
+}
+
+// Fast path for one weight: m * 2^(e-110) if e is in the window, else 0;
+// `out` records a nonzero weight outside the window.
+__device__ __forceinline__ unsigned long long absmean_fast(float w, unsigned long long acc,
+                                                           bool& out) {
+  const uint32_t u = __float_as_uint(w) & 0x7FFFFFFFu;
+  const uint32_t sh = (u >> 23) - kFastLo;  // wraps for e < kFastLo
+  out |= sh > (kFastHi - kFastLo);
+  return mad_wide_u32((u & 0x7FFFFFu) | 0x800000u, shl_clamp(1u, sh), acc);
+}
+
+// Slow path for one weight outside the fast window (zero adds nothing).
+__device__ __forceinline__ void absmean_slow(float w, unsigned long long* s_bins, bool& bad) {
   const uint32_t u = __float_as_uint(w) & 0x7FFFFFFFu;
   const uint32_t e = u >> 23;
-  const uint32_t sh = e - kFastLo;  // wraps for e < kFastLo
-  if (sh <= kFastHi - kFastLo) {
-    const unsigned long long v = (unsigned long long)((u & 0x7FFFFFu) | 0x800000u) << sh;
-    lo += v;
-    hi += (lo < v) ? 1u : 0u;
-  } else if (e == 255u) {
+  if (e - kFastLo <= kFastHi - kFastLo) return;  // counted by the fast path
+  if (e == 255u) {
     bad = true;
-  } else {
-    const uint32_t m = (u & 0x7FFFFFu) | (e ? 0x800000u : 0u);
-    if (m) atomicAdd(&s_bins[e], (unsigned long long)m);
+    return;
   }
+  const uint32_t m = (u & 0x7FFFFFu) | (e ? 0x800000u : 0u);
+  if (m) atomicAdd(&s_bins[e], (unsigned long long)m);
+}
+
+// One weight by both paths (tails).
+__device__ __forceinline__ void absmean_one(float w, unsigned long long& lo, uint32_t& hi,
+                                            unsigned long long* s_bins, bool& bad) {
+  bool out = false;
+  const unsigned long long v = absmean_fast(w, 0ull, out);
+  lo += v;
+  hi += (lo < v) ? 1u : 0u;
+  if (out) absmean_slow(w, s_bins, bad);
 }
 
 // Ternary threshold T from beta: the least float32 strictly above beta*(0.5+2^-25).
@@ -138,7 +171,7 @@ __device__ void absmean_finalize(AbsAccum* acc, int64_t n, float eps, float* bet
   *beta_out = __fadd_rn(__double2float_rn(d), eps);
 }
 
-__global__ void __launch_bounds__(kAbsThreads)
+__global__ void __launch_bounds__(kAbsThreads, 4)
 absmean_kernel(const float* __restrict__ W, int64_t n, float eps, AbsAccum* __restrict__ acc,
                float* __restrict__ beta_out) {
   __shared__ unsigned long long s_bins[256];
@@ -155,33 +188,45 @@ absmean_kernel(const float* __restrict__ W, int64_t n, float eps, AbsAccum* __re
   bool bad = false;
   const int64_t tid = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
   const int64_t nthr = int64_t(gridDim.x) * blockDim.x;
+  int64_t done = 0;  // weights [0, done) go through the batched loop
   if (aligned(W, 16)) {
+    // batches of 4 independent float4 loads per thread; 32 warps per SM keep
+    // about 64 KB per SM in flight
     const int64_t n4 = n >> 2;
+    const int64_t nb = ceil_div(n4, 4 * nthr);  // batches per thread; the last may be partial
     const float4* W4 = reinterpret_cast<const float4*>(W);
-    int64_t i = tid;
-    for (; i + 3 * nthr < n4; i += 4 * nthr) {
-      float4 v[4];
-#pragma unroll
-      for (int u = 0; u < 4; ++u) v[u] = ld_stream_f4(W4 + i + u * nthr);
+    const float4 zero4 = make_float4(0.f, 0.f, 0.f, 0.f);  // adds nothing, never "out"
+    for (int64_t b = 0; b < nb; ++b) {
+      float4 cur[4];
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
-        absmean_add(v[u].x, lo, hi, s_bins, bad);
-        absmean_add(v[u].y, lo, hi, s_bins, bad);
-        absmean_add(v[u].z, lo, hi, s_bins, bad);
-        absmean_add(v[u].w, lo, hi, s_bins, bad);
+        const int64_t i = b * 4 * nthr + tid + u * nthr;
+        cur[u] = i < n4 ? ld_stream_f4(W4 + i) : zero4;
+      }
+      unsigned long long acc = 0ull;
+      bool out = false;
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        acc = absmean_fast(cur[u].x, acc, out);
+        acc = absmean_fast(cur[u].y, acc, out);
+        acc = absmean_fast(cur[u].z, acc, out);
+        acc = absmean_fast(cur[u].w, acc, out);
+      }
+      lo += acc;
+      hi += (lo < acc) ? 1u : 0u;
+      if (__any_sync(0xffffffffu, out)) {
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          absmean_slow(cur[u].x, s_bins, bad);
+          absmean_slow(cur[u].y, s_bins, bad);
+          absmean_slow(cur[u].z, s_bins, bad);
+          absmean_slow(cur[u].w, s_bins, bad);
+        }
       }
     }
-    for (; i < n4; i += nthr) {
-      const float4 v = ld_stream_f4(W4 + i);
-      absmean_add(v.x, lo, hi, s_bins, bad);
-      absmean_add(v.y, lo, hi, s_bins, bad);
-      absmean_add(v.z, lo, hi, s_bins, bad);
-      absmean_add(v.w, lo, hi, s_bins, bad);
-    }
-    for (int64_t j = (n4 << 2) + tid; j < n; j += nthr) absmean_add(W[j], lo, hi, s_bins, bad);
-  } else {
-    for (int64_t j = tid; j < n; j += nthr) absmean_add(W[j], lo, hi, s_bins, bad);
+    done = n4 * 4;
   }
+  for (int64_t j = done + tid; j < n; j += nthr) absmean_one(W[j], lo, hi, s_bins, bad);
 
   // Exact CTA reduction of the 96-bit accumulators as three 32-bit limbs
   // (each limb sum stays below 2^40).

@@ -172,7 +172,7 @@ def _layer(bl, p, fmt, path, bias=None):
     return host(Y), Wd, beta
 
 
-PATHS = ["simt", "auto"]
+PATHS = ["simt", "gemv", "auto"]
 
 
 def _path(bl, name):
@@ -187,9 +187,32 @@ def _path(bl, name):
 def test_linear_small(bl, path, fmt, M, K, N):
     p = random_problem(M + 10 * K + 100 * N, M, K, N)
     f = bl.PACK5 if fmt == "pack5" else bl.I8
+    if bl.linear_plan(M, N, K, f, _path(bl, path))[0] < 0:
+        with pytest.raises(bl.BitLinearError) as e:
+            _layer(bl, p, f, _path(bl, path))
+        assert e.value.status == "BL_ERR_UNSUPPORTED"
+        return
     Y, _, _ = _layer(bl, p, f, _path(bl, path))
     check_ok(bl)
     assert_y_close(Y, oracle.bitlinear(p.X, p.W, p.eps)["Y"])
+
+
+@pytest.mark.parametrize("M,K,N", [
+    (1, 2560, 6912), (1, 6912, 2560), (2, 2560, 300), (3, 999, 149), (4, 2560, 1000),
+    (1, 11008, 2000),       # K split over two warp slices
+    (4, 11008, 2000),       # four rows, five slices
+    (2, 8192, 777), (4, 8192, 148), (1, 5, 3), (4, 1, 1),
+    (1, 81, 40000)])        # 271 rows per CTA in 1 KB stages: the ring of 8 is reused
+def test_gemv_parity(bl, M, K, N):
+    assert bl.linear_plan(M, N, K, bl.PACK5, bl.PATH_GEMV)[0] == bl.PATH_GEMV
+    p = random_problem(3 * M + K + N, M, K, N)
+    Y, Wd, beta = _layer(bl, p, bl.PACK5, bl.PATH_GEMV)
+    check_ok(bl)
+    assert_y_close(Y, oracle.bitlinear(p.X, p.W, p.eps)["Y"])
+    Xq, s = oracle.act_quant(p.X, p.eps)
+    acc = bl.linear_acc(dev(Xq), Wd, bl.PACK5, N, K, path=bl.PATH_GEMV)
+    check_ok(bl)
+    np.testing.assert_array_equal(host(acc), oracle.contract(Xq, oracle.ternarize(p.W, host(beta)[0])))
 
 
 def test_linear_bias(bl):
@@ -207,11 +230,16 @@ def test_linear_acc_exact(bl, path):
     Xq = rng.integers(-127, 128, (M, K)).astype(np.int8)
     Wq = rng.integers(-1, 2, (N, K)).astype(np.int8)
     ref = oracle.contract(Xq, Wq)
-    acc_i8 = bl.linear_acc(dev(Xq), dev(Wq), bl.I8, N, K, path=_path(bl, path))
-    acc_p5 = bl.linear_acc(dev(Xq), bl.pack(dev(Wq)), bl.PACK5, N, K, path=_path(bl, path))
-    check_ok(bl)
-    np.testing.assert_array_equal(host(acc_i8), ref)
-    np.testing.assert_array_equal(host(acc_p5), ref)
+    for f, Wd in ((bl.I8, dev(Wq)), (bl.PACK5, bl.pack(dev(Wq)))):
+        if bl.linear_plan(M, N, K, f, _path(bl, path))[0] < 0:
+            continue
+        acc = bl.linear_acc(dev(Xq), Wd, f, N, K, path=_path(bl, path))
+        check_ok(bl)
+        np.testing.assert_array_equal(host(acc), ref)
+    for m in (1, 2, 4):   # the GEMV's row counts
+        sub = oracle.contract(Xq[:m], Wq)
+        acc = bl.linear_acc(dev(Xq[:m]), bl.pack(dev(Wq)), bl.PACK5, N, K, path=_path(bl, path))
+        np.testing.assert_array_equal(host(acc), sub)
 
 
 def test_linear_extreme_accumulators(bl):
