@@ -181,7 +181,7 @@ class Step:
                     Wout = torch.empty((p.N, bl.pack5_ldp(p.K)), dtype=torch.uint8, device=dev)
                 else:
                     Wout = torch.empty((p.N, p.K), dtype=torch.int8, device=dev)
-                ws = bl.workspace(4096, dev)
+                ws = bl.workspace(bl.load().bl_quantize_weights_workspace_size(p.N, p.K), dev)
                 seen[key] = len(self.tensors)
                 self.tensors.append((W, beta, Wout, ws, p.N, p.K))
             X = torch.from_numpy(np.ascontiguousarray(p.X)).to(dev)
@@ -432,7 +432,7 @@ def e2e(bl, torch, probs, dev, fmt, steps, world):
     dW = [torch.empty_like(h, device=dev) for h in host_W]
     dX = [torch.empty_like(h, device=dev) for h in host_X]
     hY = [torch.empty((p.M, p.N), dtype=torch.float32).pin_memory() for p in probs]
-    ws = [bl.workspace(4096, dev) for _ in host_W]
+    ws = [bl.workspace(bl.load().bl_quantize_weights_workspace_size(1, 1), dev) for _ in host_W]
     h2d = sum(h.numel() * 4 for h in host_W) + sum(h.numel() * 4 for h in host_X)
     d2h = sum(h.numel() * 4 for h in hY)
 

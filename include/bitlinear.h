@@ -70,13 +70,15 @@ typedef enum {
   BL_PATH_AUTO = 0, /* dispatch on M, K, N and the format */
   BL_PATH_SIMT = 1, /* dp4a tile kernel: any shape, any format */
   BL_PATH_GEMV = 2, /* packed-trit decode GEMV on CUDA cores: BL_W_PACK5, M <= 4 */
-  BL_PATH_TC = 3    /* tcgen05 kind::i8 tensor-core GEMM with fused dequant */
+  BL_PATH_TC = 3    /* tcgen05 kind::i8 tensor-core GEMM with fused dequant: K >= 128;
+                       BL_W_I8 rows need ldw % 16 == 0 (packed weights are unpacked
+                       into the workspace first) */
 } bl_path;
 
 /* Packed row stride in bytes: ceil(K/5) rounded up to a multiple of 16. */
 int64_t bl_pack5_ldp(int64_t K);
 
-/* Bytes of `ws` that bl_absmean and bl_quantize_weights* need (4096). */
+/* Bytes of `ws` that bl_absmean and bl_quantize_weights* need (16384). */
 size_t bl_quantize_weights_workspace_size(int64_t N, int64_t K);
 
 /* Step 1 of the weight quantization: beta = (1/n) sum |W| + eps ("the bytes",
@@ -85,7 +87,7 @@ size_t bl_quantize_weights_workspace_size(int64_t N, int64_t K);
  *   W        [N, K] float32, contiguous, 4-byte aligned (16 bytes for full speed).
  *   eps      finite, > 0.
  *   beta_dev one float32 on the device: receives beta.
- *   ws       >= bl_quantize_weights_workspace_size(N, K) bytes (4 KB), 256-byte
+ *   ws       >= bl_quantize_weights_workspace_size(N, K) bytes (16 KB), 256-byte
  *            aligned, ZERO-FILLED before its first use (e.g. cudaMemsetAsync);
  *            every call leaves it zero-filled again, so a workspace is cleared
  *            once and reused.  Calls sharing one workspace must not overlap on
@@ -138,6 +140,9 @@ bl_status bl_quantize_act(const float* X, int64_t M, int64_t K, float eps, int8_
 /* Bytes of `ws` that bl_linear needs for this shape and format. */
 size_t bl_linear_workspace_size(int64_t M, int64_t N, int64_t K, bl_wfmt f);
 
+/* Bytes of `ws` that bl_linear_ex needs with kernel path `path` pinned. */
+size_t bl_linear_ex_workspace_size(int64_t M, int64_t N, int64_t K, bl_wfmt f, int path);
+
 /* The BitLinear forward: Y = (X_q W_q^T)(s beta) [+ bias], X_q and s computed
  * from X inside the call (deployed-path equation).
  *   X        [M, K] float32 contiguous.  M may be 0 (nothing is launched).
@@ -160,7 +165,8 @@ bl_status bl_linear_ex(const float* X, int64_t M, int64_t K, const void* W, bl_w
 
 /* The kernel path bl_linear_ex(..., path) would run for this shape (BL_PATH_*),
  * or -1 if that path cannot take it; *launches (if not NULL) receives the number
- * of kernel launches the call makes.  Host-only, no CUDA call. */
+ * of kernel launches the call makes.  Assumes contiguous weight rows (ldw = K
+ * for BL_W_I8, bl_pack5_ldp(K) for BL_W_PACK5).  Host-only, no CUDA call. */
 int bl_linear_plan(int64_t M, int64_t N, int64_t K, bl_wfmt f, int path, int* launches);
 
 /* The contraction alone: acc[m,n] = sum_k Xq[m,k] * W_q[n,k] in int32, from

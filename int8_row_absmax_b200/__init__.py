@@ -39,6 +39,7 @@ SIGNATURES = {
     "bl_unpack": (_I, [_P, _I64, _I64, _I64, _P, _P]),
     "bl_quantize_act": (_I, [_P, _I64, _I64, _F, _P, _P, _P]),
     "bl_linear_workspace_size": (_SZ, [_I64, _I64, _I64, _I]),
+    "bl_linear_ex_workspace_size": (_SZ, [_I64, _I64, _I64, _I, _I]),
     "bl_linear": (_I, [_P, _I64, _I64, _P, _I, _I64, _I64, _P, _P, _F, _P, _P, _SZ, _P]),
     "bl_linear_ex": (_I, [_P, _I64, _I64, _P, _I, _I64, _I64, _P, _P, _F, _P, _P, _SZ, _I, _P]),
     "bl_linear_noalloc": (_I, [_P, _I64, _I64, _P, _I, _I64, _I64, _P, _P, _F, _P, _P]),
@@ -229,7 +230,7 @@ def linear(X, W, fmt: int, N: int, K: int, beta, bias=None, eps: float = 1e-5,
     if X.shape[1] != K or W.shape[0] != N:
         raise ValueError("shape mismatch")
     Y = torch.empty((M, N), dtype=torch.float32, device=X.device) if out is None else out
-    need = lib.bl_linear_workspace_size(M, N, K, fmt)
+    need = lib.bl_linear_ex_workspace_size(M, N, K, fmt, path)
     ws = workspace(need, X.device) if ws is None else ws
     _check("bl_linear_ex", lib.bl_linear_ex(
         _ptr(X), M, K, _ptr(W), fmt, N, W.shape[1], _ptr(beta), _ptr(bias), eps, _ptr(Y),

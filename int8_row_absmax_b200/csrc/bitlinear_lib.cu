@@ -18,6 +18,7 @@
 #include "act_quant.cuh"
 #include "linear_simt.cuh"
 #include "gemv_pack5.cuh"
+#include "gemm_tc.cuh"
 
 namespace bl {
 namespace {
@@ -59,7 +60,14 @@ bl_status check_weights_args(const float* W, int64_t N, int64_t K, const void* o
 bl_status launch_absmean(const float* W, int64_t n, float eps, float* beta_dev, void* ws,
                          cudaStream_t st) {
   auto* acc = static_cast<AbsAccum*>(ws);
-  absmean_kernel<<<grid_for(ceil_div(n, 64), kAbsThreads, 4), kAbsThreads, 0, st>>>(W, n, eps, acc, beta_dev);
+  if (cudaFuncSetAttribute(absmean_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kAbsSmem) !=
+      cudaSuccess)
+    return BL_ERR_CUDA;
+  // one persistent CTA per SM, fewer when there are fewer 32 KB chunks
+  const int64_t chunks = ceil_div(n, kAbsChunkFloats);
+  int grid = int(chunks < num_sms() ? (chunks < 1 ? 1 : chunks) : num_sms());
+  if (grid > kAbsMaxCtas) grid = kAbsMaxCtas;
+  absmean_kernel<<<grid, kAbsThreads, kAbsSmem, st>>>(W, n, eps, acc, beta_dev);
   return launch_status();
 }
 
@@ -70,15 +78,19 @@ bl_status check_ws(const void* ws, size_t ws_bytes, size_t need) {
 
 // ---- linear --------------------------------------------------------------
 struct LinWs {
-  int64_t ldx;
-  size_t xq_off, s_off, total;
+  int64_t ldx, ldk;
+  size_t xq_off, s_off, wq_off, total;
 };
-LinWs lin_layout(int64_t M, int64_t K) {
+// X_q [M, ldx] and s [M]; with `unpacked_w`, an int8 copy of the packed weights
+// [N, ldk] for the tensor-core path.
+LinWs lin_layout(int64_t M, int64_t K, int64_t N = 0, bool unpacked_w = false) {
   LinWs l;
   l.ldx = round_up(K, 16);
+  l.ldk = round_up(K, 16);
   l.xq_off = 0;
   l.s_off = align_up(size_t(M) * size_t(l.ldx));
-  l.total = l.s_off + align_up(size_t(M) * 4 + 4);
+  l.wq_off = l.s_off + align_up(size_t(M) * 4 + 4);
+  l.total = l.wq_off + (unpacked_w ? align_up(size_t(N) * size_t(l.ldk)) : 0);
   return l;
 }
 
@@ -103,23 +115,114 @@ bl_status check_shape(int64_t M, int64_t K, int64_t N) {
 
 // Resolve the kernel path for a linear call; -1 when the pinned path cannot run it.
 // `fused_quant`: bl_linear (X in float32) rather than bl_linear_acc (X_q given).
+constexpr int64_t kTcMinM = 128;   // AUTO uses the tensor cores from this many rows
+
+// Whether the tensor-core path can take the shape: K at least one 128-byte K
+// block, and for one-trit-per-byte weights a TMA-able row stride.
+bool tc_feasible(int64_t M, int64_t N, int64_t K, bl_wfmt f, int64_t ldw, const void* W) {
+  if (M < 1 || N < 1 || K < kTcBK) return false;
+  if (f == BL_W_I8) return ldw % 16 == 0 && (W == nullptr || is_aligned(W, 16));
+  return f == BL_W_PACK5;
+}
+
 int resolve_path(int64_t M, int64_t N, int64_t K, bl_wfmt f, int path, int* launches,
-                 bool fused_quant = true) {
+                 bool fused_quant = true, int64_t ldw = -1, const void* W = nullptr) {
   const int64_t ldp = round_up(ceil_div(K, 5), 16);
+  if (ldw < 0) ldw = f == BL_W_PACK5 ? ldp : K;   // contiguous rows unless told otherwise
   const bool gemv_ok = f == BL_W_PACK5 && M >= 1 && gemv_feasible(M, N, K, ldp);
+  const bool tc_ok = tc_feasible(M, N, K, f, ldw, W);
   int p = path;
-  if (p == BL_PATH_AUTO) p = gemv_ok ? BL_PATH_GEMV : BL_PATH_SIMT;
+  if (p == BL_PATH_AUTO)
+    p = (M >= kTcMinM && tc_ok) ? BL_PATH_TC : (gemv_ok ? BL_PATH_GEMV : BL_PATH_SIMT);
   int n = 0;
   if (p == BL_PATH_SIMT) {
     n = fused_quant ? 2 : 1;  // act_quant + contraction
   } else if (p == BL_PATH_GEMV) {
     if (!gemv_ok) return -1;
     n = 1;                    // quantization fused into the GEMV
+  } else if (p == BL_PATH_TC) {
+    if (!tc_ok) return -1;
+    n = (fused_quant ? 2 : 1) + (f == BL_W_PACK5 ? 1 : 0);  // [act_quant,] [unpack,] GEMM
   } else {
     return -1;
   }
   if (launches) *launches = M == 0 ? 0 : n;
   return p;
+}
+
+// ---- tensor maps (driver entry point, so the library does not link libcuda) ---
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn encode_tiled() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// 2-D int8 [outer, inner] matrix with row stride `ld` bytes, 128-byte swizzled
+// boxes of {128, box_rows}; out-of-range elements read as zero.
+bool make_map_i8(CUtensorMap* map, const void* base, int64_t inner, int64_t outer, int64_t ld,
+                 int box_rows) {
+  EncodeTiledFn fn = encode_tiled();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {cuuint64_t(inner), cuuint64_t(outer)};
+  const cuuint64_t strides[1] = {cuuint64_t(ld)};
+  const cuuint32_t box[2] = {cuuint32_t(kTcBK), cuuint32_t(box_rows)};
+  const cuuint32_t estr[2] = {1u, 1u};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// The tcgen05 GEMM on int8 X_q [M, ldx] and int8 W_q [N, ldw].
+bl_status run_tc(const int8_t* Xq, int64_t ldx, int64_t M, int64_t K, const int8_t* Wq, int64_t ldw,
+                 int64_t N, const float* s, const float* beta, const float* bias, float* Y,
+                 int32_t* acc, cudaStream_t st) {
+  if (ldx % 16 != 0 || ldw % 16 != 0 || !is_aligned(Xq, 16) || !is_aligned(Wq, 16))
+    return BL_ERR_ALIGNMENT;
+  if (ceil_div(M, kTcBM) > 65535) return BL_ERR_UNSUPPORTED;
+  TcMaps maps;
+  if (!make_map_i8(&maps.a, Xq, K, M, ldx, kTcBM) || !make_map_i8(&maps.b, Wq, K, N, ldw, kTcBN))
+    return BL_ERR_CUDA;
+  TcArgs a;
+  a.M = M;
+  a.N = N;
+  a.K = K;
+  a.s = s;
+  a.beta = beta;
+  a.bias = bias;
+  a.Y = Y;
+  a.acc = acc;
+  const dim3 grid(unsigned(ceil_div(N, kTcBN)), unsigned(ceil_div(M, kTcBM)));
+  if (Y) {
+    if (cudaFuncSetAttribute(gemm_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kTcSmem) !=
+        cudaSuccess)
+      return BL_ERR_CUDA;
+    gemm_tc_kernel<true><<<grid, kTcThreads, kTcSmem, st>>>(maps, a);
+  } else {
+    if (cudaFuncSetAttribute(gemm_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, kTcSmem) !=
+        cudaSuccess)
+      return BL_ERR_CUDA;
+    gemm_tc_kernel<false><<<grid, kTcThreads, kTcSmem, st>>>(maps, a);
+  }
+  return launch_status();
+}
+
+// Packed weights -> int8 rows in the workspace (first version of the tensor-core path).
+bl_status unpack_rows(const uint8_t* Wp, int64_t N, int64_t K, int64_t ldp, int8_t* Wq, int64_t ldk,
+                      cudaStream_t st) {
+  const int64_t words = ceil_div(ceil_div(K, 5), 4);
+  unpack5_rows_kernel<<<grid_for(N * words, 256), 256, 0, st>>>(Wp, N, K, ldp, Wq, ldk);
+  return launch_status();
 }
 
 template <int M, int CH, bool F, bool D>
@@ -311,11 +414,14 @@ bl_status bl_quantize_act(const float* X, int64_t M, int64_t K, float eps, int8_
   return launch_status();
 }
 
+size_t bl_linear_ex_workspace_size(int64_t M, int64_t N, int64_t K, bl_wfmt f, int path) {
+  if (M < 0 || K < 1 || N < 1) return 0;
+  const int p = resolve_path(M, N, K, f, path, nullptr);
+  return lin_layout(M, K, N, p == BL_PATH_TC && f == BL_W_PACK5).total;
+}
+
 size_t bl_linear_workspace_size(int64_t M, int64_t N, int64_t K, bl_wfmt f) {
-  (void)N;
-  (void)f;
-  if (M < 0 || K < 1) return 0;
-  return lin_layout(M, K).total;
+  return bl_linear_ex_workspace_size(M, N, K, f, BL_PATH_AUTO);
 }
 
 bl_status bl_linear_ex(const float* X, int64_t M, int64_t K, const void* W, bl_wfmt f,
@@ -331,10 +437,10 @@ bl_status bl_linear_ex(const float* X, int64_t M, int64_t K, const void* W, bl_w
   if (M == 0) return BL_OK;
   if (!X || !Y || !beta_dev) return BL_ERR_INVALID_ARG;
   if (!is_aligned(X, 4) || !is_aligned(Y, 4) || (bias && !is_aligned(bias, 4))) return BL_ERR_ALIGNMENT;
-  const LinWs l = lin_layout(M, K);
-  if (!ws || !is_aligned(ws, kWsAlign) || ws_bytes < l.total) return BL_ERR_WORKSPACE;
-  const int p = resolve_path(M, N, K, f, path, nullptr);
+  const int p = resolve_path(M, N, K, f, path, nullptr, true, ldw, W);
   if (p < 0) return BL_ERR_UNSUPPORTED;
+  const LinWs l = lin_layout(M, K, N, p == BL_PATH_TC && f == BL_W_PACK5);
+  if (!ws || !is_aligned(ws, kWsAlign) || ws_bytes < l.total) return BL_ERR_WORKSPACE;
   if (p == BL_PATH_GEMV)
     return run_gemv(X, nullptr, 0, M, K, W, ldw, N, beta_dev, bias, eps, Y, nullptr, stream);
   int8_t* Xq = reinterpret_cast<int8_t*>(static_cast<char*>(ws) + l.xq_off);
@@ -342,6 +448,18 @@ bl_status bl_linear_ex(const float* X, int64_t M, int64_t K, const void* W, bl_w
   act_quant_kernel<<<unsigned(M), kActThreads, 0, stream>>>(X, K, eps, Xq, l.ldx, s);
   st = launch_status();
   if (st != BL_OK) return st;
+  if (p == BL_PATH_TC) {
+    const int8_t* Wq = static_cast<const int8_t*>(W);
+    int64_t ldq = ldw;
+    if (f == BL_W_PACK5) {
+      int8_t* scratch = reinterpret_cast<int8_t*>(static_cast<char*>(ws) + l.wq_off);
+      st = unpack_rows(static_cast<const uint8_t*>(W), N, K, ldw, scratch, l.ldk, stream);
+      if (st != BL_OK) return st;
+      Wq = scratch;
+      ldq = l.ldk;
+    }
+    return run_tc(Xq, l.ldx, M, K, Wq, ldq, N, s, beta_dev, bias, Y, nullptr, stream);
+  }
   return run_simt(Xq, l.ldx, M, K, W, f, ldw, N, s, beta_dev, bias, Y, nullptr, stream);
 }
 
@@ -375,19 +493,15 @@ bl_status bl_linear_noalloc(const float* X, int64_t M, int64_t K, const void* W,
 }
 
 size_t bl_linear_acc_workspace_size(int64_t M, int64_t N, int64_t K, bl_wfmt f, int path) {
-  (void)M;
-  (void)N;
-  (void)K;
-  (void)f;
-  (void)path;
+  if (M < 1 || N < 1 || K < 1) return 0;
+  const int p = resolve_path(M, N, K, f, path, nullptr, false);
+  if (p == BL_PATH_TC && f == BL_W_PACK5) return align_up(size_t(N) * size_t(round_up(K, 16)));
   return 0;
 }
 
 bl_status bl_linear_acc_ex(const int8_t* Xq, int64_t M, int64_t K, const void* W, bl_wfmt f,
                            int64_t N, int64_t ldw, int32_t* acc, void* ws, size_t ws_bytes,
                            int path, cudaStream_t stream) {
-  (void)ws;
-  (void)ws_bytes;
   bl_status st = check_shape(M, K, N);
   if (st != BL_OK) return st;
   st = check_w(W, f, K, ldw);
@@ -396,10 +510,30 @@ bl_status bl_linear_acc_ex(const int8_t* Xq, int64_t M, int64_t K, const void* W
   if (M == 0) return BL_OK;
   if (!Xq || !acc) return BL_ERR_INVALID_ARG;
   if (!is_aligned(acc, 4)) return BL_ERR_ALIGNMENT;
-  const int p = resolve_path(M, N, K, f, path, nullptr, false);
+  int p = resolve_path(M, N, K, f, path, nullptr, false, ldw, W);
+  // X_q given by the caller: the tensor cores need a TMA-able [M, K] int8 matrix
+  const bool tc_x_ok = K % 16 == 0 && is_aligned(Xq, 16);
+  if (p == BL_PATH_TC && !tc_x_ok) {
+    if (path == BL_PATH_TC) return BL_ERR_UNSUPPORTED;
+    p = resolve_path(M, N, K, f, BL_PATH_GEMV, nullptr, false) >= 0 ? BL_PATH_GEMV : BL_PATH_SIMT;
+  }
   if (p < 0) return BL_ERR_UNSUPPORTED;
   if (p == BL_PATH_GEMV)
     return run_gemv(nullptr, Xq, K, M, K, W, ldw, N, nullptr, nullptr, 0.f, nullptr, acc, stream);
+  if (p == BL_PATH_TC) {
+    const int8_t* Wq = static_cast<const int8_t*>(W);
+    int64_t ldq = ldw;
+    if (f == BL_W_PACK5) {
+      const size_t need = align_up(size_t(N) * size_t(round_up(K, 16)));
+      if (!ws || !is_aligned(ws, kWsAlign) || ws_bytes < need) return BL_ERR_WORKSPACE;
+      int8_t* scratch = static_cast<int8_t*>(ws);
+      bl_status st2 = unpack_rows(static_cast<const uint8_t*>(W), N, K, ldw, scratch, round_up(K, 16), stream);
+      if (st2 != BL_OK) return st2;
+      Wq = scratch;
+      ldq = round_up(K, 16);
+    }
+    return run_tc(Xq, K, M, K, Wq, ldq, N, nullptr, nullptr, nullptr, nullptr, acc, stream);
+  }
   return run_simt(Xq, K, M, K, W, f, ldw, N, nullptr, nullptr, nullptr, nullptr, acc, stream);
 }
 

@@ -8,7 +8,13 @@
 // that sit on a rounding boundary.  Every finite float32 |w| is m * 2^(e-150)
 // (m < 2^24, e the biased exponent), so the sum is an integer in units of 2^-149.
 //
-//   absmean (one launch):
+//   absmean (one launch, one persistent CTA per SM):
+//     0. the weights stream through a ring of shared-memory stages filled by
+//        32 KB bulk copies (TMA engine) that one producer warp issues; chunks
+//        are handed out dynamically from a counter in the workspace, so SMs
+//        that get their bytes sooner take more chunks instead of waiting for
+//        the slowest one; 16 consumer warps read the stages (full / empty
+//        mbarrier pair per stage, bounded waits);
 //     1. each thread adds magnitudes with exponents in a fast window [110, 141]
 //        into a 96-bit fixed-point accumulator (unit 2^-40): one mad.wide.u32 per
 //        weight adds m * 2^(e-110), where shl.b32 turns any shift outside the
@@ -18,10 +24,14 @@
 //     2. each CTA adds its three 32-bit limb sums and its non-zero bins into the
 //        workspace accumulator block with 64-bit atomics (integer adds are exact,
 //        so the total does not depend on the schedule), then takes a ticket;
-//     3. the CTA that takes the last ticket places every bin and limb at its bit
-//        offset in a 512-bit integer (word-parallel, then one carry pass), rounds
-//        it once to float64 (nearest-even), divides by n in float64 (IEEE),
-//        rounds to float32, adds eps in float32, and clears the block again.
+//     3. the CTA that takes the last ticket rounds the exact total once to
+//        float64 (nearest-even): when no exponent bin was used the total is the
+//        96-bit fixed-point sum, converted by one correctly rounded
+//        integer-to-double (a sticky bit stands for any dropped low bits);
+//        otherwise every bin and limb is placed at its bit offset in a 512-bit
+//        integer (word-parallel, then one carry pass) and rounded from there.
+//        Then it divides by n in float64 (IEEE), rounds to float32, adds eps in
+//        float32, and clears the block again.
 //     The block must therefore be zero before the first call on a workspace;
 //     every call leaves it zero.  A magic word that must read 0 catches most
 //     workspaces that were never cleared (reported as BL_ERR_WORKSPACE).
@@ -34,21 +44,30 @@
 #pragma once
 
 #include "common.cuh"
+#include "ptx.cuh"
 
 namespace bl {
 
-constexpr int kAbsThreads = 256;
+constexpr int kAbsConsumers = 512;                          // 16 consumer warps
+constexpr int kAbsThreads = kAbsConsumers + 32;             // + 1 producer warp
+constexpr int kAbsChunkFloats = 8192;                       // 32 KB per bulk copy
+constexpr uint32_t kAbsChunkBytes = kAbsChunkFloats * 4;
+constexpr int kAbsStages = 6;                               // 192 KB in flight per SM
+constexpr int kAbsSmem = kAbsStages * int(kAbsChunkBytes);
 constexpr uint32_t kFastLo = 110;  // exponent whose mantissa LSB is 2^-40
 constexpr uint32_t kFastHi = 141;  // m * 2^31 < 2^55: a batch of 16 stays below 2^59
 
 // Accumulator block at the start of the weight-quantization workspace.
+constexpr int kAbsMaxCtas = 256;
 struct AbsAccum {
-  unsigned long long limb[4];   // sums of the 32-bit limbs of the fast accumulators
   unsigned long long bins[256]; // sum of m per biased exponent outside the window
   unsigned int ticket;          // CTAs done so far in the current call
   unsigned int magic;           // must be 0: a never-cleared workspace reads non-zero
+  unsigned int next_chunk;      // next 32 KB chunk of W to hand out
+  unsigned int pad_;
+  unsigned long long slot[kAbsMaxCtas][4];  // per-CTA sums of the three 32-bit limbs
 };
-constexpr size_t kAbsWsBytes = 4096;
+constexpr size_t kAbsWsBytes = 16384;
 static_assert(sizeof(AbsAccum) <= kAbsWsBytes, "accumulator block");
 
 // 1 << s for s < 32, and 0 for any larger (unsigned) s: PTX clamps the shift.
@@ -108,145 +127,237 @@ __device__ __forceinline__ float ternary_threshold(float beta) {
 
 constexpr int kBigWords = 16;  // 512 bits; the sum is below 2^330 units of 2^-149
 
-// Step 3, run by the last CTA: the exact sum as an integer, rounded once.
-__device__ void absmean_finalize(AbsAccum* acc, int64_t n, float eps, float* beta_out,
-                                 unsigned long long* s_word, uint32_t* s_big) {
+// Step 3, run by the last CTA: the exact sum rounded once to float64.  All the
+// global reads (bins, every CTA's limb slot, the magic word) are issued at once.
+__device__ void absmean_finalize(AbsAccum* acc, int64_t n, float eps, float* beta_out, int nctas,
+                                 unsigned long long* s_binv, unsigned long long* s_limbsum,
+                                 unsigned long long* s_word, uint32_t* s_big, int* s_flag) {
   const int t = threadIdx.x;
   for (int i = t; i < kBigWords + 3; i += blockDim.x) s_word[i] = 0ull;
+  if (t < 3) s_limbsum[t] = 0ull;
+  if (t == 0) *s_flag = 0;
   __syncthreads();
-  for (int j = t; j < 258; j += blockDim.x) {
-    unsigned long long v;
-    int shift;
-    if (j < 255) {
-      v = __ldcg(&acc->bins[j]);
-      shift = (j > 0 ? j : 1) - 1;                // m * 2^(max(e,1)-150) in units of 2^-149
-    } else {
-      v = __ldcg(&acc->limb[j - 255]);
-      shift = 32 * (j - 255) + int(kFastLo) - 1;  // limb i weighs 2^(32 i) * 2^(kFastLo-150)
-    }
-    if (v) {
-      const int w = shift >> 5, b = shift & 31;
-      const unsigned long long lo64 = v << b, hi64 = b ? (v >> (64 - b)) : 0ull;
-      atomicAdd(&s_word[w], lo64 & 0xFFFFFFFFull);
-      atomicAdd(&s_word[w + 1], lo64 >> 32);
-      atomicAdd(&s_word[w + 2], hi64);
+  if (t < 255) {
+    const unsigned long long v = __ldcg(&acc->bins[t]);
+    s_binv[t] = v;
+    if (v) *s_flag = 1;                         // some magnitude outside the fast window
+  }
+  for (int c = t; c < nctas; c += blockDim.x) {
+    atomicAdd(&s_limbsum[0], __ldcg(&acc->slot[c][0]));
+    atomicAdd(&s_limbsum[1], __ldcg(&acc->slot[c][1]));
+    atomicAdd(&s_limbsum[2], __ldcg(&acc->slot[c][2]));
+  }
+  const unsigned int magic = t == 0 ? __ldcg(&acc->magic) : 0u;
+  __syncthreads();
+  const bool fast = *s_flag == 0;
+  if (!fast) {
+    for (int j = t; j < 258; j += blockDim.x) {
+      const unsigned long long w = j < 255 ? s_binv[j] : s_limbsum[j - 255];
+      // bins: m * 2^(max(e,1)-150) = m * 2^(max(e,1)-1) units of 2^-149;
+      // limb i weighs 2^(32 i) * 2^(kFastLo-150) = 2^(32 i + kFastLo - 1) units
+      const int shift = j < 255 ? (j > 0 ? j : 1) - 1 : 32 * (j - 255) + int(kFastLo) - 1;
+      if (w) {
+        const int wi = shift >> 5, b = shift & 31;
+        const unsigned long long lo64 = w << b, hi64 = b ? (w >> (64 - b)) : 0ull;
+        atomicAdd(&s_word[wi], lo64 & 0xFFFFFFFFull);
+        atomicAdd(&s_word[wi + 1], lo64 >> 32);
+        atomicAdd(&s_word[wi + 2], hi64);
+      }
     }
   }
   __syncthreads();
-  // leave the block zero for the next call
-  for (int j = t; j < 256; j += blockDim.x) acc->bins[j] = 0ull;
-  if (t < 4) acc->limb[t] = 0ull;
   if (t == 0) {
-    if (__ldcg(&acc->magic) != 0u) raise_status(kDevBadWorkspace);
-    acc->ticket = 0u;
-  }
-  if (t != 0) return;
-  unsigned long long carry = 0ull;
-  for (int i = 0; i < kBigWords; ++i) {
-    const unsigned long long sw = s_word[i] + carry;
-    s_big[i] = uint32_t(sw);
-    carry = sw >> 32;
-  }
-  int top = -1;
-  for (int i = kBigWords - 1; i >= 0; --i)
-    if (s_big[i]) { top = i * 32 + 31 - __clz(s_big[i]); break; }
-  double D = 0.0;
-  if (top >= 0) {
-    const int lsb = top - 52 > 0 ? top - 52 : 0;   // lowest bit kept in the mantissa
-    const int w0 = lsb >> 5, b0 = lsb & 31;
-    unsigned long long mant = ((unsigned long long)s_big[w0] |
-                               (w0 + 1 < kBigWords ? (unsigned long long)s_big[w0 + 1] << 32 : 0ull)) >> b0;
-    if (b0 && w0 + 2 < kBigWords) mant |= (unsigned long long)s_big[w0 + 2] << (64 - b0);
-    mant &= (1ull << (top - lsb + 1)) - 1ull;      // the bits [lsb, top]
-    if (lsb > 0) {                                 // round to nearest, ties to even
-      const int rpos = lsb - 1;
-      const int rnd = int((s_big[rpos >> 5] >> (rpos & 31)) & 1u);
-      bool sticky = (s_big[rpos >> 5] & ((1u << (rpos & 31)) - 1u)) != 0u;
-      for (int i = (rpos >> 5) - 1; i >= 0 && !sticky; --i) sticky = s_big[i] != 0u;
-      if (rnd && (sticky || (mant & 1ull))) mant += 1ull;  // 2^53 stays exact
+    double D = 0.0;
+    if (fast) {
+      // total = L0 + L1 2^32 + L2 2^64 units of 2^-40 (each L < 2^50)
+      const unsigned long long L0 = s_limbsum[0], L1 = s_limbsum[1], L2 = s_limbsum[2];
+      unsigned long long lo = L0 + (L1 << 32);
+      const unsigned long long hi = (L1 >> 32) + L2 + (lo < L0 ? 1ull : 0ull);
+      if (hi == 0ull) {
+        D = ldexp(__ull2double_rn(lo), -int(150 - kFastLo));
+      } else {
+        const int sh = 64 - __clzll(hi);            // drop sh low bits, keep a sticky bit
+        unsigned long long top = (hi << (64 - sh)) | (lo >> sh);
+        top |= (lo << (64 - sh)) != 0ull ? 1ull : 0ull;
+        D = ldexp(__ull2double_rn(top), sh - int(150 - kFastLo));
+      }
+    } else {
+      unsigned long long carry = 0ull;
+      for (int i = 0; i < kBigWords; ++i) {
+        const unsigned long long sw = s_word[i] + carry;
+        s_big[i] = uint32_t(sw);
+        carry = sw >> 32;
+      }
+      int top = -1;
+      for (int i = kBigWords - 1; i >= 0; --i)
+        if (s_big[i]) { top = i * 32 + 31 - __clz(s_big[i]); break; }
+      if (top >= 0) {
+        const int lsb = top - 52 > 0 ? top - 52 : 0;   // lowest bit kept in the mantissa
+        const int w0 = lsb >> 5, b0 = lsb & 31;
+        unsigned long long mant = ((unsigned long long)s_big[w0] |
+                                   (w0 + 1 < kBigWords ? (unsigned long long)s_big[w0 + 1] << 32 : 0ull)) >> b0;
+        if (b0 && w0 + 2 < kBigWords) mant |= (unsigned long long)s_big[w0 + 2] << (64 - b0);
+        mant &= (1ull << (top - lsb + 1)) - 1ull;      // the bits [lsb, top]
+        if (lsb > 0) {                                 // round to nearest, ties to even
+          const int rpos = lsb - 1;
+          const int rnd = int((s_big[rpos >> 5] >> (rpos & 31)) & 1u);
+          bool sticky = (s_big[rpos >> 5] & ((1u << (rpos & 31)) - 1u)) != 0u;
+          for (int i = (rpos >> 5) - 1; i >= 0 && !sticky; --i) sticky = s_big[i] != 0u;
+          if (rnd && (sticky || (mant & 1ull))) mant += 1ull;  // 2^53 stays exact
+        }
+        D = ldexp(double(mant), lsb - 149);
+      }
     }
-    D = ldexp(double(mant), lsb - 149);
+    const double d = __ddiv_rn(D, double(n));
+    *beta_out = __fadd_rn(__double2float_rn(d), eps);
+    if (magic != 0u) raise_status(kDevBadWorkspace);
+    acc->ticket = 0u;                            // leave the block clear for the next call
+    acc->next_chunk = 0u;
   }
-  const double d = __ddiv_rn(D, double(n));
-  *beta_out = __fadd_rn(__double2float_rn(d), eps);
+  for (int j = t; j < 255; j += blockDim.x)
+    if (s_binv[j]) acc->bins[j] = 0ull;
 }
 
-__global__ void __launch_bounds__(kAbsThreads, 4)
+__global__ void __launch_bounds__(kAbsThreads, 1)
 absmean_kernel(const float* __restrict__ W, int64_t n, float eps, AbsAccum* __restrict__ acc,
                float* __restrict__ beta_out) {
+  extern __shared__ __align__(128) unsigned char stage_smem[];
+  __shared__ uint64_t full[kAbsStages], empty[kAbsStages];
+  __shared__ int s_chunk[kAbsStages];
+  __shared__ int s_issued[kAbsStages];   // phases started on full[s] (copies + the stop mark)
   __shared__ unsigned long long s_bins[256];
   __shared__ unsigned long long s_limb[3];
   __shared__ unsigned long long s_word[kBigWords + 3];
   __shared__ uint32_t s_big[kBigWords];
+  __shared__ int s_flag;
+  __shared__ int s_timeout;
+  __shared__ unsigned long long s_binv[255];
   __shared__ bool s_last;
-  for (int i = threadIdx.x; i < 256; i += blockDim.x) s_bins[i] = 0ull;
-  if (threadIdx.x < 3) s_limb[threadIdx.x] = 0ull;
-  __syncthreads();
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5;
+  for (int i = tid; i < 256; i += blockDim.x) s_bins[i] = 0ull;
+  if (tid < 3) s_limb[tid] = 0ull;
 
   unsigned long long lo = 0ull;
   uint32_t hi = 0u;
   bool bad = false;
-  const int64_t tid = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
-  const int64_t nthr = int64_t(gridDim.x) * blockDim.x;
-  int64_t done = 0;  // weights [0, done) go through the batched loop
-  if (aligned(W, 16)) {
-    // batches of 4 independent float4 loads per thread; 32 warps per SM keep
-    // about 64 KB per SM in flight
-    const int64_t n4 = n >> 2;
-    const int64_t nb = ceil_div(n4, 4 * nthr);  // batches per thread; the last may be partial
-    const float4* W4 = reinterpret_cast<const float4*>(W);
-    const float4 zero4 = make_float4(0.f, 0.f, 0.f, 0.f);  // adds nothing, never "out"
-    for (int64_t b = 0; b < nb; ++b) {
-      float4 cur[4];
+  const bool tma = aligned(W, 16);
+  const int64_t nvec = tma ? (n & ~int64_t(3)) : 0;             // floats read by bulk copies
+  const int64_t nch = ceil_div(nvec, kAbsChunkFloats);
+  if (tid == 0) {
+    s_timeout = 0;
+    for (int s = 0; s < kAbsStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], kAbsConsumers / 32);
+      s_issued[s] = 0;
+    }
+    fence_mbar_init();
+  }
+  __syncthreads();
+
+  if (warp == kAbsConsumers / 32) {
+    // producer warp: lane 0 hands out chunks and issues the copies
+    if ((tid & 31) == 0) {
+      unsigned int c = atomicAdd(&acc->next_chunk, 1u);
+      for (int it = 0;; ++it) {
+        const int s = it % kAbsStages;
+        if (it >= kAbsStages && !mbar_wait(&empty[s], uint32_t(it / kAbsStages - 1) & 1u)) {
+          s_timeout = 1;
+          break;
+        }
+        if (int64_t(c) >= nch) {           // no more work: tell the consumers of stage s
+          s_chunk[s] = -1;
+          s_issued[s] += 1;
+          mbar_arrive(&full[s]);
+          break;
+        }
+        const unsigned int cur = c;
+        c = atomicAdd(&acc->next_chunk, 1u);  // the next chunk, while this copy flies
+        const int64_t f0 = int64_t(cur) * kAbsChunkFloats;
+        const uint32_t bytes = uint32_t(min(int64_t(kAbsChunkFloats), nvec - f0) * 4);
+        s_chunk[s] = int(cur);
+        s_issued[s] += 1;
+        fence_proxy_async_smem();
+        mbar_arrive_expect_tx(&full[s], bytes);
+        bulk_g2s(stage_smem + size_t(s) * kAbsChunkBytes, W + f0, bytes, &full[s]);
+      }
+    }
+  } else {
+    // consumer warps
+    for (int it = 0;; ++it) {
+      const int s = it % kAbsStages;
+      if (!mbar_wait(&full[s], uint32_t(it / kAbsStages) & 1u)) {
+        s_timeout = 1;
+        break;
+      }
+      const int c = s_chunk[s];
+      if (c < 0) break;
+      const int cnt4 = int(min(int64_t(kAbsChunkFloats), nvec - int64_t(c) * kAbsChunkFloats) >> 2);
+      const float4* src = reinterpret_cast<const float4*>(stage_smem + size_t(s) * kAbsChunkBytes);
+      float4 v[4];
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
-        const int64_t i = b * 4 * nthr + tid + u * nthr;
-        cur[u] = i < n4 ? ld_stream_f4(W4 + i) : zero4;
+        const int i = tid + u * kAbsConsumers;
+        v[u] = i < cnt4 ? src[i] : make_float4(0.f, 0.f, 0.f, 0.f);
       }
-      unsigned long long acc = 0ull;
+      __syncwarp();
+      if ((tid & 31) == 0) mbar_arrive(&empty[s]);   // this warp is done with stage s
+      unsigned long long accb = 0ull;
       bool out = false;
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
-        acc = absmean_fast(cur[u].x, acc, out);
-        acc = absmean_fast(cur[u].y, acc, out);
-        acc = absmean_fast(cur[u].z, acc, out);
-        acc = absmean_fast(cur[u].w, acc, out);
+        accb = absmean_fast(v[u].x, accb, out);
+        accb = absmean_fast(v[u].y, accb, out);
+        accb = absmean_fast(v[u].z, accb, out);
+        accb = absmean_fast(v[u].w, accb, out);
       }
-      lo += acc;
-      hi += (lo < acc) ? 1u : 0u;
+      lo += accb;
+      hi += (lo < accb) ? 1u : 0u;
       if (__any_sync(0xffffffffu, out)) {
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
-          absmean_slow(cur[u].x, s_bins, bad);
-          absmean_slow(cur[u].y, s_bins, bad);
-          absmean_slow(cur[u].z, s_bins, bad);
-          absmean_slow(cur[u].w, s_bins, bad);
+          absmean_slow(v[u].x, s_bins, bad);
+          absmean_slow(v[u].y, s_bins, bad);
+          absmean_slow(v[u].z, s_bins, bad);
+          absmean_slow(v[u].w, s_bins, bad);
         }
       }
     }
-    done = n4 * 4;
   }
-  for (int64_t j = done + tid; j < n; j += nthr) absmean_one(W[j], lo, hi, s_bins, bad);
+  __syncthreads();
+  if (s_timeout) {  // a wait gave up: report, then wait (bounded) for every stage's
+    if (tid == 0) {   // last phase so no copy is still writing when the CTA exits
+      raise_status(kDevTimeout);
+      for (int s = 0; s < kAbsStages; ++s)
+        if (s_issued[s] > 0) (void)mbar_wait(&full[s], uint32_t(s_issued[s] - 1) & 1u);
+    }
+    return;
+  }
+  // the few weights outside the bulk copies: the unaligned case, or the < 4 past them
+  if (blockIdx.x == 0 || !tma)
+    for (int64_t j = nvec + tid + (tma ? 0 : int64_t(blockIdx.x) * blockDim.x); j < n;
+         j += tma ? blockDim.x : int64_t(gridDim.x) * blockDim.x)
+      absmean_one(W[j], lo, hi, s_bins, bad);
 
   // Exact CTA reduction of the 96-bit accumulators as three 32-bit limbs
-  // (each limb sum stays below 2^40).
+  // (each limb sum stays below 2^41).
   const unsigned long long l0 = warp_sum_u64(lo & 0xFFFFFFFFull);
   const unsigned long long l1 = warp_sum_u64(lo >> 32);
   const unsigned long long l2 = warp_sum_u64((unsigned long long)hi);
-  if ((threadIdx.x & 31) == 0) {
+  if ((tid & 31) == 0) {
     atomicAdd(&s_limb[0], l0);
     atomicAdd(&s_limb[1], l1);
     atomicAdd(&s_limb[2], l2);
   }
-  if (__syncthreads_or(bad) && threadIdx.x == 0) raise_status(kDevNonFinite);
-  for (int i = threadIdx.x; i < 256; i += blockDim.x)
-    if (s_bins[i]) atomicAdd(&acc->bins[i], s_bins[i]);
-  if (threadIdx.x < 3 && s_limb[threadIdx.x]) atomicAdd(&acc->limb[threadIdx.x], s_limb[threadIdx.x]);
+  if (__syncthreads_or(bad) && tid == 0) raise_status(kDevNonFinite);
+  for (int i = tid; i < 256; i += blockDim.x)
+    if (s_bins[i]) atomicAdd(&acc->bins[i], s_bins[i]);   // rare: weights outside the window
+  if (tid < 3) acc->slot[blockIdx.x][tid] = s_limb[tid];   // plain stores, own slot
 
   // Last-CTA-done: the CTA whose ticket completes the grid finalizes.
   __threadfence();
   __syncthreads();
-  if (threadIdx.x == 0) {
+  if (tid == 0) {
     const unsigned int ticket = atomicAdd(&acc->ticket, 1u);
     if (ticket >= gridDim.x) raise_status(kDevBadWorkspace);
     s_last = (ticket == gridDim.x - 1);
@@ -254,7 +365,7 @@ absmean_kernel(const float* __restrict__ W, int64_t n, float eps, AbsAccum* __re
   __syncthreads();
   if (!s_last) return;
   __threadfence();
-  absmean_finalize(acc, n, eps, beta_out, s_word, s_big);
+  absmean_finalize(acc, n, eps, beta_out, int(gridDim.x), s_binv, s_limb, s_word, s_big, &s_flag);
 }
 
 // W [N,K] float32 -> Wq [N,K] int8 codes.

@@ -53,8 +53,8 @@ def test_status_strings(lib):
 
 def test_workspace_sizes(lib):
     assert lib.bl_quantize_weights_workspace_size(0, 5) == 0
-    assert lib.bl_quantize_weights_workspace_size(4, 4) == 4096
-    assert lib.bl_quantize_weights_workspace_size(8192, 8192) == 4096
+    assert lib.bl_quantize_weights_workspace_size(4, 4) == 16384
+    assert lib.bl_quantize_weights_workspace_size(8192, 8192) == 16384
     assert lib.bl_linear_workspace_size(16, 64, 100, 1) >= 16 * 112 + 16 * 4
 
 
@@ -89,9 +89,9 @@ NULL = None
     (lambda L: L.bl_quantize_weights(16, 4, 4, -1.0, 16, 16, 256, 1 << 20, NULL), 1),
     (lambda L: L.bl_quantize_weights(16, 4, 4, 1e-5, 16, 16, 256, 4, NULL), 4),
     (lambda L: L.bl_quantize_weights(18, 4, 4, 1e-5, 16, 16, 256, 1 << 20, NULL), 2),
-    (lambda L: L.bl_absmean(16, 4, 4, 1e-5, 16, 255, 4096, NULL), 4),
-    (lambda L: L.bl_absmean(16, 4, 4, 1e-5, 18, 256, 4096, NULL), 2),
-    (lambda L: L.bl_absmean(16, 0, 4, 1e-5, 16, 256, 4096, NULL), 1),
+    (lambda L: L.bl_absmean(16, 4, 4, 1e-5, 16, 255, 16384, NULL), 4),
+    (lambda L: L.bl_absmean(16, 4, 4, 1e-5, 18, 256, 16384, NULL), 2),
+    (lambda L: L.bl_absmean(16, 0, 4, 1e-5, 16, 256, 16384, NULL), 1),
     (lambda L: L.bl_ternarize(16, 4, 4, NULL, 16, NULL), 1),
     (lambda L: L.bl_ternarize_pack5(16, 4, 4, 16, 16, 8, NULL), 2),
     (lambda L: L.bl_quantize_weights_pack5(16, 4, 40, 1e-5, 16, 4, 16, 256, 1 << 20, NULL), 1),

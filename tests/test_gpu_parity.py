@@ -172,7 +172,7 @@ def _layer(bl, p, fmt, path, bias=None):
     return host(Y), Wd, beta
 
 
-PATHS = ["simt", "gemv", "auto"]
+PATHS = ["simt", "gemv", "tc", "auto"]
 
 
 def _path(bl, name):
@@ -215,6 +215,31 @@ def test_gemv_parity(bl, M, K, N):
     np.testing.assert_array_equal(host(acc), oracle.contract(Xq, oracle.ternarize(p.W, host(beta)[0])))
 
 
+@pytest.mark.parametrize("fmt", ["i8", "pack5"])
+@pytest.mark.parametrize("M,K,N", [(128, 128, 256), (256, 4096, 512), (300, 1000, 1000),
+                                   (129, 2560, 257), (512, 640, 96), (4, 384, 600)])
+def test_tc_parity(bl, fmt, M, K, N):
+    """tcgen05 GEMM: one or several 128 x 256 tiles, ragged M, N and K tails."""
+    f = bl.PACK5 if fmt == "pack5" else bl.I8
+    p = random_problem(7 * M + K + N, M, K, N)
+    b = np.random.default_rng(M).standard_normal(N).astype(F32)
+    if f == bl.I8 and K % 16:          # contiguous int8 rows of K bytes: not TMA-aligned
+        assert bl.linear_plan(M, N, K, f, bl.PATH_TC)[0] == -1
+        with pytest.raises(bl.BitLinearError) as e:
+            _layer(bl, p, f, bl.PATH_TC, bias=b)
+        assert e.value.status == "BL_ERR_UNSUPPORTED"
+        return
+    assert bl.linear_plan(M, N, K, f, bl.PATH_TC)[0] == bl.PATH_TC
+    Y, Wd, beta = _layer(bl, p, f, bl.PATH_TC, bias=b)
+    check_ok(bl)
+    assert_y_close(Y, oracle.bitlinear(p.X, p.W, p.eps, bias=b)["Y"])
+    if K % 16 == 0:
+        Xq, s = oracle.act_quant(p.X, p.eps)
+        acc = bl.linear_acc(dev(Xq), Wd, f, N, K, path=bl.PATH_TC)
+        check_ok(bl)
+        np.testing.assert_array_equal(host(acc), oracle.contract(Xq, oracle.ternarize(p.W, host(beta)[0])))
+
+
 def test_linear_bias(bl):
     p = random_problem(77, 5, 300, 45)
     b = np.random.default_rng(1).standard_normal(45).astype(F32)
@@ -223,23 +248,32 @@ def test_linear_bias(bl):
     assert_y_close(Y, oracle.bitlinear(p.X, p.W, p.eps, bias=b)["Y"])
 
 
+def acc_supported(bl, M, N, K, f, path):
+    """Whether bl_linear_acc_ex takes the pinned path with contiguous X_q [M, K]."""
+    if path == bl.PATH_TC:     # X_q rows of K bytes must be TMA-aligned
+        return K >= 128 and K % 16 == 0 and bl.linear_plan(M, N, K, f, path)[0] == path
+    return bl.linear_plan(M, N, K, f, path)[0] == path or path == bl.PATH_AUTO
+
+
+@pytest.mark.parametrize("K", [517, 528])
 @pytest.mark.parametrize("path", PATHS)
-def test_linear_acc_exact(bl, path):
+def test_linear_acc_exact(bl, path, K):
     rng = np.random.default_rng(3)
-    M, K, N = 37, 517, 71
+    M, N = 37, 71
+    p = _path(bl, path)
     Xq = rng.integers(-127, 128, (M, K)).astype(np.int8)
     Wq = rng.integers(-1, 2, (N, K)).astype(np.int8)
-    ref = oracle.contract(Xq, Wq)
-    for f, Wd in ((bl.I8, dev(Wq)), (bl.PACK5, bl.pack(dev(Wq)))):
-        if bl.linear_plan(M, N, K, f, _path(bl, path))[0] < 0:
-            continue
-        acc = bl.linear_acc(dev(Xq), Wd, f, N, K, path=_path(bl, path))
-        check_ok(bl)
-        np.testing.assert_array_equal(host(acc), ref)
-    for m in (1, 2, 4):   # the GEMV's row counts
-        sub = oracle.contract(Xq[:m], Wq)
-        acc = bl.linear_acc(dev(Xq[:m]), bl.pack(dev(Wq)), bl.PACK5, N, K, path=_path(bl, path))
-        np.testing.assert_array_equal(host(acc), sub)
+    for m in (M, 1, 2, 4):     # 1..4: the GEMV's row counts
+        ref = oracle.contract(Xq[:m], Wq)
+        for f, Wd in ((bl.I8, dev(Wq)), (bl.PACK5, bl.pack(dev(Wq)))):
+            if not acc_supported(bl, m, N, K, f, p):
+                with pytest.raises(bl.BitLinearError) as e:
+                    bl.linear_acc(dev(Xq[:m]), Wd, f, N, K, path=p)
+                assert e.value.status == "BL_ERR_UNSUPPORTED"
+                continue
+            acc = bl.linear_acc(dev(Xq[:m]), Wd, f, N, K, path=p)
+            check_ok(bl)
+            np.testing.assert_array_equal(host(acc), ref)
 
 
 def test_linear_extreme_accumulators(bl):
