@@ -59,6 +59,8 @@ def parse():
                     help="target CPU time of the oracle baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--path", type=int, default=0, help="pin the linear kernel path (BL_PATH_*)")
+    ap.add_argument("--concurrent", action="store_true",
+                    help="issue the step's independent weight chains on separate streams")
     return ap.parse_args()
 
 
@@ -197,26 +199,45 @@ class Step:
             n += X.numel() * 4 + Y.numel() * 4 + lws.numel()
         return n
 
-    def run(self, only=None, path=0):
-        """Issue the step on the current stream: every call, or only call `only`
-        (an index into labels())."""
-        bl = self.bl
+    def run(self, only=None, path=0, streams=None):
+        """Issue the step: every call, or only call `only` (an index into
+        labels()).  With `streams`, each weight tensor's chain (absmean,
+        ternarize, then the calls that use it) goes on its own stream, forked
+        from and joined back into the current stream."""
+        bl, torch = self.bl, self.torch
+        main = torch.cuda.current_stream()
+        if streams:
+            for st in streams:
+                st.wait_stream(main)
         k = -1
-        for W, beta, Wout, ws, N, K in self.tensors:
+        order = []
+        for ti, (W, beta, Wout, ws, N, K) in enumerate(self.tensors):
+            order.append(("w", ti, k + 1, k + 2))
+            k += 2
+        for ci in range(len(self.calls)):
             k += 1
-            if only is None or only == k:
-                bl.absmean(W, 1e-5, ws=ws, beta=beta)
-            k += 1
-            if only is None or only == k:
-                if self.fmt == bl.PACK5:
-                    bl.ternarize_pack5(W, beta, out=Wout)
+            order.append(("c", ci, k, None))
+        for kind, idx, k1, k2 in order:
+            ti = idx if kind == "w" else self.calls[idx][1]
+            st = streams[ti % len(streams)] if streams else main
+            with torch.cuda.stream(st):
+                if kind == "w":
+                    W, beta, Wout, ws, N, K = self.tensors[idx]
+                    if only is None or only == k1:
+                        bl.absmean(W, 1e-5, ws=ws, beta=beta)
+                    if only is None or only == k2:
+                        if self.fmt == bl.PACK5:
+                            bl.ternarize_pack5(W, beta, out=Wout)
+                        else:
+                            bl.ternarize(W, beta, out=Wout)
                 else:
-                    bl.ternarize(W, beta, out=Wout)
-        for X, ti, Y, lws, M, K, N, eps in self.calls:
-            k += 1
-            if only is None or only == k:
-                W, beta, Wout, ws, _, _ = self.tensors[ti]
-                bl.linear(X, Wout, self.fmt, N, K, beta, eps=eps, ws=lws, out=Y, path=path)
+                    X, ti2, Y, lws, M, K, N, eps = self.calls[idx]
+                    if only is None or only == k1:
+                        W, beta, Wout, ws, _, _ = self.tensors[ti2]
+                        bl.linear(X, Wout, self.fmt, N, K, beta, eps=eps, ws=lws, out=Y, path=path)
+        if streams:
+            for st in streams:
+                main.wait_stream(st)
 
     def labels(self):
         out = []
@@ -288,12 +309,14 @@ def run_ours(args):
 
     labels = first.labels()
     stream = torch.cuda.Stream(device=dev)
+    n_chains = min(len(first.tensors), 4) if args.concurrent else 0
+    side = [torch.cuda.Stream(device=dev) for _ in range(n_chains)]
     graphs = []
     with torch.cuda.stream(stream):
         for s in steps:
             g = torch.cuda.CUDAGraph()
             with torch.cuda.graph(g, stream=stream):
-                s.run(path=args.path)
+                s.run(path=args.path, streams=side or None)
             graphs.append(g)
     torch.cuda.synchronize()
 
@@ -389,7 +412,8 @@ def run_ours(args):
                    "l2_defeat": f"{R} rotating replicas, {R * first.nbytes() / 2**20:.0f} MiB >= 4x L2 "
                                 f"({l2 / 2**20:.0f} MiB)",
                    "step": "absmean + ternarize/pack per weight tensor, then quantize_act + "
-                           "contraction + dequant per call", "timing": "CUDA graph per replica, CUDA events"},
+                           "contraction + dequant per call", "timing": "CUDA graph per replica, CUDA events",
+                   "streams": (f"{n_chains} (one per independent weight chain)" if n_chains else "1")},
         "macs_per_step": macs_per_step,
         "linear_only": None if lin is None else {
             "gmacs": round(macs_per_step / (lin["ms"] * 1e-3) / 1e9, 1),

@@ -100,4 +100,60 @@ act_quant_kernel(const float* __restrict__ X, int64_t K, float eps, int8_t* __re
   for (int64_t i = K + threadIdx.x; i < ldq; i += kActThreads) qr[i] = 0;
 }
 
+// Single-pass variant for rows that fit in registers: each thread keeps its
+// VPT float4 of the row between the max and the quantization, so X is read
+// from memory exactly once.  Needs X rows 16-byte aligned (K % 4 == 0) and Xq
+// rows 4-byte aligned; K <= VPT * 4 * kActThreads.
+template <int VPT>
+__global__ void __launch_bounds__(kActThreads)
+act_quant_reg_kernel(const float* __restrict__ X, int64_t K, float eps, int8_t* __restrict__ Xq,
+                     int64_t ldq, float* __restrict__ s_out) {
+  __shared__ float s_red[kActThreads / 32];
+  __shared__ float s_scale;
+  const int64_t m = blockIdx.x;
+  const float4* xr = reinterpret_cast<const float4*>(X + m * K);
+  int8_t* qr = Xq + m * ldq;
+  const int K4 = int(K >> 2);
+  float4 v[VPT];
+  float amax = 0.f;
+  bool bad = false;
+#pragma unroll
+  for (int u = 0; u < VPT; ++u) {
+    const int i = threadIdx.x + u * kActThreads;
+    v[u] = i < K4 ? ld_stream_f4(xr + i) : make_float4(0.f, 0.f, 0.f, 0.f);
+    const float a = fmaxf(fmaxf(fabsf(v[u].x), fabsf(v[u].y)), fmaxf(fabsf(v[u].z), fabsf(v[u].w)));
+    bad |= !(a <= 3.402823466e38f) | (v[u].x != v[u].x) | (v[u].y != v[u].y) | (v[u].z != v[u].z) |
+           (v[u].w != v[u].w);
+    amax = fmaxf(amax, a);
+  }
+  amax = warp_max(amax);
+  if ((threadIdx.x & 31) == 0) s_red[threadIdx.x >> 5] = amax;
+  if (__syncthreads_or(bad) && threadIdx.x == 0) raise_status(kDevNonFinite);
+  if (threadIdx.x < 32) {
+    float w = threadIdx.x < kActThreads / 32 ? s_red[threadIdx.x] : 0.f;
+    w = warp_max(w);
+    if (threadIdx.x == 0) {
+      const float s = __fadd_rn(__fdiv_rn(w, float(kActQmax)), eps);
+      s_scale = s;
+      s_out[m] = s;
+    }
+  }
+  __syncthreads();
+  const float s = s_scale;
+  const float r = act_recip(s);
+#pragma unroll
+  for (int u = 0; u < VPT; ++u) {
+    const int i = threadIdx.x + u * kActThreads;
+    if (i < K4) {
+      char4 q;
+      q.x = act_code_fast(v[u].x, s, r);
+      q.y = act_code_fast(v[u].y, s, r);
+      q.z = act_code_fast(v[u].z, s, r);
+      q.w = act_code_fast(v[u].w, s, r);
+      reinterpret_cast<char4*>(qr)[i] = q;
+    }
+  }
+  for (int64_t i = K + threadIdx.x; i < ldq; i += kActThreads) qr[i] = 0;
+}
+
 }  // namespace bl

@@ -44,6 +44,22 @@ unsigned grid_for(int64_t work, int per_block, int max_blocks_per_sm = 8) {
   return unsigned(g < 1 ? 1 : g);
 }
 
+// Per-row activation quantization: the single-pass register kernel when the row
+// fits (and is 16-byte aligned), else the two-pass kernel.
+void launch_act_quant(const float* X, int64_t M, int64_t K, float eps, int8_t* Xq, int64_t ldq,
+                      float* s, cudaStream_t st) {
+  const bool vec = (K % 4) == 0 && (reinterpret_cast<uintptr_t>(X) % 16) == 0 &&
+                   (reinterpret_cast<uintptr_t>(Xq) % 4) == 0 && (ldq % 4) == 0;
+  const int64_t per_thread = ceil_div(K / 4, kActThreads);
+  const unsigned g = unsigned(M);
+  if (vec && per_thread <= 1) act_quant_reg_kernel<1><<<g, kActThreads, 0, st>>>(X, K, eps, Xq, ldq, s);
+  else if (vec && per_thread <= 2) act_quant_reg_kernel<2><<<g, kActThreads, 0, st>>>(X, K, eps, Xq, ldq, s);
+  else if (vec && per_thread <= 4) act_quant_reg_kernel<4><<<g, kActThreads, 0, st>>>(X, K, eps, Xq, ldq, s);
+  else if (vec && per_thread <= 8) act_quant_reg_kernel<8><<<g, kActThreads, 0, st>>>(X, K, eps, Xq, ldq, s);
+  else if (vec && per_thread <= 16) act_quant_reg_kernel<16><<<g, kActThreads, 0, st>>>(X, K, eps, Xq, ldq, s);
+  else act_quant_kernel<<<g, kActThreads, 0, st>>>(X, K, eps, Xq, ldq, s);
+}
+
 bl_status launch_status() {
   const cudaError_t e = cudaGetLastError();
   return e == cudaSuccess ? BL_OK : BL_ERR_CUDA;
@@ -189,7 +205,7 @@ bl_status run_tc(const int8_t* Xq, int64_t ldx, int64_t M, int64_t K, const int8
                  int32_t* acc, cudaStream_t st) {
   if (ldx % 16 != 0 || ldw % 16 != 0 || !is_aligned(Xq, 16) || !is_aligned(Wq, 16))
     return BL_ERR_ALIGNMENT;
-  if (ceil_div(M, kTcBM) > 65535) return BL_ERR_UNSUPPORTED;
+  if (ceil_div(M, kTcBM) * ceil_div(N, kTcBN) > (int64_t(1) << 31) - 1) return BL_ERR_UNSUPPORTED;
   TcMaps maps;
   if (!make_map_i8(&maps.a, Xq, K, M, ldx, kTcBM) || !make_map_i8(&maps.b, Wq, K, N, ldw, kTcBN))
     return BL_ERR_CUDA;
@@ -202,7 +218,10 @@ bl_status run_tc(const int8_t* Xq, int64_t ldx, int64_t M, int64_t K, const int8
   a.bias = bias;
   a.Y = Y;
   a.acc = acc;
-  const dim3 grid(unsigned(ceil_div(N, kTcBN)), unsigned(ceil_div(M, kTcBM)));
+  a.tiles_m = int(ceil_div(M, kTcBM));
+  a.tiles_n = int(ceil_div(N, kTcBN));
+  const int64_t tiles = int64_t(a.tiles_m) * a.tiles_n;
+  const dim3 grid(unsigned(tiles < num_sms() ? tiles : num_sms()));
   if (Y) {
     if (cudaFuncSetAttribute(gemm_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kTcSmem) !=
         cudaSuccess)
@@ -410,7 +429,7 @@ bl_status bl_quantize_act(const float* X, int64_t M, int64_t K, float eps, int8_
   if (M == 0) return BL_OK;
   if (!X || !Xq || !s || M > (int64_t(1) << 31) - 1) return BL_ERR_INVALID_ARG;
   if (!is_aligned(X, 4) || !is_aligned(s, 4)) return BL_ERR_ALIGNMENT;
-  act_quant_kernel<<<unsigned(M), kActThreads, 0, stream>>>(X, K, eps, Xq, K, s);
+  launch_act_quant(X, M, K, eps, Xq, K, s, stream);
   return launch_status();
 }
 
@@ -445,7 +464,7 @@ bl_status bl_linear_ex(const float* X, int64_t M, int64_t K, const void* W, bl_w
     return run_gemv(X, nullptr, 0, M, K, W, ldw, N, beta_dev, bias, eps, Y, nullptr, stream);
   int8_t* Xq = reinterpret_cast<int8_t*>(static_cast<char*>(ws) + l.xq_off);
   float* s = reinterpret_cast<float*>(static_cast<char*>(ws) + l.s_off);
-  act_quant_kernel<<<unsigned(M), kActThreads, 0, stream>>>(X, K, eps, Xq, l.ldx, s);
+  launch_act_quant(X, M, K, eps, Xq, l.ldx, s, stream);
   st = launch_status();
   if (st != BL_OK) return st;
   if (p == BL_PATH_TC) {

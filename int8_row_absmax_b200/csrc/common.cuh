@@ -46,6 +46,21 @@ __device__ __forceinline__ unsigned long long warp_sum_u64(unsigned long long v)
   return v;
 }
 
+// (row, column) of flat item i in rows of `per_row` items; 32-bit division
+// when the item count allows (64-bit integer division is a long software
+// routine on the GPU).
+__device__ __forceinline__ void split_index(int64_t i, int64_t per_row, bool small, int64_t& row,
+                                            int64_t& col) {
+  if (small) {
+    const uint32_t r = uint32_t(i) / uint32_t(per_row);
+    row = r;
+    col = int64_t(uint32_t(i) - r * uint32_t(per_row));
+  } else {
+    row = i / per_row;
+    col = i - row * per_row;
+  }
+}
+
 // Ternary digit d = t + 1 in {0,1,2} of a weight against the precomputed
 // threshold T (see weight_quant.cuh): |w| >= T means round(w / beta) != 0.
 __device__ __forceinline__ uint32_t trit_digit(float w, float T) {

@@ -15,10 +15,12 @@ pack5_kernel(const int8_t* __restrict__ Wq, int64_t N, int64_t K, uint8_t* __res
              int64_t ldp) {
   const int64_t words = ldp >> 2;
   const int64_t total = N * words;
+  const bool small = total < (int64_t(1) << 32);
   const bool vec = aligned(Wq, 4) && (K & 3) == 0;
   for (int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
        i += int64_t(gridDim.x) * blockDim.x) {
-    const int64_t row = i / words, g = i - row * words;
+    int64_t row, g;
+    split_index(i, words, small, row, g);
     const int64_t k0 = g * 20;
     const int8_t* wr = Wq + row * K;
     uint32_t d[20];
@@ -44,15 +46,17 @@ pack5_kernel(const int8_t* __restrict__ Wq, int64_t N, int64_t K, uint8_t* __res
 }
 
 // Wp [N,ldp] -> Wq [N,ldq] int8, the first K trits of each row.  One thread per
-// packed byte; rows beyond K are not written.
+// packed byte.
 __global__ void __launch_bounds__(256)
 unpack5_kernel(const uint8_t* __restrict__ Wp, int64_t N, int64_t K, int64_t ldp,
                int8_t* __restrict__ Wq, int64_t ldq) {
   const int64_t nb = ceil_div(K, 5);
   const int64_t total = N * nb;
+  const bool small = total < (int64_t(1) << 32);
   for (int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
        i += int64_t(gridDim.x) * blockDim.x) {
-    const int64_t row = i / nb, j = i - row * nb;
+    int64_t row, j;
+    split_index(i, nb, small, row, j);
     const uint32_t b = Wp[row * ldp + j];
     int8_t* out = Wq + row * ldq + 5 * j;
     int t5[5];

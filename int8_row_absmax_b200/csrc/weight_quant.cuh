@@ -131,10 +131,10 @@ constexpr int kBigWords = 16;  // 512 bits; the sum is below 2^330 units of 2^-1
 // global reads (bins, every CTA's limb slot, the magic word) are issued at once.
 __device__ void absmean_finalize(AbsAccum* acc, int64_t n, float eps, float* beta_out, int nctas,
                                  unsigned long long* s_binv, unsigned long long* s_limbsum,
-                                 unsigned long long* s_word, uint32_t* s_big, int* s_flag) {
+                                 unsigned long long* s_wsum, unsigned long long* s_word,
+                                 uint32_t* s_big, int* s_flag) {
   const int t = threadIdx.x;
   for (int i = t; i < kBigWords + 3; i += blockDim.x) s_word[i] = 0ull;
-  if (t < 3) s_limbsum[t] = 0ull;
   if (t == 0) *s_flag = 0;
   __syncthreads();
   if (t < 255) {
@@ -142,12 +142,31 @@ __device__ void absmean_finalize(AbsAccum* acc, int64_t n, float eps, float* bet
     s_binv[t] = v;
     if (v) *s_flag = 1;                         // some magnitude outside the fast window
   }
-  for (int c = t; c < nctas; c += blockDim.x) {
-    atomicAdd(&s_limbsum[0], __ldcg(&acc->slot[c][0]));
-    atomicAdd(&s_limbsum[1], __ldcg(&acc->slot[c][1]));
-    atomicAdd(&s_limbsum[2], __ldcg(&acc->slot[c][2]));
+  // sum every CTA's limb slot: warp shuffles, then one value per warp (no
+  // contended shared-memory atomics)
+  {
+    unsigned long long l0 = 0ull, l1 = 0ull, l2 = 0ull;
+    for (int c = t; c < nctas; c += blockDim.x) {
+      l0 += __ldcg(&acc->slot[c][0]);
+      l1 += __ldcg(&acc->slot[c][1]);
+      l2 += __ldcg(&acc->slot[c][2]);
+    }
+    l0 = warp_sum_u64(l0);
+    l1 = warp_sum_u64(l1);
+    l2 = warp_sum_u64(l2);
+    if ((t & 31) == 0) {
+      s_wsum[3 * (t >> 5) + 0] = l0;
+      s_wsum[3 * (t >> 5) + 1] = l1;
+      s_wsum[3 * (t >> 5) + 2] = l2;
+    }
   }
   const unsigned int magic = t == 0 ? __ldcg(&acc->magic) : 0u;
+  __syncthreads();
+  if (t < 3) {
+    unsigned long long v = 0ull;
+    for (int w = 0; w < int(blockDim.x >> 5); ++w) v += s_wsum[3 * w + t];
+    s_limbsum[t] = v;
+  }
   __syncthreads();
   const bool fast = *s_flag == 0;
   if (!fast) {
@@ -232,11 +251,11 @@ absmean_kernel(const float* __restrict__ W, int64_t n, float eps, AbsAccum* __re
   __shared__ int s_flag;
   __shared__ int s_timeout;
   __shared__ unsigned long long s_binv[255];
+  __shared__ unsigned long long s_wsum[3 * (kAbsThreads / 32)];
   __shared__ bool s_last;
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
   for (int i = tid; i < 256; i += blockDim.x) s_bins[i] = 0ull;
-  if (tid < 3) s_limb[tid] = 0ull;
 
   unsigned long long lo = 0ull;
   uint32_t hi = 0u;
@@ -344,15 +363,19 @@ absmean_kernel(const float* __restrict__ W, int64_t n, float eps, AbsAccum* __re
   const unsigned long long l0 = warp_sum_u64(lo & 0xFFFFFFFFull);
   const unsigned long long l1 = warp_sum_u64(lo >> 32);
   const unsigned long long l2 = warp_sum_u64((unsigned long long)hi);
-  if ((tid & 31) == 0) {
-    atomicAdd(&s_limb[0], l0);
-    atomicAdd(&s_limb[1], l1);
-    atomicAdd(&s_limb[2], l2);
+  if ((tid & 31) == 0) {                  // one slot per warp: no contended atomics
+    s_wsum[3 * warp + 0] = l0;
+    s_wsum[3 * warp + 1] = l1;
+    s_wsum[3 * warp + 2] = l2;
   }
   if (__syncthreads_or(bad) && tid == 0) raise_status(kDevNonFinite);
   for (int i = tid; i < 256; i += blockDim.x)
     if (s_bins[i]) atomicAdd(&acc->bins[i], s_bins[i]);   // rare: weights outside the window
-  if (tid < 3) acc->slot[blockIdx.x][tid] = s_limb[tid];   // plain stores, own slot
+  if (tid < 3) {                          // plain stores into this CTA's own slot
+    unsigned long long v = 0ull;
+    for (int w = 0; w < kAbsThreads / 32; ++w) v += s_wsum[3 * w + tid];
+    acc->slot[blockIdx.x][tid] = v;
+  }
 
   // Last-CTA-done: the CTA whose ticket completes the grid finalizes.
   __threadfence();
@@ -365,7 +388,8 @@ absmean_kernel(const float* __restrict__ W, int64_t n, float eps, AbsAccum* __re
   __syncthreads();
   if (!s_last) return;
   __threadfence();
-  absmean_finalize(acc, n, eps, beta_out, int(gridDim.x), s_binv, s_limb, s_word, s_big, &s_flag);
+  absmean_finalize(acc, n, eps, beta_out, int(gridDim.x), s_binv, s_limb, s_wsum, s_word, s_big,
+                   &s_flag);
 }
 
 // W [N,K] float32 -> Wq [N,K] int8 codes.
@@ -400,10 +424,12 @@ ternarize_pack5_kernel(const float* __restrict__ W, int64_t N, int64_t K,
   const float T = ternary_threshold(*beta);
   const int64_t words = ldp >> 2;
   const int64_t total = N * words;
+  const bool small = total < (int64_t(1) << 32);
   const bool vec = aligned(W, 16) && (K & 3) == 0;
   for (int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
        i += int64_t(gridDim.x) * blockDim.x) {
-    const int64_t row = i / words, g = i - row * words;
+    int64_t row, g;
+    split_index(i, words, small, row, g);
     const int64_t k0 = g * 20;
     const float* wr = W + row * K;
     uint32_t d[20];
