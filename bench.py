@@ -4,9 +4,10 @@
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload 2] [--impl ours|reference]
 
 A step is one pass of the whole BitLinear hot path over one batch of the
-workload: for every weight tensor, absmean beta (a1) and ternarize + pack
-(a2, a3); for every call, per-row int8 quantization of X, the ternary x int8
-contraction and the fused dequant (a4-a6).  The default workload is batch-1
+workload: for every weight tensor, absmean beta, ternarize and pack (a1-a3,
+one library call: a single streaming pass over W in one launch); for every
+call, per-row int8 quantization of X, the ternary x int8 contraction and the
+fused dequant (a4-a6).  The default workload is batch-1
 decode: (K,N) = (2560,6912) and (6912,2560) with packed trits, M = 1.
 
 Timing: inputs are resident in HBM; R replicas of every buffer rotate so each
@@ -171,7 +172,7 @@ class Step:
 
     def __init__(self, bl, torch, probs, dev, fmt):
         self.bl, self.torch, self.fmt = bl, torch, fmt
-        self.tensors = []          # weight tensors: (W, beta, Wout, absmean ws)
+        self.tensors = []          # weight tensors: (W, beta, Wout, quantizer ws, N, K)
         self.calls = []            # linear calls: (X, tensor index, Y, lin ws, M, K, N)
         seen = {}
         for p in probs:
@@ -201,8 +202,8 @@ class Step:
 
     def run(self, only=None, path=0, streams=None):
         """Issue the step: every call, or only call `only` (an index into
-        labels()).  With `streams`, each weight tensor's chain (absmean,
-        ternarize, then the calls that use it) goes on its own stream, forked
+        labels()).  With `streams`, each weight tensor's chain (its
+        quantization, then the calls that use it) goes on its own stream, forked
         from and joined back into the current stream."""
         bl, torch = self.bl, self.torch
         main = torch.cuda.current_stream()
@@ -212,8 +213,8 @@ class Step:
         k = -1
         order = []
         for ti, (W, beta, Wout, ws, N, K) in enumerate(self.tensors):
-            order.append(("w", ti, k + 1, k + 2))
-            k += 2
+            order.append(("w", ti, k + 1, None))
+            k += 1
         for ci in range(len(self.calls)):
             k += 1
             order.append(("c", ci, k, None))
@@ -224,12 +225,10 @@ class Step:
                 if kind == "w":
                     W, beta, Wout, ws, N, K = self.tensors[idx]
                     if only is None or only == k1:
-                        bl.absmean(W, 1e-5, ws=ws, beta=beta)
-                    if only is None or only == k2:
                         if self.fmt == bl.PACK5:
-                            bl.ternarize_pack5(W, beta, out=Wout)
+                            bl.quantize_weights_pack5(W, 1e-5, ws=ws, out=Wout, beta=beta)
                         else:
-                            bl.ternarize(W, beta, out=Wout)
+                            bl.quantize_weights(W, 1e-5, ws=ws, out=Wout, beta=beta)
                 else:
                     X, ti2, Y, lws, M, K, N, eps = self.calls[idx]
                     if only is None or only == k1:
@@ -242,7 +241,7 @@ class Step:
     def labels(self):
         out = []
         for i, (W, beta, Wout, ws, N, K) in enumerate(self.tensors):
-            out += [("absmean", i), ("ternarize_pack5" if self.fmt == self.bl.PACK5 else "ternarize", i)]
+            out.append(("wquant", i))
         for j, c in enumerate(self.calls):
             out.append(("linear", j))
         return out
@@ -251,9 +250,7 @@ class Step:
 def algorithmic_bytes(kind, N, K, M, fmt):
     """Bytes each kind of call must move at minimum (inputs read + outputs written)."""
     wbytes = N * math.ceil(K / 5) if fmt == 1 else N * K
-    if kind == "absmean":
-        return 4 * N * K
-    if kind.startswith("ternarize"):
+    if kind == "wquant":          # read W once, write the codes
         return 4 * N * K + wbytes
     if kind == "linear":
         return wbytes + 4 * M * K + 4 * M * N
@@ -367,36 +364,39 @@ def run_ours(args):
             del g
     shapes = {}
     for i, (W, beta, Wout, ws, N, Kd) in enumerate(first.tensors):
-        shapes[("absmean", i)] = (N, Kd, 0)
-        shapes[(labels[2 * i + 1][0], i)] = (N, Kd, 0)
+        # the single-pass quantizer (1 cooperative launch) whenever the library
+        # sized the workspace for it, else absmean + ternarize (2)
+        shapes[("wquant", i)] = (N, Kd, 0, 1 if ws.numel() > 16384 else 2)
     for j, (X, ti, Y, lws, M, Kd, N, eps) in enumerate(first.calls):
-        shapes[("linear", j)] = (N, Kd, M)
+        shapes[("linear", j)] = (N, Kd, M, bl.linear_plan(M, N, Kd, fmt, args.path)[1])
     kinds = {}
     for lab, v in per_call.items():
         kind = lab[0]
-        N, Kd, M = shapes[lab]
+        N, Kd, M, nl = shapes[lab]
         d = kinds.setdefault(kind, {"ms": 0.0, "bytes": 0, "launches": 0})
         d["ms"] += float(np.mean(v))
         d["bytes"] += algorithmic_bytes(kind, N, Kd, M, fmt)
-        d["launches"] += 1 if kind != "linear" else bl.linear_plan(M, N, Kd, fmt, args.path)[1]
+        d["launches"] += nl
     peaks = measured_peaks()
-    kern_names = {"absmean": "absmean_kernel", "ternarize_pack5": "ternarize_pack5_kernel",
-                  "ternarize": "ternarize_i8_kernel", "linear": "linear"}
+    kern_names = {"wquant": "wquant_kernel", "linear": "linear"}
     kernels = {}
     for kind, d in kinds.items():
         gbs = d["bytes"] / (d["ms"] * 1e-3) / 1e9
         kernels[kind] = {"ms_per_step": round(d["ms"], 5), "algorithmic_bytes": d["bytes"],
                          "launches": d["launches"], "achieved_gbs": round(gbs, 1),
                          "frac_hbm": round(gbs / peaks["hbm_gbs"], 4)}
-    # the dominant single-kernel call (linear may be two launches: act quant + contraction)
-    single = [k for k in kinds if k != "linear" or kinds[k]["launches"] == len(first.calls)]
-    dom = max(single, key=lambda k: kinds[k]["ms"])
+    # the dominant call of the step (the weight call is one launch for tensors
+    # of 2^20 weights and more; the linear call is activation quantization plus
+    # the contraction, or one fused launch for the GEMV)
+    dom = max(kinds, key=lambda k: kinds[k]["ms"])
     dkind = kinds[dom]
     achieved = dkind["bytes"] / (dkind["ms"] * 1e-3) / 1e9
     roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"],
                 "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
                 "traffic": ncu_traffic(kern_names[dom], args.workload),
-                "kernel": kern_names[dom], "peak_source": peaks["source"] + " (MEASURED_PEAKS.json hbm_gbs)"
+                "kernel": kern_names[dom], "call_launches": dkind["launches"] // max(
+                    1, len(first.tensors) if dom == "wquant" else len(first.calls)),
+                "peak_source": peaks["source"] + " (MEASURED_PEAKS.json hbm_gbs)"
                 if peaks["source"] == "measured" else "fallback 6.65 TB/s"}
 
     launches_per_step = sum(d["launches"] for d in kinds.values())
@@ -411,8 +411,8 @@ def run_ours(args):
                    "weight_format": wl.fmt, "parallelism": f"dp{world} (independent batches)",
                    "l2_defeat": f"{R} rotating replicas, {R * first.nbytes() / 2**20:.0f} MiB >= 4x L2 "
                                 f"({l2 / 2**20:.0f} MiB)",
-                   "step": "absmean + ternarize/pack per weight tensor, then quantize_act + "
-                           "contraction + dequant per call", "timing": "CUDA graph per replica, CUDA events",
+                   "step": "absmean + ternarize + pack per weight tensor (one call), then "
+                           "quantize_act + contraction + dequant per call", "timing": "CUDA graph per replica, CUDA events",
                    "streams": (f"{n_chains} (one per independent weight chain)" if n_chains else "1")},
         "macs_per_step": macs_per_step,
         "linear_only": None if lin is None else {
@@ -456,7 +456,7 @@ def e2e(bl, torch, probs, dev, fmt, steps, world):
     dW = [torch.empty_like(h, device=dev) for h in host_W]
     dX = [torch.empty_like(h, device=dev) for h in host_X]
     hY = [torch.empty((p.M, p.N), dtype=torch.float32).pin_memory() for p in probs]
-    ws = [bl.workspace(bl.load().bl_quantize_weights_workspace_size(1, 1), dev) for _ in host_W]
+    ws = [bl.workspace(bl.load().bl_quantize_weights_workspace_size(*h.shape), dev) for h in host_W]
     h2d = sum(h.numel() * 4 for h in host_W) + sum(h.numel() * 4 for h in host_X)
     d2h = sum(h.numel() * 4 for h in hY)
 

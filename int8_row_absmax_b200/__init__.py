@@ -118,13 +118,13 @@ def workspace(nbytes: int, device):
     return torch.zeros(max(int(nbytes), 256), dtype=torch.uint8, device=device)
 
 
-def quantize_weights(W, eps: float = 1e-5, ws=None):
+def quantize_weights(W, eps: float = 1e-5, ws=None, out=None, beta=None):
     """W [N,K] float32 -> (Wq int8 [N,K], beta float32 [1] on the device)."""
     torch, lib = _torch(), load()
     _dev(W, torch.float32)
     N, K = W.shape
-    Wq = torch.empty((N, K), dtype=torch.int8, device=W.device)
-    beta = torch.empty(1, dtype=torch.float32, device=W.device)
+    Wq = torch.empty((N, K), dtype=torch.int8, device=W.device) if out is None else out
+    beta = torch.empty(1, dtype=torch.float32, device=W.device) if beta is None else beta
     need = lib.bl_quantize_weights_workspace_size(N, K)
     ws = workspace(need, W.device) if ws is None else ws
     _check("bl_quantize_weights", lib.bl_quantize_weights(

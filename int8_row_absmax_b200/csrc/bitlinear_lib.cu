@@ -14,6 +14,7 @@
 #include "bitlinear.h"
 #include "common.cuh"
 #include "weight_quant.cuh"
+#include "weight_fused.cuh"
 #include "pack.cuh"
 #include "act_quant.cuh"
 #include "linear_simt.cuh"
@@ -85,6 +86,44 @@ bl_status launch_absmean(const float* W, int64_t n, float eps, float* beta_dev, 
   if (grid > kAbsMaxCtas) grid = kAbsMaxCtas;
   absmean_kernel<<<grid, kAbsThreads, kAbsSmem, st>>>(W, n, eps, acc, beta_dev);
   return launch_status();
+}
+
+// Whether the single-pass quantizer applies: large enough to pay for its extra
+// launches, 16-byte rows for the bulk copies, column index within 17 bits.
+bool fused_shape(int64_t N, int64_t K) { return N * K >= kFusedMinN && K % 4 == 0 && K <= 131072; }
+
+// a1-a3 in one read of W: one cooperative launch (all CTAs resident, for the
+// kernel's two grid barriers).  Returns BL_ERR_UNSUPPORTED, with nothing
+// launched, when the device cannot hold the grid at once.
+bl_status launch_wquant_fused(const float* W, int64_t N, int64_t K, float eps, void* out,
+                              int64_t ldo, bool packed, float* beta_dev, void* ws,
+                              cudaStream_t st) {
+  auto* acc = static_cast<AbsAccum*>(ws);
+  auto* list = reinterpret_cast<unsigned long long*>(static_cast<char*>(ws) + kFuListOff);
+  const int64_t ngroups = N * ceil_div(K, 20);
+  const int64_t nch = ceil_div(ngroups, kFuGroups);
+  const void* fn = packed ? reinterpret_cast<const void*>(wquant_kernel<true>)
+                          : reinterpret_cast<const void*>(wquant_kernel<false>);
+  if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, kFuSmem) != cudaSuccess)
+    return BL_ERR_CUDA;
+  int per_sm = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, kAbsThreads, kFuSmem) != cudaSuccess)
+    return BL_ERR_CUDA;
+  int grid = num_sms() * per_sm;
+  if (grid > kAbsMaxCtas) grid = kAbsMaxCtas;
+  if (int64_t(grid) > nch) grid = int(nch);
+  if (grid < 1) return BL_ERR_UNSUPPORTED;
+  int cap = int(fused_cap_w(ngroups, grid));
+  uint32_t stride = chunk_stride(nch, grid);
+  const int64_t gpr = ceil_div(K, 20);
+  uint32_t gpr_magic = gpr > 1 ? uint32_t(((uint64_t(1) << 32) + uint64_t(gpr) - 1) / uint64_t(gpr)) : 0u;
+  void* args[] = {&W, &N, &K, &eps, &out, &ldo, &acc, &list, &cap, &stride, &gpr_magic, &beta_dev};
+  const cudaError_t e = cudaLaunchCooperativeKernel(fn, grid, kAbsThreads, args, kFuSmem, st);
+  if (e == cudaErrorCooperativeLaunchTooLarge) {
+    (void)cudaGetLastError();
+    return BL_ERR_UNSUPPORTED;
+  }
+  return e == cudaSuccess ? BL_OK : BL_ERR_CUDA;
 }
 
 bl_status check_ws(const void* ws, size_t ws_bytes, size_t need) {
@@ -353,7 +392,7 @@ int64_t bl_pack5_ldp(int64_t K) { return K < 1 ? 0 : round_up(ceil_div(K, 5), 16
 
 size_t bl_quantize_weights_workspace_size(int64_t N, int64_t K) {
   if (N < 1 || K < 1) return 0;
-  return kAbsWsBytes;
+  return fused_shape(N, K) ? fused_ws_bytes(N, K) : kAbsWsBytes;
 }
 
 bl_status bl_absmean(const float* W, int64_t N, int64_t K, float eps, float* beta_dev, void* ws,
@@ -391,6 +430,14 @@ bl_status bl_quantize_weights(const float* W, int64_t N, int64_t K, float eps, i
                               float* beta_dev, void* ws, size_t ws_bytes, cudaStream_t stream) {
   bl_status st = check_weights_args(W, N, K, Wq);
   if (st != BL_OK) return st;
+  if (!eps_ok(eps)) return BL_ERR_INVALID_ARG;
+  if (!beta_dev) return BL_ERR_INVALID_ARG;
+  if (!is_aligned(beta_dev, 4)) return BL_ERR_ALIGNMENT;
+  if ((st = check_ws(ws, ws_bytes, kAbsWsBytes)) != BL_OK) return st;
+  if (fused_shape(N, K) && is_aligned(W, 16) && is_aligned(Wq, 4) && ws_bytes >= fused_ws_bytes(N, K)) {
+    st = launch_wquant_fused(W, N, K, eps, Wq, K, false, beta_dev, ws, stream);
+    if (st != BL_ERR_UNSUPPORTED) return st;
+  }
   st = bl_absmean(W, N, K, eps, beta_dev, ws, ws_bytes, stream);
   if (st != BL_OK) return st;
   return bl_ternarize(W, N, K, beta_dev, Wq, stream);
@@ -403,6 +450,14 @@ bl_status bl_quantize_weights_pack5(const float* W, int64_t N, int64_t K, float 
   if (st != BL_OK) return st;
   if (ldp < ceil_div(K, 5)) return BL_ERR_INVALID_ARG;
   if (ldp % 16 != 0 || !is_aligned(Wp, 16)) return BL_ERR_ALIGNMENT;
+  if (!eps_ok(eps)) return BL_ERR_INVALID_ARG;
+  if (!beta_dev) return BL_ERR_INVALID_ARG;
+  if (!is_aligned(beta_dev, 4)) return BL_ERR_ALIGNMENT;
+  if ((st = check_ws(ws, ws_bytes, kAbsWsBytes)) != BL_OK) return st;
+  if (fused_shape(N, K) && is_aligned(W, 16) && ws_bytes >= fused_ws_bytes(N, K)) {
+    st = launch_wquant_fused(W, N, K, eps, Wp, ldp, true, beta_dev, ws, stream);
+    if (st != BL_ERR_UNSUPPORTED) return st;
+  }
   st = bl_absmean(W, N, K, eps, beta_dev, ws, ws_bytes, stream);
   if (st != BL_OK) return st;
   return bl_ternarize_pack5(W, N, K, beta_dev, Wp, ldp, stream);

@@ -66,6 +66,20 @@ struct AbsAccum {
   unsigned int next_chunk;      // next 32 KB chunk of W to hand out
   unsigned int pad_;
   unsigned long long slot[kAbsMaxCtas][4];  // per-CTA sums of the three 32-bit limbs
+  // single-pass quantization (weight_fused.cuh): the fix-up mode chosen by the
+  // last CTA, the fall-back flags, the two grid barriers and the exit count (all
+  // zero between calls), and each CTA's sums of sampled run means
+  unsigned int mode;
+  unsigned int overflow;
+  unsigned int bar_a;
+  unsigned int flag_b;
+  unsigned int exit_cnt;
+  unsigned int bins_used;
+  unsigned long long tot[3];        // exact pass: the three 32-bit limb sums over all CTAs
+  double dsum;                      // float64 sum of |w| over all CTAs
+  unsigned int ticket2;             // exact pass: CTAs done
+  unsigned int flag_c;              // exact pass: beta published
+  double est_part[kAbsMaxCtas][2];  // per CTA: sampled chunk mean (-1: none) and its square
 };
 constexpr size_t kAbsWsBytes = 16384;
 static_assert(sizeof(AbsAccum) <= kAbsWsBytes, "accumulator block");
@@ -94,11 +108,13 @@ __device__ __forceinline__ unsigned long long absmean_fast(float w, unsigned lon
   return mad_wide_u32((u & 0x7FFFFFu) | 0x800000u, shl_clamp(1u, sh), acc);
 }
 
-// Slow path for one weight outside the fast window (zero adds nothing).
-__device__ __forceinline__ void absmean_slow(float w, unsigned long long* s_bins, bool& bad) {
+// Slow path for one weight outside the fast window [lo_e, lo_e + 31] (zero adds
+// nothing).
+__device__ __forceinline__ void absmean_slow(float w, unsigned long long* s_bins, bool& bad,
+                                             uint32_t lo_e = kFastLo) {
   const uint32_t u = __float_as_uint(w) & 0x7FFFFFFFu;
   const uint32_t e = u >> 23;
-  if (e - kFastLo <= kFastHi - kFastLo) return;  // counted by the fast path
+  if (e - lo_e <= kFastHi - kFastLo) return;  // counted by the fast path
   if (e == 255u) {
     bad = true;
     return;
@@ -129,10 +145,12 @@ constexpr int kBigWords = 16;  // 512 bits; the sum is below 2^330 units of 2^-1
 
 // Step 3, run by the last CTA: the exact sum rounded once to float64.  All the
 // global reads (bins, every CTA's limb slot, the magic word) are issued at once.
-__device__ void absmean_finalize(AbsAccum* acc, int64_t n, float eps, float* beta_out, int nctas,
+// The limbs are in units of 2^(lo_e - 150).  Returns beta in thread 0 (other
+// threads: 0).
+__device__ float absmean_finalize(AbsAccum* acc, int64_t n, float eps, float* beta_out, int nctas,
                                  unsigned long long* s_binv, unsigned long long* s_limbsum,
                                  unsigned long long* s_wsum, unsigned long long* s_word,
-                                 uint32_t* s_big, int* s_flag) {
+                                 uint32_t* s_big, int* s_flag, uint32_t lo_e = kFastLo) {
   const int t = threadIdx.x;
   for (int i = t; i < kBigWords + 3; i += blockDim.x) s_word[i] = 0ull;
   if (t == 0) *s_flag = 0;
@@ -173,8 +191,8 @@ __device__ void absmean_finalize(AbsAccum* acc, int64_t n, float eps, float* bet
     for (int j = t; j < 258; j += blockDim.x) {
       const unsigned long long w = j < 255 ? s_binv[j] : s_limbsum[j - 255];
       // bins: m * 2^(max(e,1)-150) = m * 2^(max(e,1)-1) units of 2^-149;
-      // limb i weighs 2^(32 i) * 2^(kFastLo-150) = 2^(32 i + kFastLo - 1) units
-      const int shift = j < 255 ? (j > 0 ? j : 1) - 1 : 32 * (j - 255) + int(kFastLo) - 1;
+      // limb i weighs 2^(32 i) * 2^(lo_e-150) = 2^(32 i + lo_e - 1) units
+      const int shift = j < 255 ? (j > 0 ? j : 1) - 1 : 32 * (j - 255) + int(lo_e) - 1;
       if (w) {
         const int wi = shift >> 5, b = shift & 31;
         const unsigned long long lo64 = w << b, hi64 = b ? (w >> (64 - b)) : 0ull;
@@ -185,20 +203,21 @@ __device__ void absmean_finalize(AbsAccum* acc, int64_t n, float eps, float* bet
     }
   }
   __syncthreads();
+  float beta = 0.f;
   if (t == 0) {
     double D = 0.0;
     if (fast) {
-      // total = L0 + L1 2^32 + L2 2^64 units of 2^-40 (each L < 2^50)
+      // total = L0 + L1 2^32 + L2 2^64 units of 2^(lo_e-150) (each L < 2^50)
       const unsigned long long L0 = s_limbsum[0], L1 = s_limbsum[1], L2 = s_limbsum[2];
       unsigned long long lo = L0 + (L1 << 32);
       const unsigned long long hi = (L1 >> 32) + L2 + (lo < L0 ? 1ull : 0ull);
       if (hi == 0ull) {
-        D = ldexp(__ull2double_rn(lo), -int(150 - kFastLo));
+        D = ldexp(__ull2double_rn(lo), int(lo_e) - 150);
       } else {
         const int sh = 64 - __clzll(hi);            // drop sh low bits, keep a sticky bit
         unsigned long long top = (hi << (64 - sh)) | (lo >> sh);
         top |= (lo << (64 - sh)) != 0ull ? 1ull : 0ull;
-        D = ldexp(__ull2double_rn(top), sh - int(150 - kFastLo));
+        D = ldexp(__ull2double_rn(top), sh + int(lo_e) - 150);
       }
     } else {
       unsigned long long carry = 0ull;
@@ -228,13 +247,15 @@ __device__ void absmean_finalize(AbsAccum* acc, int64_t n, float eps, float* bet
       }
     }
     const double d = __ddiv_rn(D, double(n));
-    *beta_out = __fadd_rn(__double2float_rn(d), eps);
+    beta = __fadd_rn(__double2float_rn(d), eps);
+    *beta_out = beta;
     if (magic != 0u) raise_status(kDevBadWorkspace);
     acc->ticket = 0u;                            // leave the block clear for the next call
     acc->next_chunk = 0u;
   }
   for (int j = t; j < 255; j += blockDim.x)
     if (s_binv[j]) acc->bins[j] = 0ull;
+  return beta;
 }
 
 __global__ void __launch_bounds__(kAbsThreads, 1)
@@ -392,13 +413,9 @@ absmean_kernel(const float* __restrict__ W, int64_t n, float eps, AbsAccum* __re
                    &s_flag);
 }
 
-// W [N,K] float32 -> Wq [N,K] int8 codes.
-__global__ void __launch_bounds__(256)
-ternarize_i8_kernel(const float* __restrict__ W, int64_t n, const float* __restrict__ beta,
-                    int8_t* __restrict__ Wq) {
-  const float T = ternary_threshold(*beta);
-  const int64_t tid = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
-  const int64_t nthr = int64_t(gridDim.x) * blockDim.x;
+// W [N,K] float32 -> Wq [N,K] int8 codes, grid-stride from thread `tid`.
+__device__ __forceinline__ void ternarize_i8_range(const float* __restrict__ W, int64_t n, float T,
+                                                   int8_t* __restrict__ Wq, int64_t tid, int64_t nthr) {
   if (aligned(W, 16) && aligned(Wq, 4)) {
     const int64_t n4 = n >> 2;
     for (int64_t i = tid; i < n4; i += nthr) {
@@ -416,42 +433,61 @@ ternarize_i8_kernel(const float* __restrict__ W, int64_t n, const float* __restr
   }
 }
 
-// W [N,K] float32 -> Wp [N,ldp] packed bytes.  One thread per 4 output bytes
-// (20 weights): a 32-bit store, and five 128-bit loads when the group is whole.
 __global__ void __launch_bounds__(256)
-ternarize_pack5_kernel(const float* __restrict__ W, int64_t N, int64_t K,
-                       const float* __restrict__ beta, uint8_t* __restrict__ Wp, int64_t ldp) {
-  const float T = ternary_threshold(*beta);
+ternarize_i8_kernel(const float* __restrict__ W, int64_t n, const float* __restrict__ beta,
+                    int8_t* __restrict__ Wq) {
+  ternarize_i8_range(W, n, ternary_threshold(*beta), Wq, int64_t(blockIdx.x) * blockDim.x + threadIdx.x,
+                     int64_t(gridDim.x) * blockDim.x);
+}
+
+// The packed word g of row `row` (weights 20g .. 20g+19; digit 1 past K).
+__device__ __forceinline__ uint32_t ternarize_pack5_word(const float* __restrict__ W, int64_t K,
+                                                         float T, bool vec, int64_t row, int64_t g) {
+  const int64_t k0 = g * 20;
+  const float* wr = W + row * K;
+  uint32_t d[20];
+  if (vec && k0 + 20 <= K) {
+#pragma unroll
+    for (int v = 0; v < 5; ++v) {
+      const float4 f = ld_stream_f4(reinterpret_cast<const float4*>(wr + k0) + v);
+      d[4 * v + 0] = trit_digit(f.x, T);
+      d[4 * v + 1] = trit_digit(f.y, T);
+      d[4 * v + 2] = trit_digit(f.z, T);
+      d[4 * v + 3] = trit_digit(f.w, T);
+    }
+  } else {
+#pragma unroll
+    for (int k = 0; k < 20; ++k) d[k] = (k0 + k < K) ? trit_digit(wr[k0 + k], T) : 1u;
+  }
+  uint32_t word = 0u;
+#pragma unroll
+  for (int b = 0; b < 4; ++b)
+    word |= pack5_digits(d[5 * b], d[5 * b + 1], d[5 * b + 2], d[5 * b + 3], d[5 * b + 4]) << (8 * b);
+  return word;
+}
+
+// W [N,K] float32 -> Wp [N,ldp] packed bytes, grid-stride from thread `first`
+// with stride `nthr`.  One thread per 4 output bytes (20 weights): a 32-bit
+// store, and five 128-bit loads when the group is whole.
+__device__ __forceinline__ void ternarize_pack5_range(const float* __restrict__ W, int64_t N,
+                                                      int64_t K, float T, uint8_t* __restrict__ Wp,
+                                                      int64_t ldp, int64_t first, int64_t nthr) {
   const int64_t words = ldp >> 2;
   const int64_t total = N * words;
   const bool small = total < (int64_t(1) << 32);
   const bool vec = aligned(W, 16) && (K & 3) == 0;
-  for (int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
-       i += int64_t(gridDim.x) * blockDim.x) {
+  for (int64_t i = first; i < total; i += nthr) {
     int64_t row, g;
     split_index(i, words, small, row, g);
-    const int64_t k0 = g * 20;
-    const float* wr = W + row * K;
-    uint32_t d[20];
-    if (vec && k0 + 20 <= K) {
-#pragma unroll
-      for (int v = 0; v < 5; ++v) {
-        const float4 f = ld_stream_f4(reinterpret_cast<const float4*>(wr + k0) + v);
-        d[4 * v + 0] = trit_digit(f.x, T);
-        d[4 * v + 1] = trit_digit(f.y, T);
-        d[4 * v + 2] = trit_digit(f.z, T);
-        d[4 * v + 3] = trit_digit(f.w, T);
-      }
-    } else {
-#pragma unroll
-      for (int k = 0; k < 20; ++k) d[k] = (k0 + k < K) ? trit_digit(wr[k0 + k], T) : 1u;
-    }
-    uint32_t word = 0u;
-#pragma unroll
-    for (int b = 0; b < 4; ++b)
-      word |= pack5_digits(d[5 * b], d[5 * b + 1], d[5 * b + 2], d[5 * b + 3], d[5 * b + 4]) << (8 * b);
-    *reinterpret_cast<uint32_t*>(Wp + row * ldp + 4 * g) = word;
+    *reinterpret_cast<uint32_t*>(Wp + row * ldp + 4 * g) = ternarize_pack5_word(W, K, T, vec, row, g);
   }
+}
+
+__global__ void __launch_bounds__(256)
+ternarize_pack5_kernel(const float* __restrict__ W, int64_t N, int64_t K,
+                       const float* __restrict__ beta, uint8_t* __restrict__ Wp, int64_t ldp) {
+  ternarize_pack5_range(W, N, K, ternary_threshold(*beta), Wp, ldp,
+                        int64_t(blockIdx.x) * blockDim.x + threadIdx.x, int64_t(gridDim.x) * blockDim.x);
 }
 
 }  // namespace bl

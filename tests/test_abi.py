@@ -54,7 +54,16 @@ def test_status_strings(lib):
 def test_workspace_sizes(lib):
     assert lib.bl_quantize_weights_workspace_size(0, 5) == 0
     assert lib.bl_quantize_weights_workspace_size(4, 4) == 16384
-    assert lib.bl_quantize_weights_workspace_size(8192, 8192) == 16384
+    # below 2^20 weights, or rows that are not whole 16-byte units: the two-pass
+    # kernels and their 16 KB accumulator block
+    assert lib.bl_quantize_weights_workspace_size(1023, 1024) == 16384
+    assert lib.bl_quantize_weights_workspace_size(8192, 8190) == 16384
+    # the single-pass quantizer adds per-warp lists of 20-weight groups to
+    # re-code (8 bytes each, room for 1/8 of the groups) after the block
+    big = lib.bl_quantize_weights_workspace_size(8192, 8192)
+    assert big % 256 == 0 and big >= 16384 + 8192 * (8192 // 20 + 1)
+    assert big < 8192 * 8192                      # well under the 4 n bytes of W
+    assert lib.bl_quantize_weights_workspace_size(1024, 1024) > 16384
     assert lib.bl_linear_workspace_size(16, 64, 100, 1) >= 16 * 112 + 16 * 4
 
 

@@ -103,6 +103,172 @@ def test_ternary_rounding_boundary(bl):
     assert len(set(ref.ravel()[:80:10].tolist())) > 1   # the boundary really splits
 
 
+# ------------------------------------------- single-pass weight quantizer ---
+# Byte offset of the fix-up mode word in the accumulator block at the start of
+# the workspace (after bins[256], four 32-bit counters and slot[256][4]):
+# 0 = listed band weights recoded, 1 = whole tensor re-ternarized.
+MODE_OFFSET = 256 * 8 + 16 + 256 * 32
+
+
+def _quantize_single_pass(bl, W, fmt, ws=None):
+    N, K = W.shape
+    lib = bl.load()
+    if ws is None:
+        ws = bl.workspace(lib.bl_quantize_weights_workspace_size(N, K), "cuda")
+    assert ws.numel() > 16384, "shape should take the single-pass quantizer"
+    if fmt == "pack5":
+        out, beta = bl.quantize_weights_pack5(dev(W), 1e-5, ws=ws)
+    else:
+        out, beta = bl.quantize_weights(dev(W), 1e-5, ws=ws)
+    mode = int(host(ws[MODE_OFFSET:MODE_OFFSET + 4]).view(np.uint32)[0])
+    return host(out), host(beta)[0], mode, ws
+
+
+def _expect_codes(W, fmt):
+    rb = oracle.absmean_beta(W, 1e-5)
+    q = oracle.ternarize(W, rb)
+    return rb, (oracle.pack5(q) if fmt == "pack5" else q)
+
+
+@pytest.mark.parametrize("fmt", ["i8", "pack5"])
+@pytest.mark.parametrize("N,K", [(512, 2560), (300, 3508), (8000, 132), (262144, 4), (1024, 1040)])
+def test_single_pass_gaussian(bl, fmt, N, K):
+    """Gaussian weights: the sampled band holds T, so only the band weights are
+    recoded (mode 0); chunks of several rows, ragged last groups and pad bytes."""
+    p = random_problem(N + 3 * K, 1, K, N)
+    out, beta, mode, _ = _quantize_single_pass(bl, p.W, fmt)
+    rb, ref = _expect_codes(p.W, fmt)
+    check_ok(bl)
+    assert beta == rb
+    np.testing.assert_array_equal(out, ref)
+    assert mode == 0
+
+
+@pytest.mark.parametrize("fmt", ["i8", "pack5"])
+def test_single_pass_wide_range_and_zeros(bl, fmt):
+    """Exponent bins, subnormals and exact zeros inside the single pass."""
+    rng = np.random.default_rng(15)
+    W = (rng.standard_normal((1100, 1000)) * 0.02).astype(F32)
+    W.ravel()[::7] *= F32(2.0 ** 30)
+    W.ravel()[3::11] *= F32(2.0 ** -40)
+    W.ravel()[5::13] = F32(1e-42)
+    W.ravel()[2::17] = F32(0.0)
+    out, beta, _, _ = _quantize_single_pass(bl, W, fmt)
+    rb, ref = _expect_codes(W, fmt)
+    check_ok(bl)
+    assert beta == rb
+    np.testing.assert_array_equal(out, ref)
+
+
+@pytest.mark.parametrize("fmt", ["i8", "pack5"])
+def test_single_pass_band_overflow_falls_back(bl, fmt):
+    """Half the magnitudes sit a hair below T (|w| = 1/3 with beta ~ 2/3): the
+    band lists overflow and the fix-up re-ternarizes the whole tensor."""
+    rng = np.random.default_rng(16)
+    mag = np.where(rng.random((1024, 1024)) < 0.5, F32(1.0), F32(1.0 / 3.0)).astype(F32)
+    W = (mag * np.where(rng.random(mag.shape) < 0.5, F32(-1), F32(1))).astype(F32)
+    out, beta, mode, _ = _quantize_single_pass(bl, W, fmt)
+    rb, ref = _expect_codes(W, fmt)
+    check_ok(bl)
+    assert beta == rb
+    np.testing.assert_array_equal(out, ref)
+    assert mode == 1
+
+
+def test_single_pass_unrepresentative_sample_falls_back(bl):
+    """Weights shrunk 1000x in every chunk the CTAs read first (chunk i*stride
+    mod nch for the first handouts, stride ~ nch/grid and coprime to nch, one
+    CTA per SM): the sampled band misses the exact T, and the whole tensor is
+    re-ternarized."""
+    import math
+    import torch
+    N, K = 4096, 4096
+    p = random_problem(77, 1, K, N)
+    W = p.W.copy()
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    nch = -(-N * (-(-K // 20)) // 512)
+    grid = min(sms, 256, nch)
+    stride = max(1, nch // grid)
+    while math.gcd(stride, nch) != 1:
+        stride += 1
+    flat = W.ravel()
+    for i in range(3 * grid):          # generous: every early handout
+        c = (i * stride) % nch
+        g0, g1 = c * 512, min(N * 205, c * 512 + 512)
+        r0, r1 = g0 // 205, (g1 - 1) // 205
+        f0 = r0 * K + 20 * (g0 - r0 * 205)
+        f1 = r1 * K + min(K, 20 * (g1 - 1 - r1 * 205) + 20)
+        flat[f0:f1] *= F32(1e-3)
+    out, beta, mode, ws = _quantize_single_pass(bl, W, "pack5")
+    rb, ref = _expect_codes(W, "pack5")
+    check_ok(bl)
+    assert beta == rb
+    np.testing.assert_array_equal(out, ref)
+    assert mode == 1
+    # the same workspace again, now with a representative tensor: back to mode 0
+    out2, beta2, mode2, _ = _quantize_single_pass(bl, p.W, "pack5", ws=ws)
+    rb2, ref2 = _expect_codes(p.W, "pack5")
+    check_ok(bl)
+    assert beta2 == rb2 and mode2 == 0
+    np.testing.assert_array_equal(out2, ref2)
+
+
+@pytest.mark.parametrize("fmt", ["i8", "pack5"])
+def test_single_pass_uncertified_mean_takes_exact_pass(bl, fmt):
+    """Half the weights 1.0, half the next float up: the exact mean 1 + 2^-24
+    is a float32 rounding tie, so the float64 sum cannot certify beta and the
+    kernel adds every magnitude again exactly (ties to even: beta = 1 + eps)."""
+    rng = np.random.default_rng(17)
+    mag = np.where(rng.permutation(1024 * 1024) < 512 * 1024, F32(1.0),
+                   np.nextafter(F32(1.0), F32(2.0))).astype(F32).reshape(1024, 1024)
+    W = (mag * np.where(rng.random(mag.shape) < 0.5, F32(-1), F32(1))).astype(F32)
+    out, beta, _, _ = _quantize_single_pass(bl, W, fmt)
+    rb, ref = _expect_codes(W, fmt)
+    check_ok(bl)
+    assert rb == F32(F32(1.0) + F32(1e-5))
+    assert beta == rb
+    np.testing.assert_array_equal(out, ref)
+
+
+def test_single_pass_nonfinite_is_reported(bl):
+    W = random_problem(19, 1, 1024, 1024).W.copy()
+    W[700, 33] = np.inf
+    _quantize_single_pass(bl, W, "pack5")
+    assert bl.sync_status() == "BL_ERR_NONFINITE"
+    check_ok(bl)
+    # the workspace is clear again: a finite tensor on it is exact
+    p = random_problem(20, 1, 1024, 1024)
+    lib = bl.load()
+    ws = bl.workspace(lib.bl_quantize_weights_workspace_size(1024, 1024), "cuda")
+    _quantize_single_pass(bl, W, "pack5", ws=ws)
+    assert bl.sync_status() == "BL_ERR_NONFINITE"
+    out, beta, _, _ = _quantize_single_pass(bl, p.W, "pack5", ws=ws)
+    rb, ref = _expect_codes(p.W, "pack5")
+    check_ok(bl)
+    assert beta == rb
+    np.testing.assert_array_equal(out, ref)
+
+
+def test_single_pass_workspace_reuse_and_two_pass_agree(bl):
+    """The workspace is left clear: repeated calls, and the two-pass kernels on
+    the same workspace, give identical results."""
+    p = random_problem(91, 1, 2560, 6912)
+    lib = bl.load()
+    ws = bl.workspace(lib.bl_quantize_weights_workspace_size(6912, 2560), "cuda")
+    first = _quantize_single_pass(bl, p.W, "pack5", ws=ws)
+    second = _quantize_single_pass(bl, p.W, "pack5", ws=ws)
+    Wd = dev(p.W)
+    beta = bl.absmean(Wd, 1e-5, ws=ws)
+    Wp = host(bl.ternarize_pack5(Wd, beta))
+    third = _quantize_single_pass(bl, p.W, "pack5", ws=ws)
+    check_ok(bl)
+    for r in (second, third):
+        assert r[1] == first[1]
+        np.testing.assert_array_equal(r[0], first[0])
+    assert host(beta)[0] == first[1]
+    np.testing.assert_array_equal(Wp, first[0])
+
+
 def test_nonfinite_weight_is_reported(bl):
     W = np.ones((4, 8), F32)
     W[2, 3] = np.inf
