@@ -34,13 +34,34 @@ __device__ __forceinline__ float act_recip(float s) {
 // real quotient y = x / s by at most 1.5 ulp(y) <= 1.5 * 2^-17 < 2^-16, and
 // float32(y) is within 2^-18 of y.  So unless y' lies within 2^-15 of a
 // half-integer, y, float32(y) and y' all round to the same integer; the rare
-// near-tie values take the exact division.
+// near-tie values take the exact division.  The rounding itself is t = y +
+// 1.5 * 2^23 (round to nearest even, exact for |y| <= 127), so the code is the
+// low byte of t's bits (two's complement) and no conversion instruction is
+// needed.  Returned in the low byte.
+__device__ __forceinline__ uint32_t act_code_bits(float x, float s, float r) {
+  const float y = fminf(fmaxf(__fmul_rn(x, r), -float(kActQmax)), float(kActQmax));
+  const float t = __fadd_rn(y, 12582912.0f);
+  const float d = __fsub_rn(y, __fsub_rn(t, 12582912.0f));
+  if (r == 0.f || fabsf(fabsf(d) - 0.5f) < 3.0517578125e-05f)
+    return uint32_t(uint8_t(int8_t(act_code_slow(x, s))));
+  return __float_as_uint(t) & 0xFFu;
+}
 __device__ __forceinline__ int8_t act_code_fast(float x, float s, float r) {
-  const float y = __fmul_rn(x, r);
-  const float q = rintf(y);
-  if (r == 0.f || fabsf(fabsf(__fsub_rn(y, q)) - 0.5f) < 3.0517578125e-05f)
-    return int8_t(act_code_slow(x, s));
-  return int8_t(int(fminf(fmaxf(q, -float(kActQmax)), float(kActQmax))));
+  return int8_t(uint8_t(act_code_bits(x, s, r)));
+}
+// act_code_bits without its branch: the caller redoes the codes with act_code
+// when `tie` comes back set (near a half-integer, or r == 0).
+__device__ __forceinline__ uint32_t act_code_try(float x, float r, bool& tie) {
+  const float y = fminf(fmaxf(__fmul_rn(x, r), -float(kActQmax)), float(kActQmax));
+  const float t = __fadd_rn(y, 12582912.0f);
+  const float d = __fsub_rn(y, __fsub_rn(t, 12582912.0f));
+  tie |= fabsf(fabsf(d) - 0.5f) < 3.0517578125e-05f;
+  return __float_as_uint(t) & 0xFFu;
+}
+// Four codes packed little-endian into one word.
+__device__ __forceinline__ uint32_t act_codes4(float4 v, float s, float r) {
+  return __byte_perm(__byte_perm(act_code_bits(v.x, s, r), act_code_bits(v.y, s, r), 0x0040),
+                     __byte_perm(act_code_bits(v.z, s, r), act_code_bits(v.w, s, r), 0x0040), 0x5410);
 }
 
 // One CTA per row: pass 1 finds max|x| (warp shuffles, then across warps), pass
@@ -89,12 +110,7 @@ act_quant_kernel(const float* __restrict__ X, int64_t K, float eps, int8_t* __re
 
   for (int64_t i = threadIdx.x; i < K4; i += kActThreads) {
     const float4 v = reinterpret_cast<const float4*>(xr)[i];
-    char4 q;
-    q.x = act_code_fast(v.x, s, r);
-    q.y = act_code_fast(v.y, s, r);
-    q.z = act_code_fast(v.z, s, r);
-    q.w = act_code_fast(v.w, s, r);
-    reinterpret_cast<char4*>(qr)[i] = q;
+    reinterpret_cast<uint32_t*>(qr)[i] = act_codes4(v, s, r);
   }
   for (int64_t i = (K4 << 2) + threadIdx.x; i < K; i += kActThreads) qr[i] = act_code_fast(xr[i], s, r);
   for (int64_t i = K + threadIdx.x; i < ldq; i += kActThreads) qr[i] = 0;
@@ -144,14 +160,7 @@ act_quant_reg_kernel(const float* __restrict__ X, int64_t K, float eps, int8_t* 
 #pragma unroll
   for (int u = 0; u < VPT; ++u) {
     const int i = threadIdx.x + u * kActThreads;
-    if (i < K4) {
-      char4 q;
-      q.x = act_code_fast(v[u].x, s, r);
-      q.y = act_code_fast(v[u].y, s, r);
-      q.z = act_code_fast(v[u].z, s, r);
-      q.w = act_code_fast(v[u].w, s, r);
-      reinterpret_cast<char4*>(qr)[i] = q;
-    }
+    if (i < K4) reinterpret_cast<uint32_t*>(qr)[i] = act_codes4(v[u], s, r);
   }
   for (int64_t i = K + threadIdx.x; i < ldq; i += kActThreads) qr[i] = 0;
 }

@@ -9,10 +9,10 @@
 // Per CTA (one per SM, persistent over a contiguous block of rows):
 //   * the rows' packed bytes arrive by 1-D bulk copies (TMA engine) into a ring
 //     of shared-memory stages, all issued up front when they fit;
-//   * the same kind of copies bring the decode table (a constant table in global
-//     memory) and the float32 X rows into shared memory; the CTA then quantizes
-//     X itself (per-row absmax, then exactly the codes of bl_quantize_act) into
-//     a layout matched to the decode;
+//   * the same kind of copy brings the float32 X rows into shared memory while
+//     the CTA builds the decode table there; the CTA then quantizes X itself
+//     (per-row absmax, then exactly the codes of bl_quantize_act) into a layout
+//     matched to the decode;
 //   * decode: a packed byte b holds digits d_k = floor(b/3^k) mod 3, trit t_k =
 //     d_k - 1.  A 243-entry table gives (t0,t1,t2,t3) as four int8; every lane has
 //     its own copy at b*256 + 4*lane, so 32 lanes never collide on a bank, and one
@@ -41,24 +41,6 @@ constexpr int kGemvMaxRS = 32;
 // The decode table as it sits in shared memory: word b*64 + l (l < 32) holds
 // trits t0..t3 of byte b as int8, one copy per lane; words 32..63 of a row are
 // unused, so the row pitch is 256 bytes and a byte_perm builds the address.
-struct GemvLut {
-  uint32_t w[243 * 64];
-};
-constexpr GemvLut gemv_make_lut() {
-  GemvLut t{};
-  for (int b = 0; b < 243; ++b) {
-    uint32_t v = 0;
-    int x = b;
-    for (int k = 0; k < 4; ++k) {
-      v |= uint32_t(uint8_t(int8_t(x % 3 - 1))) << (8 * k);
-      x /= 3;
-    }
-    for (int l = 0; l < 32; ++l) t.w[b * 64 + l] = v;
-  }
-  return t;
-}
-__device__ __align__(128) const GemvLut g_gemv_lut = gemv_make_lut();
-static_assert(sizeof(GemvLut) == kLutBytes, "decode table size");
 constexpr uint32_t kGemvXSmemMax = 64 * 1024;   // float32 X staged in shared memory up to this
 
 struct GemvArgs {
@@ -169,13 +151,30 @@ __global__ void __launch_bounds__(kGemvMaxWarps * 32, 1) gemv_pack5_kernel(const
   }
   __syncthreads();
   if (tid == 0) {
-    mbar_arrive_expect_tx(bar_x, uint32_t(kLutBytes) + a.xf_bytes);
-    bulk_g2s(smem, &g_gemv_lut, uint32_t(kLutBytes), bar_x);
-    if (a.xf_bytes) bulk_g2s(smem + a.xf_off, a.X, a.xf_bytes, bar_x);
+    if (a.xf_bytes) {
+      mbar_arrive_expect_tx(bar_x, a.xf_bytes);
+      bulk_g2s(smem + a.xf_off, a.X, a.xf_bytes, bar_x);
+    }
     for (int s = 0; s < nstage && s < nst; ++s) issue(s, s);
   }
   for (int i = tid; i < M * RS; i += nthr) part[i] = 0;
-  const bool xready = mbar_wait(bar_x, 0u);
+  // the decode table, built in place while the copies fly: word b*64 + l holds
+  // trits t0..t3 of byte b (one copy per lane l).  Lane l of a warp computes the
+  // word of byte 32 i + l once; shuffles spread each word to its 32 slots.
+  for (int blk = warp; blk < 8; blk += nthr >> 5) {
+    const uint32_t bl = uint32_t(blk * 32 + lane);
+    const uint32_t b1 = (bl * 171u) >> 9, b2 = (bl * 57u) >> 9, b3 = (bl * 19u) >> 9;  // bl/3, /9, /27
+    const uint32_t d0 = bl - 3u * b1, d1 = b1 - 3u * b2, d2 = b2 - 3u * b3, d3 = b3 - 3u * ((bl * 203u) >> 14);
+    const uint32_t v = ((d0 + 255u) & 0xFFu) | ((d1 + 255u) & 0xFFu) << 8 | ((d2 + 255u) & 0xFFu) << 16 |
+                       ((d3 + 255u) & 0xFFu) << 24;
+#pragma unroll 8
+    for (int i = 0; i < 32; ++i) {
+      const uint32_t e = uint32_t(blk * 32 + i);
+      const uint32_t vi = __shfl_sync(0xffffffffu, v, i);
+      if (e < 243u) reinterpret_cast<uint32_t*>(smem)[e * 64u + uint32_t(lane)] = vi;
+    }
+  }
+  const bool xready = a.xf_bytes ? mbar_wait(bar_x, 0u) : true;
   if (!__syncthreads_and(xready)) {
     if (tid == 0) {
       raise_status(kDevTimeout);
@@ -186,12 +185,13 @@ __global__ void __launch_bounds__(kGemvMaxWarps * 32, 1) gemv_pack5_kernel(const
 
   // 2. quantized x in decode order: for weight word g (packed bytes 4g..4g+3,
   //    weights 20g..20g+19) five words: x[5j..5j+3] for j = 4g+i (i<4), then
-  //    x[5j+4] for the four j.  One thread per (row, word); all rows at once.
-  const int W4 = int(ldp >> 2);                 // weight words per row
+  //    x[5j+4] for the four j.  Element k = 5j + r goes to byte 20g + 4i + r
+  //    (r < 4) or 20g + 16 + i (r = 4); positions past K hold 0.  Four elements
+  //    per thread and step, all rows.
   const int kpad = int(5 * ldp);
-  const int items = M * W4;
   unsigned char* xb = reinterpret_cast<unsigned char*>(xst);
   const float* xsrc = a.xf_bytes ? reinterpret_cast<const float*>(smem + a.xf_off) : a.X;
+  float scm[M];
   if (kFused) {
     const bool xvec = aligned(xsrc, 16) && (K & 3) == 0;
     const int64_t K4 = xvec ? (K >> 2) : 0;
@@ -216,53 +216,53 @@ __global__ void __launch_bounds__(kGemvMaxWarps * 32, 1) gemv_pack5_kernel(const
       if (lane == 0) s_redf[m * kGemvMaxWarps + warp] = w;
     }
     if (__syncthreads_or(bad) && tid == 0) raise_status(kDevNonFinite);
-    if (tid < M) {
-      float v = 0.f;
-      for (int w = 0; w < nthr / 32; ++w) v = fmaxf(v, s_redf[tid * kGemvMaxWarps + w]);
-      s_scale[tid] = __fadd_rn(__fdiv_rn(v, float(kActQmax)), a.eps);
+    // every warp forms the row scales from the per-warp maxima (no extra barrier)
+#pragma unroll
+    for (int m = 0; m < M; ++m) {
+      const float w = warp_max(lane < (nthr >> 5) ? s_redf[m * kGemvMaxWarps + lane] : 0.f);
+      scm[m] = __fadd_rn(__fdiv_rn(w, float(kActQmax)), a.eps);
+      if (tid == 0) s_scale[m] = scm[m];
     }
-    __syncthreads();
   }
   int x4part[M];
 #pragma unroll
-  for (int m = 0; m < M; ++m) x4part[m] = 0;
-  for (int it = tid; it < items; it += nthr) {
-    const int m = it / W4, g = it - m * W4;
-    const int k0 = 20 * g;
-    int q[20];
-    if (kFused) {
-      const float sc = s_scale[m], rc = act_recip(sc);
-      const float* xr = xsrc + int64_t(m) * K + k0;
-      if (k0 + 20 <= K && aligned(xr, 16)) {
+  for (int m = 0; m < M; ++m) {
+    x4part[m] = 0;
+    unsigned char* xbm = xb + int64_t(m) * kpad;
+    const float* xr = kFused ? xsrc + int64_t(m) * K : nullptr;
+    const int8_t* xq = kFused ? nullptr : a.Xq + int64_t(m) * a.ldxq;
+    const float sc = kFused ? scm[m] : 0.f, rc = kFused ? act_recip(sc) : 0.f;
+    for (int i4 = tid; i4 < (kpad >> 2); i4 += nthr) {
+      const int k = 4 * i4;
+      uint32_t c[4];
+      if (kFused) {
+        bool tie = rc == 0.f;
+        if (k + 4 <= K && aligned(xr + k, 16)) {
+          const float4 f = *reinterpret_cast<const float4*>(xr + k);
+          c[0] = act_code_try(f.x, rc, tie);
+          c[1] = act_code_try(f.y, rc, tie);
+          c[2] = act_code_try(f.z, rc, tie);
+          c[3] = act_code_try(f.w, rc, tie);
+        } else {
 #pragma unroll
-        for (int v4 = 0; v4 < 5; ++v4) {
-          const float4 f = reinterpret_cast<const float4*>(xr)[v4];
-          q[4 * v4] = act_code_fast(f.x, sc, rc);
-          q[4 * v4 + 1] = act_code_fast(f.y, sc, rc);
-          q[4 * v4 + 2] = act_code_fast(f.z, sc, rc);
-          q[4 * v4 + 3] = act_code_fast(f.w, sc, rc);
+          for (int e = 0; e < 4; ++e) c[e] = k + e < K ? act_code_try(xr[k + e], rc, tie) : 0u;
         }
+        if (tie)   // rare: a quotient near a half-integer; exact division
+          for (int e = 0; e < 4 && k + e < K; ++e) c[e] = uint32_t(uint8_t(int8_t(act_code_slow(xr[k + e], sc))));
       } else {
-        for (int e = 0; e < 20; ++e) q[e] = (k0 + e < K) ? act_code_fast(xr[e], sc, rc) : 0;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) c[e] = k + e < K ? uint32_t(uint8_t(xq[k + e])) : 0u;
       }
-    } else {
-      const int8_t* xr = a.Xq + int64_t(m) * a.ldxq + k0;
-      for (int e = 0; e < 20; ++e) q[e] = (k0 + e < K) ? int(xr[e]) : 0;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const uint32_t kk = uint32_t(k + e);
+        const uint32_t j = __umulhi(kk, 0xCCCCCCCDu) >> 2;     // kk / 5
+        const uint32_t r = kk - 5u * j;
+        const uint32_t off = 20u * (j >> 2) + (r < 4u ? 4u * (j & 3u) + r : 16u + (j & 3u));
+        xbm[off] = uint8_t(c[e]);
+        if (r == 4u) x4part[m] += int(int8_t(uint8_t(c[e])));
+      }
     }
-    uint32_t w5[5];
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-      w5[i] = uint32_t(uint8_t(q[5 * i])) | uint32_t(uint8_t(q[5 * i + 1])) << 8 |
-              uint32_t(uint8_t(q[5 * i + 2])) << 16 | uint32_t(uint8_t(q[5 * i + 3])) << 24;
-    w5[4] = uint32_t(uint8_t(q[4])) | uint32_t(uint8_t(q[9])) << 8 | uint32_t(uint8_t(q[14])) << 16 |
-            uint32_t(uint8_t(q[19])) << 24;
-    uint32_t* dst = reinterpret_cast<uint32_t*>(xb + int64_t(m) * kpad + 20 * g);
-#pragma unroll
-    for (int i = 0; i < 5; ++i) dst[i] = w5[i];
-    const int s4 = q[4] + q[9] + q[14] + q[19];
-#pragma unroll
-    for (int mm = 0; mm < M; ++mm)
-      if (mm == m) x4part[mm] += s4;
   }
 #pragma unroll
   for (int m = 0; m < M; ++m) {
@@ -276,7 +276,6 @@ __global__ void __launch_bounds__(kGemvMaxWarps * 32, 1) gemv_pack5_kernel(const
     for (int w = 0; w < nthr / 32; ++w) t += s_redi[tid * kGemvMaxWarps + w];
     s_x4sum[tid] = t;
   }
-  __syncthreads();
 
   // 4. this lane's x registers: chunks c0 + lane + 32 i of its K slice
   const int sl = warp % a.S, grp = warp / a.S;
