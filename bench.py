@@ -168,13 +168,20 @@ def ncu_traffic(kernel: str, workload: int):
 
 # ------------------------------------------------------------- the step ----
 class Step:
-    """Device buffers and API calls for one replica of the workload's step."""
+    """Device buffers and API calls for one replica of the workload's step.
+
+    A weight tensor used by one call runs as one BitLinear forward call (weight
+    quantization, activation quantization, contraction, dequant); a tensor shared
+    by several calls is quantized once, then each call runs the linear alone."""
 
     def __init__(self, bl, torch, probs, dev, fmt):
         self.bl, self.torch, self.fmt = bl, torch, fmt
-        self.tensors = []          # weight tensors: (W, beta, Wout, quantizer ws, N, K)
-        self.calls = []            # linear calls: (X, tensor index, Y, lin ws, M, K, N)
-        seen = {}
+        lib = bl.load()
+        self.tensors = []          # weight tensors: (W, beta, Wout, ws, N, K)
+        self.calls = []            # calls: (X, tensor index, Y, ws, M, K, N, eps)
+        seen, uses = {}, {}
+        for p in probs:
+            uses[id(p.W)] = uses.get(id(p.W), 0) + 1
         for p in probs:
             key = id(p.W)
             if key not in seen:
@@ -184,67 +191,76 @@ class Step:
                     Wout = torch.empty((p.N, bl.pack5_ldp(p.K)), dtype=torch.uint8, device=dev)
                 else:
                     Wout = torch.empty((p.N, p.K), dtype=torch.int8, device=dev)
-                ws = bl.workspace(bl.load().bl_quantize_weights_workspace_size(p.N, p.K), dev)
+                fused = uses[key] == 1
+                nb = (lib.bl_bitlinear_forward_workspace_size(p.M, p.N, p.K, fmt) if fused
+                      else lib.bl_quantize_weights_workspace_size(p.N, p.K))
+                ws = bl.workspace(nb, dev)
                 seen[key] = len(self.tensors)
-                self.tensors.append((W, beta, Wout, ws, p.N, p.K))
+                self.tensors.append((W, beta, Wout, ws, p.N, p.K, fused))
             X = torch.from_numpy(np.ascontiguousarray(p.X)).to(dev)
             Y = torch.empty((p.M, p.N), dtype=torch.float32, device=dev)
-            lws = bl.workspace(bl.linear_workspace_size(p.M, p.N, p.K, fmt), dev)
+            fused = self.tensors[seen[key]][6]
+            lws = (self.tensors[seen[key]][3] if fused
+                   else bl.workspace(bl.linear_workspace_size(p.M, p.N, p.K, fmt), dev))
             self.calls.append((X, seen[key], Y, lws, p.M, p.K, p.N, p.eps))
 
     def nbytes(self):
         n = 0
-        for W, beta, Wout, ws, N, K in self.tensors:
+        for W, beta, Wout, ws, N, K, fused in self.tensors:
             n += W.numel() * 4 + Wout.numel()
         for X, ti, Y, lws, M, K, N, eps in self.calls:
-            n += X.numel() * 4 + Y.numel() * 4 + lws.numel()
+            n += X.numel() * 4 + Y.numel() * 4 + (0 if self.tensors[ti][6] else lws.numel())
         return n
 
+    def order(self):
+        """(kind, index) in issue order: shared tensors' quantization, then calls."""
+        out = [("wquant", ti) for ti, t in enumerate(self.tensors) if not t[6]]
+        for ci, c in enumerate(self.calls):
+            out.append(("forward" if self.tensors[c[1]][6] else "linear", ci))
+        return out
+
     def run(self, only=None, path=0, streams=None):
-        """Issue the step: every call, or only call `only` (an index into
-        labels()).  With `streams`, each weight tensor's chain (its
-        quantization, then the calls that use it) goes on its own stream, forked
-        from and joined back into the current stream."""
+        """Issue the step, or only entry `only` of order().  With `streams`,
+        each weight tensor's chain goes on its own stream, forked from and
+        joined back into the current stream."""
         bl, torch = self.bl, self.torch
         main = torch.cuda.current_stream()
         if streams:
             for st in streams:
                 st.wait_stream(main)
-        k = -1
-        order = []
-        for ti, (W, beta, Wout, ws, N, K) in enumerate(self.tensors):
-            order.append(("w", ti, k + 1, None))
-            k += 1
-        for ci in range(len(self.calls)):
-            k += 1
-            order.append(("c", ci, k, None))
-        for kind, idx, k1, k2 in order:
-            ti = idx if kind == "w" else self.calls[idx][1]
+        for k, (kind, idx) in enumerate(self.order()):
+            if only is not None and only != k:
+                continue
+            ti = idx if kind == "wquant" else self.calls[idx][1]
             st = streams[ti % len(streams)] if streams else main
             with torch.cuda.stream(st):
-                if kind == "w":
-                    W, beta, Wout, ws, N, K = self.tensors[idx]
-                    if only is None or only == k1:
-                        if self.fmt == bl.PACK5:
-                            bl.quantize_weights_pack5(W, 1e-5, ws=ws, out=Wout, beta=beta)
-                        else:
-                            bl.quantize_weights(W, 1e-5, ws=ws, out=Wout, beta=beta)
+                if kind == "wquant":
+                    W, beta, Wout, ws, N, K, _ = self.tensors[idx]
+                    if self.fmt == bl.PACK5:
+                        bl.quantize_weights_pack5(W, 1e-5, ws=ws, out=Wout, beta=beta)
+                    else:
+                        bl.quantize_weights(W, 1e-5, ws=ws, out=Wout, beta=beta)
                 else:
                     X, ti2, Y, lws, M, K, N, eps = self.calls[idx]
-                    if only is None or only == k1:
-                        W, beta, Wout, ws, _, _ = self.tensors[ti2]
+                    W, beta, Wout, ws, _, _, _ = self.tensors[ti2]
+                    if kind == "forward":
+                        bl.bitlinear_forward(X, W, self.fmt, eps=eps, ws=ws, w_out=Wout, beta=beta, out=Y)
+                    else:
                         bl.linear(X, Wout, self.fmt, N, K, beta, eps=eps, ws=lws, out=Y, path=path)
         if streams:
             for st in streams:
                 main.wait_stream(st)
 
     def labels(self):
-        out = []
-        for i, (W, beta, Wout, ws, N, K) in enumerate(self.tensors):
-            out.append(("wquant", i))
-        for j, c in enumerate(self.calls):
-            out.append(("linear", j))
-        return out
+        return self.order()
+
+
+def forward_launches(bl, M, N, K, fmt, path):
+    """Kernel launches of one bl_bitlinear_forward call."""
+    if M <= 4 and N * K >= 2 ** 20 and K % 4 == 0 and M * K * 4 <= 48 * 1024 and path == 0:
+        return 1
+    q = 1 if (N * K >= 2 ** 20 and K % 4 == 0) else 2
+    return q + bl.linear_plan(M, N, K, fmt, path)[1]
 
 
 def algorithmic_bytes(kind, N, K, M, fmt):
@@ -254,6 +270,8 @@ def algorithmic_bytes(kind, N, K, M, fmt):
         return 4 * N * K + wbytes
     if kind == "linear":
         return wbytes + 4 * M * K + 4 * M * N
+    if kind == "forward":         # read W and X once, write the codes and Y
+        return 4 * N * K + wbytes + 4 * M * K + 4 * M * N
     raise ValueError(kind)
 
 
@@ -363,12 +381,15 @@ def run_ours(args):
             per_call[lab] = [c0.elapsed_time(c1) / (4 * reps * R)]
             del g
     shapes = {}
-    for i, (W, beta, Wout, ws, N, Kd) in enumerate(first.tensors):
-        # the single-pass quantizer (1 cooperative launch) whenever the library
-        # sized the workspace for it, else absmean + ternarize (2)
-        shapes[("wquant", i)] = (N, Kd, 0, 1 if ws.numel() > 16384 else 2)
-    for j, (X, ti, Y, lws, M, Kd, N, eps) in enumerate(first.calls):
-        shapes[("linear", j)] = (N, Kd, M, bl.linear_plan(M, N, Kd, fmt, args.path)[1])
+    for kind, idx in labels:
+        if kind == "wquant":
+            W, beta, Wout, ws, N, Kd, _ = first.tensors[idx]
+            shapes[(kind, idx)] = (N, Kd, 0, 1 if ws.numel() > 16384 else 2)
+        else:
+            X, ti, Y, lws, M, Kd, N, eps = first.calls[idx]
+            nl = (forward_launches(bl, M, N, Kd, fmt, args.path) if kind == "forward"
+                  else bl.linear_plan(M, N, Kd, fmt, args.path)[1])
+            shapes[(kind, idx)] = (N, Kd, M, nl)
     kinds = {}
     for lab, v in per_call.items():
         kind = lab[0]
@@ -378,7 +399,8 @@ def run_ours(args):
         d["bytes"] += algorithmic_bytes(kind, N, Kd, M, fmt)
         d["launches"] += nl
     peaks = measured_peaks()
-    kern_names = {"wquant": "wquant_kernel", "linear": "linear"}
+    kern_names = {"wquant": "wquant_kernel", "linear": "linear",
+                  "forward": "wquant_kernel (BitLinear forward)"}
     kernels = {}
     for kind, d in kinds.items():
         gbs = d["bytes"] / (d["ms"] * 1e-3) / 1e9
@@ -394,8 +416,8 @@ def run_ours(args):
     roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"],
                 "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
                 "traffic": ncu_traffic(kern_names[dom], args.workload),
-                "kernel": kern_names[dom], "call_launches": dkind["launches"] // max(
-                    1, len(first.tensors) if dom == "wquant" else len(first.calls)),
+                "kernel": kern_names[dom], "call_launches": dkind["launches"] / max(
+                    1, sum(1 for k, _ in labels if k == dom)),
                 "peak_source": peaks["source"] + " (MEASURED_PEAKS.json hbm_gbs)"
                 if peaks["source"] == "measured" else "fallback 6.65 TB/s"}
 
@@ -411,8 +433,8 @@ def run_ours(args):
                    "weight_format": wl.fmt, "parallelism": f"dp{world} (independent batches)",
                    "l2_defeat": f"{R} rotating replicas, {R * first.nbytes() / 2**20:.0f} MiB >= 4x L2 "
                                 f"({l2 / 2**20:.0f} MiB)",
-                   "step": "absmean + ternarize + pack per weight tensor (one call), then "
-                           "quantize_act + contraction + dequant per call", "timing": "CUDA graph per replica, CUDA events",
+                   "step": "per call: absmean beta, ternarize + pack W, per-row int8 X, "
+                           "contraction, dequant (one bl_bitlinear_forward call per weight tensor)", "timing": "CUDA graph per replica, CUDA events",
                    "streams": (f"{n_chains} (one per independent weight chain)" if n_chains else "1")},
         "macs_per_step": macs_per_step,
         "linear_only": None if lin is None else {
@@ -446,7 +468,12 @@ def run_ours(args):
 
 
 def e2e(bl, torch, probs, dev, fmt, steps, world):
-    """The step through the public API with pinned host inputs copied in and Y copied out."""
+    """The step through the public API with pinned host inputs copied in and Y
+    copied out: one bl_bitlinear_forward per single-use weight tensor, else
+    quantize once and run the linear per call."""
+    uses = {}
+    for p in probs:
+        uses[id(p.W)] = uses.get(id(p.W), 0) + 1
     host_W, host_X, seen = [], [], {}
     for p in probs:
         if id(p.W) not in seen:
@@ -456,7 +483,14 @@ def e2e(bl, torch, probs, dev, fmt, steps, world):
     dW = [torch.empty_like(h, device=dev) for h in host_W]
     dX = [torch.empty_like(h, device=dev) for h in host_X]
     hY = [torch.empty((p.M, p.N), dtype=torch.float32).pin_memory() for p in probs]
-    ws = [bl.workspace(bl.load().bl_quantize_weights_workspace_size(*h.shape), dev) for h in host_W]
+    lib = bl.load()
+    ws = {}
+    for j, p in enumerate(probs):
+        i = seen[id(p.W)]
+        if uses[id(p.W)] == 1:
+            ws[i] = bl.workspace(lib.bl_bitlinear_forward_workspace_size(p.M, p.N, p.K, fmt), dev)
+        elif i not in ws:
+            ws[i] = bl.workspace(lib.bl_quantize_weights_workspace_size(p.N, p.K), dev)
     h2d = sum(h.numel() * 4 for h in host_W) + sum(h.numel() * 4 for h in host_X)
     d2h = sum(h.numel() * 4 for h in hY)
 
@@ -465,15 +499,20 @@ def e2e(bl, torch, probs, dev, fmt, steps, world):
             d.copy_(h, non_blocking=True)
         for h, d in zip(host_X, dX):
             d.copy_(h, non_blocking=True)
-        packed = []
+        packed = {}
         for i, W in enumerate(dW):
-            if fmt == bl.PACK5:
-                packed.append(bl.quantize_weights_pack5(W, 1e-5, ws=ws[i]))
-            else:
-                packed.append(bl.quantize_weights(W, 1e-5, ws=ws[i]))
+            if i in ws and ws[i].numel() and any(uses[id(p.W)] > 1 and seen[id(p.W)] == i for p in probs):
+                if fmt == bl.PACK5:
+                    packed[i] = bl.quantize_weights_pack5(W, 1e-5, ws=ws[i])
+                else:
+                    packed[i] = bl.quantize_weights(W, 1e-5, ws=ws[i])
         for j, p in enumerate(probs):
-            Wd, beta = packed[seen[id(p.W)]]
-            Y = bl.linear(dX[j], Wd, fmt, p.N, p.K, beta, eps=p.eps)
+            i = seen[id(p.W)]
+            if uses[id(p.W)] == 1:
+                Y = bl.bitlinear_forward(dX[j], dW[i], fmt, eps=p.eps, ws=ws[i])[0]
+            else:
+                Wd, beta = packed[i]
+                Y = bl.linear(dX[j], Wd, fmt, p.N, p.K, beta, eps=p.eps)
             hY[j].copy_(Y, non_blocking=True)
 
     one()

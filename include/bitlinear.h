@@ -156,6 +156,30 @@ bl_status bl_linear(const float* X, int64_t M, int64_t K, const void* W, bl_wfmt
                     int64_t ldw, const float* beta_dev, const float* bias, float eps, float* Y,
                     void* ws, size_t ws_bytes, cudaStream_t stream);
 
+/* The BitLinear forward pass, steps 1-6 in one call: the weight tensor's beta
+ * and codes (as bl_quantize_weights / bl_quantize_weights_pack5), then
+ * Y = (X_q W_q^T)(s beta) [+ bias] (as bl_linear) -- the layer of "ultragraph
+ * -- when the graph is the 1-bit LLM, part 2", sections "the bytes" and
+ * "autograd on a byte-graph", where every forward quantizes both operands.
+ *   X        [M, K] float32 contiguous (16-byte aligned for the one-launch path).
+ *   W        [N, K] float32 contiguous.
+ *   f, Wout  the codes written out: BL_W_PACK5 [N, ldo] (ldo % 16 == 0,
+ *            ldo >= ceil(K/5), 16-byte aligned) or BL_W_I8 [N, K] (ldo == K).
+ *   beta_dev receives beta; bias [N] float32 or NULL; Y [M, N] float32.
+ *   eps      the epsilon of both quantizers.
+ *   ws       >= bl_bitlinear_forward_workspace_size(M, N, K, f) bytes, 256-byte
+ *            aligned, zero-filled before its first use (as for
+ *            bl_quantize_weights); calls sharing it must not overlap.
+ * For M <= 4 (decode) and tensors of 2^20+ weights with K % 4 == 0 and
+ * M*K*4 <= 48 KB, one cooperative launch reads W once and computes everything;
+ * other shapes run bl_quantize_weights* and bl_linear.  Results are identical
+ * either way.  Errors as for those two calls. */
+size_t bl_bitlinear_forward_workspace_size(int64_t M, int64_t N, int64_t K, bl_wfmt f);
+bl_status bl_bitlinear_forward(const float* X, int64_t M, int64_t K, const float* W, bl_wfmt f,
+                               int64_t N, float eps, void* Wout, int64_t ldo, float* beta_dev,
+                               const float* bias, float* Y, void* ws, size_t ws_bytes,
+                               cudaStream_t stream);
+
 /* bl_linear with the kernel path pinned (BL_PATH_*); BL_ERR_UNSUPPORTED when the
  * pinned path cannot take the shape.  Results are identical across paths. */
 bl_status bl_linear_ex(const float* X, int64_t M, int64_t K, const void* W, bl_wfmt f,

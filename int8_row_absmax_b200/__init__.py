@@ -43,6 +43,8 @@ SIGNATURES = {
     "bl_linear": (_I, [_P, _I64, _I64, _P, _I, _I64, _I64, _P, _P, _F, _P, _P, _SZ, _P]),
     "bl_linear_ex": (_I, [_P, _I64, _I64, _P, _I, _I64, _I64, _P, _P, _F, _P, _P, _SZ, _I, _P]),
     "bl_linear_noalloc": (_I, [_P, _I64, _I64, _P, _I, _I64, _I64, _P, _P, _F, _P, _P]),
+    "bl_bitlinear_forward_workspace_size": (_SZ, [_I64, _I64, _I64, _I]),
+    "bl_bitlinear_forward": (_I, [_P, _I64, _I64, _P, _I, _I64, _F, _P, _I64, _P, _P, _P, _P, _SZ, _P]),
     "bl_linear_plan": (_I, [_I64, _I64, _I64, _I, _I, ctypes.POINTER(ctypes.c_int)]),
     "bl_linear_acc": (_I, [_P, _I64, _I64, _P, _I, _I64, _I64, _P, _P]),
     "bl_linear_acc_workspace_size": (_SZ, [_I64, _I64, _I64, _I, _I]),
@@ -236,6 +238,29 @@ def linear(X, W, fmt: int, N: int, K: int, beta, bias=None, eps: float = 1e-5,
         _ptr(X), M, K, _ptr(W), fmt, N, W.shape[1], _ptr(beta), _ptr(bias), eps, _ptr(Y),
         _ptr(ws), ws.numel(), path, _stream(torch, X)))
     return Y
+
+
+def bitlinear_forward(X, W, fmt: int = PACK5, bias=None, eps: float = 1e-5, ws=None, w_out=None,
+                      beta=None, out=None):
+    """The BitLinear forward: W [N,K] and X [M,K] float32 -> (Y [M,N], codes, beta).
+    Codes: packed [N, ldp] uint8 (PACK5) or int8 [N,K] (I8)."""
+    torch, lib = _torch(), load()
+    _dev(X, torch.float32)
+    _dev(W, torch.float32)
+    M, K = X.shape
+    N = W.shape[0]
+    if W.shape[1] != K:
+        raise ValueError("shape mismatch")
+    if w_out is None:
+        w_out = (torch.empty((N, pack5_ldp(K)), dtype=torch.uint8, device=W.device) if fmt == PACK5
+                 else torch.empty((N, K), dtype=torch.int8, device=W.device))
+    beta = torch.empty(1, dtype=torch.float32, device=W.device) if beta is None else beta
+    Y = torch.empty((M, N), dtype=torch.float32, device=X.device) if out is None else out
+    ws = workspace(lib.bl_bitlinear_forward_workspace_size(M, N, K, fmt), W.device) if ws is None else ws
+    _check("bl_bitlinear_forward", lib.bl_bitlinear_forward(
+        _ptr(X), M, K, _ptr(W), fmt, N, eps, _ptr(w_out), w_out.shape[1], _ptr(beta), _ptr(bias),
+        _ptr(Y), _ptr(ws), ws.numel(), _stream(torch, X)))
+    return Y, w_out, beta
 
 
 NOALLOC_SCRATCH_BYTES = 16 << 20

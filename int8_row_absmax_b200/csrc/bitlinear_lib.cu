@@ -93,37 +93,74 @@ bl_status launch_absmean(const float* W, int64_t n, float eps, float* beta_dev, 
 bool fused_shape(int64_t N, int64_t K) { return N * K >= kFusedMinN && K % 4 == 0 && K <= 131072; }
 
 // a1-a3 in one read of W: one cooperative launch (all CTAs resident, for the
-// kernel's two grid barriers).  Returns BL_ERR_UNSUPPORTED, with nothing
+// kernel's two grid barriers); with M > 0 rows of X also a4-a6 (the BitLinear
+// forward) in the same launch.  Returns BL_ERR_UNSUPPORTED, with nothing
 // launched, when the device cannot hold the grid at once.
+template <bool kPacked, int kM>
+const void* wquant_fn() {
+  return reinterpret_cast<const void*>(wquant_kernel<kPacked, kM>);
+}
+const void* wquant_pick(bool packed, int M) {
+  switch (M) {
+    case 0: return packed ? wquant_fn<true, 0>() : wquant_fn<false, 0>();
+    case 1: return packed ? wquant_fn<true, 1>() : wquant_fn<false, 1>();
+    case 2: return packed ? wquant_fn<true, 2>() : wquant_fn<false, 2>();
+    case 3: return packed ? wquant_fn<true, 3>() : wquant_fn<false, 3>();
+    default: return packed ? wquant_fn<true, 4>() : wquant_fn<false, 4>();
+  }
+}
+
 bl_status launch_wquant_fused(const float* W, int64_t N, int64_t K, float eps, void* out,
                               int64_t ldo, bool packed, float* beta_dev, void* ws,
-                              cudaStream_t st) {
-  auto* acc = static_cast<AbsAccum*>(ws);
-  auto* list = reinterpret_cast<unsigned long long*>(static_cast<char*>(ws) + kFuListOff);
+                              cudaStream_t st, int64_t M = 0, const float* X = nullptr,
+                              const float* bias = nullptr, float* Y = nullptr) {
+  WqArgs a;
+  a.W = W;
+  a.N = N;
+  a.K = K;
+  a.eps = eps;
+  a.out = out;
+  a.ldo = ldo;
+  a.acc = static_cast<AbsAccum*>(ws);
+  a.yacc = reinterpret_cast<int*>(static_cast<char*>(ws) + kFuListOff);
+  a.list = reinterpret_cast<unsigned long long*>(static_cast<char*>(ws) + kFuListOff +
+                                                 fused_acc_bytes(M, N));
+  a.beta_out = beta_dev;
+  a.X = X;
+  a.bias = bias;
+  a.Y = Y;
   const int64_t ngroups = N * ceil_div(K, 20);
   const int64_t nch = ceil_div(ngroups, kFuGroups);
-  const void* fn = packed ? reinterpret_cast<const void*>(wquant_kernel<true>)
-                          : reinterpret_cast<const void*>(wquant_kernel<false>);
-  if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, kFuSmem) != cudaSuccess)
+  const int stages = M > 0 ? kFuStagesFwd : kFuStages;
+  a.xf_off = uint32_t(stages) * kFuStageBytes;
+  const int smem = int(a.xf_off + uint32_t(M * K * 4));
+  const void* fn = wquant_pick(packed, int(M));
+  if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
     return BL_ERR_CUDA;
   int per_sm = 0;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, kAbsThreads, kFuSmem) != cudaSuccess)
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, kAbsThreads, smem) != cudaSuccess)
     return BL_ERR_CUDA;
   int grid = num_sms() * per_sm;
   if (grid > kAbsMaxCtas) grid = kAbsMaxCtas;
   if (int64_t(grid) > nch) grid = int(nch);
   if (grid < 1) return BL_ERR_UNSUPPORTED;
-  int cap = int(fused_cap_w(ngroups, grid));
-  uint32_t stride = chunk_stride(nch, grid);
+  a.cap_w = int(fused_cap_w(ngroups, grid));
+  a.stride = chunk_stride(nch, grid);
   const int64_t gpr = ceil_div(K, 20);
-  uint32_t gpr_magic = gpr > 1 ? uint32_t(((uint64_t(1) << 32) + uint64_t(gpr) - 1) / uint64_t(gpr)) : 0u;
-  void* args[] = {&W, &N, &K, &eps, &out, &ldo, &acc, &list, &cap, &stride, &gpr_magic, &beta_dev};
-  const cudaError_t e = cudaLaunchCooperativeKernel(fn, grid, kAbsThreads, args, kFuSmem, st);
+  a.gpr_magic = gpr > 1 ? uint32_t(((uint64_t(1) << 32) + uint64_t(gpr) - 1) / uint64_t(gpr)) : 0u;
+  void* args[] = {&a};
+  const cudaError_t e = cudaLaunchCooperativeKernel(fn, grid, kAbsThreads, args, size_t(smem), st);
   if (e == cudaErrorCooperativeLaunchTooLarge) {
     (void)cudaGetLastError();
     return BL_ERR_UNSUPPORTED;
   }
   return e == cudaSuccess ? BL_OK : BL_ERR_CUDA;
+}
+
+// Whether the forward can run inside the single-pass launch.
+bool fused_forward_ok(int64_t M, int64_t N, int64_t K, const float* X, const float* W) {
+  return M >= 1 && M <= kFwdMaxM && fused_shape(N, K) && N < (int64_t(1) << 31) &&
+         uint64_t(M * K * 4) <= kFwdXBytesMax && is_aligned(X, 16) && is_aligned(W, 16);
 }
 
 bl_status check_ws(const void* ws, size_t ws_bytes, size_t need) {
@@ -392,7 +429,7 @@ int64_t bl_pack5_ldp(int64_t K) { return K < 1 ? 0 : round_up(ceil_div(K, 5), 16
 
 size_t bl_quantize_weights_workspace_size(int64_t N, int64_t K) {
   if (N < 1 || K < 1) return 0;
-  return fused_shape(N, K) ? fused_ws_bytes(N, K) : kAbsWsBytes;
+  return fused_shape(N, K) ? fused_ws_bytes(N, K, 0) : kAbsWsBytes;
 }
 
 bl_status bl_absmean(const float* W, int64_t N, int64_t K, float eps, float* beta_dev, void* ws,
@@ -434,7 +471,7 @@ bl_status bl_quantize_weights(const float* W, int64_t N, int64_t K, float eps, i
   if (!beta_dev) return BL_ERR_INVALID_ARG;
   if (!is_aligned(beta_dev, 4)) return BL_ERR_ALIGNMENT;
   if ((st = check_ws(ws, ws_bytes, kAbsWsBytes)) != BL_OK) return st;
-  if (fused_shape(N, K) && is_aligned(W, 16) && is_aligned(Wq, 4) && ws_bytes >= fused_ws_bytes(N, K)) {
+  if (fused_shape(N, K) && is_aligned(W, 16) && is_aligned(Wq, 4) && ws_bytes >= fused_ws_bytes(N, K, 0)) {
     st = launch_wquant_fused(W, N, K, eps, Wq, K, false, beta_dev, ws, stream);
     if (st != BL_ERR_UNSUPPORTED) return st;
   }
@@ -454,13 +491,54 @@ bl_status bl_quantize_weights_pack5(const float* W, int64_t N, int64_t K, float 
   if (!beta_dev) return BL_ERR_INVALID_ARG;
   if (!is_aligned(beta_dev, 4)) return BL_ERR_ALIGNMENT;
   if ((st = check_ws(ws, ws_bytes, kAbsWsBytes)) != BL_OK) return st;
-  if (fused_shape(N, K) && is_aligned(W, 16) && ws_bytes >= fused_ws_bytes(N, K)) {
+  if (fused_shape(N, K) && is_aligned(W, 16) && ws_bytes >= fused_ws_bytes(N, K, 0)) {
     st = launch_wquant_fused(W, N, K, eps, Wp, ldp, true, beta_dev, ws, stream);
     if (st != BL_ERR_UNSUPPORTED) return st;
   }
   st = bl_absmean(W, N, K, eps, beta_dev, ws, ws_bytes, stream);
   if (st != BL_OK) return st;
   return bl_ternarize_pack5(W, N, K, beta_dev, Wp, ldp, stream);
+}
+
+size_t bl_bitlinear_forward_workspace_size(int64_t M, int64_t N, int64_t K, bl_wfmt f) {
+  if (M < 1 || N < 1 || K < 1 || (f != BL_W_I8 && f != BL_W_PACK5)) return 0;
+  const size_t two = align_up(bl_quantize_weights_workspace_size(N, K)) + bl_linear_workspace_size(M, N, K, f);
+  size_t one = 0;
+  if (M <= kFwdMaxM && fused_shape(N, K) && N < (int64_t(1) << 31) && uint64_t(M * K * 4) <= kFwdXBytesMax)
+    one = fused_ws_bytes(N, K, M);
+  return align_up(two > one ? two : one);
+}
+
+bl_status bl_bitlinear_forward(const float* X, int64_t M, int64_t K, const float* W, bl_wfmt f,
+                               int64_t N, float eps, void* Wout, int64_t ldo, float* beta_dev,
+                               const float* bias, float* Y, void* ws, size_t ws_bytes,
+                               cudaStream_t stream) {
+  bl_status st = check_weights_args(W, N, K, Wout);
+  if (st != BL_OK) return st;
+  if (!X || !Y || !beta_dev || M < 1 || !eps_ok(eps)) return BL_ERR_INVALID_ARG;
+  if ((st = check_shape(M, K, N)) != BL_OK) return st;
+  if (f == BL_W_PACK5) {
+    if (ldo < ceil_div(K, 5)) return BL_ERR_INVALID_ARG;
+    if (ldo % 16 != 0 || !is_aligned(Wout, 16)) return BL_ERR_ALIGNMENT;
+  } else if (f == BL_W_I8) {
+    if (ldo != K) return BL_ERR_INVALID_ARG;
+  } else {
+    return BL_ERR_INVALID_ARG;
+  }
+  if (!is_aligned(beta_dev, 4) || !is_aligned(X, 4) || !is_aligned(Y, 4)) return BL_ERR_ALIGNMENT;
+  if ((st = check_ws(ws, ws_bytes, bl_bitlinear_forward_workspace_size(M, N, K, f))) != BL_OK) return st;
+  if (fused_forward_ok(M, N, K, X, W) && (f == BL_W_PACK5 || is_aligned(Wout, 4))) {
+    st = launch_wquant_fused(W, N, K, eps, Wout, ldo, f == BL_W_PACK5, beta_dev, ws, stream, M, X, bias, Y);
+    if (st != BL_ERR_UNSUPPORTED) return st;
+  }
+  // otherwise the two calls: weight quantization, then the linear
+  const size_t q = align_up(bl_quantize_weights_workspace_size(N, K));
+  st = f == BL_W_PACK5
+           ? bl_quantize_weights_pack5(W, N, K, eps, static_cast<uint8_t*>(Wout), ldo, beta_dev, ws, q, stream)
+           : bl_quantize_weights(W, N, K, eps, static_cast<int8_t*>(Wout), beta_dev, ws, q, stream);
+  if (st != BL_OK) return st;
+  return bl_linear(X, M, K, Wout, f, N, ldo, beta_dev, bias, eps, Y, static_cast<char*>(ws) + q,
+                   ws_bytes - q, stream);
 }
 
 bl_status bl_pack(const int8_t* Wq, int64_t N, int64_t K, uint8_t* Wp, int64_t ldp,

@@ -19,16 +19,17 @@
 //      handed out dynamically).  Every weight's magnitude is added in float64,
 //      and each 20-weight group is coded against T_hi at once: |w| >= T_hi gives
 //      +-1, anything else 0; a group holding a weight with T_lo <= |w| < T_hi has
-//      its index appended to the warp's list.  The CTA that finishes last
-//      certifies beta: the float64 total T is within E = (L + 4) 2^-52 T of the
-//      exact sum (L = the longest chain of float64 additions, all addends being
-//      non-negative), and beta = float32(float64(S) / n) + eps is monotone in
-//      S, so when T - E and T + E give the same beta that is the exact beta.
-//      Otherwise (a mean within about 1e-13 of a float32 rounding boundary, or
-//      a non-finite sum) every CTA adds the magnitudes again exactly, as
-//      integers in units of 2^-149 (the absmean_kernel method), and the last
-//      one rounds the exact total.  With beta and T known, mode 0 if
-//      T_lo <= T <= T_hi and no list overflowed, else mode 1; grid barrier B;
+//      its index appended to the warp's list.  At grid barrier B (all CTAs
+//      have added their float64 sums) every CTA certifies beta from the same
+//      total: T is within E = (L + 4) 2^-52 T of the exact sum (L = the
+//      longest chain of float64 additions, all addends being non-negative), and
+//      beta = float32(float64(S) / n) + eps is monotone in S, so when T - E and
+//      T + E give the same beta that is the exact beta.  Otherwise (a mean
+//      within about 1e-13 of a float32 rounding boundary, or a non-finite sum)
+//      every CTA adds the magnitudes again exactly, as integers in units of
+//      2^-149 (the absmean_kernel method), and the last one rounds the exact
+//      total.  With beta and T known: mode 0 if T_lo <= T <= T_hi and no list
+//      overflowed, else mode 1;
 //   2. mode 0: each warp re-codes the groups on its list from W against T;
 //      mode 1: the grid re-ternarizes the whole tensor.
 //
@@ -37,8 +38,18 @@
 // codes equal those of the two-pass kernels (and of the IEEE division) for any
 // input; the sample only decides how much work phase 2 has.  Every wait is
 // bounded: a barrier that times out records kDevTimeout and forces mode 1.
+//
+// The BitLinear forward for M <= 4 rows of X (decode) rides on the same pass
+// (kM > 0): while phase 0 waits, every CTA quantizes X (per-row absmax, the
+// codes of bl_quantize_act) into shared memory as small integer floats; in
+// phase 1 each group adds sum_k t_k x_q[k] (exact in float32: |sum| <= 20*127)
+// into int32 row accumulators (a row-segmented warp reduction, one atomic per
+// segment); phase 2 adds, for every re-coded group, the exact difference
+// between its final and provisional codes; the CTA that leaves last writes
+// Y = float(acc) (s beta) [+ b] and clears the accumulators.
 #pragma once
 
+#include "act_quant.cuh"
 #include "weight_quant.cuh"
 
 namespace bl {
@@ -47,7 +58,10 @@ constexpr int kFuGroups = kAbsConsumers;               // 20-weight groups per c
 constexpr int kFuStageFloats = kFuGroups * 20;         // 10240 floats
 constexpr uint32_t kFuStageBytes = kFuStageFloats * 4; // 40 KB
 constexpr int kFuStages = 5;                           // 200 KB in flight per SM
+constexpr int kFuStagesFwd = 4;                        // with the forward: room for X codes
 constexpr int kFuPreStages = 2;                        // issued before the band is known
+constexpr int kFwdMaxM = 4;
+constexpr uint32_t kFwdXBytesMax = 48 * 1024;          // float X codes in shared memory
 constexpr int kFuSmem = kFuStages * int(kFuStageBytes);
 constexpr int kFuWarps = kAbsConsumers / 32;           // lists per CTA
 constexpr int64_t kFusedMinN = int64_t(1) << 20;       // smaller tensors take the two-pass path
@@ -63,11 +77,34 @@ __host__ __device__ inline int64_t fused_cap_w(int64_t ngroups, int grid) {
 
 // Workspace bytes for any grid up to kAbsMaxCtas CTAs (8-byte list entries):
 // grid*16*cap_w <= grid*16*(18 + ngroups/(grid*128)) <= 288*kAbsMaxCtas + ngroups/8.
-__host__ __device__ inline size_t fused_ws_bytes(int64_t N, int64_t K) {
+// With the forward (M rows), int32 row accumulators [M, N] come first.
+__host__ __device__ inline size_t fused_acc_bytes(int64_t M, int64_t N) {
+  return (size_t(M) * size_t(N) * 4 + 255) & ~size_t(255);
+}
+__host__ __device__ inline size_t fused_ws_bytes(int64_t N, int64_t K, int64_t M = 0) {
   const int64_t ngroups = N * ((K + 19) / 20);
   const size_t entries = size_t(288) * kAbsMaxCtas + size_t(ngroups / 8 + 1);
-  return (kFuListOff + entries * 8 + 255) & ~size_t(255);
+  return (kFuListOff + fused_acc_bytes(M, N) + entries * 8 + 255) & ~size_t(255);
 }
+
+struct WqArgs {
+  const float* W;
+  int64_t N, K;
+  float eps;
+  void* out;                       // packed [N, ldo] or int8 [N, ldo = K]
+  int64_t ldo;
+  AbsAccum* acc;                   // accumulator block (workspace start)
+  unsigned long long* list;        // per-warp lists of groups to re-code
+  int cap_w;
+  uint32_t stride, gpr_magic;
+  float* beta_out;
+  // the forward (kM > 0)
+  const float* X;                  // [M, K] float32, 16-byte aligned
+  const float* bias;               // [N] or nullptr
+  float* Y;                        // [M, N]
+  int* yacc;                       // [M, N] int32 row sums (cleared in phase 0)
+  uint32_t xf_off;                 // shared-memory offset of the X codes
+};
 
 // A chunk order whose first `grid` entries are spread over the tensor: handout
 // i takes chunk (i * stride) mod nch, stride ~ nch / grid and coprime to nch.
@@ -214,21 +251,51 @@ __device__ inline float beta_from_limbs(unsigned long long L0, unsigned long lon
   return __fadd_rn(__double2float_rn(__ddiv_rn(D, double(n))), eps);
 }
 
-// out: packed [N, ldo] (kPacked) or int8 [N, ldo = K].  Chunks are 512
-// consecutive 20-weight groups in row-major group order (a group never crosses a
-// row, so a chunk is one contiguous range of W); consumer thread t takes group t
-// of every chunk: five 128-bit shared-memory loads, 20 weights, one output word.
-// list: per warp, cap_w 8-byte entries (row << 32 | group).
-template <bool kPacked>
+// [x >= T] for the step constants c, with the sign of x: -1, 0 or +1 as a float.
+__device__ __forceinline__ float signed_step(float x, StepConst c) {
+  return __uint_as_float(__float_as_uint(step_ge(fabsf(x), c)) | (__float_as_uint(x) & 0x80000000u));
+}
+
+// The code of bl_quantize_act as a float (-127 .. 127); `tie` as in act_code_try.
+__device__ __forceinline__ float act_codef_try(float x, float r, bool& tie) {
+  const float y = fminf(fmaxf(__fmul_rn(x, r), -float(kActQmax)), float(kActQmax));
+  const float q = __fsub_rn(__fadd_rn(y, 12582912.0f), 12582912.0f);
+  tie |= fabsf(fabsf(__fsub_rn(y, q)) - 0.5f) < 3.0517578125e-05f;
+  return q;
+}
+
+// Adds v into yacc[m * N + key] once per run of equal keys among the warp's
+// lanes (keys of one warp are non-decreasing; key -1: nothing).
+__device__ __forceinline__ void add_by_row(int* yacc, int64_t idx_base, int key, int v, int lane) {
+  if (__shfl_sync(0xffffffffu, key, 0) == __shfl_sync(0xffffffffu, key, 31)) {  // one row: the usual case
+    const int t = __reduce_add_sync(0xffffffffu, v);
+    if (lane == 0 && key >= 0 && t != 0) atomicAdd(yacc + idx_base + key, t);
+    return;
+  }
+#pragma unroll
+  for (int d = 1; d < 32; d <<= 1) {
+    const int vv = __shfl_down_sync(0xffffffffu, v, d);
+    const int kk = __shfl_down_sync(0xffffffffu, key, d);
+    if (lane + d < 32 && kk == key) v += vv;
+  }
+  const int kp = __shfl_up_sync(0xffffffffu, key, 1);
+  if (key >= 0 && (lane == 0 || kp != key) && v != 0) atomicAdd(yacc + idx_base + key, v);
+}
+
+// Chunks are 512 consecutive 20-weight groups in row-major group order (a group
+// never crosses a row, so a chunk is one contiguous range of W); consumer thread
+// t takes group t of every chunk: five 128-bit shared-memory loads, 20 weights,
+// one output word.  list: per warp, cap_w 8-byte entries (row << 32 | group).
+template <bool kPacked, int kM>
 __global__ void __launch_bounds__(kAbsThreads, 1)
-wquant_kernel(const float* __restrict__ W, int64_t N, int64_t K, float eps, void* __restrict__ out,
-              int64_t ldo, AbsAccum* __restrict__ acc, unsigned long long* __restrict__ list,
-              int cap_w, uint32_t stride, uint32_t gpr_magic, float* __restrict__ beta_out) {
+wquant_kernel(const __grid_constant__ WqArgs a) {
+  constexpr int kStages = kM > 0 ? kFuStagesFwd : kFuStages;
+  constexpr int kMM = kM > 0 ? kM : 1;
   extern __shared__ __align__(128) unsigned char stage_smem[];
-  __shared__ uint64_t full[kFuStages], empty[kFuStages];
-  __shared__ long long s_row0[kFuStages];
-  __shared__ int s_g0[kFuStages], s_ng[kFuStages];
-  __shared__ int s_issued[kFuStages];
+  __shared__ uint64_t full[kStages], empty[kStages];
+  __shared__ long long s_row0[kStages];
+  __shared__ int s_g0[kStages], s_ng[kStages];
+  __shared__ int s_issued[kStages];
   __shared__ unsigned long long s_bins[256];
   __shared__ unsigned long long s_limb[3];
   __shared__ unsigned long long s_word[kBigWords + 3];
@@ -240,9 +307,20 @@ wquant_kernel(const float* __restrict__ W, int64_t N, int64_t K, float eps, void
   __shared__ double s_dpart[kAbsThreads / 32];
   __shared__ float s_samp[kFuWarps];
   __shared__ int s_scnt[kFuWarps];
+  __shared__ float s_xred[kMM][kFuWarps];
+  __shared__ float s_xs[kMM];
   __shared__ bool s_last;
   __shared__ TernBand s_band;
   __shared__ int s_mode, s_next;
+  __shared__ float s_beta;
+  const float* __restrict__ W = a.W;
+  const int64_t N = a.N, K = a.K, ldo = a.ldo;
+  const float eps = a.eps;
+  void* __restrict__ out = a.out;
+  AbsAccum* __restrict__ acc = a.acc;
+  const int cap_w = a.cap_w;
+  float* __restrict__ beta_out = a.beta_out;
+  const float* xf = reinterpret_cast<const float*>(stage_smem + a.xf_off);  // kM > 0 only
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
   for (int i = tid; i < 256; i += blockDim.x) s_bins[i] = 0ull;
@@ -252,10 +330,10 @@ wquant_kernel(const float* __restrict__ W, int64_t N, int64_t K, float eps, void
   const int64_t n = N * K;
   const int n_static = nch >= 2 * int64_t(gridDim.x) ? int(nch / gridDim.x) - 1 : 0;
   // q / gpr for q < gpr + 512: hi32(q * ceil(2^32 / gpr)) is exact while q * gpr < 2^32
-  auto div_gpr = [&](uint32_t q) -> uint32_t { return gpr == 1 ? q : __umulhi(q, gpr_magic); };
+  auto div_gpr = [&](uint32_t q) -> uint32_t { return gpr == 1 ? q : __umulhi(q, a.gpr_magic); };
   if (tid == 0) {
     s_timeout = 0;
-    for (int s = 0; s < kFuStages; ++s) {
+    for (int s = 0; s < kStages; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], kFuWarps);
       s_issued[s] = 0;
@@ -266,19 +344,19 @@ wquant_kernel(const float* __restrict__ W, int64_t N, int64_t K, float eps, void
 
   double da0 = 0.0, da1 = 0.0;                      // this thread's float64 sums of |w|
   int wcount = 0;                                   // this warp's list length
-  unsigned long long* wl = list + int64_t(blockIdx.x * kFuWarps + (warp < kFuWarps ? warp : 0)) * cap_w;
+  unsigned long long* wl = a.list + int64_t(blockIdx.x * kFuWarps + (warp < kFuWarps ? warp : 0)) * cap_w;
   if (warp == kFuWarps) {
     // producer warp: lane 0 hands out chunks and issues the copies; only the
     // first kFuPreStages go out before the band is known, so the first chunk
-    // and barrier A do not queue behind a full ring's worth of copies
-    // handouts: this CTA's first n_static are blockIdx.x + k * grid (so its
+    // and barrier A do not queue behind a full ring's worth of copies.
+    // Handouts: this CTA's first n_static are blockIdx.x + k * grid (so its
     // first one is its share of the stratified sample), the tail comes from a
-    // counter whose next value is always requested one handout ahead
+    // counter whose next value is always requested one handout ahead.
     unsigned int tail = 0u;
     bool more = true;
     auto issue = [&](int it) -> bool {   // false: stop marker sent, or a wait gave up
-      const int s = it % kFuStages;
-      if (it >= kFuStages && !mbar_wait(&empty[s], uint32_t(it / kFuStages - 1) & 1u)) {
+      const int s = it % kStages;
+      if (it >= kStages && !mbar_wait(&empty[s], uint32_t(it / kStages - 1) & 1u)) {
         s_timeout = 1;
         return false;
       }
@@ -295,7 +373,7 @@ wquant_kernel(const float* __restrict__ W, int64_t N, int64_t K, float eps, void
         mbar_arrive(&full[s]);
         return false;
       }
-      const int64_t chunk = int64_t((static_cast<unsigned long long>(h) * stride) % uint64_t(nch));
+      const int64_t chunk = int64_t((static_cast<unsigned long long>(h) * a.stride) % uint64_t(nch));
       const int64_t G0 = chunk * kFuGroups;
       const int64_t G1 = min(ngroups, G0 + kFuGroups);
       const int64_t row0 = G0 / gpr, g0 = G0 - row0 * gpr;
@@ -322,9 +400,59 @@ wquant_kernel(const float* __restrict__ W, int64_t N, int64_t K, float eps, void
     if (lane == 0)
       for (; more; ++it) more = issue(it);
   } else {
-    // ---- phase 0: the first chunk's mean |w| is this CTA's sample ----
+    // ---- phase 0: X codes (forward), then this CTA's sample and barrier A ----
+    if constexpr (kM > 0) {
+      // the row sums start at zero: cleared here, before barrier A, so every
+      // CTA's clearing is visible before any CTA adds into them
+      for (int64_t i = int64_t(blockIdx.x) * kAbsConsumers + tid; i < int64_t(kM) * N;
+           i += int64_t(gridDim.x) * kAbsConsumers)
+        a.yacc[i] = 0;
+      float* xw = reinterpret_cast<float*>(stage_smem + a.xf_off);
+      const int K4 = int(K >> 2);                    // K % 4 == 0, X 16-byte aligned
+      bool badx = false;
+#pragma unroll
+      for (int m = 0; m < kM; ++m) {
+        const float4* xr = reinterpret_cast<const float4*>(a.X + int64_t(m) * K);
+        float mx = 0.f;
+        for (int i = tid; i < K4; i += kAbsConsumers) {
+          const float4 v = __ldg(xr + i);
+          const float t = fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w)));
+          badx |= !(t <= 3.402823466e38f) | (v.x != v.x) | (v.y != v.y) | (v.z != v.z) | (v.w != v.w);
+          mx = fmaxf(mx, t);
+        }
+        mx = warp_max(mx);
+        if (lane == 0) s_xred[m][warp] = mx;
+      }
+      if (badx) raise_status(kDevNonFinite);
+      named_bar_sync(1, kAbsConsumers);
+#pragma unroll
+      for (int m = 0; m < kM; ++m) {
+        const float w = warp_max(lane < kFuWarps ? s_xred[m][lane] : 0.f);
+        const float sc = __fadd_rn(__fdiv_rn(w, float(kActQmax)), eps);
+        const float rc = act_recip(sc);
+        if (tid == 0) s_xs[m] = sc;
+        const float4* xr = reinterpret_cast<const float4*>(a.X + int64_t(m) * K);
+        float4* xo = reinterpret_cast<float4*>(xw + int64_t(m) * K);
+        for (int i = tid; i < K4; i += kAbsConsumers) {
+          const float4 v = __ldg(xr + i);
+          bool tie = rc == 0.f;
+          float4 q;
+          q.x = act_codef_try(v.x, rc, tie);
+          q.y = act_codef_try(v.y, rc, tie);
+          q.z = act_codef_try(v.z, rc, tie);
+          q.w = act_codef_try(v.w, rc, tie);
+          if (tie) {   // rare: a quotient near a half-integer; exact division
+            q.x = float(act_code_slow(v.x, sc));
+            q.y = float(act_code_slow(v.y, sc));
+            q.z = float(act_code_slow(v.z, sc));
+            q.w = float(act_code_slow(v.w, sc));
+          }
+          xo[i] = q;
+        }
+      }
+    }
     {
-      float a = 0.f;
+      float sa = 0.f;
       int cnt = 0;
       if (mbar_wait(&full[0], 0u)) {
         const int ng = s_ng[0];
@@ -334,29 +462,29 @@ wquant_kernel(const float* __restrict__ W, int64_t N, int64_t K, float eps, void
           const int g = int(q - dr * uint32_t(gpr));
           cnt = int(min(int64_t(20), K - 20 * int64_t(g)));
           const float* gs = reinterpret_cast<const float*>(stage_smem) + (int(dr) * int(K) + 20 * (g - s_g0[0]));
-          for (int k = 0; k < cnt; ++k) a += fabsf(gs[k]);
+          for (int k = 0; k < cnt; ++k) sa += fabsf(gs[k]);
         }
       } else {
         s_timeout = 1;
       }
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) {
-        a += __shfl_xor_sync(0xffffffffu, a, o);
+        sa += __shfl_xor_sync(0xffffffffu, sa, o);
         cnt += __shfl_xor_sync(0xffffffffu, cnt, o);
       }
       if (lane == 0) {
-        s_samp[warp] = a;
+        s_samp[warp] = sa;
         s_scnt[warp] = cnt;
       }
       named_bar_sync(1, kAbsConsumers);
       if (tid == 0) {
-        double sa = 0.0;
+        double ssum = 0.0;
         int64_t sc = 0;
         for (int w = 0; w < kFuWarps; ++w) {
-          sa += double(s_samp[w]);
+          ssum += double(s_samp[w]);
           sc += s_scnt[w];
         }
-        const double m = sc > 0 ? sa / double(sc) : -1.0;
+        const double m = sc > 0 ? ssum / double(sc) : -1.0;
         acc->est_part[blockIdx.x][0] = m;
         acc->est_part[blockIdx.x][1] = m * m;
         __threadfence();
@@ -379,8 +507,8 @@ wquant_kernel(const float* __restrict__ W, int64_t N, int64_t K, float eps, void
     const StepConst sc_hi = s_band.ok ? step_const(s_band.hi) : StepConst{__int_as_float(0x7F800000), 1.f};
     const StepConst sc_lo = s_band.ok ? step_const(s_band.lo) : StepConst{__int_as_float(0x7F800000), 1.f};
     for (int it = 0;; ++it) {
-      const int s = it % kFuStages;
-      if (!mbar_wait(&full[s], uint32_t(it / kFuStages) & 1u)) {
+      const int s = it % kStages;
+      if (!mbar_wait(&full[s], uint32_t(it / kStages) & 1u)) {
         s_timeout = 1;
         break;
       }
@@ -409,25 +537,49 @@ wquant_kernel(const float* __restrict__ W, int64_t N, int64_t K, float eps, void
       float y[4] = {0.f, 0.f, 0.f, 0.f};   // packed: per byte, sum of trit * 3^k
       float t8[20];                        // int8: the trits
       float nband = 0.f;                   // weights with T_lo <= |w| < T_hi
+      float dot[kMM];                      // forward: sum_k t_k x_q[k]
 #pragma unroll
-      for (int P = 0; P < 20; ++P) {
-        const float x = f4get(f[P >> 2], P & 3);
-        const float ax = fabsf(x);
-        if (P & 1)
-          da1 = __dadd_rn(da1, double(ax));
-        else
-          da0 = __dadd_rn(da0, double(ax));
-        const float mh = step_ge(ax, sc_hi);
-        const float ml = step_ge(ax, sc_lo);
-        nband = __fadd_rn(nband, __fsub_rn(ml, mh));
-        const uint32_t sgn = __float_as_uint(x) & 0x80000000u;
-        if (kPacked) {
-          const float p3 = __uint_as_float(
-              __float_as_uint(float(P % 5 == 0 ? 1 : P % 5 == 1 ? 3 : P % 5 == 2 ? 9 : P % 5 == 3 ? 27 : 81)) | sgn);
-          y[P / 5] = __fmaf_rn(mh, p3, y[P / 5]);
-        } else {
-          t8[P] = __uint_as_float(__float_as_uint(mh) | sgn);
+      for (int m = 0; m < kMM; ++m) dot[m] = 0.f;
+#pragma unroll
+      for (int v = 0; v < 5; ++v) {
+        float4 xv[kMM];
+        if constexpr (kM > 0) {
+#pragma unroll
+          for (int m = 0; m < kM; ++m)
+            xv[m] = active && 4 * v < nk ? reinterpret_cast<const float4*>(xf + int64_t(m) * K + 20 * g)[v]
+                                         : make_float4(0.f, 0.f, 0.f, 0.f);
         }
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int P = 4 * v + j;
+          const float x = f4get(f[v], j);
+          const float ax = fabsf(x);
+          if (P & 1)
+            da1 = __dadd_rn(da1, double(ax));
+          else
+            da0 = __dadd_rn(da0, double(ax));
+          const float mh = step_ge(ax, sc_hi);
+          const float ml = step_ge(ax, sc_lo);
+          nband = __fadd_rn(nband, __fsub_rn(ml, mh));
+          const uint32_t sgn = __float_as_uint(x) & 0x80000000u;
+          if (kPacked) {
+            const float p3 = __uint_as_float(
+                __float_as_uint(float(P % 5 == 0 ? 1 : P % 5 == 1 ? 3 : P % 5 == 2 ? 9 : P % 5 == 3 ? 27 : 81)) | sgn);
+            y[P / 5] = __fmaf_rn(mh, p3, y[P / 5]);
+          } else {
+            t8[P] = __uint_as_float(__float_as_uint(mh) | sgn);
+          }
+          if constexpr (kM > 0) {
+            const float t = __uint_as_float(__float_as_uint(mh) | sgn);
+#pragma unroll
+            for (int m = 0; m < kM; ++m) dot[m] = __fmaf_rn(t, f4get(xv[m], j), dot[m]);
+          }
+        }
+      }
+      if constexpr (kM > 0) {
+#pragma unroll
+        for (int m = 0; m < kM; ++m)
+          add_by_row(a.yacc, int64_t(m) * N, active ? int(row) : -1, active ? __float2int_rn(dot[m]) : 0, lane);
       }
       // groups holding a band weight: one ballot, one list store per such lane
       const uint32_t pend = __ballot_sync(0xffffffffu, active && nband > 0.f);
@@ -441,11 +593,11 @@ wquant_kernel(const float* __restrict__ W, int64_t N, int64_t K, float eps, void
       if (active) {
         if (kPacked) {
           // byte = 121 + y: exact in the low mantissa bits of y + 2^23 + 121
-          uint32_t v[4];
+          uint32_t vb[4];
 #pragma unroll
-          for (int j = 0; j < 4; ++j) v[j] = __float_as_uint(__fadd_rn(y[j], 8388729.0f));
+          for (int j = 0; j < 4; ++j) vb[j] = __float_as_uint(__fadd_rn(y[j], 8388729.0f));
           uint32_t* orow = reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(out) + row * ldo);
-          orow[g] = __byte_perm(__byte_perm(v[0], v[1], 0x0040), __byte_perm(v[2], v[3], 0x0040), 0x5410);
+          orow[g] = __byte_perm(__byte_perm(vb[0], vb[1], 0x0040), __byte_perm(vb[2], vb[3], 0x0040), 0x5410);
           if (g == int(gpr) - 1)
             for (int64_t j = gpr; j < (ldo >> 2); ++j) orow[j] = 0x79797979u;  // pad bytes: 121
         } else {
@@ -473,7 +625,7 @@ wquant_kernel(const float* __restrict__ W, int64_t N, int64_t K, float eps, void
     // workspace ends clear; mode 1 then re-codes everything
     raise_status(kDevTimeout);
     atomicOr(&acc->overflow, 2u);
-    for (int s = 0; s < kFuStages; ++s)
+    for (int s = 0; s < kStages; ++s)
       if (s_issued[s] > 0) (void)mbar_wait(&full[s], uint32_t(s_issued[s] - 1) & 1u);
   }
 
@@ -490,17 +642,16 @@ wquant_kernel(const float* __restrict__ W, int64_t N, int64_t K, float eps, void
     for (int w = 0; w < kAbsThreads / 32; ++w) d = __dadd_rn(d, s_dpart[w]);
     atomicAdd(&acc->dsum, d);
     __threadfence();
-    const unsigned int ticket = atomicAdd(&acc->ticket, 1u);
+    const unsigned int ticket = atomicAdd(&acc->ticket, 1u);   // grid barrier B: arrive
     if (ticket >= gridDim.x) raise_status(kDevBadWorkspace);
-    s_last = (ticket == gridDim.x - 1);
   }
   __threadfence();
   __syncthreads();
-  // while beta is being finished: each lane loads its first listed group into
+  // while the other CTAs finish: each lane loads its first listed group into
   // registers, and warms L2 with the rest of the list
   int64_t prow = -1, pg = 0;
   float4 pf[5];
-  if (!s_last && warp < kFuWarps) {
+  if (warp < kFuWarps) {
     const int cnt = min(wcount, cap_w);
     if (lane < cnt) {
       const unsigned long long ent = __ldcg(wl + lane);
@@ -513,17 +664,18 @@ wquant_kernel(const float* __restrict__ W, int64_t N, int64_t K, float eps, void
     }
     for (int e = lane + 32; e < cnt; e += 32) {
       const unsigned long long ent = __ldcg(wl + e);
-      const float* a = W + int64_t(ent >> 32) * K + 20 * int64_t(ent & 0xFFFFFFFFull);
-      asm volatile("prefetch.global.L2 [%0];" ::"l"(a));
-      asm volatile("prefetch.global.L2 [%0];" ::"l"(a + 19));
+      const float* p = W + int64_t(ent >> 32) * K + 20 * int64_t(ent & 0xFFFFFFFFull);
+      asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
+      asm volatile("prefetch.global.L2 [%0];" ::"l"(p + 19));
     }
   }
   if (tid == 0) {
-    if (s_last) {
-      __threadfence();
+    // barrier B: every CTA, once all have added their sums, certifies beta
+    // itself from the same total (identical results everywhere)
+    if (wait_u32_geq(&acc->ticket, gridDim.x)) {
       const double T = __ldcg(&acc->dsum);
       const unsigned int ovf = __ldcg(&acc->overflow);
-      if (__ldcg(&acc->magic) != 0u) raise_status(kDevBadWorkspace);
+      if (blockIdx.x == 0 && __ldcg(&acc->magic) != 0u) raise_status(kDevBadWorkspace);
       // longest addition chain: 10 per group in each of a thread's two sums (a
       // thread adds one group per chunk of its CTA: at most the static ones and
       // the whole tail), their sum, the warp tree, the warps, and one per CTA
@@ -532,29 +684,20 @@ wquant_kernel(const float* __restrict__ W, int64_t N, int64_t K, float eps, void
       const double L = 10.0 * max_chunks + 1.0 + 5.0 + double(kAbsThreads / 32) + double(gridDim.x);
       const double E = (L + 4.0) * 2.220446049250313e-16 * T;
       const float beta = certified_beta(T, E, n, eps);
-      acc->dsum = 0.0;
-      acc->ticket = 0u;
-      acc->next_chunk = 0u;
       if (beta == beta) {
-        *beta_out = beta;
+        if (blockIdx.x == 0) *beta_out = beta;
+        s_beta = beta;
         const uint32_t tb = __float_as_uint(ternary_threshold(beta));
         const TernBand bd = s_band;
         s_mode = (bd.ok && bd.lo <= tb && tb <= bd.hi && ovf == 0u) ? 0 : 1;
-        acc->mode = uint32_t(s_mode);
+        if (blockIdx.x == 0) acc->mode = uint32_t(s_mode);   // for inspection only
         s_next = 1;
-        st_release_u32(&acc->flag_b, 1u);   // grid barrier B: beta and the mode are out
       } else {
-        s_next = 2;
-        st_release_u32(&acc->flag_b, 2u);   // not certified: everyone adds exactly
+        s_next = 2;                          // not certified: everyone adds exactly
       }
     } else {
-      if (wait_u32_geq(&acc->flag_b, 1u)) {
-        s_next = int(ld_acquire_u32(&acc->flag_b));
-        if (s_next == 1) s_mode = int(__ldcg(&acc->mode));
-      } else {
-        raise_status(kDevTimeout);
-        s_next = 0;                          // leave the provisional codes
-      }
+      raise_status(kDevTimeout);
+      s_next = 0;                            // leave the provisional codes
     }
   }
   __syncthreads();
@@ -613,6 +756,7 @@ wquant_kernel(const float* __restrict__ W, int64_t N, int64_t K, float eps, void
         if (tid == 0) *beta_out = beta;
       }
       if (tid == 0) {
+        s_beta = beta;
         const uint32_t tb = __float_as_uint(ternary_threshold(beta));
         const TernBand bd = s_band;
         s_mode = (bd.ok && bd.lo <= tb && tb <= bd.hi && __ldcg(&acc->overflow) == 0u) ? 0 : 1;
@@ -627,6 +771,7 @@ wquant_kernel(const float* __restrict__ W, int64_t N, int64_t K, float eps, void
     } else if (tid == 0) {
       if (wait_u32_geq(&acc->flag_c, 1u)) {
         s_mode = int(__ldcg(&acc->mode));
+        s_beta = __ldcg(beta_out);
       } else {
         raise_status(kDevTimeout);
         s_next = 0;
@@ -635,71 +780,125 @@ wquant_kernel(const float* __restrict__ W, int64_t N, int64_t K, float eps, void
     __syncthreads();
   }
 
-  // ---- phase 2: re-code against the exact T ----
+  // ---- phase 2: re-code against the exact T (and correct the forward sums) ----
   if (s_next != 0) {
     const int mode = s_mode;
-    const float T = ternary_threshold(__ldcg(beta_out));
+    const float T = ternary_threshold(s_beta);
+    const StepConst sc_old = s_band.ok ? step_const(s_band.hi) : StepConst{__int_as_float(0x7F800000), 1.f};
+    // one group: final codes into `out`; for the forward, the difference
+    // between final and provisional codes dotted with the X codes
+    auto recode = [&](int64_t row, int64_t g, const float4 (&w4)[5]) {
+      const int nk = int(min(int64_t(20), K - 20 * g));
+      if (kPacked) {
+        uint32_t d[20];
+#pragma unroll
+        for (int P = 0; P < 20; ++P) d[P] = P < nk ? trit_digit(f4get(w4[P >> 2], P & 3), T) : 1u;
+        uint32_t word = 0u;
+#pragma unroll
+        for (int b = 0; b < 4; ++b)
+          word |= pack5_digits(d[5 * b], d[5 * b + 1], d[5 * b + 2], d[5 * b + 3], d[5 * b + 4]) << (8 * b);
+        reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(out) + row * ldo)[g] = word;
+      } else {
+        uint32_t* o = reinterpret_cast<uint32_t*>(static_cast<int8_t*>(out) + row * ldo + 20 * g);
+#pragma unroll
+        for (int j = 0; j < 5; ++j)
+          if (4 * j < nk)
+            o[j] = uint32_t(uint8_t(trit_code(w4[j].x, T))) | uint32_t(uint8_t(trit_code(w4[j].y, T))) << 8 |
+                   uint32_t(uint8_t(trit_code(w4[j].z, T))) << 16 | uint32_t(uint8_t(trit_code(w4[j].w, T))) << 24;
+      }
+      if constexpr (kM > 0) {
+#pragma unroll
+        for (int m = 0; m < kM; ++m) {
+          float dd = 0.f;
+#pragma unroll
+          for (int P = 0; P < 20; ++P) {
+            if (P < nk) {
+              const float x = f4get(w4[P >> 2], P & 3);
+              const float tdiff = float(trit_code(x, T)) - signed_step(x, sc_old);
+              dd = __fmaf_rn(tdiff, xf[int64_t(m) * K + 20 * g + P], dd);
+            }
+          }
+          const int di = __float2int_rn(dd);
+          if (di != 0) atomicAdd(a.yacc + int64_t(m) * N + row, di);
+        }
+      }
+    };
     if (mode == 0) {
       if (warp < kFuWarps) {
         const int cnt = min(wcount, cap_w);
         int e0 = lane;
         if (prow >= 0) {   // the preloaded group
-          const int nk = int(min(int64_t(20), K - 20 * pg));
-          if (kPacked) {
-            uint32_t d[20];
-#pragma unroll
-            for (int P = 0; P < 20; ++P) d[P] = P < nk ? trit_digit(f4get(pf[P >> 2], P & 3), T) : 1u;
-            uint32_t word = 0u;
-#pragma unroll
-            for (int b = 0; b < 4; ++b)
-              word |= pack5_digits(d[5 * b], d[5 * b + 1], d[5 * b + 2], d[5 * b + 3], d[5 * b + 4]) << (8 * b);
-            reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(out) + prow * ldo)[pg] = word;
-          } else {
-            uint32_t* o = reinterpret_cast<uint32_t*>(static_cast<int8_t*>(out) + prow * ldo + 20 * pg);
-#pragma unroll
-            for (int j = 0; j < 5; ++j)
-              if (4 * j < nk)
-                o[j] = uint32_t(uint8_t(trit_code(pf[j].x, T))) | uint32_t(uint8_t(trit_code(pf[j].y, T))) << 8 |
-                       uint32_t(uint8_t(trit_code(pf[j].z, T))) << 16 | uint32_t(uint8_t(trit_code(pf[j].w, T))) << 24;
-          }
+          recode(prow, pg, pf);
           e0 = lane + 32;
         }
         for (int e = e0; e < cnt; e += 32) {
           const unsigned long long ent = __ldcg(wl + e);
           const int64_t row = int64_t(ent >> 32);
           const int64_t g = int64_t(ent & 0xFFFFFFFFull);
-          if (kPacked) {
-            reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(out) + row * ldo)[g] =
-                ternarize_pack5_word(W, K, T, true, row, g);   // W 16-byte aligned, K % 4 == 0
-          } else {
-            const float* wr = W + row * K + 20 * g;
-            uint32_t* o = reinterpret_cast<uint32_t*>(static_cast<int8_t*>(out) + row * ldo + 20 * g);
-            const int nk = int(min(int64_t(20), K - 20 * g));
-            for (int j = 0; 4 * j < nk; ++j) {
-              const float4 v = ld_stream_f4(reinterpret_cast<const float4*>(wr) + j);
-              o[j] = uint32_t(uint8_t(trit_code(v.x, T))) | uint32_t(uint8_t(trit_code(v.y, T))) << 8 |
-                     uint32_t(uint8_t(trit_code(v.z, T))) << 16 | uint32_t(uint8_t(trit_code(v.w, T))) << 24;
-            }
-          }
+          const int nk = int(min(int64_t(20), K - 20 * g));
+          const float4* src = reinterpret_cast<const float4*>(W + row * K + 20 * g);
+          float4 w4[5];
+#pragma unroll
+          for (int v = 0; v < 5; ++v) w4[v] = (4 * v < nk) ? ld_stream_f4(src + v) : make_float4(0.f, 0.f, 0.f, 0.f);
+          recode(row, g, w4);
         }
       }
-    } else {
+    } else if (kM == 0) {
       const int64_t t0 = int64_t(blockIdx.x) * blockDim.x + tid;
       const int64_t nthr = int64_t(gridDim.x) * blockDim.x;
       if (kPacked)
         ternarize_pack5_range(W, N, K, T, static_cast<uint8_t*>(out), ldo, t0, nthr);
       else
         ternarize_i8_range(W, n, T, static_cast<int8_t*>(out), t0, nthr);
+    } else {
+      // every group, with its forward correction; the pad words keep 121
+      for (int64_t i = int64_t(blockIdx.x) * blockDim.x + tid; i < ngroups; i += int64_t(gridDim.x) * blockDim.x) {
+        const int64_t row = i / gpr, g = i - row * gpr;
+        const int nk = int(min(int64_t(20), K - 20 * g));
+        const float4* src = reinterpret_cast<const float4*>(W + row * K + 20 * g);
+        float4 w4[5];
+#pragma unroll
+        for (int v = 0; v < 5; ++v) w4[v] = (4 * v < nk) ? ld_stream_f4(src + v) : make_float4(0.f, 0.f, 0.f, 0.f);
+        recode(row, g, w4);
+      }
     }
   }
-  // the CTA that leaves last clears the barriers and flags for the next call
+  // exit.  Plain quantizer: the CTA that leaves last clears the counters and
+  // flags.  Forward: grid barrier C (every CTA's corrections are in), each CTA
+  // writes its slice of Y = float(acc) (s beta) [+ b], and the CTA that finishes
+  // that last clears the counters and flags.
+  __threadfence();
   __syncthreads();
-  if (tid == 0 && atomicAdd(&acc->exit_cnt, 1u) == gridDim.x - 1) {
+  unsigned int* const done = kM > 0 ? &acc->exit2 : &acc->exit_cnt;
+  if constexpr (kM > 0) {
+    if (tid == 0) {
+      atomicAdd(&acc->exit_cnt, 1u);
+      if (!wait_u32_geq(&acc->exit_cnt, gridDim.x)) raise_status(kDevTimeout);
+    }
+    __syncthreads();
+    const float beta = s_beta;
+    const int64_t per = ceil_div(N, int64_t(gridDim.x));
+    const int64_t n0 = int64_t(blockIdx.x) * per, n1 = min(N, n0 + per);
+#pragma unroll
+    for (int m = 0; m < kM; ++m) {
+      const float sb = __fmul_rn(s_xs[m], beta);
+      for (int64_t i = n0 + tid; i < n1; i += blockDim.x) {
+        float yv = __fmul_rn(float(__ldcg(a.yacc + int64_t(m) * N + i)), sb);
+        if (a.bias) yv = __fadd_rn(yv, __ldg(a.bias + i));
+        a.Y[int64_t(m) * N + i] = yv;
+      }
+    }
+    __syncthreads();
+  }
+  if (tid == 0 && atomicAdd(done, 1u) == gridDim.x - 1) {
     acc->bar_a = 0u;
-    acc->flag_b = 0u;
     acc->flag_c = 0u;
     acc->overflow = 0u;
     acc->exit_cnt = 0u;
+    acc->exit2 = 0u;
+    acc->ticket = 0u;
+    acc->next_chunk = 0u;
+    acc->dsum = 0.0;
   }
 }
 

@@ -79,6 +79,8 @@ struct AbsAccum {
   double dsum;                      // float64 sum of |w| over all CTAs
   unsigned int ticket2;             // exact pass: CTAs done
   unsigned int flag_c;              // exact pass: beta published
+  unsigned int exit2;               // forward: CTAs done writing Y
+  unsigned int pad4_;
   double est_part[kAbsMaxCtas][2];  // per CTA: sampled chunk mean (-1: none) and its square
 };
 constexpr size_t kAbsWsBytes = 16384;

@@ -269,6 +269,74 @@ def test_single_pass_workspace_reuse_and_two_pass_agree(bl):
     np.testing.assert_array_equal(Wp, first[0])
 
 
+# ------------------------------------------------------- the fused forward ---
+def _forward_check(bl, X, W, fmt, bias=None, eps=1e-5):
+    fmt_c = bl.PACK5 if fmt == "pack5" else bl.I8
+    Y, Wd, beta = bl.bitlinear_forward(dev(X), dev(W), fmt_c, None if bias is None else dev(bias), eps)
+    ref = oracle.bitlinear(X, W, eps, bias)
+    check_ok(bl)
+    assert host(beta)[0] == ref["beta"]
+    codes = oracle.pack5(ref["Wq"]) if fmt == "pack5" else ref["Wq"]
+    np.testing.assert_array_equal(host(Wd), codes)
+    assert_y_close(host(Y), ref["Y"])
+
+
+@pytest.mark.parametrize("fmt", ["pack5", "i8"])
+@pytest.mark.parametrize("M,K,N", [(1, 2560, 6912), (1, 6912, 2560), (2, 1040, 1024), (3, 3508, 300),
+                                   (4, 132, 8000), (1, 12288, 128)])
+def test_forward_one_launch(bl, fmt, M, K, N):
+    """M <= 4: weight quantization, activation quantization, contraction and
+    dequant in the single pass over W; Y bit-identical to the oracle."""
+    p = random_problem(M * 1000 + K + N, M, K, N)
+    bias = (np.random.default_rng(M + K).standard_normal(N) * 0.1).astype(F32) if M % 2 else None
+    _forward_check(bl, p.X, p.W, fmt, bias)
+
+
+def test_forward_decode_outliers(bl):
+    """The decode workload's activations (1% of entries x20) through the forward."""
+    for p in problems(2):
+        _forward_check(bl, p.X, p.W, "pack5")
+
+
+@pytest.mark.parametrize("fmt", ["pack5", "i8"])
+def test_forward_band_overflow_corrects_sums(bl, fmt):
+    """Mode 1 (every group re-coded): the row sums get every group's correction."""
+    rng = np.random.default_rng(21)
+    mag = np.where(rng.random((1024, 1024)) < 0.5, F32(1.0), F32(1.0 / 3.0)).astype(F32)
+    W = (mag * np.where(rng.random(mag.shape) < 0.5, F32(-1), F32(1))).astype(F32)
+    X = rng.standard_normal((2, 1024)).astype(F32)
+    _forward_check(bl, X, W, fmt)
+
+
+def test_forward_uncertified_mean(bl):
+    """The float32 rounding tie of beta (exact pass) inside the forward."""
+    rng = np.random.default_rng(22)
+    mag = np.where(rng.permutation(1024 * 1024) < 512 * 1024, F32(1.0),
+                   np.nextafter(F32(1.0), F32(2.0))).astype(F32).reshape(1024, 1024)
+    W = (mag * np.where(rng.random(mag.shape) < 0.5, F32(-1), F32(1))).astype(F32)
+    X = rng.standard_normal((1, 1024)).astype(F32)
+    _forward_check(bl, X, W, "pack5")
+
+
+@pytest.mark.parametrize("M,K,N", [(5, 1040, 1024), (1, 1001, 1100), (64, 256, 256), (1, 40, 30)])
+def test_forward_two_call_shapes(bl, M, K, N):
+    """Shapes outside the one-launch path (M > 4, K % 4 != 0, small tensors)."""
+    p = random_problem(M + K + N + 7, M, K, N)
+    _forward_check(bl, p.X, p.W, "pack5")
+    _forward_check(bl, p.X, p.W, "i8")
+
+
+def test_forward_repeat_same_workspace(bl):
+    p = random_problem(23, 1, 2560, 6912)
+    lib = bl.load()
+    ws = bl.workspace(lib.bl_bitlinear_forward_workspace_size(1, 6912, 2560, bl.PACK5), "cuda")
+    outs = [host(bl.bitlinear_forward(dev(p.X), dev(p.W), bl.PACK5, ws=ws)[0]) for _ in range(3)]
+    check_ok(bl)
+    for o in outs[1:]:
+        np.testing.assert_array_equal(o, outs[0])
+    assert_y_close(outs[0], oracle.bitlinear(p.X, p.W, 1e-5)["Y"])
+
+
 def test_nonfinite_weight_is_reported(bl):
     W = np.ones((4, 8), F32)
     W[2, 3] = np.inf
