@@ -375,6 +375,21 @@ def test_quantize_act(bl, M, K):
     np.testing.assert_array_equal(host(Xq), rq)
 
 
+@pytest.mark.parametrize("M,K", [(600, 4096), (700, 1000), (320, 12288), (1000, 12)])
+def test_quantize_act_many_rows(bl, M, K):
+    """Many rows take the persistent bulk-copy kernel (rows streamed through a
+    ring of shared-memory stages); codes and scales as the oracle's."""
+    rng = np.random.default_rng(M + K)
+    X = rng.standard_normal((M, K)).astype(F32)
+    X[::17] *= F32(40.0)
+    X[5] = 0.0
+    Xq, s = bl.quantize_act(dev(X), 1e-5)
+    rq, rs = oracle.act_quant(X, 1e-5)
+    check_ok(bl)
+    np.testing.assert_array_equal(host(s), rs)
+    np.testing.assert_array_equal(host(Xq), rq)
+
+
 def test_quantize_act_ties_and_zero_rows(bl):
     X = np.zeros((4, 9), F32)
     X[0] = [127, 0.5, 1.5, 2.5, -0.5, -1.5, -2.5, 126.5, -127]
