@@ -207,7 +207,7 @@ bl_status check_shape(int64_t M, int64_t K, int64_t N) {
 
 // Resolve the kernel path for a linear call; -1 when the pinned path cannot run it.
 // `fused_quant`: bl_linear (X in float32) rather than bl_linear_acc (X_q given).
-constexpr int64_t kTcMinM = 128;   // AUTO uses the tensor cores from this many rows
+constexpr int64_t kTcMinM = 5;     // AUTO: tensor cores above the GEMV's M <= 4 (measured faster than dp4a from M = 5)
 
 // Whether the tensor-core path can take the shape: K at least one 128-byte K
 // block, and for one-trit-per-byte weights a TMA-able row stride.
@@ -276,14 +276,35 @@ bool make_map_i8(CUtensorMap* map, const void* base, int64_t inner, int64_t oute
 }
 
 // The tcgen05 GEMM on int8 X_q [M, ldx] and int8 W_q [N, ldw].
+template <int kBN>
+bl_status launch_tc(const TcMaps& maps, const TcArgs& a, bool dequant, cudaStream_t st) {
+  const int64_t tiles = int64_t(a.tiles_m) * a.tiles_n;
+  const dim3 grid(unsigned(tiles < num_sms() ? tiles : num_sms()));
+  constexpr int smem = TcCfg<kBN>::kSmem;
+  if (dequant) {
+    if (cudaFuncSetAttribute(gemm_tc_kernel<true, kBN>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+        cudaSuccess)
+      return BL_ERR_CUDA;
+    gemm_tc_kernel<true, kBN><<<grid, kTcThreads, smem, st>>>(maps, a);
+  } else {
+    if (cudaFuncSetAttribute(gemm_tc_kernel<false, kBN>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+        cudaSuccess)
+      return BL_ERR_CUDA;
+    gemm_tc_kernel<false, kBN><<<grid, kTcThreads, smem, st>>>(maps, a);
+  }
+  return launch_status();
+}
+
 bl_status run_tc(const int8_t* Xq, int64_t ldx, int64_t M, int64_t K, const int8_t* Wq, int64_t ldw,
                  int64_t N, const float* s, const float* beta, const float* bias, float* Y,
                  int32_t* acc, cudaStream_t st) {
   if (ldx % 16 != 0 || ldw % 16 != 0 || !is_aligned(Xq, 16) || !is_aligned(Wq, 16))
     return BL_ERR_ALIGNMENT;
-  if (ceil_div(M, kTcBM) * ceil_div(N, kTcBN) > (int64_t(1) << 31) - 1) return BL_ERR_UNSUPPORTED;
+  // 64-wide tiles when the 256-wide ones would leave SMs idle
+  const int bn = ceil_div(M, kTcBM) * ceil_div(N, kTcBN) < num_sms() ? 64 : 256;
+  if (ceil_div(M, kTcBM) * ceil_div(N, bn) > (int64_t(1) << 31) - 1) return BL_ERR_UNSUPPORTED;
   TcMaps maps;
-  if (!make_map_i8(&maps.a, Xq, K, M, ldx, kTcBM) || !make_map_i8(&maps.b, Wq, K, N, ldw, kTcBN))
+  if (!make_map_i8(&maps.a, Xq, K, M, ldx, kTcBM) || !make_map_i8(&maps.b, Wq, K, N, ldw, bn))
     return BL_ERR_CUDA;
   TcArgs a;
   a.M = M;
@@ -295,21 +316,8 @@ bl_status run_tc(const int8_t* Xq, int64_t ldx, int64_t M, int64_t K, const int8
   a.Y = Y;
   a.acc = acc;
   a.tiles_m = int(ceil_div(M, kTcBM));
-  a.tiles_n = int(ceil_div(N, kTcBN));
-  const int64_t tiles = int64_t(a.tiles_m) * a.tiles_n;
-  const dim3 grid(unsigned(tiles < num_sms() ? tiles : num_sms()));
-  if (Y) {
-    if (cudaFuncSetAttribute(gemm_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kTcSmem) !=
-        cudaSuccess)
-      return BL_ERR_CUDA;
-    gemm_tc_kernel<true><<<grid, kTcThreads, kTcSmem, st>>>(maps, a);
-  } else {
-    if (cudaFuncSetAttribute(gemm_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, kTcSmem) !=
-        cudaSuccess)
-      return BL_ERR_CUDA;
-    gemm_tc_kernel<false><<<grid, kTcThreads, kTcSmem, st>>>(maps, a);
-  }
-  return launch_status();
+  a.tiles_n = int(ceil_div(N, bn));
+  return bn == 64 ? launch_tc<64>(maps, a, Y != nullptr, st) : launch_tc<256>(maps, a, Y != nullptr, st);
 }
 
 // Packed weights -> int8 rows in the workspace (first version of the tensor-core path).

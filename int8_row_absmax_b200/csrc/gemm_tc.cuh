@@ -6,11 +6,12 @@
 // section "autograd on a byte-graph".  With many token rows the layer is a dense
 // GEMM, so it runs on the 5th-generation tensor cores.
 //
-// Persistent kernel, one CTA per SM walking 128 x 256 output tiles:
+// Persistent kernel, one CTA per SM walking 128 x kBN output tiles (kBN = 256,
+// or 64 when 256-wide tiles would leave SMs idle):
 //   * warp 0 (one thread): TMA loads of A = X_q [128 x 128 B] and B = W_q
-//     [256 x 128 B] tiles (128-byte swizzle) into a 4-stage shared-memory ring;
-//   * warp 1 (one thread): tcgen05.mma, M=128 N=256 K=32, four per stage, into
-//     one of two 256-column TMEM accumulators; tcgen05.commit releases each
+//     [kBN x 128 B] tiles (128-byte swizzle) into a 4- (8-) stage shared-memory ring;
+//   * warp 1 (one thread): tcgen05.mma, M=128 N=kBN K=32, four per stage, into
+//     one of two kBN-column TMEM accumulators; tcgen05.commit releases each
 //     stage, and the accumulator once a tile's K loop is done;
 //   * warps 2..5: the epilogue, each warp draining its 32 TMEM lanes (tile rows)
 //     with tcgen05.ld, y = float32(acc) * (s_m * beta) [+ b_n], float32 stores;
@@ -27,12 +28,17 @@
 namespace bl {
 
 constexpr int kTcBM = 128, kTcBN = 256, kTcBK = 128;
-constexpr int kTcStages = 4;
 constexpr int kTcStageA = kTcBM * kTcBK;             // 16 KB
-constexpr int kTcStageB = kTcBN * kTcBK;             // 32 KB
-constexpr int kTcSmem = kTcStages * (kTcStageA + kTcStageB) + 1024;  // + alignment slack
 constexpr int kTcThreads = 192;                       // producer, MMA, 4 epilogue warps
-constexpr uint32_t kTcTmemCols = 512;                 // two 256-column accumulators
+// Tile width kBN = 256 (4 stages of 16 + 32 KB), or 64 when the 256-wide tiles
+// would leave SMs idle (small M: N / 256 tiles only; 8 stages of 16 + 8 KB).
+template <int kBN>
+struct TcCfg {
+  static constexpr int kStages = kBN == 256 ? 4 : 8;
+  static constexpr int kStageB = kBN * kTcBK;
+  static constexpr int kSmem = kStages * (kTcStageA + kStageB) + 1024;   // + alignment slack
+  static constexpr uint32_t kTmemCols = 2 * kBN;                         // two accumulators
+};
 
 struct alignas(64) TcMaps {
   CUtensorMap a;   // X_q [M, K] int8, row stride ldx
@@ -49,9 +55,12 @@ struct TcArgs {
   int tiles_m, tiles_n;
 };
 
-template <bool kDequant>
+template <bool kDequant, int kBN = kTcBN>
 __global__ void __launch_bounds__(kTcThreads, 1)
 gemm_tc_kernel(const __grid_constant__ TcMaps maps, const TcArgs a) {
+  constexpr int kTcStages = TcCfg<kBN>::kStages;
+  constexpr int kTcStageB = TcCfg<kBN>::kStageB;
+  constexpr uint32_t kTcTmemCols = TcCfg<kBN>::kTmemCols;
   extern __shared__ unsigned char smem_raw[];
   __shared__ uint64_t full[kTcStages], empty[kTcStages], acc_full[2], acc_empty[2], drain;
   __shared__ uint32_t s_tmem;
@@ -102,14 +111,14 @@ gemm_tc_kernel(const __grid_constant__ TcMaps maps, const TcArgs a) {
           unsigned char* sa = smem + s * (kTcStageA + kTcStageB);
           mbar_arrive_expect_tx(&full[s], uint32_t(kTcStageA + kTcStageB));
           tma_load_2d(sa, &maps.a, kb * kTcBK, tm * kTcBM, &full[s]);
-          tma_load_2d(sa + kTcStageA, &maps.b, kb * kTcBK, tn * kTcBN, &full[s]);
+          tma_load_2d(sa + kTcStageA, &maps.b, kb * kTcBK, tn * kBN, &full[s]);
         }
       }
     }
   } else if (warp == 1) {
     if (lane == 0) {
       // MMA issuer
-      constexpr uint32_t idesc = umma_idesc_i8(kTcBM, kTcBN);
+      constexpr uint32_t idesc = umma_idesc_i8(kTcBM, kBN);
       int it = 0, u = 0;
       for (int t = blockIdx.x; t < ntiles && !*err; t += gridDim.x, ++u) {
         const int b = u & 1;
@@ -118,7 +127,7 @@ gemm_tc_kernel(const __grid_constant__ TcMaps maps, const TcArgs a) {
           break;
         }
         tc_fence_after();
-        const uint32_t d = tmem + uint32_t(b * kTcBN);
+        const uint32_t d = tmem + uint32_t(b * kBN);
         bool ok = true;
         for (int kb = 0; kb < nkb; ++kb, ++it) {
           const int s = it % kTcStages;
@@ -160,12 +169,12 @@ gemm_tc_kernel(const __grid_constant__ TcMaps maps, const TcArgs a) {
       tc_fence_after();
       const int tm = t / a.tiles_n, tn = t - tm * a.tiles_n;
       const int64_t m = int64_t(tm) * kTcBM + row;
-      const int64_t n0 = int64_t(tn) * kTcBN;
-      const uint32_t taddr = tmem + (uint32_t(q * 32) << 16) + uint32_t(b * kTcBN);
+      const int64_t n0 = int64_t(tn) * kBN;
+      const uint32_t taddr = tmem + (uint32_t(q * 32) << 16) + uint32_t(b * kBN);
       float sbm = 0.f;
       if (kDequant && m < a.M) sbm = __fmul_rn(a.s[m], beta);
 #pragma unroll 1
-      for (int c = 0; c < kTcBN / 32; ++c) {
+      for (int c = 0; c < kBN / 32; ++c) {
         uint32_t r[32];
         tmem_ld32(taddr + uint32_t(c * 32), r);
         tmem_ld_wait();

@@ -489,6 +489,20 @@ def test_tc_parity(bl, fmt, M, K, N):
         np.testing.assert_array_equal(host(acc), oracle.contract(Xq, oracle.ternarize(p.W, host(beta)[0])))
 
 
+@pytest.mark.parametrize("fmt", ["i8", "pack5"])
+@pytest.mark.parametrize("M,K,N", [(5, 6912, 2560), (40, 2560, 6912), (127, 1040, 1000), (9, 128, 70)])
+def test_small_m_tensor_core_auto(bl, fmt, M, K, N):
+    """5 <= M < 128 with AUTO: the tcgen05 GEMM with 64-wide tiles (the 256-wide
+    ones would leave SMs idle); ragged N tails inside a 64-wide tile."""
+    f = bl.PACK5 if fmt == "pack5" else bl.I8
+    assert bl.linear_plan(M, N, K, f, bl.PATH_AUTO)[0] == bl.PATH_TC
+    p = random_problem(M * 31 + K + N, M, K, N)
+    Y, Wd, beta = _layer(bl, p, f, bl.PATH_AUTO)
+    ref = oracle.bitlinear(p.X, p.W, p.eps)
+    check_ok(bl)
+    assert_y_close(Y, ref["Y"])
+
+
 def test_linear_bias(bl):
     p = random_problem(77, 5, 300, 45)
     b = np.random.default_rng(1).standard_normal(45).astype(F32)
