@@ -207,6 +207,10 @@ bl_status check_shape(int64_t M, int64_t K, int64_t N) {
 
 // Resolve the kernel path for a linear call; -1 when the pinned path cannot run it.
 // `fused_quant`: bl_linear (X in float32) rather than bl_linear_acc (X_q given).
+// Packed weights are decoded inside the tensor-core GEMM for up to this many
+// 128-row tiles; beyond, they are unpacked to int8 once and the GEMM reads those.
+constexpr int64_t kTcDecodeMaxTilesM = 4;
+bool tc_unpack(int64_t M, bl_wfmt f) { return f == BL_W_PACK5 && ceil_div(M, int64_t(kTcBM)) > kTcDecodeMaxTilesM; }
 constexpr int64_t kTcMinM = 5;     // AUTO: tensor cores above the GEMV's M <= 4 (measured faster than dp4a from M = 5)
 
 // Whether the tensor-core path can take the shape: K at least one 128-byte K
@@ -234,7 +238,7 @@ int resolve_path(int64_t M, int64_t N, int64_t K, bl_wfmt f, int path, int* laun
     n = 1;                    // quantization fused into the GEMV
   } else if (p == BL_PATH_TC) {
     if (!tc_ok) return -1;
-    n = (fused_quant ? 2 : 1) + (f == BL_W_PACK5 ? 1 : 0);  // [act_quant,] [unpack,] GEMM
+    n = (fused_quant ? 2 : 1) + (tc_unpack(M, f) ? 1 : 0);  // [act_quant,] [unpack,] GEMM
   } else {
     return -1;
   }
@@ -275,36 +279,54 @@ bool make_map_i8(CUtensorMap* map, const void* base, int64_t inner, int64_t oute
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// The tcgen05 GEMM on int8 X_q [M, ldx] and int8 W_q [N, ldw].
-template <int kBN>
+// Packed W [N, ldp] bytes as 128-byte x rows boxes with the 128-byte swizzle
+// (the decoder warps' reads of four rows then spread over the banks);
+// out-of-range bytes are 0 (they only meet zero X columns).
+bool make_map_packed(CUtensorMap* map, const void* base, int64_t ldp, int64_t N, int box_rows) {
+  EncodeTiledFn fn = encode_tiled();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {cuuint64_t(ldp), cuuint64_t(N)};
+  const cuuint64_t strides[1] = {cuuint64_t(ldp)};
+  const cuuint32_t box[2] = {128u, cuuint32_t(box_rows)};
+  const cuuint32_t estr[2] = {1u, 1u};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// The tcgen05 GEMM on int8 X_q [M, ldx] and int8 W_q [N, ldw] (or packed W
+// [N, ldw = ldp], decoded inside the kernel).
+template <int kBN, bool kPacked>
 bl_status launch_tc(const TcMaps& maps, const TcArgs& a, bool dequant, cudaStream_t st) {
   const int64_t tiles = int64_t(a.tiles_m) * a.tiles_n;
   const dim3 grid(unsigned(tiles < num_sms() ? tiles : num_sms()));
-  constexpr int smem = TcCfg<kBN>::kSmem;
+  constexpr int smem = TcCfg<kBN, kPacked>::kSmem;
+  constexpr int threads = TcCfg<kBN, kPacked>::kThreads;
   if (dequant) {
-    if (cudaFuncSetAttribute(gemm_tc_kernel<true, kBN>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
-        cudaSuccess)
+    if (cudaFuncSetAttribute(gemm_tc_kernel<true, kBN, kPacked>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             smem) != cudaSuccess)
       return BL_ERR_CUDA;
-    gemm_tc_kernel<true, kBN><<<grid, kTcThreads, smem, st>>>(maps, a);
+    gemm_tc_kernel<true, kBN, kPacked><<<grid, threads, smem, st>>>(maps, a);
   } else {
-    if (cudaFuncSetAttribute(gemm_tc_kernel<false, kBN>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
-        cudaSuccess)
+    if (cudaFuncSetAttribute(gemm_tc_kernel<false, kBN, kPacked>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             smem) != cudaSuccess)
       return BL_ERR_CUDA;
-    gemm_tc_kernel<false, kBN><<<grid, kTcThreads, smem, st>>>(maps, a);
+    gemm_tc_kernel<false, kBN, kPacked><<<grid, threads, smem, st>>>(maps, a);
   }
   return launch_status();
 }
 
-bl_status run_tc(const int8_t* Xq, int64_t ldx, int64_t M, int64_t K, const int8_t* Wq, int64_t ldw,
-                 int64_t N, const float* s, const float* beta, const float* bias, float* Y,
+bl_status run_tc(const int8_t* Xq, int64_t ldx, int64_t M, int64_t K, const void* W, int64_t ldw,
+                 bool packed, int64_t N, const float* s, const float* beta, const float* bias, float* Y,
                  int32_t* acc, cudaStream_t st) {
-  if (ldx % 16 != 0 || ldw % 16 != 0 || !is_aligned(Xq, 16) || !is_aligned(Wq, 16))
+  if (ldx % 16 != 0 || ldw % 16 != 0 || !is_aligned(Xq, 16) || !is_aligned(W, 16))
     return BL_ERR_ALIGNMENT;
   // 64-wide tiles when the 256-wide ones would leave SMs idle
   const int bn = ceil_div(M, kTcBM) * ceil_div(N, kTcBN) < num_sms() ? 64 : 256;
   if (ceil_div(M, kTcBM) * ceil_div(N, bn) > (int64_t(1) << 31) - 1) return BL_ERR_UNSUPPORTED;
   TcMaps maps;
-  if (!make_map_i8(&maps.a, Xq, K, M, ldx, kTcBM) || !make_map_i8(&maps.b, Wq, K, N, ldw, bn))
+  if (!make_map_i8(&maps.a, Xq, K, M, ldx, kTcBM)) return BL_ERR_CUDA;
+  if (packed ? !make_map_packed(&maps.b, W, ldw, N, bn) : !make_map_i8(&maps.b, W, K, N, ldw, bn))
     return BL_ERR_CUDA;
   TcArgs a;
   a.M = M;
@@ -317,10 +339,14 @@ bl_status run_tc(const int8_t* Xq, int64_t ldx, int64_t M, int64_t K, const int8
   a.acc = acc;
   a.tiles_m = int(ceil_div(M, kTcBM));
   a.tiles_n = int(ceil_div(N, bn));
-  return bn == 64 ? launch_tc<64>(maps, a, Y != nullptr, st) : launch_tc<256>(maps, a, Y != nullptr, st);
+  const bool dq = Y != nullptr;
+  if (packed) return bn == 64 ? launch_tc<64, true>(maps, a, dq, st) : launch_tc<256, true>(maps, a, dq, st);
+  return bn == 64 ? launch_tc<64, false>(maps, a, dq, st) : launch_tc<256, false>(maps, a, dq, st);
 }
 
-// Packed weights -> int8 rows in the workspace (first version of the tensor-core path).
+// Packed weights -> int8 rows in the workspace, for tensor-core GEMMs with more
+// than kTcDecodeMaxTilesM row tiles (decoding inside the GEMM would repeat for
+// every row tile there).
 bl_status unpack_rows(const uint8_t* Wp, int64_t N, int64_t K, int64_t ldp, int8_t* Wq, int64_t ldk,
                       cudaStream_t st) {
   const int64_t words = ceil_div(ceil_div(K, 5), 4);
@@ -577,7 +603,7 @@ bl_status bl_quantize_act(const float* X, int64_t M, int64_t K, float eps, int8_
 size_t bl_linear_ex_workspace_size(int64_t M, int64_t N, int64_t K, bl_wfmt f, int path) {
   if (M < 0 || K < 1 || N < 1) return 0;
   const int p = resolve_path(M, N, K, f, path, nullptr);
-  return lin_layout(M, K, N, p == BL_PATH_TC && f == BL_W_PACK5).total;
+  return lin_layout(M, K, N, p == BL_PATH_TC && tc_unpack(M, f)).total;
 }
 
 size_t bl_linear_workspace_size(int64_t M, int64_t N, int64_t K, bl_wfmt f) {
@@ -599,7 +625,7 @@ bl_status bl_linear_ex(const float* X, int64_t M, int64_t K, const void* W, bl_w
   if (!is_aligned(X, 4) || !is_aligned(Y, 4) || (bias && !is_aligned(bias, 4))) return BL_ERR_ALIGNMENT;
   const int p = resolve_path(M, N, K, f, path, nullptr, true, ldw, W);
   if (p < 0) return BL_ERR_UNSUPPORTED;
-  const LinWs l = lin_layout(M, K, N, p == BL_PATH_TC && f == BL_W_PACK5);
+  const LinWs l = lin_layout(M, K, N, p == BL_PATH_TC && tc_unpack(M, f));
   if (!ws || !is_aligned(ws, kWsAlign) || ws_bytes < l.total) return BL_ERR_WORKSPACE;
   if (p == BL_PATH_GEMV)
     return run_gemv(X, nullptr, 0, M, K, W, ldw, N, beta_dev, bias, eps, Y, nullptr, stream);
@@ -609,16 +635,13 @@ bl_status bl_linear_ex(const float* X, int64_t M, int64_t K, const void* W, bl_w
   st = launch_status();
   if (st != BL_OK) return st;
   if (p == BL_PATH_TC) {
-    const int8_t* Wq = static_cast<const int8_t*>(W);
-    int64_t ldq = ldw;
-    if (f == BL_W_PACK5) {
+    if (tc_unpack(M, f)) {
       int8_t* scratch = reinterpret_cast<int8_t*>(static_cast<char*>(ws) + l.wq_off);
       st = unpack_rows(static_cast<const uint8_t*>(W), N, K, ldw, scratch, l.ldk, stream);
       if (st != BL_OK) return st;
-      Wq = scratch;
-      ldq = l.ldk;
+      return run_tc(Xq, l.ldx, M, K, scratch, l.ldk, false, N, s, beta_dev, bias, Y, nullptr, stream);
     }
-    return run_tc(Xq, l.ldx, M, K, Wq, ldq, N, s, beta_dev, bias, Y, nullptr, stream);
+    return run_tc(Xq, l.ldx, M, K, W, ldw, f == BL_W_PACK5, N, s, beta_dev, bias, Y, nullptr, stream);
   }
   return run_simt(Xq, l.ldx, M, K, W, f, ldw, N, s, beta_dev, bias, Y, nullptr, stream);
 }
@@ -655,7 +678,7 @@ bl_status bl_linear_noalloc(const float* X, int64_t M, int64_t K, const void* W,
 size_t bl_linear_acc_workspace_size(int64_t M, int64_t N, int64_t K, bl_wfmt f, int path) {
   if (M < 1 || N < 1 || K < 1) return 0;
   const int p = resolve_path(M, N, K, f, path, nullptr, false);
-  if (p == BL_PATH_TC && f == BL_W_PACK5) return align_up(size_t(N) * size_t(round_up(K, 16)));
+  if (p == BL_PATH_TC && tc_unpack(M, f)) return align_up(size_t(N) * size_t(round_up(K, 16)));
   return 0;
 }
 
@@ -681,18 +704,16 @@ bl_status bl_linear_acc_ex(const int8_t* Xq, int64_t M, int64_t K, const void* W
   if (p == BL_PATH_GEMV)
     return run_gemv(nullptr, Xq, K, M, K, W, ldw, N, nullptr, nullptr, 0.f, nullptr, acc, stream);
   if (p == BL_PATH_TC) {
-    const int8_t* Wq = static_cast<const int8_t*>(W);
-    int64_t ldq = ldw;
-    if (f == BL_W_PACK5) {
+    if (tc_unpack(M, f)) {
       const size_t need = align_up(size_t(N) * size_t(round_up(K, 16)));
       if (!ws || !is_aligned(ws, kWsAlign) || ws_bytes < need) return BL_ERR_WORKSPACE;
       int8_t* scratch = static_cast<int8_t*>(ws);
       bl_status st2 = unpack_rows(static_cast<const uint8_t*>(W), N, K, ldw, scratch, round_up(K, 16), stream);
       if (st2 != BL_OK) return st2;
-      Wq = scratch;
-      ldq = round_up(K, 16);
+      return run_tc(Xq, K, M, K, scratch, round_up(K, 16), false, N, nullptr, nullptr, nullptr, nullptr, acc,
+                    stream);
     }
-    return run_tc(Xq, K, M, K, Wq, ldq, N, nullptr, nullptr, nullptr, nullptr, acc, stream);
+    return run_tc(Xq, K, M, K, W, ldw, f == BL_W_PACK5, N, nullptr, nullptr, nullptr, nullptr, acc, stream);
   }
   return run_simt(Xq, K, M, K, W, f, ldw, N, nullptr, nullptr, nullptr, nullptr, acc, stream);
 }

@@ -503,6 +503,18 @@ def test_small_m_tensor_core_auto(bl, fmt, M, K, N):
     assert_y_close(Y, ref["Y"])
 
 
+@pytest.mark.parametrize("M,K,N", [(385, 1300, 9500), (129, 700, 19000), (640, 1040, 300)])
+def test_tc_packed_routes(bl, M, K, N):
+    """Packed weights on the tensor cores, both routes: decoded inside the GEMM
+    for up to 4 row tiles of 128 (the first two shapes have enough tiles for the
+    256-wide ones, and K ends inside a packed super-tile of 640 trits), unpacked
+    to int8 once beyond that (the third: one more launch)."""
+    p = random_problem(M + 3 * K + 7 * N, M, K, N)
+    path, n = bl.linear_plan(M, N, K, bl.PACK5, bl.PATH_AUTO)
+    assert path == bl.PATH_TC and n == (3 if M > 4 * 128 else 2)
+    _sampled_check(bl, p, bl.PACK5, n_samples=4096, seed=M)
+
+
 def test_linear_bias(bl):
     p = random_problem(77, 5, 300, 45)
     b = np.random.default_rng(1).standard_normal(45).astype(F32)
