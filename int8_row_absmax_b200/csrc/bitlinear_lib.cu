@@ -171,18 +171,20 @@ bl_status check_ws(const void* ws, size_t ws_bytes, size_t need) {
 // ---- linear --------------------------------------------------------------
 struct LinWs {
   int64_t ldx, ldk;
-  size_t xq_off, s_off, wq_off, total;
+  size_t xq_off, s_off, wq_off, tc_off, total;
 };
 // X_q [M, ldx] and s [M]; with `unpacked_w`, an int8 copy of the packed weights
-// [N, ldk] for the tensor-core path.
-LinWs lin_layout(int64_t M, int64_t K, int64_t N = 0, bool unpacked_w = false) {
+// [N, ldk] for the tensor-core path; then `tc_bytes` for the tensor-core GEMM's
+// K-split partials.
+LinWs lin_layout(int64_t M, int64_t K, int64_t N = 0, bool unpacked_w = false, size_t tc_bytes = 0) {
   LinWs l;
   l.ldx = round_up(K, 16);
   l.ldk = round_up(K, 16);
   l.xq_off = 0;
   l.s_off = align_up(size_t(M) * size_t(l.ldx));
   l.wq_off = l.s_off + align_up(size_t(M) * 4 + 4);
-  l.total = l.wq_off + (unpacked_w ? align_up(size_t(N) * size_t(l.ldk)) : 0);
+  l.tc_off = l.wq_off + (unpacked_w ? align_up(size_t(N) * size_t(l.ldk)) : 0);
+  l.total = l.tc_off + tc_bytes;
   return l;
 }
 
@@ -211,6 +213,31 @@ bl_status check_shape(int64_t M, int64_t K, int64_t N) {
 // 128-row tiles; beyond, they are unpacked to int8 once and the GEMM reads those.
 constexpr int64_t kTcDecodeMaxTilesM = 4;
 bool tc_unpack(int64_t M, bl_wfmt f) { return f == BL_W_PACK5 && ceil_div(M, int64_t(kTcBM)) > kTcDecodeMaxTilesM; }
+
+// K split of the tensor-core GEMM: with fewer 128 x 256 tiles than SMs, each
+// tile's K is cut into `split` ranges of whole 640-wide chunks (at most
+// kTcMaxSplit), whose int32 partial tiles [split, M, N] live in the workspace;
+// tc_reduce_kernel sums them (one more launch).
+// The split is planned for B200's 148 SMs (a fixed figure, so that planning
+// and workspace sizes need no device query; the grid is still capped by the
+// device's own SM count).
+constexpr int64_t kTcSplitSms = 148;
+struct TcSplit {
+  int64_t tiles;
+  int split;
+  size_t bytes;
+};
+TcSplit tc_split(int64_t M, int64_t N, int64_t K) {
+  TcSplit r;
+  r.tiles = ceil_div(M, int64_t(kTcBM)) * ceil_div(N, int64_t(kTcBN));
+  const int64_t nch = ceil_div(ceil_div(K, int64_t(kTcBK)), int64_t(kTcChunk));
+  int64_t sp = kTcSplitSms / (r.tiles > 0 ? r.tiles : 1);
+  if (sp > nch) sp = nch;
+  if (sp > kTcMaxSplit) sp = kTcMaxSplit;
+  r.split = int(sp < 1 ? 1 : sp);
+  r.bytes = r.split > 1 ? align_up(size_t(r.split) * size_t(M) * size_t(N) * 4) : 0;
+  return r;
+}
 constexpr int64_t kTcMinM = 5;     // AUTO: tensor cores above the GEMV's M <= 4 (measured faster than dp4a from M = 5)
 
 // Whether the tensor-core path can take the shape: K at least one 128-byte K
@@ -238,7 +265,8 @@ int resolve_path(int64_t M, int64_t N, int64_t K, bl_wfmt f, int path, int* laun
     n = 1;                    // quantization fused into the GEMV
   } else if (p == BL_PATH_TC) {
     if (!tc_ok) return -1;
-    n = (fused_quant ? 2 : 1) + (tc_unpack(M, f) ? 1 : 0);  // [act_quant,] [unpack,] GEMM
+    // [act_quant,] [unpack,] GEMM [, K-split reduction]
+    n = (fused_quant ? 2 : 1) + (tc_unpack(M, f) ? 1 : 0) + (tc_split(M, N, K).split > 1 ? 1 : 0);
   } else {
     return -1;
   }
@@ -296,37 +324,39 @@ bool make_map_packed(CUtensorMap* map, const void* base, int64_t ldp, int64_t N,
 
 // The tcgen05 GEMM on int8 X_q [M, ldx] and int8 W_q [N, ldw] (or packed W
 // [N, ldw = ldp], decoded inside the kernel).
-template <int kBN, bool kPacked>
+template <bool kPacked>
 bl_status launch_tc(const TcMaps& maps, const TcArgs& a, bool dequant, cudaStream_t st) {
-  const int64_t tiles = int64_t(a.tiles_m) * a.tiles_n;
-  const dim3 grid(unsigned(tiles < num_sms() ? tiles : num_sms()));
-  constexpr int smem = TcCfg<kBN, kPacked>::kSmem;
-  constexpr int threads = TcCfg<kBN, kPacked>::kThreads;
+  const int64_t work = int64_t(a.tiles_m) * a.tiles_n * a.split;
+  const dim3 grid(unsigned(work < num_sms() ? work : num_sms()));
+  constexpr int smem = TcCfg<kPacked>::kSmem;
+  constexpr int threads = TcCfg<kPacked>::kThreads;
   if (dequant) {
-    if (cudaFuncSetAttribute(gemm_tc_kernel<true, kBN, kPacked>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             smem) != cudaSuccess)
+    if (cudaFuncSetAttribute(gemm_tc_kernel<true, kPacked>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+        cudaSuccess)
       return BL_ERR_CUDA;
-    gemm_tc_kernel<true, kBN, kPacked><<<grid, threads, smem, st>>>(maps, a);
+    gemm_tc_kernel<true, kPacked><<<grid, threads, smem, st>>>(maps, a);
   } else {
-    if (cudaFuncSetAttribute(gemm_tc_kernel<false, kBN, kPacked>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             smem) != cudaSuccess)
+    if (cudaFuncSetAttribute(gemm_tc_kernel<false, kPacked>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+        cudaSuccess)
       return BL_ERR_CUDA;
-    gemm_tc_kernel<false, kBN, kPacked><<<grid, threads, smem, st>>>(maps, a);
+    gemm_tc_kernel<false, kPacked><<<grid, threads, smem, st>>>(maps, a);
   }
   return launch_status();
 }
 
 bl_status run_tc(const int8_t* Xq, int64_t ldx, int64_t M, int64_t K, const void* W, int64_t ldw,
                  bool packed, int64_t N, const float* s, const float* beta, const float* bias, float* Y,
-                 int32_t* acc, cudaStream_t st) {
+                 int32_t* acc, void* tcws, size_t tcws_bytes, cudaStream_t st) {
   if (ldx % 16 != 0 || ldw % 16 != 0 || !is_aligned(Xq, 16) || !is_aligned(W, 16))
     return BL_ERR_ALIGNMENT;
-  // 64-wide tiles when the 256-wide ones would leave SMs idle
-  const int bn = ceil_div(M, kTcBM) * ceil_div(N, kTcBN) < num_sms() ? 64 : 256;
-  if (ceil_div(M, kTcBM) * ceil_div(N, bn) > (int64_t(1) << 31) - 1) return BL_ERR_UNSUPPORTED;
+  // no workspace (tcws null): no K split
+  TcSplit sp = tc_split(M, N, K);
+  if (!tcws) sp.split = 1;
+  if (sp.tiles > (int64_t(1) << 28)) return BL_ERR_UNSUPPORTED;
+  if (sp.split > 1 && (!is_aligned(tcws, kWsAlign) || tcws_bytes < sp.bytes)) return BL_ERR_WORKSPACE;
   TcMaps maps;
   if (!make_map_i8(&maps.a, Xq, K, M, ldx, kTcBM)) return BL_ERR_CUDA;
-  if (packed ? !make_map_packed(&maps.b, W, ldw, N, bn) : !make_map_i8(&maps.b, W, K, N, ldw, bn))
+  if (packed ? !make_map_packed(&maps.b, W, ldw, N, kTcBN) : !make_map_i8(&maps.b, W, K, N, ldw, kTcBN))
     return BL_ERR_CUDA;
   TcArgs a;
   a.M = M;
@@ -338,10 +368,19 @@ bl_status run_tc(const int8_t* Xq, int64_t ldx, int64_t M, int64_t K, const void
   a.Y = Y;
   a.acc = acc;
   a.tiles_m = int(ceil_div(M, kTcBM));
-  a.tiles_n = int(ceil_div(N, bn));
+  a.tiles_n = int(ceil_div(N, kTcBN));
+  a.split = sp.split;
+  a.part = sp.split > 1 ? static_cast<int32_t*>(tcws) : nullptr;
   const bool dq = Y != nullptr;
-  if (packed) return bn == 64 ? launch_tc<64, true>(maps, a, dq, st) : launch_tc<256, true>(maps, a, dq, st);
-  return bn == 64 ? launch_tc<64, false>(maps, a, dq, st) : launch_tc<256, false>(maps, a, dq, st);
+  const bl_status r = packed ? launch_tc<true>(maps, a, dq, st) : launch_tc<false>(maps, a, dq, st);
+  if (r != BL_OK || sp.split == 1) return r;
+  const int64_t work = (N % 4 == 0 ? M * (N / 4) : M * N);
+  if (dq)
+    tc_reduce_kernel<true><<<grid_for(work, 256), 256, 0, st>>>(a.part, sp.split, M, N, s, beta, bias, Y, nullptr);
+  else
+    tc_reduce_kernel<false><<<grid_for(work, 256), 256, 0, st>>>(a.part, sp.split, M, N, nullptr, nullptr, nullptr,
+                                                                nullptr, acc);
+  return launch_status();
 }
 
 // Packed weights -> int8 rows in the workspace, for tensor-core GEMMs with more
@@ -603,7 +642,8 @@ bl_status bl_quantize_act(const float* X, int64_t M, int64_t K, float eps, int8_
 size_t bl_linear_ex_workspace_size(int64_t M, int64_t N, int64_t K, bl_wfmt f, int path) {
   if (M < 0 || K < 1 || N < 1) return 0;
   const int p = resolve_path(M, N, K, f, path, nullptr);
-  return lin_layout(M, K, N, p == BL_PATH_TC && tc_unpack(M, f)).total;
+  return lin_layout(M, K, N, p == BL_PATH_TC && tc_unpack(M, f), p == BL_PATH_TC ? tc_split(M, N, K).bytes : 0)
+      .total;
 }
 
 size_t bl_linear_workspace_size(int64_t M, int64_t N, int64_t K, bl_wfmt f) {
@@ -625,7 +665,8 @@ bl_status bl_linear_ex(const float* X, int64_t M, int64_t K, const void* W, bl_w
   if (!is_aligned(X, 4) || !is_aligned(Y, 4) || (bias && !is_aligned(bias, 4))) return BL_ERR_ALIGNMENT;
   const int p = resolve_path(M, N, K, f, path, nullptr, true, ldw, W);
   if (p < 0) return BL_ERR_UNSUPPORTED;
-  const LinWs l = lin_layout(M, K, N, p == BL_PATH_TC && tc_unpack(M, f));
+  const LinWs l =
+      lin_layout(M, K, N, p == BL_PATH_TC && tc_unpack(M, f), p == BL_PATH_TC ? tc_split(M, N, K).bytes : 0);
   if (!ws || !is_aligned(ws, kWsAlign) || ws_bytes < l.total) return BL_ERR_WORKSPACE;
   if (p == BL_PATH_GEMV)
     return run_gemv(X, nullptr, 0, M, K, W, ldw, N, beta_dev, bias, eps, Y, nullptr, stream);
@@ -639,9 +680,11 @@ bl_status bl_linear_ex(const float* X, int64_t M, int64_t K, const void* W, bl_w
       int8_t* scratch = reinterpret_cast<int8_t*>(static_cast<char*>(ws) + l.wq_off);
       st = unpack_rows(static_cast<const uint8_t*>(W), N, K, ldw, scratch, l.ldk, stream);
       if (st != BL_OK) return st;
-      return run_tc(Xq, l.ldx, M, K, scratch, l.ldk, false, N, s, beta_dev, bias, Y, nullptr, stream);
+      return run_tc(Xq, l.ldx, M, K, scratch, l.ldk, false, N, s, beta_dev, bias, Y, nullptr,
+                    static_cast<char*>(ws) + l.tc_off, l.total - l.tc_off, stream);
     }
-    return run_tc(Xq, l.ldx, M, K, W, ldw, f == BL_W_PACK5, N, s, beta_dev, bias, Y, nullptr, stream);
+    return run_tc(Xq, l.ldx, M, K, W, ldw, f == BL_W_PACK5, N, s, beta_dev, bias, Y, nullptr,
+                  static_cast<char*>(ws) + l.tc_off, l.total - l.tc_off, stream);
   }
   return run_simt(Xq, l.ldx, M, K, W, f, ldw, N, s, beta_dev, bias, Y, nullptr, stream);
 }
@@ -678,13 +721,15 @@ bl_status bl_linear_noalloc(const float* X, int64_t M, int64_t K, const void* W,
 size_t bl_linear_acc_workspace_size(int64_t M, int64_t N, int64_t K, bl_wfmt f, int path) {
   if (M < 1 || N < 1 || K < 1) return 0;
   const int p = resolve_path(M, N, K, f, path, nullptr, false);
-  if (p == BL_PATH_TC && tc_unpack(M, f)) return align_up(size_t(N) * size_t(round_up(K, 16)));
-  return 0;
+  if (p != BL_PATH_TC) return 0;
+  return (tc_unpack(M, f) ? align_up(size_t(N) * size_t(round_up(K, 16))) : 0) + tc_split(M, N, K).bytes;
 }
 
-bl_status bl_linear_acc_ex(const int8_t* Xq, int64_t M, int64_t K, const void* W, bl_wfmt f,
-                           int64_t N, int64_t ldw, int32_t* acc, void* ws, size_t ws_bytes,
-                           int path, cudaStream_t stream) {
+// no_ws: bl_linear_acc, which takes no workspace: packed weights are then
+// decoded inside the tensor-core GEMM at any M, and K is not split.
+static bl_status linear_acc_impl(const int8_t* Xq, int64_t M, int64_t K, const void* W, bl_wfmt f, int64_t N,
+                          int64_t ldw, int32_t* acc, void* ws, size_t ws_bytes, int path, bool no_ws,
+                          cudaStream_t stream) {
   bl_status st = check_shape(M, K, N);
   if (st != BL_OK) return st;
   st = check_w(W, f, K, ldw);
@@ -704,23 +749,34 @@ bl_status bl_linear_acc_ex(const int8_t* Xq, int64_t M, int64_t K, const void* W
   if (p == BL_PATH_GEMV)
     return run_gemv(nullptr, Xq, K, M, K, W, ldw, N, nullptr, nullptr, 0.f, nullptr, acc, stream);
   if (p == BL_PATH_TC) {
-    if (tc_unpack(M, f)) {
-      const size_t need = align_up(size_t(N) * size_t(round_up(K, 16)));
-      if (!ws || !is_aligned(ws, kWsAlign) || ws_bytes < need) return BL_ERR_WORKSPACE;
+    const bool unp = !no_ws && tc_unpack(M, f);
+    const size_t wq = unp ? align_up(size_t(N) * size_t(round_up(K, 16))) : 0;
+    const size_t need = no_ws ? 0 : wq + tc_split(M, N, K).bytes;
+    if (need && (!ws || !is_aligned(ws, kWsAlign) || ws_bytes < need)) return BL_ERR_WORKSPACE;
+    void* tcws = need > wq ? static_cast<char*>(ws) + wq : nullptr;
+    const size_t tcb = need > wq ? ws_bytes - wq : 0;
+    if (unp) {
       int8_t* scratch = static_cast<int8_t*>(ws);
       bl_status st2 = unpack_rows(static_cast<const uint8_t*>(W), N, K, ldw, scratch, round_up(K, 16), stream);
       if (st2 != BL_OK) return st2;
       return run_tc(Xq, K, M, K, scratch, round_up(K, 16), false, N, nullptr, nullptr, nullptr, nullptr, acc,
-                    stream);
+                    tcws, tcb, stream);
     }
-    return run_tc(Xq, K, M, K, W, ldw, f == BL_W_PACK5, N, nullptr, nullptr, nullptr, nullptr, acc, stream);
+    return run_tc(Xq, K, M, K, W, ldw, f == BL_W_PACK5, N, nullptr, nullptr, nullptr, nullptr, acc, tcws, tcb,
+                  stream);
   }
   return run_simt(Xq, K, M, K, W, f, ldw, N, nullptr, nullptr, nullptr, nullptr, acc, stream);
 }
 
+bl_status bl_linear_acc_ex(const int8_t* Xq, int64_t M, int64_t K, const void* W, bl_wfmt f,
+                           int64_t N, int64_t ldw, int32_t* acc, void* ws, size_t ws_bytes,
+                           int path, cudaStream_t stream) {
+  return linear_acc_impl(Xq, M, K, W, f, N, ldw, acc, ws, ws_bytes, path, false, stream);
+}
+
 bl_status bl_linear_acc(const int8_t* Xq, int64_t M, int64_t K, const void* W, bl_wfmt f,
                         int64_t N, int64_t ldw, int32_t* acc, cudaStream_t stream) {
-  return bl_linear_acc_ex(Xq, M, K, W, f, N, ldw, acc, nullptr, 0, BL_PATH_AUTO, stream);
+  return linear_acc_impl(Xq, M, K, W, f, N, ldw, acc, nullptr, 0, BL_PATH_AUTO, true, stream);
 }
 
 bl_status bl_sync_status(cudaStream_t stream) {

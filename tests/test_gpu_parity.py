@@ -492,8 +492,9 @@ def test_tc_parity(bl, fmt, M, K, N):
 @pytest.mark.parametrize("fmt", ["i8", "pack5"])
 @pytest.mark.parametrize("M,K,N", [(5, 6912, 2560), (40, 2560, 6912), (127, 1040, 1000), (9, 128, 70)])
 def test_small_m_tensor_core_auto(bl, fmt, M, K, N):
-    """5 <= M < 128 with AUTO: the tcgen05 GEMM with 64-wide tiles (the 256-wide
-    ones would leave SMs idle); ragged N tails inside a 64-wide tile."""
+    """5 <= M < 128 with AUTO: the tcgen05 GEMM with K split across CTAs (few
+    128 x 256 tiles), the partials summed by the reduction kernel; ragged N
+    tails inside a tile."""
     f = bl.PACK5 if fmt == "pack5" else bl.I8
     assert bl.linear_plan(M, N, K, f, bl.PATH_AUTO)[0] == bl.PATH_TC
     p = random_problem(M * 31 + K + N, M, K, N)
@@ -506,12 +507,18 @@ def test_small_m_tensor_core_auto(bl, fmt, M, K, N):
 @pytest.mark.parametrize("M,K,N", [(385, 1300, 9500), (129, 700, 19000), (640, 1040, 300)])
 def test_tc_packed_routes(bl, M, K, N):
     """Packed weights on the tensor cores, both routes: decoded inside the GEMM
-    for up to 4 row tiles of 128 (the first two shapes have enough tiles for the
-    256-wide ones, and K ends inside a packed super-tile of 640 trits), unpacked
-    to int8 once beyond that (the third: one more launch)."""
+    for up to 4 row tiles of 128 (the first two shapes fill the SMs without a K
+    split, and K ends inside a 640-trit chunk), unpacked to int8 once beyond
+    that (the third, whose K is also split in two)."""
     p = random_problem(M + 3 * K + 7 * N, M, K, N)
     path, n = bl.linear_plan(M, N, K, bl.PACK5, bl.PATH_AUTO)
-    assert path == bl.PATH_TC and n == (3 if M > 4 * 128 else 2)
+    # act_quant + GEMM, + unpack beyond 4 row tiles, + the K-split reduction
+    # when there are fewer 128 x 256 tiles than half of 148 SMs (and K has at
+    # least two 640-wide chunks)
+    tiles = -(-M // 128) * -(-N // 256)
+    chunks = -(-(-(-K // 128)) // 5)
+    split = min(148 // tiles, chunks, 8)
+    assert path == bl.PATH_TC and n == 2 + (M > 4 * 128) + (split > 1)
     _sampled_check(bl, p, bl.PACK5, n_samples=4096, seed=M)
 
 
