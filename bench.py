@@ -142,13 +142,34 @@ def measured_peaks():
     return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "source": "fallback"}
 
 
-def kernel_source_hash():
+# The sources a profiled kernel is built from: its header chain, and the lines
+# of the library source that name it (its launcher and launch configuration).
+KERNEL_SOURCES = {
+    "wquant_kernel": (("weight_fused.cuh", "weight_quant.cuh", "act_quant.cuh", "common.cuh", "ptx.cuh"),
+                      ("wquant", "kFu", "fused")),
+}
+
+
+def kernel_source_hash(kernel=None):
+    """Hash of the sources `kernel` is built from (all CUDA sources if it has no
+    entry in KERNEL_SOURCES): a stored ncu figure is used only while it matches."""
     h = hashlib.sha256()
     d = os.path.join(ROOT, "int8_row_absmax_b200", "csrc")
-    for f in sorted(os.listdir(d)):
-        if f.endswith((".cu", ".cuh")):
-            with open(os.path.join(d, f), "rb") as fh:
-                h.update(f.encode() + fh.read())
+    spec = KERNEL_SOURCES.get(kernel)
+    if spec is None:
+        for f in sorted(os.listdir(d)):
+            if f.endswith((".cu", ".cuh")):
+                with open(os.path.join(d, f), "rb") as fh:
+                    h.update(f.encode() + fh.read())
+        return h.hexdigest()[:16]
+    files, keys = spec
+    for f in files:
+        with open(os.path.join(d, f), "rb") as fh:
+            h.update(f.encode() + fh.read())
+    with open(os.path.join(d, "bitlinear_lib.cu")) as fh:
+        for line in fh:
+            if any(k in line for k in keys):
+                h.update(line.encode())
     return h.hexdigest()[:16]
 
 
@@ -161,7 +182,7 @@ def ncu_traffic(kernel: str, workload: int):
     with open(p) as fh:
         d = json.load(fh)
     rec = d.get(f"{kernel}@{workload}")
-    if not rec or rec.get("source_hash") != kernel_source_hash():
+    if not rec or rec.get("source_hash") != kernel_source_hash(kernel):
         return None
     return rec.get("dram_bytes_per_launch")
 

@@ -71,8 +71,11 @@ typedef enum {
   BL_PATH_SIMT = 1, /* dp4a tile kernel: any shape, any format */
   BL_PATH_GEMV = 2, /* packed-trit decode GEMV on CUDA cores: BL_W_PACK5, M <= 4 */
   BL_PATH_TC = 3    /* tcgen05 kind::i8 tensor-core GEMM with fused dequant: K >= 128;
-                       BL_W_I8 rows need ldw % 16 == 0 (packed weights are unpacked
-                       into the workspace first) */
+                       BL_W_I8 rows need ldw % 16 == 0.  Packed weights are decoded
+                       inside the GEMM for M <= 512 and unpacked into the workspace
+                       beyond; with fewer 128 x 256 output tiles than 148, K is split
+                       across CTAs and the int32 partials [split, M, N] go to the
+                       workspace (one more launch sums them; exact) */
 } bl_path;
 
 /* Packed row stride in bytes: ceil(K/5) rounded up to a multiple of 16. */
@@ -195,7 +198,9 @@ int bl_linear_plan(int64_t M, int64_t N, int64_t K, bl_wfmt f, int path, int* la
 
 /* The contraction alone: acc[m,n] = sum_k Xq[m,k] * W_q[n,k] in int32, from
  * pre-quantized activations Xq [M, K] int8 contiguous; acc [M, N] int32.
- * (The integer product x_q W_q^T of the deployed-path equation.) */
+ * (The integer product x_q W_q^T of the deployed-path equation.)  Needs no
+ * workspace: on the tensor cores packed weights are then decoded inside the
+ * GEMM at any M and K is not split. */
 bl_status bl_linear_acc(const int8_t* Xq, int64_t M, int64_t K, const void* W, bl_wfmt f,
                         int64_t N, int64_t ldw, int32_t* acc, cudaStream_t stream);
 
@@ -221,8 +226,10 @@ bl_status bl_linear_acc_ex(const int8_t* Xq, int64_t M, int64_t K, const void* W
  * BL_LINEAR_NOALLOC_SCRATCH_BYTES that every GPU loading the library holds until
  * the process exits.  Nothing is allocated: no cudaMalloc, cudaFree or
  * allocating library routine is called.
- *   - Shapes whose bl_linear_workspace_size(M, N, K, f) exceeds the array are
- *     rejected with BL_ERR_WORKSPACE before anything is launched.
+ *   - Shapes whose bl_linear_workspace_size(M, N, K, f) exceeds the array run
+ *     the tensor-core GEMM without its K split (whose partials are most of
+ *     that workspace) if the rest fits; otherwise they are rejected with
+ *     BL_ERR_WORKSPACE before anything is launched.
  *   - The first call on each device looks up the array's device address with
  *     cudaGetSymbolAddress (with that device current); make that first call
  *     before any stream capture.

@@ -646,14 +646,21 @@ size_t bl_linear_ex_workspace_size(int64_t M, int64_t N, int64_t K, bl_wfmt f, i
       .total;
 }
 
+// bl_linear's workspace without the tensor-core K split's partials.
+static size_t linear_ws_nosplit(int64_t M, int64_t N, int64_t K, bl_wfmt f) {
+  const int p = resolve_path(M, N, K, f, BL_PATH_AUTO, nullptr);
+  return lin_layout(M, K, N, p == BL_PATH_TC && tc_unpack(M, f), 0).total;
+}
+
 size_t bl_linear_workspace_size(int64_t M, int64_t N, int64_t K, bl_wfmt f) {
   return bl_linear_ex_workspace_size(M, N, K, f, BL_PATH_AUTO);
 }
 
-bl_status bl_linear_ex(const float* X, int64_t M, int64_t K, const void* W, bl_wfmt f,
-                       int64_t N, int64_t ldw, const float* beta_dev, const float* bias,
-                       float eps, float* Y, void* ws, size_t ws_bytes, int path,
-                       cudaStream_t stream) {
+// allow_split = false: the tensor-core GEMM runs without a K split (no partials
+// in the workspace), for bl_linear_noalloc when the split would not fit.
+static bl_status linear_impl(const float* X, int64_t M, int64_t K, const void* W, bl_wfmt f, int64_t N,
+                             int64_t ldw, const float* beta_dev, const float* bias, float eps, float* Y,
+                             void* ws, size_t ws_bytes, int path, bool allow_split, cudaStream_t stream) {
   bl_status st = check_shape(M, K, N);
   if (st != BL_OK) return st;
   if (!eps_ok(eps)) return BL_ERR_INVALID_ARG;
@@ -665,9 +672,10 @@ bl_status bl_linear_ex(const float* X, int64_t M, int64_t K, const void* W, bl_w
   if (!is_aligned(X, 4) || !is_aligned(Y, 4) || (bias && !is_aligned(bias, 4))) return BL_ERR_ALIGNMENT;
   const int p = resolve_path(M, N, K, f, path, nullptr, true, ldw, W);
   if (p < 0) return BL_ERR_UNSUPPORTED;
-  const LinWs l =
-      lin_layout(M, K, N, p == BL_PATH_TC && tc_unpack(M, f), p == BL_PATH_TC ? tc_split(M, N, K).bytes : 0);
+  const size_t tcb = (p == BL_PATH_TC && allow_split) ? tc_split(M, N, K).bytes : 0;
+  const LinWs l = lin_layout(M, K, N, p == BL_PATH_TC && tc_unpack(M, f), tcb);
   if (!ws || !is_aligned(ws, kWsAlign) || ws_bytes < l.total) return BL_ERR_WORKSPACE;
+  void* tcws = tcb ? static_cast<char*>(ws) + l.tc_off : nullptr;   // null: no K split
   if (p == BL_PATH_GEMV)
     return run_gemv(X, nullptr, 0, M, K, W, ldw, N, beta_dev, bias, eps, Y, nullptr, stream);
   int8_t* Xq = reinterpret_cast<int8_t*>(static_cast<char*>(ws) + l.xq_off);
@@ -680,13 +688,18 @@ bl_status bl_linear_ex(const float* X, int64_t M, int64_t K, const void* W, bl_w
       int8_t* scratch = reinterpret_cast<int8_t*>(static_cast<char*>(ws) + l.wq_off);
       st = unpack_rows(static_cast<const uint8_t*>(W), N, K, ldw, scratch, l.ldk, stream);
       if (st != BL_OK) return st;
-      return run_tc(Xq, l.ldx, M, K, scratch, l.ldk, false, N, s, beta_dev, bias, Y, nullptr,
-                    static_cast<char*>(ws) + l.tc_off, l.total - l.tc_off, stream);
+      return run_tc(Xq, l.ldx, M, K, scratch, l.ldk, false, N, s, beta_dev, bias, Y, nullptr, tcws, tcb, stream);
     }
-    return run_tc(Xq, l.ldx, M, K, W, ldw, f == BL_W_PACK5, N, s, beta_dev, bias, Y, nullptr,
-                  static_cast<char*>(ws) + l.tc_off, l.total - l.tc_off, stream);
+    return run_tc(Xq, l.ldx, M, K, W, ldw, f == BL_W_PACK5, N, s, beta_dev, bias, Y, nullptr, tcws, tcb, stream);
   }
   return run_simt(Xq, l.ldx, M, K, W, f, ldw, N, s, beta_dev, bias, Y, nullptr, stream);
+}
+
+bl_status bl_linear_ex(const float* X, int64_t M, int64_t K, const void* W, bl_wfmt f,
+                       int64_t N, int64_t ldw, const float* beta_dev, const float* bias,
+                       float eps, float* Y, void* ws, size_t ws_bytes, int path,
+                       cudaStream_t stream) {
+  return linear_impl(X, M, K, W, f, N, ldw, beta_dev, bias, eps, Y, ws, ws_bytes, path, true, stream);
 }
 
 int bl_linear_plan(int64_t M, int64_t N, int64_t K, bl_wfmt f, int path, int* launches) {
@@ -710,12 +723,13 @@ bl_status bl_linear_noalloc(const float* X, int64_t M, int64_t K, const void* W,
   if (!eps_ok(eps)) return BL_ERR_INVALID_ARG;
   if ((st = check_w(W, f, K, ldw)) != BL_OK) return st;
   if (M == 0) return BL_OK;
-  const size_t need = bl_linear_workspace_size(M, N, K, f);
-  if (need > BL_LINEAR_NOALLOC_SCRATCH_BYTES) return BL_ERR_WORKSPACE;
+  // the tensor-core K split only if its partials fit the array as well
+  const bool split = bl_linear_workspace_size(M, N, K, f) <= BL_LINEAR_NOALLOC_SCRATCH_BYTES;
+  if (!split && linear_ws_nosplit(M, N, K, f) > BL_LINEAR_NOALLOC_SCRATCH_BYTES) return BL_ERR_WORKSPACE;
   void* scratch = noalloc_scratch_ptr();
   if (!scratch) return BL_ERR_CUDA;
-  return bl_linear_ex(X, M, K, W, f, N, ldw, beta_dev, bias, eps, Y, scratch,
-                      BL_LINEAR_NOALLOC_SCRATCH_BYTES, BL_PATH_AUTO, stream);
+  return linear_impl(X, M, K, W, f, N, ldw, beta_dev, bias, eps, Y, scratch, BL_LINEAR_NOALLOC_SCRATCH_BYTES,
+                     BL_PATH_AUTO, split, stream);
 }
 
 size_t bl_linear_acc_workspace_size(int64_t M, int64_t N, int64_t K, bl_wfmt f, int path) {

@@ -65,3 +65,23 @@ def test_noalloc_rejects_shapes_beyond_its_scratch(bl):
     code = lib.bl_linear_noalloc(X.data_ptr(), M, K, W.data_ptr(), bl.PACK5, 16, W.shape[1],
                                  beta.data_ptr(), None, 1e-5, Y.data_ptr(), None)
     assert bl.STATUS[code] == "BL_ERR_WORKSPACE"
+
+
+def test_noalloc_drops_the_k_split_when_its_partials_do_not_fit(bl):
+    """M = 512, K = 11008, N = 4096 on the tensor cores: 64 tiles of 128 x 256, so
+    bl_linear splits K in two and its workspace (5.6 MB of X_q + 16.8 MB of
+    int32 partials) exceeds the 16 MB array; bl_linear_noalloc runs the GEMM
+    unsplit instead and must give the same Y (integer sums are exact)."""
+    import torch
+    M, K, N = 512, 11008, 4096
+    lib = bl.load()
+    assert lib.bl_linear_workspace_size(M, N, K, bl.PACK5) > bl.NOALLOC_SCRATCH_BYTES
+    rng = np.random.default_rng(11)
+    W = torch.from_numpy(rng.standard_normal((N, K), dtype=np.float32) * np.float32(0.02)).cuda()
+    Wd, beta = bl.quantize_weights_pack5(W, 1e-5)
+    X = torch.from_numpy(rng.standard_normal((M, K), dtype=np.float32)).cuda()
+    ref = bl.linear(X, Wd, bl.PACK5, N, K, beta, eps=1e-5)
+    Y = torch.full((M, N), float("nan"), dtype=torch.float32, device="cuda")
+    assert _noalloc(bl, X, Wd, bl.PACK5, N, K, beta, Y, 1e-5) == 0
+    assert bl.sync_status() == "BL_OK"
+    np.testing.assert_array_equal(Y.cpu().numpy(), ref.cpu().numpy())
