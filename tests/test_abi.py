@@ -112,3 +112,39 @@ NULL = None
 ])
 def test_host_validation(lib, case, expect):
     assert case(lib) == expect
+
+
+def _cdiv(a, b):
+    return -(-a // b)
+
+
+def _al(v):
+    return _cdiv(v, 256) * 256
+
+
+@pytest.mark.parametrize("M,K,N", [(5, 8192, 8192), (64, 2560, 6912), (129, 700, 19000), (512, 4096, 11008),
+                                   (640, 1040, 300), (4096, 4096, 11008), (8, 128, 256), (300, 1000, 1000)])
+def test_tensor_core_plan_and_workspace(lib, M, K, N):
+    """The tensor-core plan, on the host: act_quant + GEMM, + the unpack of packed
+    weights beyond 4 row tiles of 128, + the reduction of a K split, which is
+    taken when the 128 x 256 tiles are fewer than half of 148 SMs and K has at
+    least two 640-wide chunks (at most 8 splits).  The workspace holds X_q [M,
+    ldx] and s, then the int8 copy of W_q, then the split's int32 partials."""
+    tiles = _cdiv(M, 128) * _cdiv(N, 256)
+    split = max(1, min(148 // tiles, _cdiv(_cdiv(K, 128), 5), 8))
+    n = ctypes.c_int(0)
+    assert lib.bl_linear_plan(M, N, K, pkg.PACK5, pkg.PATH_TC, ctypes.byref(n)) == pkg.PATH_TC
+    assert n.value == 2 + (M > 512) + (split > 1)
+    ldx = _cdiv(K, 16) * 16
+    extra = (_al(N * ldx) if M > 512 else 0) + (_al(split * M * N * 4) if split > 1 else 0)
+    assert lib.bl_linear_ex_workspace_size(M, N, K, pkg.PACK5, pkg.PATH_TC) == _al(M * ldx) + _al(M * 4 + 4) + extra
+    assert lib.bl_linear_acc_workspace_size(M, N, K, pkg.PACK5, pkg.PATH_TC) == extra
+
+
+def test_auto_path_crossover(lib):
+    """AUTO: the decode GEMV for M <= 4 (packed weights), the tensor cores from M = 5."""
+    n = ctypes.c_int(0)
+    for M in (1, 2, 3, 4):
+        assert lib.bl_linear_plan(M, 4096, 4096, pkg.PACK5, pkg.PATH_AUTO, ctypes.byref(n)) == pkg.PATH_GEMV
+    for M in (5, 8, 100, 4096):
+        assert lib.bl_linear_plan(M, 4096, 4096, pkg.PACK5, pkg.PATH_AUTO, ctypes.byref(n)) == pkg.PATH_TC

@@ -522,6 +522,25 @@ def test_tc_packed_routes(bl, M, K, N):
     _sampled_check(bl, p, bl.PACK5, n_samples=4096, seed=M)
 
 
+def test_linear_acc_without_workspace_decodes_in_the_gemm(bl):
+    """bl_linear_acc takes no workspace: at M = 640 (5 row tiles) with packed
+    weights the tensor-core GEMM then decodes the trits itself instead of
+    reading an unpacked copy, and K is not split; acc must equal the exact
+    contraction."""
+    import torch
+    M, K, N = 640, 1040, 300
+    p = random_problem(M + K + N + 5, M, K, N)
+    Wd, beta = bl.quantize_weights_pack5(dev(p.W), p.eps)
+    Xq, _ = oracle.act_quant(p.X, p.eps)
+    Xd = dev(Xq)
+    acc = torch.empty((M, N), dtype=torch.int32, device="cuda")
+    st = bl.load().bl_linear_acc(Xd.data_ptr(), M, K, Wd.data_ptr(), bl.PACK5, N, Wd.shape[1],
+                                 acc.data_ptr(), None)
+    assert bl.STATUS[st] == "BL_OK"
+    check_ok(bl)
+    np.testing.assert_array_equal(host(acc), oracle.contract(Xq, oracle.ternarize(p.W, host(beta)[0])))
+
+
 def test_linear_bias(bl):
     p = random_problem(77, 5, 300, 45)
     b = np.random.default_rng(1).standard_normal(45).astype(F32)
