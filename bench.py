@@ -22,6 +22,12 @@ none sit inside the timed step graphs).  SM clocks and throttle reasons are
 sampled through NVML during the timed region.  `e2e` repeats the step through the public Python API
 with the step's inputs copied from pinned host memory and Y copied back.
 
+Roofline: the dominant call's algorithmic bytes over its live duration against
+the measured HBM copy rate; when every contraction of the step runs on the
+int8 tensor cores (M >= 5), int8 operations over the live duration of the
+bl_linear calls against the measured sustained bf16 GEMM rate x 2 instead (the
+HBM figure then moves to `roofline_weight_path`).
+
 Under torchrun each rank runs its own independently seeded batch (weak
 scaling, no data-path collective); only the timing reduction crosses ranks.
 `--impl reference` times the CPU oracle instead (rank 0 only).
@@ -138,8 +144,24 @@ def measured_peaks():
         with open(p) as fh:
             d = json.load(fh)
         return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]),
+                "bf16_tflops_sustained": float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
                 "source": "measured"}
-    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "source": "fallback"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+def tensor_roofline(macs, ms, peaks):
+    """Roofline of a step whose contractions all run on the int8 tensor cores:
+    int8 operations (2 per multiply-add) per second over the live duration of
+    the bl_linear calls, against the measured sustained bf16 GEMM rate times 2
+    (the nominal dense int8 : bf16 ratio, 4.5 : 2.25 PFLOP/s)."""
+    achieved = 2.0 * macs / (ms * 1e-3) / 1e12
+    peak = 2.0 * peaks["bf16_tflops_sustained"]
+    return {"bound": "tensor", "achieved": round(achieved, 1), "peak": round(peak, 1), "unit": "TFLOP/s",
+            "frac": round(achieved / peak, 4), "traffic": None, "kernel": "gemm_tc_kernel", "call": "bl_linear",
+            "ops": "int8: 2 per multiply-add, over whole bl_linear calls (activation quantization, "
+                   "[unpack,] GEMM [, K-split reduction])",
+            "peak_source": ("measured sustained bf16 x 2 (MEASURED_PEAKS.json bf16_tflops_sustained)"
+                            if peaks["source"] == "measured" else "fallback 1.4 PFLOP/s bf16 sustained x 2")}
 
 
 # The sources a profiled kernel is built from: its header chain, and the lines
@@ -477,6 +499,11 @@ def run_ours(args):
     }
     if line["linear_only"] is not None:
         line["linear_only"]["frac_hbm"] = round(line["linear_only"]["weight_stream_gbs"] / peaks["hbm_gbs"], 4)
+    # every contraction on the tensor cores: the step is bound by them, not by HBM
+    if lin is not None and all(bl.linear_plan(c[4], c[6], c[5], fmt, args.path)[0] == bl.PATH_TC
+                               for c in first.calls):
+        line["roofline_weight_path"] = roofline
+        line["roofline"] = tensor_roofline(macs_per_step, lin["ms"], peaks)
 
     # ---- end to end through the public API, host buffers -------------------
     line["e2e"] = e2e(bl, torch, probs, dev, fmt, args.e2e_steps, world)
