@@ -14,14 +14,15 @@ What it computes, and where the method is stated (page title, then section):
 * ``act_quant`` -- same page, section "the bytes" and the per-token fix in
   section "attention, as graph ops": s = max_i |x_i| / 127 + eps per row,
   x_q = clip(round(x / s), -127, 127), the symmetric range [-127, 127].
-* ``contract`` and ``dequant`` -- same page, section "autograd on a byte-graph",
-  deployed-path equation y = (x_q W_q^T)(s beta) + b: an integer matmul, then
+* ``contract`` (and ``contract_f64``, the same product by a float64 matmul
+  that is exact for these integer codes) and ``dequant`` -- same page, section
+  "autograd on a byte-graph", deployed-path equation y = (x_q W_q^T)(s beta) + b: an integer matmul, then
   one rescale by the row scale times beta.
 * ``pack5`` / ``unpack5`` -- "ultragraph-1bit 0.12.0" (PyPI), sections "A whole
   ternary GPT" and "Layout" (5 ternary values per byte, ~1.6 bits/weight), and
   "a 1-bit llm, from scratch", tl;dr (1.6 bits each).  Byte = sum_k (t_k+1) 3^k.
 
-Readings where the pages leave a step open (each is also listed in the design doc):
+Readings taken where the pages leave a step open:
 
 1. Precision.  The pages' arrays are numpy float32, so every quantizer step is
    IEEE-754 float32 with round-to-nearest-even, in the order written.
@@ -47,6 +48,7 @@ from .layer import (  # noqa: F401
     act_quant,
     bitlinear,
     contract,
+    contract_f64,
     contract_entries,
     dequant,
     pack5,

@@ -111,6 +111,24 @@ def contract(Xq: np.ndarray, Wq: np.ndarray) -> np.ndarray:
     return acc.astype(np.int32)
 
 
+def contract_f64(Xq: np.ndarray, Wq: np.ndarray) -> np.ndarray:
+    """acc = x_q W_q^T as a float64 matrix product of the integer codes.
+
+    The same definition as ``contract``, for full-size cases where an int64
+    product is too slow: every product and every partial sum is an integer of
+    magnitude at most 127 * K, far below 2^53, so float64 represents each one
+    exactly and the result does not depend on how the library orders the sum.
+    """
+    Xq = np.asarray(Xq)
+    Wq = np.asarray(Wq)
+    if 127 * Xq.shape[1] >= 2 ** 53:
+        raise OverflowError("partial sums may exceed 2^53")
+    acc = Xq.astype(np.float64) @ Wq.astype(np.float64).T
+    if acc.size and np.max(np.abs(acc)) >= 2 ** 31:
+        raise OverflowError("accumulator exceeds int32")
+    return acc.astype(np.int32)
+
+
 def contract_entries(Xq_rows: np.ndarray, Wq_rows: np.ndarray) -> np.ndarray:
     """Selected outputs one by one: acc_i = sum_k Xq_rows[i,k] * Wq_rows[i,k]."""
     a = np.asarray(Xq_rows).astype(np.int64)

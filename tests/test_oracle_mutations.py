@@ -70,6 +70,10 @@ def _contract_transposed_w(Xq, Wq):
     return (np.asarray(Xq).astype(np.int64) @ Wq.astype(np.int64).T).astype(np.int32)
 
 
+def _contract_f64_no_widening(Xq, Wq):
+    return (np.asarray(Xq) @ np.asarray(Wq).T).astype(np.int32)   # int8 sums wrap
+
+
 def _dequant_acc_times_s_first(acc, s, beta, bias=None):
     y = (np.asarray(acc).astype(F32) * np.asarray(s, F32).reshape(-1, 1)) * F32(beta)
     return y if bias is None else y + np.asarray(bias, F32)
@@ -85,6 +89,7 @@ MUTANTS = {
     "act_quant": [_act_quant_half_away, _act_quant_per_tensor, _act_quant_128],
     "pack5": [_pack_big_endian],
     "contract": [_contract_transposed_w],
+    "contract_f64": [_contract_f64_no_widening],
     "dequant": [_dequant_acc_times_s_first],
 }
 

@@ -218,6 +218,28 @@ def test_contract_extremes():
     assert acc.tolist() == [[127 * K, -127 * K], [-127 * K, 127 * K]]
 
 
+def test_contract_f64_equals_integer_contract():
+    """The float64 product of the codes is the exact integer product: random
+    codes, the extremes, and a column-sliced (transposition-sensitive) case."""
+    rng = np.random.default_rng(57)
+    for M, N, K in ((7, 5, 33), (16, 16, 1000), (3, 40, 6912)):
+        Xq = rng.integers(-127, 128, (M, K)).astype(np.int8)
+        Wq = rng.integers(-1, 2, (N, K)).astype(np.int8)
+        np.testing.assert_array_equal(oracle.contract_f64(Xq, Wq), oracle.contract(Xq, Wq))
+        np.testing.assert_array_equal(oracle.contract_f64(Xq[:, :K // 2], Wq[:, :K // 2]),
+                                      oracle.contract(Xq[:, :K // 2], Wq[:, :K // 2]))
+    K = 131072
+    Xq = np.full((2, K), 127, np.int8)
+    Xq[1] = -127
+    Wq = np.ones((2, K), np.int8)
+    Wq[1, ::2] = -1
+    acc = oracle.contract_f64(Xq, Wq)
+    assert acc.tolist() == [[127 * K, 0], [-127 * K, 0]]
+    sq = rng.integers(-1, 2, (9, 9)).astype(np.int8)
+    xs = rng.integers(-127, 128, (4, 9)).astype(np.int8)
+    assert np.array_equal(oracle.contract_f64(xs, sq), oracle.contract(xs, sq))
+
+
 # ---------------------------------------------------------------- dequant ---
 @pytest.mark.parametrize("case", GOLD["dequant"], ids=lambda c: c["name"])
 def test_dequant_hand_worked(case):
