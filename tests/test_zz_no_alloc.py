@@ -77,11 +77,20 @@ def test_noalloc_drops_the_k_split_when_its_partials_do_not_fit(bl):
     lib = bl.load()
     assert lib.bl_linear_workspace_size(M, N, K, bl.PACK5) > bl.NOALLOC_SCRATCH_BYTES
     rng = np.random.default_rng(11)
-    W = torch.from_numpy(rng.standard_normal((N, K), dtype=np.float32) * np.float32(0.02)).cuda()
-    Wd, beta = bl.quantize_weights_pack5(W, 1e-5)
-    X = torch.from_numpy(rng.standard_normal((M, K), dtype=np.float32)).cuda()
+    Wh = rng.standard_normal((N, K), dtype=np.float32) * np.float32(0.02)
+    Xh = rng.standard_normal((M, K), dtype=np.float32)
+    Wd, beta = bl.quantize_weights_pack5(torch.from_numpy(Wh).cuda(), 1e-5)
+    X = torch.from_numpy(Xh).cuda()
     ref = bl.linear(X, Wd, bl.PACK5, N, K, beta, eps=1e-5)
     Y = torch.full((M, N), float("nan"), dtype=torch.float32, device="cuda")
     assert _noalloc(bl, X, Wd, bl.PACK5, N, K, beta, Y, 1e-5) == 0
     assert bl.sync_status() == "BL_OK"
-    np.testing.assert_array_equal(Y.cpu().numpy(), ref.cpu().numpy())
+    got = Y.cpu().numpy()
+    np.testing.assert_array_equal(got, ref.cpu().numpy())
+    # and every element against the oracle itself
+    import oracle
+    rb = oracle.absmean_beta(Wh, 1e-5)
+    assert beta.cpu().numpy()[0] == rb
+    Xq, s = oracle.act_quant(Xh, 1e-5)
+    acc = oracle.contract_f64(Xq, oracle.ternarize(Wh, rb))
+    np.testing.assert_array_equal(got, oracle.dequant(acc, s, rb))
