@@ -69,7 +69,8 @@ typedef enum {
 typedef enum {
   BL_PATH_AUTO = 0, /* dispatch on M, K, N and the format */
   BL_PATH_SIMT = 1, /* dp4a tile kernel: any shape, any format */
-  BL_PATH_GEMV = 2, /* packed-trit decode GEMV on CUDA cores: BL_W_PACK5, M <= 4 */
+  BL_PATH_GEMV = 2, /* packed-trit decode GEMV on CUDA cores: BL_W_PACK5, M <= 4; one
+                       launch, activation quantization inside */
   BL_PATH_TC = 3    /* tcgen05 kind::i8 tensor-core GEMM with fused dequant: K >= 128;
                        BL_W_I8 rows need ldw % 16 == 0.  Packed weights are decoded
                        inside the GEMM for M <= 512 and unpacked into the workspace
@@ -77,6 +78,19 @@ typedef enum {
                        across CTAs and the int32 partials [split, M, N] go to the
                        workspace (one more launch sums them; exact) */
 } bl_path;
+
+/* Flags OR'd into the `path` argument of bl_linear_ex and bl_linear_acc_ex,
+ * and passed as `flags` to bl_linear_group.
+ *
+ * BL_FLAG_STATIC_WEIGHTS: the caller guarantees that W is not written by any
+ * kernel that may still be running when the call is issued (for instance
+ * weights quantized once and only read while decoding).  The decode GEMV is
+ * launched with programmatic dependent launch in every case, so its prologue
+ * overlaps the previous kernel on the stream; with this flag it also starts
+ * copying W into shared memory before that kernel has finished, and waits for
+ * it only before reading X and writing Y.  Results are identical with and
+ * without the flag; a call that breaks the guarantee may read stale weights. */
+#define BL_FLAG_STATIC_WEIGHTS 0x100
 
 /* Packed row stride in bytes: ceil(K/5) rounded up to a multiple of 16. */
 int64_t bl_pack5_ldp(int64_t K);
@@ -140,7 +154,8 @@ bl_status bl_unpack(const uint8_t* Wp, int64_t N, int64_t K, int64_t ldp, int8_t
 bl_status bl_quantize_act(const float* X, int64_t M, int64_t K, float eps, int8_t* Xq,
                           float* s, cudaStream_t stream);
 
-/* Bytes of `ws` that bl_linear needs for this shape and format. */
+/* Bytes of `ws` that bl_linear needs for this shape and format (0 for shapes
+ * that take the decode GEMV: ws may then be NULL). */
 size_t bl_linear_workspace_size(int64_t M, int64_t N, int64_t K, bl_wfmt f);
 
 /* Bytes of `ws` that bl_linear_ex needs with kernel path `path` pinned. */
@@ -154,7 +169,8 @@ size_t bl_linear_ex_workspace_size(int64_t M, int64_t N, int64_t K, bl_wfmt f, i
  *   beta_dev the tensor's beta on the device (from bl_quantize_weights*).
  *   bias     [N] float32 or NULL.
  *   Y        [M, N] float32 contiguous output.
- *   ws       >= bl_linear_workspace_size(M, N, K, f) bytes, 256-byte aligned. */
+ *   ws       >= bl_linear_workspace_size(M, N, K, f) bytes, 256-byte aligned
+ *            (NULL when that size is 0). */
 bl_status bl_linear(const float* X, int64_t M, int64_t K, const void* W, bl_wfmt f, int64_t N,
                     int64_t ldw, const float* beta_dev, const float* bias, float eps, float* Y,
                     void* ws, size_t ws_bytes, cudaStream_t stream);
@@ -183,8 +199,9 @@ bl_status bl_bitlinear_forward(const float* X, int64_t M, int64_t K, const float
                                const float* bias, float* Y, void* ws, size_t ws_bytes,
                                cudaStream_t stream);
 
-/* bl_linear with the kernel path pinned (BL_PATH_*); BL_ERR_UNSUPPORTED when the
- * pinned path cannot take the shape.  Results are identical across paths. */
+/* bl_linear with the kernel path pinned (BL_PATH_*, optionally OR'd with
+ * BL_FLAG_STATIC_WEIGHTS); BL_ERR_UNSUPPORTED when the pinned path cannot take
+ * the shape.  Results are identical across paths. */
 bl_status bl_linear_ex(const float* X, int64_t M, int64_t K, const void* W, bl_wfmt f,
                        int64_t N, int64_t ldw, const float* beta_dev, const float* bias,
                        float eps, float* Y, void* ws, size_t ws_bytes, int path,
@@ -210,6 +227,36 @@ size_t bl_linear_acc_workspace_size(int64_t M, int64_t N, int64_t K, bl_wfmt f, 
 bl_status bl_linear_acc_ex(const int8_t* Xq, int64_t M, int64_t K, const void* W, bl_wfmt f,
                            int64_t N, int64_t ldw, int32_t* acc, void* ws, size_t ws_bytes,
                            int path, cudaStream_t stream);
+
+/* One call of bl_linear_group: the arguments of bl_linear, minus the workspace. */
+typedef struct {
+  const float* X;        /* [M, K] float32 */
+  int64_t M, K;
+  const void* W;         /* weights in format f, [N, ldw] */
+  int64_t N, ldw;
+  bl_wfmt f;
+  float eps;
+  const float* beta_dev;
+  const float* bias;     /* [N] or NULL */
+  float* Y;              /* [M, N] float32 */
+} bl_linear_call;
+
+/* Bytes of `ws` that bl_linear_group needs for these calls (0 when every call
+ * takes the decode GEMV). */
+size_t bl_linear_group_workspace_size(const bl_linear_call* calls, int count);
+
+/* Several independent BitLinear forwards (deployed-path equation, as bl_linear)
+ * in as few launches as possible: the calls that take the decode GEMV (packed
+ * weights, M <= 4) run in one launch per M, up to four problems each, so their
+ * weight streams share one grid (for instance the projections of one decode
+ * step that read the same or separate activations); the other calls run as
+ * bl_linear would, each with its own part of `ws`.  Results are bit-identical
+ * to `count` bl_linear calls.  The calls must be independent: no call's Y may
+ * overlap another call's X, W, beta, bias or Y.  `flags`: 0 or
+ * BL_FLAG_STATIC_WEIGHTS.  Every call is validated before anything launches;
+ * errors as for bl_linear. */
+bl_status bl_linear_group(const bl_linear_call* calls, int count, int flags, void* ws, size_t ws_bytes,
+                          cudaStream_t stream);
 
 /* Size of the scratch array built into the library for bl_linear_noalloc. */
 #define BL_LINEAR_NOALLOC_SCRATCH_BYTES ((size_t)16 << 20)

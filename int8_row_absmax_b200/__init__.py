@@ -20,6 +20,7 @@ LIB_PATH = os.path.join(PKG_DIR, "libbitlinear.so")
 
 I8, PACK5 = 0, 1                       # bl_wfmt
 PATH_AUTO, PATH_SIMT, PATH_GEMV, PATH_TC = 0, 1, 2, 3   # bl_path
+FLAG_STATIC_WEIGHTS = 0x100            # BL_FLAG_STATIC_WEIGHTS
 
 STATUS = {0: "BL_OK", 1: "BL_ERR_INVALID_ARG", 2: "BL_ERR_ALIGNMENT", 3: "BL_ERR_UNSUPPORTED",
           4: "BL_ERR_WORKSPACE", 5: "BL_ERR_CUDA", 6: "BL_ERR_DEVICE_TIMEOUT",
@@ -27,6 +28,15 @@ STATUS = {0: "BL_OK", 1: "BL_ERR_INVALID_ARG", 2: "BL_ERR_ALIGNMENT", 3: "BL_ERR
 
 # Every symbol the header declares, with (restype, argtypes).
 _P, _I64, _SZ, _F, _I = ctypes.c_void_p, ctypes.c_int64, ctypes.c_size_t, ctypes.c_float, ctypes.c_int
+
+
+class LinearCall(ctypes.Structure):
+    """bl_linear_call: one call of bl_linear_group (field order and types as in the header)."""
+    _fields_ = [("X", _P), ("M", _I64), ("K", _I64), ("W", _P), ("N", _I64), ("ldw", _I64),
+                ("f", _I), ("eps", _F), ("beta_dev", _P), ("bias", _P), ("Y", _P)]
+
+
+_CALLS = ctypes.POINTER(LinearCall)
 SIGNATURES = {
     "bl_pack5_ldp": (_I64, [_I64]),
     "bl_quantize_weights_workspace_size": (_SZ, [_I64, _I64]),
@@ -42,6 +52,8 @@ SIGNATURES = {
     "bl_linear_ex_workspace_size": (_SZ, [_I64, _I64, _I64, _I, _I]),
     "bl_linear": (_I, [_P, _I64, _I64, _P, _I, _I64, _I64, _P, _P, _F, _P, _P, _SZ, _P]),
     "bl_linear_ex": (_I, [_P, _I64, _I64, _P, _I, _I64, _I64, _P, _P, _F, _P, _P, _SZ, _I, _P]),
+    "bl_linear_group_workspace_size": (_SZ, [_CALLS, _I]),
+    "bl_linear_group": (_I, [_CALLS, _I, _I, _P, _SZ, _P]),
     "bl_linear_noalloc": (_I, [_P, _I64, _I64, _P, _I, _I64, _I64, _P, _P, _F, _P, _P]),
     "bl_bitlinear_forward_workspace_size": (_SZ, [_I64, _I64, _I64, _I]),
     "bl_bitlinear_forward": (_I, [_P, _I64, _I64, _P, _I, _I64, _F, _P, _I64, _P, _P, _P, _P, _SZ, _P]),
@@ -224,20 +236,58 @@ def linear_workspace_size(M: int, N: int, K: int, fmt: int) -> int:
 
 
 def linear(X, W, fmt: int, N: int, K: int, beta, bias=None, eps: float = 1e-5,
-           path: int = PATH_AUTO, ws=None, out=None):
-    """Y = (X_q W_q^T)(s beta) + bias for X [M,K] float32 and W in format fmt."""
+           path: int = PATH_AUTO, ws=None, out=None, static_weights: bool = False):
+    """Y = (X_q W_q^T)(s beta) + bias for X [M,K] float32 and W in format fmt.
+    static_weights: W is not written by a kernel still in flight (BL_FLAG_STATIC_WEIGHTS)."""
     torch, lib = _torch(), load()
+    path = path | (FLAG_STATIC_WEIGHTS if static_weights else 0)
     _dev(X, torch.float32)
     M = X.shape[0]
     if X.shape[1] != K or W.shape[0] != N:
         raise ValueError("shape mismatch")
     Y = torch.empty((M, N), dtype=torch.float32, device=X.device) if out is None else out
     need = lib.bl_linear_ex_workspace_size(M, N, K, fmt, path)
-    ws = workspace(need, X.device) if ws is None else ws
+    if ws is None and need:
+        ws = workspace(need, X.device)
     _check("bl_linear_ex", lib.bl_linear_ex(
         _ptr(X), M, K, _ptr(W), fmt, N, W.shape[1], _ptr(beta), _ptr(bias), eps, _ptr(Y),
-        _ptr(ws), ws.numel(), path, _stream(torch, X)))
+        _ptr(ws), 0 if ws is None else ws.numel(), path, _stream(torch, X)))
     return Y
+
+
+def _call_array(calls, outs=None):
+    torch = _torch()
+    arr = (LinearCall * max(1, len(calls)))()
+    Ys = []
+    for i, (X, W, fmt, N, K, beta, bias, eps) in enumerate(calls):
+        _dev(X, torch.float32)
+        M = X.shape[0]
+        if X.shape[1] != K or W.shape[0] != N:
+            raise ValueError("shape mismatch")
+        Y = torch.empty((M, N), dtype=torch.float32, device=X.device) if outs is None else outs[i]
+        Ys.append(Y)
+        arr[i] = LinearCall(_ptr(X), M, K, _ptr(W), N, W.shape[1], fmt, eps, _ptr(beta), _ptr(bias), _ptr(Y))
+    return arr, Ys
+
+
+def linear_group_workspace_size(calls) -> int:
+    arr, _ = _call_array(calls, outs=[None] * len(calls))
+    return int(load().bl_linear_group_workspace_size(arr, len(calls)))
+
+
+def linear_group(calls, static_weights: bool = False, ws=None, outs=None):
+    """bl_linear_group: several independent linears, calls = [(X, W, fmt, N, K, beta, bias, eps)];
+    returns the list of Y (written into `outs` when given)."""
+    torch, lib = _torch(), load()
+    arr, Ys = _call_array(calls, outs)
+    need = lib.bl_linear_group_workspace_size(arr, len(calls))
+    if ws is None and need:
+        ws = workspace(need, calls[0][0].device)
+    stream = _stream(torch, calls[0][0]) if calls else None
+    _check("bl_linear_group", lib.bl_linear_group(
+        arr, len(calls), FLAG_STATIC_WEIGHTS if static_weights else 0, _ptr(ws),
+        0 if ws is None else ws.numel(), stream))
+    return Ys
 
 
 def bitlinear_forward(X, W, fmt: int = PACK5, bias=None, eps: float = 1e-5, ws=None, w_out=None,
@@ -278,9 +328,11 @@ def linear_noalloc(X, W, fmt: int, N: int, K: int, beta, out, bias=None, eps: fl
     return out
 
 
-def linear_acc(Xq, W, fmt: int, N: int, K: int, path: int = PATH_AUTO, ws=None):
+def linear_acc(Xq, W, fmt: int, N: int, K: int, path: int = PATH_AUTO, ws=None,
+               static_weights: bool = False):
     """acc = X_q W_q^T in int32 from pre-quantized Xq [M,K] int8."""
     torch, lib = _torch(), load()
+    path = path | (FLAG_STATIC_WEIGHTS if static_weights else 0)
     _dev(Xq, torch.int8)
     M = Xq.shape[0]
     acc = torch.empty((M, N), dtype=torch.int32, device=Xq.device)

@@ -25,6 +25,7 @@ namespace bl {
 namespace {
 
 constexpr size_t kWsAlign = 256;
+constexpr int kPathMask = 0xFF;   // the BL_PATH_* bits of a `path` argument (flags above)
 
 size_t align_up(size_t v) { return (v + kWsAlign - 1) / kWsAlign * kWsAlign; }
 
@@ -393,63 +394,108 @@ bl_status unpack_rows(const uint8_t* Wp, int64_t N, int64_t K, int64_t ldp, int8
   return launch_status();
 }
 
-template <int M, int CH, bool F, bool D>
-bl_status launch_gemv_inst(const GemvPlan& P, const GemvArgs& a, cudaStream_t st) {
-  auto kern = gemv_pack5_kernel<M, CH, F, D>;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kGemvMaxSmem) != cudaSuccess)
+// ---- decode GEMV launches -------------------------------------------------
+// One problem of a GEMV launch: Y from float32 X, or acc from X_q.
+struct GemvCall {
+  const float* X;
+  const int8_t* Xq;
+  int64_t ldxq;
+  const void* W;
+  int64_t ldw, N, K;
+  const float* beta;
+  const float* bias;
+  float eps;
+  float* Y;
+  int32_t* acc;
+};
+
+template <int M, int CH, bool F>
+bl_status launch_gemv_inst(const GemvArgs& a, int grid, uint32_t smem, cudaStream_t st) {
+  constexpr int kMinBlocks = (M * CH == 1) ? 2 : 1;    // two CTAs per SM when their data fit
+  auto kern = gemv_pack5_kernel<M, CH, F, kMinBlocks>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kGemvMaxSmem)) != cudaSuccess)
     return BL_ERR_CUDA;
-  kern<<<P.grid, P.nwarps * 32, P.smem, st>>>(a);
-  return launch_status();
+  // programmatic dependent launch: the kernel's prologue (and, with static
+  // weights, its weight copies) may overlap the previous kernel on the stream;
+  // it waits (griddepcontrol.wait) before touching X, Y or acc
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(unsigned(grid));
+  cfg.blockDim = dim3(kGemvThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, a) == cudaSuccess ? launch_status() : BL_ERR_CUDA;
 }
 
-template <bool F, bool D>
-bl_status launch_gemv_fd(const GemvPlan& P, const GemvArgs& a, cudaStream_t st) {
-  switch (P.M * 8 + P.CH) {
-    case 1 * 8 + 1: return launch_gemv_inst<1, 1, F, D>(P, a, st);
-    case 1 * 8 + 2: return launch_gemv_inst<1, 2, F, D>(P, a, st);
-    case 1 * 8 + 3: return launch_gemv_inst<1, 3, F, D>(P, a, st);
-    case 1 * 8 + 4: return launch_gemv_inst<1, 4, F, D>(P, a, st);
-    case 2 * 8 + 1: return launch_gemv_inst<2, 1, F, D>(P, a, st);
-    case 2 * 8 + 2: return launch_gemv_inst<2, 2, F, D>(P, a, st);
-    case 3 * 8 + 1: return launch_gemv_inst<3, 1, F, D>(P, a, st);
-    case 4 * 8 + 1: return launch_gemv_inst<4, 1, F, D>(P, a, st);
+template <bool F>
+bl_status launch_gemv_f(int M, int ch, const GemvArgs& a, int grid, uint32_t smem, cudaStream_t st) {
+  switch (M * 8 + ch) {
+    case 1 * 8 + 1: return launch_gemv_inst<1, 1, F>(a, grid, smem, st);
+    case 1 * 8 + 2: return launch_gemv_inst<1, 2, F>(a, grid, smem, st);
+    case 1 * 8 + 4: return launch_gemv_inst<1, 4, F>(a, grid, smem, st);
+    case 2 * 8 + 1: return launch_gemv_inst<2, 1, F>(a, grid, smem, st);
+    case 2 * 8 + 2: return launch_gemv_inst<2, 2, F>(a, grid, smem, st);
+    case 3 * 8 + 1: return launch_gemv_inst<3, 1, F>(a, grid, smem, st);
+    case 4 * 8 + 1: return launch_gemv_inst<4, 1, F>(a, grid, smem, st);
   }
   return BL_ERR_UNSUPPORTED;
 }
 
-// The packed-trit GEMV: Y from float32 X (fused quantization) or acc from X_q.
+// Up to kGemvMaxProbs problems with the same M in one launch; every call
+// either quantizes float32 X (fused) or reads given X_q (not fused).
+bl_status run_gemv_group(int64_t M, const GemvCall* c, int n, bool prefetch, cudaStream_t st) {
+  if (n < 1 || n > kGemvMaxProbs || M < 1 || M > kGemvMaxM) return BL_ERR_UNSUPPORTED;
+  const bool fused = c[0].X != nullptr;
+  int ch = 1;
+  double total = 0.0;
+  for (int i = 0; i < n; ++i) {
+    if ((c[i].X != nullptr) != fused) return BL_ERR_UNSUPPORTED;
+    const int chi = gemv_chunks_per_lane(M, c[i].ldw);
+    if (chi == 0) return BL_ERR_UNSUPPORTED;
+    ch = chi > ch ? chi : ch;
+    total += double(c[i].N) * double(c[i].ldw);
+  }
+  GemvArgs a = {};
+  a.nprob = n;
+  a.prefetch = prefetch ? 1 : 0;
+  int cta = 0;
+  uint32_t smem = 0;
+  for (int i = 0; i < n; ++i) {
+    int64_t want = int64_t(double(kGemvCtas) * double(c[i].N) * double(c[i].ldw) / total + 0.5);
+    if (want < 1) want = 1;
+    if (want > c[i].N) want = c[i].N;
+    GemvProb& P = a.p[i];
+    if (!gemv_plan_prob(M, c[i].N, c[i].K, c[i].ldw, int(want), ch, P)) return BL_ERR_UNSUPPORTED;
+    P.X = c[i].X;
+    P.Xq = c[i].Xq;
+    P.ldxq = c[i].ldxq;
+    P.Wp = static_cast<const uint8_t*>(c[i].W);
+    P.N = c[i].N;
+    P.K = c[i].K;
+    P.ldp = c[i].ldw;
+    P.beta = c[i].beta;
+    P.bias = c[i].bias;
+    P.eps = c[i].eps;
+    P.Y = c[i].Y;
+    P.acc = c[i].acc;
+    P.cta0 = cta;
+    cta += int(ceil_div(c[i].N, int64_t(P.rows_per_cta)));   // every CTA has at least one row
+    smem = P.smem > smem ? P.smem : smem;
+  }
+  return fused ? launch_gemv_f<true>(int(M), ch, a, cta, smem, st)
+               : launch_gemv_f<false>(int(M), ch, a, cta, smem, st);
+}
+
+// The packed-trit GEMV for one call: Y from float32 X (fused quantization) or acc from X_q.
 bl_status run_gemv(const float* X, const int8_t* Xq, int64_t ldxq, int64_t M, int64_t K,
                    const void* W, int64_t ldw, int64_t N, const float* beta, const float* bias,
-                   float eps, float* Y, int32_t* acc, cudaStream_t st) {
-  GemvPlan P;
-  const bool x_copyable = X && is_aligned(X, 16) && (K % 4) == 0;
-  if (!gemv_make_plan(M, N, K, ldw, num_sms(), P, x_copyable)) return BL_ERR_UNSUPPORTED;
-  GemvArgs a;
-  a.X = X;
-  a.Xq = Xq;
-  a.ldxq = ldxq;
-  a.Wp = static_cast<const uint8_t*>(W);
-  a.N = N;
-  a.K = K;
-  a.ldp = ldw;
-  a.beta = beta;
-  a.bias = bias;
-  a.eps = eps;
-  a.Y = Y;
-  a.acc = acc;
-  a.S = P.S;
-  a.slice = P.slice;
-  a.G = P.G;
-  a.RS = P.RS;
-  a.nstage = P.nstage;
-  a.rows_per_cta = P.rows_per_cta;
-  a.xstage_off = P.xstage_off;
-  a.part_off = P.part_off;
-  a.bar_off = P.bar_off;
-  a.stage_off = P.stage_off;
-  a.xf_off = P.xf_off;
-  a.xf_bytes = P.xf_bytes;
-  return Y ? launch_gemv_fd<true, true>(P, a, st) : launch_gemv_fd<false, false>(P, a, st);
+                   float eps, float* Y, int32_t* acc, bool prefetch, cudaStream_t st) {
+  GemvCall c = {X, Xq, ldxq, W, ldw, N, K, beta, bias, eps, Y, acc};
+  return run_gemv_group(M, &c, 1, prefetch, st);
 }
 
 bl_status run_simt(const int8_t* Xq, int64_t ldx, int64_t M, int64_t K, const void* W,
@@ -641,7 +687,9 @@ bl_status bl_quantize_act(const float* X, int64_t M, int64_t K, float eps, int8_
 
 size_t bl_linear_ex_workspace_size(int64_t M, int64_t N, int64_t K, bl_wfmt f, int path) {
   if (M < 0 || K < 1 || N < 1) return 0;
+  path &= kPathMask;
   const int p = resolve_path(M, N, K, f, path, nullptr);
+  if (p == BL_PATH_GEMV) return 0;   // activation quantization inside the GEMV: no scratch
   return lin_layout(M, K, N, p == BL_PATH_TC && tc_unpack(M, f), p == BL_PATH_TC ? tc_split(M, N, K).bytes : 0)
       .total;
 }
@@ -649,6 +697,7 @@ size_t bl_linear_ex_workspace_size(int64_t M, int64_t N, int64_t K, bl_wfmt f, i
 // bl_linear's workspace without the tensor-core K split's partials.
 static size_t linear_ws_nosplit(int64_t M, int64_t N, int64_t K, bl_wfmt f) {
   const int p = resolve_path(M, N, K, f, BL_PATH_AUTO, nullptr);
+  if (p == BL_PATH_GEMV) return 0;
   return lin_layout(M, K, N, p == BL_PATH_TC && tc_unpack(M, f), 0).total;
 }
 
@@ -656,28 +705,38 @@ size_t bl_linear_workspace_size(int64_t M, int64_t N, int64_t K, bl_wfmt f) {
   return bl_linear_ex_workspace_size(M, N, K, f, BL_PATH_AUTO);
 }
 
+// The argument checks of bl_linear (M == 0 passes once the rest is valid).
+static bl_status check_linear(const float* X, int64_t M, int64_t K, const void* W, bl_wfmt f, int64_t N,
+                              int64_t ldw, const float* beta_dev, const float* bias, float eps, const float* Y) {
+  bl_status st = check_shape(M, K, N);
+  if (st != BL_OK) return st;
+  if (!eps_ok(eps)) return BL_ERR_INVALID_ARG;
+  st = check_w(W, f, K, ldw);
+  if (st != BL_OK || M == 0) return st;
+  if (!X || !Y || !beta_dev) return BL_ERR_INVALID_ARG;
+  if (!is_aligned(X, 4) || !is_aligned(Y, 4) || (bias && !is_aligned(bias, 4))) return BL_ERR_ALIGNMENT;
+  return BL_OK;
+}
+
 // allow_split = false: the tensor-core GEMM runs without a K split (no partials
 // in the workspace), for bl_linear_noalloc when the split would not fit.
 static bl_status linear_impl(const float* X, int64_t M, int64_t K, const void* W, bl_wfmt f, int64_t N,
                              int64_t ldw, const float* beta_dev, const float* bias, float eps, float* Y,
                              void* ws, size_t ws_bytes, int path, bool allow_split, cudaStream_t stream) {
-  bl_status st = check_shape(M, K, N);
-  if (st != BL_OK) return st;
-  if (!eps_ok(eps)) return BL_ERR_INVALID_ARG;
-  st = check_w(W, f, K, ldw);
-  if (st != BL_OK) return st;
+  const bool static_w = (path & BL_FLAG_STATIC_WEIGHTS) != 0;
+  if (path & ~(kPathMask | BL_FLAG_STATIC_WEIGHTS)) return BL_ERR_INVALID_ARG;
+  path &= kPathMask;
   if (path < BL_PATH_AUTO || path > BL_PATH_TC) return BL_ERR_INVALID_ARG;
-  if (M == 0) return BL_OK;
-  if (!X || !Y || !beta_dev) return BL_ERR_INVALID_ARG;
-  if (!is_aligned(X, 4) || !is_aligned(Y, 4) || (bias && !is_aligned(bias, 4))) return BL_ERR_ALIGNMENT;
+  bl_status st = check_linear(X, M, K, W, f, N, ldw, beta_dev, bias, eps, Y);
+  if (st != BL_OK || M == 0) return st;
   const int p = resolve_path(M, N, K, f, path, nullptr, true, ldw, W);
   if (p < 0) return BL_ERR_UNSUPPORTED;
+  if (p == BL_PATH_GEMV)   // needs no workspace
+    return run_gemv(X, nullptr, 0, M, K, W, ldw, N, beta_dev, bias, eps, Y, nullptr, static_w, stream);
   const size_t tcb = (p == BL_PATH_TC && allow_split) ? tc_split(M, N, K).bytes : 0;
   const LinWs l = lin_layout(M, K, N, p == BL_PATH_TC && tc_unpack(M, f), tcb);
   if (!ws || !is_aligned(ws, kWsAlign) || ws_bytes < l.total) return BL_ERR_WORKSPACE;
   void* tcws = tcb ? static_cast<char*>(ws) + l.tc_off : nullptr;   // null: no K split
-  if (p == BL_PATH_GEMV)
-    return run_gemv(X, nullptr, 0, M, K, W, ldw, N, beta_dev, bias, eps, Y, nullptr, stream);
   int8_t* Xq = reinterpret_cast<int8_t*>(static_cast<char*>(ws) + l.xq_off);
   float* s = reinterpret_cast<float*>(static_cast<char*>(ws) + l.s_off);
   launch_act_quant(X, M, K, eps, Xq, l.ldx, s, stream);
@@ -703,6 +762,7 @@ bl_status bl_linear_ex(const float* X, int64_t M, int64_t K, const void* W, bl_w
 }
 
 int bl_linear_plan(int64_t M, int64_t N, int64_t K, bl_wfmt f, int path, int* launches) {
+  path &= kPathMask;
   if (check_shape(M, K, N) != BL_OK || (f != BL_W_I8 && f != BL_W_PACK5)) return -1;
   if (path < BL_PATH_AUTO || path > BL_PATH_TC) return -1;
   return resolve_path(M, N, K, f, path, launches);
@@ -713,6 +773,61 @@ bl_status bl_linear(const float* X, int64_t M, int64_t K, const void* W, bl_wfmt
                     void* ws, size_t ws_bytes, cudaStream_t stream) {
   return bl_linear_ex(X, M, K, W, f, N, ldw, beta_dev, bias, eps, Y, ws, ws_bytes,
                       BL_PATH_AUTO, stream);
+}
+
+// Whether a call of a group takes the decode GEMV (and so needs no workspace).
+static bool group_gemv(const bl_linear_call& c) {
+  return c.M >= 1 && resolve_path(c.M, c.N, c.K, c.f, BL_PATH_AUTO, nullptr, true, c.ldw, c.W) == BL_PATH_GEMV;
+}
+
+size_t bl_linear_group_workspace_size(const bl_linear_call* calls, int count) {
+  if (!calls || count < 1) return 0;
+  size_t t = 0;
+  for (int i = 0; i < count; ++i)
+    if (calls[i].M > 0 && !group_gemv(calls[i])) t += align_up(bl_linear_workspace_size(calls[i].M, calls[i].N, calls[i].K, calls[i].f));
+  return t;
+}
+
+bl_status bl_linear_group(const bl_linear_call* calls, int count, int flags, void* ws, size_t ws_bytes,
+                          cudaStream_t stream) {
+  if (count < 0 || (count > 0 && !calls)) return BL_ERR_INVALID_ARG;
+  if (flags & ~BL_FLAG_STATIC_WEIGHTS) return BL_ERR_INVALID_ARG;
+  // every call is checked before anything is launched
+  for (int i = 0; i < count; ++i) {
+    const bl_linear_call& c = calls[i];
+    const bl_status st = check_linear(c.X, c.M, c.K, c.W, c.f, c.N, c.ldw, c.beta_dev, c.bias, c.eps, c.Y);
+    if (st != BL_OK) return st;
+  }
+  const size_t need = bl_linear_group_workspace_size(calls, count);
+  if (need && (!ws || !is_aligned(ws, kWsAlign) || ws_bytes < need)) return BL_ERR_WORKSPACE;
+  // decode-GEMV calls: one launch per M, up to kGemvMaxProbs problems each
+  for (int64_t m = 1; m <= kGemvMaxM; ++m) {
+    GemvCall g[kGemvMaxProbs];
+    int n = 0;
+    for (int i = 0; i <= count; ++i) {
+      if (i < count && calls[i].M == m && group_gemv(calls[i])) {
+        const bl_linear_call& c = calls[i];
+        g[n++] = GemvCall{c.X, nullptr, 0, c.W, c.ldw, c.N, c.K, c.beta_dev, c.bias, c.eps, c.Y, nullptr};
+      }
+      if (n == kGemvMaxProbs || (i == count && n > 0)) {
+        const bl_status st = run_gemv_group(m, g, n, (flags & BL_FLAG_STATIC_WEIGHTS) != 0, stream);
+        if (st != BL_OK) return st;
+        n = 0;
+      }
+    }
+  }
+  // the rest, each as bl_linear with its own part of the workspace
+  size_t off = 0;
+  for (int i = 0; i < count; ++i) {
+    const bl_linear_call& c = calls[i];
+    if (c.M == 0 || group_gemv(c)) continue;
+    const size_t wsz = bl_linear_workspace_size(c.M, c.N, c.K, c.f);
+    const bl_status st = linear_impl(c.X, c.M, c.K, c.W, c.f, c.N, c.ldw, c.beta_dev, c.bias, c.eps, c.Y,
+                                     static_cast<char*>(ws) + off, wsz, BL_PATH_AUTO | flags, true, stream);
+    if (st != BL_OK) return st;
+    off += align_up(wsz);
+  }
+  return BL_OK;
 }
 
 bl_status bl_linear_noalloc(const float* X, int64_t M, int64_t K, const void* W, bl_wfmt f,
@@ -734,6 +849,7 @@ bl_status bl_linear_noalloc(const float* X, int64_t M, int64_t K, const void* W,
 
 size_t bl_linear_acc_workspace_size(int64_t M, int64_t N, int64_t K, bl_wfmt f, int path) {
   if (M < 1 || N < 1 || K < 1) return 0;
+  path &= kPathMask;
   const int p = resolve_path(M, N, K, f, path, nullptr, false);
   if (p != BL_PATH_TC) return 0;
   return (tc_unpack(M, f) ? align_up(size_t(N) * size_t(round_up(K, 16))) : 0) + tc_split(M, N, K).bytes;
@@ -744,6 +860,9 @@ size_t bl_linear_acc_workspace_size(int64_t M, int64_t N, int64_t K, bl_wfmt f, 
 static bl_status linear_acc_impl(const int8_t* Xq, int64_t M, int64_t K, const void* W, bl_wfmt f, int64_t N,
                           int64_t ldw, int32_t* acc, void* ws, size_t ws_bytes, int path, bool no_ws,
                           cudaStream_t stream) {
+  const bool static_w = (path & BL_FLAG_STATIC_WEIGHTS) != 0;
+  if (path & ~(kPathMask | BL_FLAG_STATIC_WEIGHTS)) return BL_ERR_INVALID_ARG;
+  path &= kPathMask;
   bl_status st = check_shape(M, K, N);
   if (st != BL_OK) return st;
   st = check_w(W, f, K, ldw);
@@ -761,7 +880,7 @@ static bl_status linear_acc_impl(const int8_t* Xq, int64_t M, int64_t K, const v
   }
   if (p < 0) return BL_ERR_UNSUPPORTED;
   if (p == BL_PATH_GEMV)
-    return run_gemv(nullptr, Xq, K, M, K, W, ldw, N, nullptr, nullptr, 0.f, nullptr, acc, stream);
+    return run_gemv(nullptr, Xq, K, M, K, W, ldw, N, nullptr, nullptr, 0.f, nullptr, acc, static_w, stream);
   if (p == BL_PATH_TC) {
     const bool unp = !no_ws && tc_unpack(M, f);
     const size_t wq = unp ? align_up(size_t(N) * size_t(round_up(K, 16))) : 0;

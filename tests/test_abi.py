@@ -86,10 +86,10 @@ NULL = None
     # unknown format / path
     (lambda L: L.bl_linear(16, 1, 8, 16, 7, 4, 16, 16, NULL, 1e-5, 16, 256, 1 << 20, NULL), 1),
     (lambda L: L.bl_linear_ex(16, 1, 8, 16, 1, 4, 16, 16, NULL, 1e-5, 16, 256, 1 << 20, 9, NULL), 1),
-    # workspace missing / too small / unaligned
-    (lambda L: L.bl_linear(16, 4, 8, 16, 1, 4, 16, 16, NULL, 1e-5, 16, NULL, 0, NULL), 4),
-    (lambda L: L.bl_linear(16, 4, 8, 16, 1, 4, 16, 16, NULL, 1e-5, 16, 256, 8, NULL), 4),
-    (lambda L: L.bl_linear(16, 4, 8, 16, 1, 4, 16, 16, NULL, 1e-5, 16, 257, 1 << 20, NULL), 4),
+    # workspace missing / too small / unaligned (M = 5: not the decode GEMV, which needs none)
+    (lambda L: L.bl_linear(16, 5, 8, 16, 1, 4, 16, 16, NULL, 1e-5, 16, NULL, 0, NULL), 4),
+    (lambda L: L.bl_linear(16, 5, 8, 16, 1, 4, 16, 16, NULL, 1e-5, 16, 256, 8, NULL), 4),
+    (lambda L: L.bl_linear(16, 5, 8, 16, 1, 4, 16, 16, NULL, 1e-5, 16, 257, 1 << 20, NULL), 4),
     # M == 0 is a no-op success, nothing launched
     (lambda L: L.bl_linear(NULL, 0, 8, 16, 1, 4, 16, 16, NULL, 1e-5, NULL, NULL, 0, NULL), 0),
     (lambda L: L.bl_quantize_act(NULL, 0, 8, 1e-5, NULL, NULL, NULL), 0),
@@ -141,6 +141,14 @@ def test_tensor_core_plan_and_workspace(lib, M, K, N):
     assert lib.bl_linear_acc_workspace_size(M, N, K, pkg.PACK5, pkg.PATH_TC) == extra
 
 
+def test_decode_gemv_needs_no_workspace(lib):
+    for M in (1, 2, 3, 4):
+        assert lib.bl_linear_workspace_size(M, 6912, 2560, pkg.PACK5) == 0
+        assert lib.bl_linear_ex_workspace_size(M, 6912, 2560, pkg.PACK5, pkg.PATH_GEMV) == 0
+    assert lib.bl_linear_workspace_size(5, 6912, 2560, pkg.PACK5) > 0
+    assert lib.bl_linear_workspace_size(1, 6912, 2560, pkg.I8) > 0      # one trit per byte: not the GEMV
+
+
 def test_auto_path_crossover(lib):
     """AUTO: the decode GEMV for M <= 4 (packed weights), the tensor cores from M = 5."""
     n = ctypes.c_int(0)
@@ -148,3 +156,53 @@ def test_auto_path_crossover(lib):
         assert lib.bl_linear_plan(M, 4096, 4096, pkg.PACK5, pkg.PATH_AUTO, ctypes.byref(n)) == pkg.PATH_GEMV
     for M in (5, 8, 100, 4096):
         assert lib.bl_linear_plan(M, 4096, 4096, pkg.PACK5, pkg.PATH_AUTO, ctypes.byref(n)) == pkg.PATH_TC
+
+
+def test_linear_call_struct_layout_matches_the_header(tmp_path):
+    """The binding's bl_linear_call mirrors the C struct: size and every field's
+    offset, as a C compiler lays them out from the header."""
+    fields = [f for f, _ in pkg.LinearCall._fields_]
+    src = tmp_path / "layout.c"
+    src.write_text("#include <stdio.h>\n#include <stddef.h>\n#include \"bitlinear.h\"\nint main(void){\n"
+                   "printf(\"%zu\\n\", sizeof(bl_linear_call));\n" +
+                   "".join(f"printf(\"%zu\\n\", offsetof(bl_linear_call, {f}));\n" for f in fields) +
+                   "return 0;}\n")
+    exe = tmp_path / "layout"
+    subprocess.run(["gcc", "-I", os.path.join(ROOT, "include"), "-I", "/usr/local/cuda/include",
+                    str(src), "-o", str(exe)], check=True)
+    out = [int(v) for v in subprocess.run([str(exe)], capture_output=True, text=True, check=True).stdout.split()]
+    assert out[0] == ctypes.sizeof(pkg.LinearCall)
+    assert out[1:] == [getattr(pkg.LinearCall, f).offset for f in fields]
+
+
+def test_linear_group_host_checks(lib):
+    """Group calls are validated before any launch; decode-GEMV calls need no
+    workspace, the others need bl_linear's; flags other than
+    BL_FLAG_STATIC_WEIGHTS are rejected; an empty group is a no-op."""
+    C = pkg.LinearCall
+    gemv = C(16, 1, 2560, 16, 6912, 512, pkg.PACK5, 1e-5, 16, None, 16)
+    tc = C(16, 64, 2560, 16, 6912, 512, pkg.PACK5, 1e-5, 16, None, 16)
+    arr = (C * 2)(gemv, tc)
+    assert lib.bl_linear_group_workspace_size(arr, 1) == 0
+    assert lib.bl_linear_group_workspace_size(arr, 2) == _al(lib.bl_linear_workspace_size(64, 6912, 2560, pkg.PACK5))
+    assert lib.bl_linear_group(arr, 0, 0, None, 0, None) == 0
+    assert lib.bl_linear_group(arr, 1, 0x1, None, 0, None) == 1            # unknown flag
+    assert lib.bl_linear_group(arr, 2, 0, None, 0, None) == 4              # workspace missing
+    bad = (C * 2)(gemv, C(16, 1, 2560, 17, 6912, 512, pkg.PACK5, 1e-5, 16, None, 16))
+    assert lib.bl_linear_group(bad, 2, 0, None, 0, None) == 2              # unaligned packed W
+    neg = (C * 1)(C(16, 1, 2560, 16, 6912, 512, pkg.PACK5, 0.0, 16, None, 16))
+    assert lib.bl_linear_group(neg, 1, 0, None, 0, None) == 1              # eps <= 0
+
+
+def test_static_weights_flag_is_a_flag(lib):
+    """BL_FLAG_STATIC_WEIGHTS rides on `path` without changing the plan or the
+    workspace; other high bits are rejected."""
+    n = ctypes.c_int(0)
+    F = pkg.FLAG_STATIC_WEIGHTS
+    for M in (1, 4, 64):
+        for path in (pkg.PATH_AUTO, pkg.PATH_GEMV, pkg.PATH_TC):
+            assert lib.bl_linear_plan(M, 6912, 2560, pkg.PACK5, path | F, ctypes.byref(n)) == \
+                lib.bl_linear_plan(M, 6912, 2560, pkg.PACK5, path, ctypes.byref(n))
+            assert lib.bl_linear_ex_workspace_size(M, 6912, 2560, pkg.PACK5, path | F) == \
+                lib.bl_linear_ex_workspace_size(M, 6912, 2560, pkg.PACK5, path)
+    assert lib.bl_linear_ex(16, 1, 8, 16, 1, 4, 16, 16, NULL, 1e-5, 16, 256, 1 << 20, 0x200, NULL) == 1

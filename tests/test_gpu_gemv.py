@@ -1,0 +1,148 @@
+"""The decode GEMV's launch modes against the oracle: several problems in one
+launch (bl_linear_group), weights streamed before the dependency wait
+(BL_FLAG_STATIC_WEIGHTS), and back-to-back launches that overlap through
+programmatic dependent launch -- including chains whose next input is the
+previous output, and weights rewritten by the kernel right before the GEMV.
+"""
+import numpy as np
+import pytest
+
+import oracle
+from workloads import problems, random_problem
+
+pytestmark = pytest.mark.gpu
+F32 = np.float32
+
+
+def dev(a):
+    import torch
+    return torch.from_numpy(np.ascontiguousarray(a)).cuda()
+
+
+def host(t):
+    return t.cpu().numpy()
+
+
+def assert_y_exact(y, ref):
+    y, ref = np.asarray(y, np.float64), np.asarray(ref, np.float64)
+    rel = np.abs(y - ref) / np.maximum(np.abs(ref), 1e-30)
+    assert rel.size == 0 or float(rel.max()) <= 1e-6, f"max rel err {rel.max():.3e}"
+    np.testing.assert_array_equal(y, ref)
+
+
+class _P:
+    """A weight tensor alone, as the quantization helper takes it."""
+    def __init__(self, W):
+        self.W, self.eps = W, 1e-5
+
+
+def quantized(bl, p, fmt=None):
+    fmt = bl.PACK5 if fmt is None else fmt
+    fn = bl.quantize_weights_pack5 if fmt == bl.PACK5 else bl.quantize_weights
+    return fn(dev(p.W), p.eps)
+
+
+@pytest.mark.parametrize("static", [False, True])
+def test_group_decode_workload(bl, static):
+    """Both decode-workload layers in one launch, every output against the oracle."""
+    ps = list(problems(2))
+    calls, refs = [], []
+    for p in ps:
+        Wd, beta = quantized(bl, p)
+        calls.append((dev(p.X), Wd, bl.PACK5, p.N, p.K, beta, None, p.eps))
+        refs.append(oracle.bitlinear(p.X, p.W, p.eps)["Y"])
+    lib = bl.load()
+    arr = (bl.LinearCall * 2)()
+    for i, (X, Wd, f, N, K, beta, _, eps) in enumerate(calls):
+        arr[i] = bl.LinearCall(X.data_ptr(), 1, K, Wd.data_ptr(), N, Wd.shape[1], f, eps, beta.data_ptr(), None, 0)
+    assert lib.bl_linear_group_workspace_size(arr, 2) == 0
+    Ys = bl.linear_group(calls, static_weights=static)
+    assert bl.sync_status() == "BL_OK"
+    for Y, ref in zip(Ys, refs):
+        assert_y_exact(host(Y), ref)
+
+
+def test_group_mixed_calls(bl):
+    """Six decode calls (M = 1 and 2, ragged K, bias) -- two launches for M = 1
+    (at most four problems each) and one for M = 2 -- beside a tensor-core call
+    and a one-trit-per-byte call that take bl_linear's own paths."""
+    specs = [(1, 2560, 700), (1, 999, 1500), (1, 6912, 257), (1, 40, 3000), (1, 8192, 64),
+             (2, 3000, 500), (64, 1040, 300), (3, 77, 90)]
+    calls, refs = [], []
+    for i, (M, K, N) in enumerate(specs):
+        p = random_problem(900 + i, M, K, N)
+        fmt = bl.I8 if i == len(specs) - 1 else bl.PACK5
+        Wd, beta = quantized(bl, p, fmt)
+        bias = (np.random.default_rng(i).standard_normal(N) * 0.1).astype(F32) if i % 2 else None
+        calls.append((dev(p.X), Wd, fmt, N, K, beta, None if bias is None else dev(bias), p.eps))
+        refs.append(oracle.bitlinear(p.X, p.W, p.eps, bias)["Y"])
+    Ys = bl.linear_group(calls, static_weights=True)
+    assert bl.sync_status() == "BL_OK"
+    for Y, ref in zip(Ys, refs):
+        assert_y_exact(host(Y), ref)
+
+
+@pytest.mark.parametrize("M,K,N", [(1, 50000, 300), (2, 50000, 200), (2, 20000, 333), (4, 40000, 129),
+                                   (3, 12345, 1000)])
+def test_gemv_long_rows(bl, M, K, N):
+    """Rows of up to 10000 packed bytes: several 16-byte chunks per lane and up
+    to 16 warps per row slice."""
+    p = random_problem(M * 7 + K + N, M, K, N)
+    Wd, beta = quantized(bl, p)
+    assert bl.linear_plan(M, N, K, bl.PACK5)[0] == bl.PATH_GEMV
+    for static in (False, True):
+        Y = bl.linear(dev(p.X), Wd, bl.PACK5, N, K, beta, eps=p.eps, static_weights=static)
+        assert bl.sync_status() == "BL_OK"
+        assert_y_exact(host(Y), oracle.bitlinear(p.X, p.W, p.eps)["Y"])
+
+
+def test_chain_output_feeds_next_input(bl):
+    """Twelve GEMVs back to back on one stream, each reading the previous one's
+    Y as its X (K = N), with static weights: the dependency wait must order
+    every X read after the previous kernel's writes."""
+    import torch
+    K = N = 2560
+    rng = np.random.default_rng(5)
+    Ws = [(rng.standard_normal((N, K), dtype=np.float32) * F32(0.02 * (1 + i % 3))) for i in range(3)]
+    Wq = [quantized(bl, _P(W)) for W in Ws]
+    X0 = rng.standard_normal((1, K), dtype=np.float32)
+    bufs = [dev(X0)] + [torch.empty((1, N), dtype=torch.float32, device="cuda") for _ in range(12)]
+    for i in range(12):
+        Wd, beta = Wq[i % 3]
+        bl.linear(bufs[i], Wd, bl.PACK5, N, K, beta, out=bufs[i + 1], static_weights=True)
+    assert bl.sync_status() == "BL_OK"
+    x = X0
+    for i in range(12):
+        x = oracle.bitlinear(x, Ws[i % 3], 1e-5)["Y"]
+        assert_y_exact(host(bufs[i + 1]), x)
+
+
+def test_weights_rewritten_right_before_the_gemv(bl):
+    """Without the static-weights flag the GEMV reads W only after the kernel
+    before it has finished: quantize into the same packed buffer, then the
+    linear, five times with different weights and no synchronization."""
+    import torch
+    K, N = 6912, 2560
+    Wp = torch.empty((N, bl.pack5_ldp(K)), dtype=torch.uint8, device="cuda")
+    beta = torch.empty(1, dtype=torch.float32, device="cuda")
+    ws = bl.workspace(bl.load().bl_quantize_weights_workspace_size(N, K), "cuda")
+    outs, refs = [], []
+    for i in range(5):
+        p = random_problem(4000 + i, 1, K, N, w_sigma=0.01 * (i + 1))
+        bl.quantize_weights_pack5(dev(p.W), p.eps, ws=ws, out=Wp, beta=beta)
+        outs.append(bl.linear(dev(p.X), Wp, bl.PACK5, N, K, beta, eps=p.eps))
+        refs.append(oracle.bitlinear(p.X, p.W, p.eps)["Y"])
+    assert bl.sync_status() == "BL_OK"
+    for Y, ref in zip(outs, refs):
+        assert_y_exact(host(Y), ref)
+
+
+def test_integer_product_with_static_weights(bl):
+    """bl_linear_acc_ex on the GEMV with the flag: the exact integer product."""
+    rng = np.random.default_rng(8)
+    for M, K, N in ((1, 2560, 6912), (4, 6912, 2560), (3, 1001, 77)):
+        Xq = rng.integers(-127, 128, (M, K)).astype(np.int8)
+        Wq = rng.integers(-1, 2, (N, K)).astype(np.int8)
+        acc = bl.linear_acc(dev(Xq), bl.pack(dev(Wq)), bl.PACK5, N, K, path=bl.PATH_GEMV, static_weights=True)
+        assert bl.sync_status() == "BL_OK"
+        np.testing.assert_array_equal(host(acc), oracle.contract(Xq, Wq))
