@@ -22,6 +22,11 @@ What it computes, and where the method is stated (page title, then section):
   ternary GPT" and "Layout" (5 ternary values per byte, ~1.6 bits/weight), and
   "a 1-bit llm, from scratch", tl;dr (1.6 bits each).  Byte = sum_k (t_k+1) 3^k.
 
+* ``checkpoint.write_deployed`` / ``checkpoint.read_deployed`` -- "ultragraph-1bit
+  0.12.0" (PyPI), section "A whole ternary GPT": the deployed checkpoint keeps
+  the ternary weights at five per byte plus the float32 pieces (beta, biases),
+  byte-exact; the file layout is read in ``oracle/checkpoint.py``.
+
 Readings taken where the pages leave a step open:
 
 1. Precision.  The pages' arrays are numpy float32, so every quantizer step is
@@ -38,6 +43,10 @@ Readings taken where the pages leave a step open:
 6. Packing runs along K in order: trit 5j+k of a row is digit k (little-endian)
    of byte j; trits past K are 0 (digit 1), so an all-padding byte is 121; the
    row stride ``ldp`` is ceil(K/5) rounded up to 16 bytes.
+
+7. The deployed checkpoint's layout (the pages fix only its density and
+   byte-exactness): little-endian records of name, N, K, flags, beta bits,
+   the packed rows without their 16-byte padding, then the bias.
 
 Every function here is pinned by ``tests/test_oracle_pins.py`` against hand-
 worked values, closed forms, invariants or brute force; none is unpinned.

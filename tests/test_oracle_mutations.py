@@ -74,6 +74,24 @@ def _contract_f64_no_widening(Xq, Wq):
     return (np.asarray(Xq) @ np.asarray(Wq).T).astype(np.int32)   # int8 sums wrap
 
 
+def _write_deployed_padded_rows(layers):
+    import struct
+    from oracle import checkpoint as ck
+    out = [ck.MAGIC, struct.pack("<III", ck.VERSION, len(layers), 0)]
+    for L in layers:
+        name = L.get("name", "").encode()
+        Wq = np.asarray(L["Wq"])
+        N, K = Wq.shape
+        bias = L.get("bias")
+        out += [struct.pack("<I", len(name)), name,
+                struct.pack("<QQII", N, K, 1 if bias is not None else 0,
+                            int(np.float32(L["beta"]).view(np.uint32))),
+                ob.pack5(Wq).tobytes()]                       # rows keep their 16-byte padding
+        if bias is not None:
+            out.append(np.asarray(bias, "<f4").tobytes())
+    return b"".join(out)
+
+
 def _dequant_acc_times_s_first(acc, s, beta, bias=None):
     y = (np.asarray(acc).astype(F32) * np.asarray(s, F32).reshape(-1, 1)) * F32(beta)
     return y if bias is None else y + np.asarray(bias, F32)
@@ -92,6 +110,14 @@ MUTANTS = {
     "contract_f64": [_contract_f64_no_widening],
     "dequant": [_dequant_acc_times_s_first],
 }
+
+
+def test_checkpoint_pins_reject_padded_rows(monkeypatch):
+    from oracle import checkpoint as ck
+    monkeypatch.setattr(ck, "write_deployed", _write_deployed_padded_rows)
+    rc = pytest.main(["-q", "-x", "-p", "no:cacheprovider",
+                      __file__.replace("test_oracle_mutations.py", "test_oracle_checkpoint.py")])
+    assert rc != 0
 
 
 @pytest.mark.parametrize("name,mutant", [(n, f) for n, fs in MUTANTS.items() for f in fs],
