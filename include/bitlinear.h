@@ -51,7 +51,8 @@ typedef enum {
   BL_ERR_WORKSPACE = 4,      /* ws NULL, too small, unaligned, or (device) not cleared */
   BL_ERR_CUDA = 5,           /* a CUDA runtime call or launch failed */
   BL_ERR_DEVICE_TIMEOUT = 6, /* a bounded device-side wait gave up */
-  BL_ERR_NONFINITE = 7       /* a kernel met a NaN or Inf input */
+  BL_ERR_NONFINITE = 7,      /* a kernel met a NaN or Inf input */
+  BL_ERR_IO = 8              /* a checkpoint file could not be written or read, or is malformed */
 } bl_status;
 
 /* Weight storage formats. */
@@ -288,6 +289,50 @@ bl_status bl_linear_group(const bl_linear_call* calls, int count, int flags, voi
 bl_status bl_linear_noalloc(const float* X, int64_t M, int64_t K, const void* W, bl_wfmt f,
                             int64_t N, int64_t ldw, const float* beta_dev, const float* bias,
                             float eps, float* Y, cudaStream_t stream);
+
+/* ---- deployed checkpoint ---------------------------------------------------
+ * "ultragraph-1bit 0.12.0" (PyPI), section "A whole ternary GPT": a deployed
+ * checkpoint stores the ternary weights at five per byte (~1.6 bits each) plus
+ * the float32 pieces, and a model loaded from it computes exactly what the
+ * model that wrote it computes, straight from the stored bytes.  File layout
+ * (little-endian, no padding):
+ *   "BLT5", version u32 = 1, count u32, reserved u32 = 0, then per layer:
+ *   name_len u32 (<= 255), name bytes, N u64, K u64, flags u32 (bit 0: bias),
+ *   beta u32 (float32 bits), the packed rows (N * ceil(K/5) bytes: BL_W_PACK5
+ *   rows without their padding), [bias: N float32].
+ * These calls are synchronous: they wait for the work queued on `stream`, copy
+ * through host staging buffers (at most 64 MB, malloc'd and freed inside the
+ * call; no device memory is allocated) and return when the copies are done.
+ * A file that cannot be opened, written or read, that is truncated or has
+ * trailing bytes, or that holds a byte above 242 in its packed rows gives
+ * BL_ERR_IO; a failed save removes the partial file. */
+typedef struct {
+  const char* name;        /* NUL-terminated, at most 255 bytes; NULL = "" */
+  int64_t N, K;
+  const uint8_t* Wp;       /* device, packed trits [N, ldp] (BL_W_PACK5) */
+  int64_t ldp;             /* >= ceil(K/5) */
+  const float* beta_dev;   /* device, the tensor's beta */
+  const float* bias_dev;   /* device [N] float32, or NULL (no bias stored) */
+} bl_deployed_layer;
+
+/* Writes `count` layers to `path` (replacing it). */
+bl_status bl_save_deployed(const char* path, const bl_deployed_layer* layers, int count, cudaStream_t stream);
+
+/* The number of layers in the checkpoint at `path` (the whole file is checked). */
+bl_status bl_deployed_count(const char* path, int* count);
+
+/* Layer `index`'s shape, whether it stores a bias, and its name (copied into
+ * `name`, at most name_cap - 1 bytes and a NUL; NULL to skip).  Host only. */
+bl_status bl_deployed_layer_info(const char* path, int index, int64_t* N, int64_t* K, int* has_bias, char* name,
+                                 size_t name_cap);
+
+/* Layer `index` into device buffers: Wp [N, ldp] (ldp % 16 == 0, >= ceil(K/5),
+ * 16-byte aligned; bytes past ceil(K/5) in each row are set to 121, five zero
+ * trits, exactly as bl_pack writes them), beta_dev (one float32, bit for bit),
+ * bias_dev ([N] float32; NULL to skip; BL_ERR_INVALID_ARG if the layer has no
+ * bias). */
+bl_status bl_load_deployed_layer(const char* path, int index, uint8_t* Wp, int64_t ldp, float* beta_dev,
+                                 float* bias_dev, cudaStream_t stream);
 
 /* Synchronizes `stream`, then reads and clears this device's status word:
  * BL_ERR_DEVICE_TIMEOUT or BL_ERR_NONFINITE if a kernel recorded one, BL_ERR_CUDA

@@ -24,7 +24,7 @@ FLAG_STATIC_WEIGHTS = 0x100            # BL_FLAG_STATIC_WEIGHTS
 
 STATUS = {0: "BL_OK", 1: "BL_ERR_INVALID_ARG", 2: "BL_ERR_ALIGNMENT", 3: "BL_ERR_UNSUPPORTED",
           4: "BL_ERR_WORKSPACE", 5: "BL_ERR_CUDA", 6: "BL_ERR_DEVICE_TIMEOUT",
-          7: "BL_ERR_NONFINITE"}
+          7: "BL_ERR_NONFINITE", 8: "BL_ERR_IO"}
 
 # Every symbol the header declares, with (restype, argtypes).
 _P, _I64, _SZ, _F, _I = ctypes.c_void_p, ctypes.c_int64, ctypes.c_size_t, ctypes.c_float, ctypes.c_int
@@ -37,6 +37,15 @@ class LinearCall(ctypes.Structure):
 
 
 _CALLS = ctypes.POINTER(LinearCall)
+
+
+class DeployedLayer(ctypes.Structure):
+    """bl_deployed_layer: one layer for bl_save_deployed (as in the header)."""
+    _fields_ = [("name", ctypes.c_char_p), ("N", _I64), ("K", _I64), ("Wp", _P), ("ldp", _I64),
+                ("beta_dev", _P), ("bias_dev", _P)]
+
+
+_LAYERS = ctypes.POINTER(DeployedLayer)
 SIGNATURES = {
     "bl_pack5_ldp": (_I64, [_I64]),
     "bl_quantize_weights_workspace_size": (_SZ, [_I64, _I64]),
@@ -61,6 +70,11 @@ SIGNATURES = {
     "bl_linear_acc": (_I, [_P, _I64, _I64, _P, _I, _I64, _I64, _P, _P]),
     "bl_linear_acc_workspace_size": (_SZ, [_I64, _I64, _I64, _I, _I]),
     "bl_linear_acc_ex": (_I, [_P, _I64, _I64, _P, _I, _I64, _I64, _P, _P, _SZ, _I, _P]),
+    "bl_save_deployed": (_I, [ctypes.c_char_p, _LAYERS, _I, _P]),
+    "bl_deployed_count": (_I, [ctypes.c_char_p, ctypes.POINTER(ctypes.c_int)]),
+    "bl_deployed_layer_info": (_I, [ctypes.c_char_p, _I, ctypes.POINTER(_I64), ctypes.POINTER(_I64),
+                                    ctypes.POINTER(ctypes.c_int), ctypes.c_char_p, _SZ]),
+    "bl_load_deployed_layer": (_I, [ctypes.c_char_p, _I, _P, _I64, _P, _P, _P]),
     "bl_sync_status": (_I, [_P]),
     "bl_status_string": (ctypes.c_char_p, [_I]),
 }
@@ -343,6 +357,40 @@ def linear_acc(Xq, W, fmt: int, N: int, K: int, path: int = PATH_AUTO, ws=None,
         _ptr(Xq), M, K, _ptr(W), fmt, N, W.shape[1], _ptr(acc), _ptr(ws),
         0 if ws is None else ws.numel(), path, _stream(torch, Xq)))
     return acc
+
+
+def save_deployed(path: str, layers):
+    """bl_save_deployed: layers = [dict(name, Wp [N, ldp] uint8, K, beta [1], bias [N] or None)]."""
+    torch, lib = _torch(), load()
+    arr = (DeployedLayer * max(1, len(layers)))()
+    for i, L in enumerate(layers):
+        Wp = _dev(L["Wp"], torch.uint8)
+        arr[i] = DeployedLayer(L.get("name", "").encode(), Wp.shape[0], L["K"], _ptr(Wp), Wp.shape[1],
+                               _ptr(L["beta"]), _ptr(L.get("bias")))
+    stream = _stream(torch, layers[0]["Wp"]) if layers else ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    _check("bl_save_deployed", lib.bl_save_deployed(path.encode(), arr, len(layers), stream))
+
+
+def load_deployed(path: str, device=None):
+    """bl_deployed_count / bl_deployed_layer_info / bl_load_deployed_layer: every
+    layer into new device tensors: dict(name, N, K, Wp [N, pack5_ldp(K)], beta, bias)."""
+    torch, lib = _torch(), load()
+    device = torch.device("cuda") if device is None else device
+    n = ctypes.c_int(0)
+    _check("bl_deployed_count", lib.bl_deployed_count(path.encode(), ctypes.byref(n)))
+    out = []
+    for i in range(n.value):
+        N, K, hb = _I64(0), _I64(0), ctypes.c_int(0)
+        name = ctypes.create_string_buffer(256)
+        _check("bl_deployed_layer_info", lib.bl_deployed_layer_info(
+            path.encode(), i, ctypes.byref(N), ctypes.byref(K), ctypes.byref(hb), name, 256))
+        Wp = torch.empty((N.value, pack5_ldp(K.value)), dtype=torch.uint8, device=device)
+        beta = torch.empty(1, dtype=torch.float32, device=device)
+        bias = torch.empty(N.value, dtype=torch.float32, device=device) if hb.value else None
+        _check("bl_load_deployed_layer", lib.bl_load_deployed_layer(
+            path.encode(), i, _ptr(Wp), Wp.shape[1], _ptr(beta), _ptr(bias), _stream(torch, Wp)))
+        out.append({"name": name.value.decode(), "N": N.value, "K": K.value, "Wp": Wp, "beta": beta, "bias": bias})
+    return out
 
 
 def sync_status(device=None) -> str:

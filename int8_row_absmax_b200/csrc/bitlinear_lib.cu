@@ -20,6 +20,7 @@
 #include "linear_simt.cuh"
 #include "gemv_pack5.cuh"
 #include "gemm_tc.cuh"
+#include "deployed_io.cuh"
 
 namespace bl {
 namespace {
@@ -912,6 +913,191 @@ bl_status bl_linear_acc(const int8_t* Xq, int64_t M, int64_t K, const void* W, b
   return linear_acc_impl(Xq, M, K, W, f, N, ldw, acc, nullptr, 0, BL_PATH_AUTO, true, stream);
 }
 
+// ---- deployed checkpoint ------------------------------------------------------
+bl_status bl_save_deployed(const char* path, const bl_deployed_layer* layers, int count, cudaStream_t stream) {
+  if (!path || count < 0 || (count > 0 && !layers)) return BL_ERR_INVALID_ARG;
+  for (int i = 0; i < count; ++i) {
+    const bl_deployed_layer& L = layers[i];
+    if (L.N < 1 || L.K < 1 || L.K > kMaxK || L.N > (int64_t(1) << 40) || !L.Wp || !L.beta_dev) return BL_ERR_INVALID_ARG;
+    if (L.ldp < ceil_div(L.K, 5)) return BL_ERR_INVALID_ARG;
+    if (L.name && strlen(L.name) > io::kMaxName) return BL_ERR_INVALID_ARG;
+  }
+  if (count > 0 && cudaStreamSynchronize(stream) != cudaSuccess) return BL_ERR_CUDA;
+  io::File file;
+  file.f = fopen(path, "wb");
+  if (!file.f) return BL_ERR_IO;
+  bl_status st = BL_OK;
+  unsigned char h[24];
+  memcpy(h, io::kMagic, 4);
+  io::put_u32(h + 4, io::kVersion);
+  io::put_u32(h + 8, uint32_t(count));
+  io::put_u32(h + 12, 0u);
+  if (fwrite(h, 1, 16, file.f) != 16) st = BL_ERR_IO;
+  unsigned char* buf = nullptr;
+  for (int i = 0; i < count && st == BL_OK; ++i) {
+    const bl_deployed_layer& L = layers[i];
+    const uint32_t nlen = L.name ? uint32_t(strlen(L.name)) : 0u;
+    uint32_t beta_bits = 0;
+    if (cudaMemcpyAsync(&beta_bits, L.beta_dev, 4, cudaMemcpyDeviceToHost, stream) != cudaSuccess ||
+        cudaStreamSynchronize(stream) != cudaSuccess) {
+      st = BL_ERR_CUDA;
+      break;
+    }
+    io::put_u32(h, nlen);
+    if (fwrite(h, 1, 4, file.f) != 4 || (nlen && fwrite(L.name, 1, nlen, file.f) != nlen)) {
+      st = BL_ERR_IO;
+      break;
+    }
+    io::put_u64(h, uint64_t(L.N));
+    io::put_u64(h + 8, uint64_t(L.K));
+    io::put_u32(h + 16, L.bias_dev ? 1u : 0u);
+    io::put_u32(h + 20, beta_bits);
+    if (fwrite(h, 1, 24, file.f) != 24) {
+      st = BL_ERR_IO;
+      break;
+    }
+    const size_t cb = size_t(ceil_div(L.K, 5));
+    const int64_t rows_per = int64_t(io::kIoChunk / cb) > 0 ? int64_t(io::kIoChunk / cb) : 1;
+    if (!buf && !(buf = static_cast<unsigned char*>(malloc(io::kIoChunk > cb ? io::kIoChunk : cb)))) {
+      st = BL_ERR_IO;
+      break;
+    }
+    for (int64_t r0 = 0; r0 < L.N && st == BL_OK; r0 += rows_per) {
+      const int64_t nr = L.N - r0 < rows_per ? L.N - r0 : rows_per;
+      if (cudaMemcpy2DAsync(buf, cb, L.Wp + r0 * L.ldp, size_t(L.ldp), cb, size_t(nr), cudaMemcpyDeviceToHost,
+                            stream) != cudaSuccess ||
+          cudaStreamSynchronize(stream) != cudaSuccess)
+        st = BL_ERR_CUDA;
+      else if (fwrite(buf, 1, cb * size_t(nr), file.f) != cb * size_t(nr))
+        st = BL_ERR_IO;
+    }
+    if (st == BL_OK && L.bias_dev) {
+      const int64_t per = int64_t(io::kIoChunk / 4);
+      for (int64_t n0 = 0; n0 < L.N && st == BL_OK; n0 += per) {
+        const int64_t nn = L.N - n0 < per ? L.N - n0 : per;
+        float* fb = reinterpret_cast<float*>(buf);
+        if (cudaMemcpyAsync(fb, L.bias_dev + n0, size_t(nn) * 4, cudaMemcpyDeviceToHost, stream) != cudaSuccess ||
+            cudaStreamSynchronize(stream) != cudaSuccess) {
+          st = BL_ERR_CUDA;
+          break;
+        }
+        for (int64_t j = 0; j < nn; ++j) {   // little-endian float32 bits
+          uint32_t u;
+          memcpy(&u, fb + j, 4);
+          io::put_u32(buf + 4 * j, u);
+        }
+        if (fwrite(buf, 1, size_t(nn) * 4, file.f) != size_t(nn) * 4) st = BL_ERR_IO;
+      }
+    }
+  }
+  free(buf);
+  if (fclose(file.f) != 0 && st == BL_OK) st = BL_ERR_IO;
+  file.f = nullptr;
+  if (st != BL_OK) remove(path);
+  return st;
+}
+
+bl_status bl_deployed_count(const char* path, int* count) {
+  if (!path || !count) return BL_ERR_INVALID_ARG;
+  io::File file;
+  const int n = io::open_checked(path, file);
+  if (n < 0) return BL_ERR_IO;
+  io::Record r;
+  for (int i = 0; i < n; ++i)
+    if (!io::read_record(file.f, r)) return BL_ERR_IO;
+  const long end = ftell(file.f);
+  if (fseek(file.f, 0, SEEK_END) != 0 || ftell(file.f) != end) return BL_ERR_IO;   // short or trailing bytes
+  *count = n;
+  return BL_OK;
+}
+
+bl_status bl_deployed_layer_info(const char* path, int index, int64_t* N, int64_t* K, int* has_bias, char* name,
+                                 size_t name_cap) {
+  if (!path || index < 0) return BL_ERR_INVALID_ARG;
+  int n = 0;
+  bl_status st = bl_deployed_count(path, &n);
+  if (st != BL_OK) return st;
+  if (index >= n) return BL_ERR_INVALID_ARG;
+  io::File file;
+  io::Record r;
+  if (io::open_checked(path, file) < 0 || !io::seek_layer(file, index, r)) return BL_ERR_IO;
+  if (N) *N = int64_t(r.N);
+  if (K) *K = int64_t(r.K);
+  if (has_bias) *has_bias = int(r.flags & 1u);
+  if (name && name_cap) {
+    strncpy(name, r.name, name_cap - 1);
+    name[name_cap - 1] = '\0';
+  }
+  return BL_OK;
+}
+
+bl_status bl_load_deployed_layer(const char* path, int index, uint8_t* Wp, int64_t ldp, float* beta_dev,
+                                 float* bias_dev, cudaStream_t stream) {
+  if (!path || index < 0 || !Wp || !beta_dev) return BL_ERR_INVALID_ARG;
+  int n = 0;
+  bl_status st = bl_deployed_count(path, &n);
+  if (st != BL_OK) return st;
+  if (index >= n) return BL_ERR_INVALID_ARG;
+  io::File file;
+  io::Record r;
+  if (io::open_checked(path, file) < 0 || !io::seek_layer(file, index, r)) return BL_ERR_IO;
+  const int64_t N = int64_t(r.N), K = int64_t(r.K);
+  const size_t cb = size_t(ceil_div(K, 5));
+  if (ldp < int64_t(cb)) return BL_ERR_INVALID_ARG;
+  if (ldp % 16 != 0 || !is_aligned(Wp, 16) || !is_aligned(beta_dev, 4)) return BL_ERR_ALIGNMENT;
+  if (bias_dev && !(r.flags & 1u)) return BL_ERR_INVALID_ARG;
+  if (fseek(file.f, r.packed_off, SEEK_SET) != 0) return BL_ERR_IO;
+  if (cudaStreamSynchronize(stream) != cudaSuccess) return BL_ERR_CUDA;
+  const int64_t rows_per = int64_t(io::kIoChunk / cb) > 0 ? int64_t(io::kIoChunk / cb) : 1;
+  unsigned char* buf = static_cast<unsigned char*>(malloc(io::kIoChunk > cb ? io::kIoChunk : cb));
+  if (!buf) return BL_ERR_IO;
+  for (int64_t r0 = 0; r0 < N && st == BL_OK; r0 += rows_per) {
+    const int64_t nr = N - r0 < rows_per ? N - r0 : rows_per;
+    const size_t nb = cb * size_t(nr);
+    if (fread(buf, 1, nb, file.f) != nb) {
+      st = BL_ERR_IO;
+      break;
+    }
+    for (size_t j = 0; j < nb; ++j)
+      if (buf[j] > 242) st = BL_ERR_IO;    // not a five-trit code
+    if (st == BL_OK && (cudaMemcpy2DAsync(Wp + r0 * ldp, size_t(ldp), buf, cb, cb, size_t(nr), cudaMemcpyHostToDevice,
+                                          stream) != cudaSuccess ||
+                        cudaStreamSynchronize(stream) != cudaSuccess))
+      st = BL_ERR_CUDA;
+  }
+  // whole padding bytes of every row: five zero trits each
+  if (st == BL_OK && ldp > int64_t(cb) &&
+      cudaMemset2DAsync(Wp + cb, size_t(ldp), 121, size_t(ldp) - cb, size_t(N), stream) != cudaSuccess)
+    st = BL_ERR_CUDA;
+  if (st == BL_OK) {
+    float beta;
+    memcpy(&beta, &r.beta_bits, 4);
+    if (cudaMemcpyAsync(beta_dev, &beta, 4, cudaMemcpyHostToDevice, stream) != cudaSuccess ||
+        cudaStreamSynchronize(stream) != cudaSuccess)
+      st = BL_ERR_CUDA;
+  }
+  if (st == BL_OK && bias_dev) {
+    const int64_t per = int64_t(io::kIoChunk / 4);
+    for (int64_t n0 = 0; n0 < N && st == BL_OK; n0 += per) {
+      const int64_t nn = N - n0 < per ? N - n0 : per;
+      if (fread(buf, 1, size_t(nn) * 4, file.f) != size_t(nn) * 4) {
+        st = BL_ERR_IO;
+        break;
+      }
+      float* fb = reinterpret_cast<float*>(buf);
+      for (int64_t j = 0; j < nn; ++j) {
+        const uint32_t u = io::get_u32(buf + 4 * j);
+        memcpy(fb + j, &u, 4);
+      }
+      if (cudaMemcpyAsync(bias_dev + n0, fb, size_t(nn) * 4, cudaMemcpyHostToDevice, stream) != cudaSuccess ||
+          cudaStreamSynchronize(stream) != cudaSuccess)
+        st = BL_ERR_CUDA;
+    }
+  }
+  free(buf);
+  return st;
+}
+
 bl_status bl_sync_status(cudaStream_t stream) {
   if (cudaStreamSynchronize(stream) != cudaSuccess) return BL_ERR_CUDA;
   unsigned int word = 0u, zero = 0u;
@@ -933,6 +1119,7 @@ const char* bl_status_string(bl_status s) {
     case BL_ERR_CUDA: return "BL_ERR_CUDA";
     case BL_ERR_DEVICE_TIMEOUT: return "BL_ERR_DEVICE_TIMEOUT";
     case BL_ERR_NONFINITE: return "BL_ERR_NONFINITE";
+    case BL_ERR_IO: return "BL_ERR_IO";
   }
   return "BL_ERR_UNKNOWN";
 }

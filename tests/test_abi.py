@@ -206,3 +206,38 @@ def test_static_weights_flag_is_a_flag(lib):
             assert lib.bl_linear_ex_workspace_size(M, 6912, 2560, pkg.PACK5, path | F) == \
                 lib.bl_linear_ex_workspace_size(M, 6912, 2560, pkg.PACK5, path)
     assert lib.bl_linear_ex(16, 1, 8, 16, 1, 4, 16, 16, NULL, 1e-5, 16, 256, 1 << 20, 0x200, NULL) == 1
+
+
+def test_deployed_checkpoint_host_side(lib, tmp_path):
+    """The checkpoint reader's host side against files the oracle writes: layer
+    count, shapes, names and bias flags; malformed files give BL_ERR_IO; a
+    save of no layers writes the oracle's header bytes."""
+    import numpy as np
+    from oracle import checkpoint
+    rng = np.random.default_rng(3)
+    layers = [{"name": "attn.q", "Wq": rng.integers(-1, 2, (7, 33)).astype(np.int8), "beta": np.float32(0.02)},
+              {"name": "", "Wq": rng.integers(-1, 2, (2, 5)).astype(np.int8), "beta": np.float32(1),
+               "bias": np.ones(2, np.float32)}]
+    data = checkpoint.write_deployed(layers)
+    path = tmp_path / "m.blt"
+    path.write_bytes(data)
+    n = ctypes.c_int(-1)
+    assert lib.bl_deployed_count(str(path).encode(), ctypes.byref(n)) == 0 and n.value == 2
+    N, K, hb = ctypes.c_int64(), ctypes.c_int64(), ctypes.c_int()
+    name = ctypes.create_string_buffer(256)
+    for i, (eN, eK, eb, en) in enumerate(((7, 33, 0, b"attn.q"), (2, 5, 1, b""))):
+        assert lib.bl_deployed_layer_info(str(path).encode(), i, ctypes.byref(N), ctypes.byref(K),
+                                          ctypes.byref(hb), name, 256) == 0
+        assert (N.value, K.value, hb.value, name.value) == (eN, eK, eb, en)
+    short = ctypes.create_string_buffer(4)
+    assert lib.bl_deployed_layer_info(str(path).encode(), 0, None, None, None, short, 4) == 0
+    assert short.value == b"att"
+    assert lib.bl_deployed_layer_info(str(path).encode(), 2, None, None, None, None, 0) == 1
+    for bad in (data[:-1], data + b"\0", b"XLT5" + data[4:], data[:4] + b"\2\0\0\0" + data[8:], b""):
+        path.write_bytes(bad)
+        assert lib.bl_deployed_count(str(path).encode(), ctypes.byref(n)) == 8
+    assert lib.bl_deployed_count(str(tmp_path / "missing.blt").encode(), ctypes.byref(n)) == 8
+    empty = tmp_path / "empty.blt"
+    assert lib.bl_save_deployed(str(empty).encode(), None, 0, None) == 0
+    assert empty.read_bytes() == checkpoint.write_deployed([])
+    assert lib.bl_save_deployed(str(tmp_path / "no_dir" / "x.blt").encode(), None, 0, None) == 8
