@@ -290,6 +290,32 @@ bl_status bl_linear_noalloc(const float* X, int64_t M, int64_t K, const void* W,
                             int64_t N, int64_t ldw, const float* beta_dev, const float* bias,
                             float eps, float* Y, cudaStream_t stream);
 
+/* ---- straight-through backward --------------------------------------------
+ * "ultragraph -- when the graph is the 1-bit LLM, part 2", section "autograd on
+ * a byte-graph, and the straight-through lie": the backward of y = (x_q W_q^T)
+ * (s beta) + b treats the quantizers and the per-row scale as the identity, so
+ *     dX = dY W  [M, K],   dW = dY^T X  [N, K],   db = sum over rows of dY  [N],
+ * with W the float32 master weights [N, K] and X the float32 input [M, K].
+ *
+ * Bytes of `ws` that bl_linear_backward needs (float32 hi/lo splits of the
+ * operands of one product at a time). */
+size_t bl_linear_backward_workspace_size(int64_t M, int64_t N, int64_t K);
+
+/* The three gradients; any of dX, dW, db may be NULL to skip it.
+ *   dY [M, N], X [M, K], W [N, K], dX [M, K], dW [N, K], db [N]: float32,
+ *   contiguous, 4-byte aligned.  X may be NULL when dW is, W when dX is.
+ *   ws  >= bl_linear_backward_workspace_size(M, N, K) bytes, 256-byte aligned
+ *       (may be NULL when dX and dW are both NULL).
+ * The products run on the tensor cores (tcgen05 kind::tf32, float32
+ * accumulators) with every float32 operand split into two tf32 parts, a = a_hi
+ * + a_lo, and the three products a_hi b_hi + a_hi b_lo + a_lo b_hi: each
+ * product is then within about 3 * 2^-22 |a b| of the exact one, and an output
+ * is within (3 * 2^-22 + (n + 1) 2^-24) sum |a b| of the exact sum, n being
+ * the 3 * ceil(Kc / 8) accumulator updates over the contraction length Kc.
+ * db is summed in float64 and rounded once.  M == 0 launches nothing. */
+bl_status bl_linear_backward(const float* dY, const float* X, const float* W, int64_t M, int64_t N, int64_t K,
+                             float* dX, float* dW, float* db, void* ws, size_t ws_bytes, cudaStream_t stream);
+
 /* ---- deployed checkpoint ---------------------------------------------------
  * "ultragraph-1bit 0.12.0" (PyPI), section "A whole ternary GPT": a deployed
  * checkpoint stores the ternary weights at five per byte (~1.6 bits each) plus

@@ -70,6 +70,8 @@ SIGNATURES = {
     "bl_linear_acc": (_I, [_P, _I64, _I64, _P, _I, _I64, _I64, _P, _P]),
     "bl_linear_acc_workspace_size": (_SZ, [_I64, _I64, _I64, _I, _I]),
     "bl_linear_acc_ex": (_I, [_P, _I64, _I64, _P, _I, _I64, _I64, _P, _P, _SZ, _I, _P]),
+    "bl_linear_backward_workspace_size": (_SZ, [_I64, _I64, _I64]),
+    "bl_linear_backward": (_I, [_P, _P, _P, _I64, _I64, _I64, _P, _P, _P, _P, _SZ, _P]),
     "bl_save_deployed": (_I, [ctypes.c_char_p, _LAYERS, _I, _P]),
     "bl_deployed_count": (_I, [ctypes.c_char_p, ctypes.POINTER(ctypes.c_int)]),
     "bl_deployed_layer_info": (_I, [ctypes.c_char_p, _I, ctypes.POINTER(_I64), ctypes.POINTER(_I64),
@@ -357,6 +359,25 @@ def linear_acc(Xq, W, fmt: int, N: int, K: int, path: int = PATH_AUTO, ws=None,
         _ptr(Xq), M, K, _ptr(W), fmt, N, W.shape[1], _ptr(acc), _ptr(ws),
         0 if ws is None else ws.numel(), path, _stream(torch, Xq)))
     return acc
+
+
+def linear_backward(dY, X, W, want=("dX", "dW", "db"), ws=None):
+    """Straight-through backward: (dX [M,K], dW [N,K], db [N]) float32; entries
+    not in `want` come back as None."""
+    torch, lib = _torch(), load()
+    _dev(dY, torch.float32)
+    M, N = dY.shape
+    K = W.shape[1] if W is not None else X.shape[1]
+    dX = torch.empty((M, K), dtype=torch.float32, device=dY.device) if "dX" in want else None
+    dW = torch.empty((N, K), dtype=torch.float32, device=dY.device) if "dW" in want else None
+    db = torch.empty((N,), dtype=torch.float32, device=dY.device) if "db" in want else None
+    need = lib.bl_linear_backward_workspace_size(M, N, K) if (dX is not None or dW is not None) else 0
+    if ws is None and need:
+        ws = workspace(need, dY.device)
+    _check("bl_linear_backward", lib.bl_linear_backward(
+        _ptr(dY), _ptr(X), _ptr(W), M, N, K, _ptr(dX), _ptr(dW), _ptr(db), _ptr(ws),
+        0 if ws is None else ws.numel(), _stream(torch, dY)))
+    return dX, dW, db
 
 
 def save_deployed(path: str, layers):

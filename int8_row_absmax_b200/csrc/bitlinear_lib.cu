@@ -21,6 +21,7 @@
 #include "gemv_pack5.cuh"
 #include "gemm_tc.cuh"
 #include "deployed_io.cuh"
+#include "ste_backward.cuh"
 
 namespace bl {
 namespace {
@@ -322,6 +323,41 @@ bool make_map_packed(CUtensorMap* map, const void* base, int64_t ldp, int64_t N,
   return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// float32 [outer, inner] (row stride ld floats, a multiple of 4) as 128-byte
+// swizzled boxes of {32, box_rows}; out-of-range elements read as zero.
+bool make_map_f32(CUtensorMap* map, const void* base, int64_t inner, int64_t outer, int64_t ld, int box_rows) {
+  EncodeTiledFn fn = encode_tiled();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {cuuint64_t(inner), cuuint64_t(outer)};
+  const cuuint64_t strides[1] = {cuuint64_t(ld) * 4};
+  const cuuint32_t box[2] = {cuuint32_t(kBwBK), cuuint32_t(box_rows)};
+  const cuuint32_t estr[2] = {1u, 1u};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// D [Mr, Nc] = A B^T over Kc from the hi/lo splits of A [Mr, ld] and B [Nc, ld].
+bl_status run_tf32x3(const float* ahi, const float* alo, const float* bhi, const float* blo, int64_t ld, int64_t Mr,
+                     int64_t Nc, int64_t Kc, float* D, cudaStream_t st) {
+  BwMaps maps;
+  if (!make_map_f32(&maps.a_hi, ahi, Kc, Mr, ld, kBwBM) || !make_map_f32(&maps.a_lo, alo, Kc, Mr, ld, kBwBM) ||
+      !make_map_f32(&maps.b_hi, bhi, Kc, Nc, ld, kBwBN) || !make_map_f32(&maps.b_lo, blo, Kc, Nc, ld, kBwBN))
+    return BL_ERR_CUDA;
+  BwArgs a;
+  a.Mr = Mr;
+  a.Nc = Nc;
+  a.Kc = Kc;
+  a.D = D;
+  a.tiles_m = int(ceil_div(Mr, int64_t(kBwBM)));
+  a.tiles_n = int(ceil_div(Nc, int64_t(kBwBN)));
+  const int64_t work = int64_t(a.tiles_m) * a.tiles_n;
+  if (cudaFuncSetAttribute(gemm_tf32x3_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kBwSmem) != cudaSuccess)
+    return BL_ERR_CUDA;
+  gemm_tf32x3_kernel<<<unsigned(work < num_sms() ? work : num_sms()), kBwThreads, kBwSmem, st>>>(maps, a);
+  return launch_status();
 }
 
 // The tcgen05 GEMM on int8 X_q [M, ldx] and int8 W_q [N, ldw] (or packed W
@@ -911,6 +947,73 @@ bl_status bl_linear_acc_ex(const int8_t* Xq, int64_t M, int64_t K, const void* W
 bl_status bl_linear_acc(const int8_t* Xq, int64_t M, int64_t K, const void* W, bl_wfmt f,
                         int64_t N, int64_t ldw, int32_t* acc, cudaStream_t stream) {
   return linear_acc_impl(Xq, M, K, W, f, N, ldw, acc, nullptr, 0, BL_PATH_AUTO, true, stream);
+}
+
+// ---- straight-through backward ---------------------------------------------------
+struct BwLayout {
+  int64_t ldN, ldM;
+  size_t dx_a, dx_b, dw_a, dw_b, total;   // bytes of one hi (or lo) array of each operand
+};
+static BwLayout bw_layout(int64_t M, int64_t N, int64_t K) {
+  BwLayout l;
+  l.ldN = round_up(N, 4);
+  l.ldM = round_up(M, 4);
+  l.dx_a = align_up(size_t(M) * size_t(l.ldN) * 4);
+  l.dx_b = align_up(size_t(K) * size_t(l.ldN) * 4);
+  l.dw_a = align_up(size_t(N) * size_t(l.ldM) * 4);
+  l.dw_b = align_up(size_t(K) * size_t(l.ldM) * 4);
+  const size_t dx = 2 * (l.dx_a + l.dx_b), dw = 2 * (l.dw_a + l.dw_b);
+  l.total = dx > dw ? dx : dw;
+  return l;
+}
+
+size_t bl_linear_backward_workspace_size(int64_t M, int64_t N, int64_t K) {
+  if (M < 1 || N < 1 || K < 1) return 0;
+  return bw_layout(M, N, K).total;
+}
+
+bl_status bl_linear_backward(const float* dY, const float* X, const float* W, int64_t M, int64_t N, int64_t K,
+                             float* dX, float* dW, float* db, void* ws, size_t ws_bytes, cudaStream_t stream) {
+  if (M < 0 || N < 1 || K < 1 || M > (int64_t(1) << 31) - 1 || N > (int64_t(1) << 31) - 1 ||
+      K > (int64_t(1) << 31) - 1)
+    return BL_ERR_INVALID_ARG;
+  if (M == 0) return BL_OK;
+  if (!dY || (dX && !W) || (dW && !X)) return BL_ERR_INVALID_ARG;
+  for (const void* p : {static_cast<const void*>(dY), static_cast<const void*>(X), static_cast<const void*>(W),
+                        static_cast<const void*>(dX), static_cast<const void*>(dW), static_cast<const void*>(db)})
+    if (p && !is_aligned(p, 4)) return BL_ERR_ALIGNMENT;
+  const BwLayout l = bw_layout(M, N, K);
+  if ((dX || dW) && (!ws || !is_aligned(ws, kWsAlign) || ws_bytes < l.total)) return BL_ERR_WORKSPACE;
+  char* w = static_cast<char*>(ws);
+  bl_status st = BL_OK;
+  if (dX) {   // dX [M, K] = dY [M, N] W [N, K]: A = dY (K-major over n), B = W^T [K, N]
+    float* ahi = reinterpret_cast<float*>(w);
+    float* alo = reinterpret_cast<float*>(w + l.dx_a);
+    float* bhi = reinterpret_cast<float*>(w + 2 * l.dx_a);
+    float* blo = reinterpret_cast<float*>(w + 2 * l.dx_a + l.dx_b);
+    split_tf32_kernel<false><<<grid_for(M * l.ldN, 256), 256, 0, stream>>>(dY, M, N, N, ahi, alo, l.ldN);
+    split_tf32_kernel<true><<<grid_for(ceil_div(l.ldN, 32) * ceil_div(K, 32), 1), 256, 0, stream>>>(W, N, K, K, bhi,
+                                                                                                   blo, l.ldN);
+    if ((st = launch_status()) != BL_OK) return st;
+    if ((st = run_tf32x3(ahi, alo, bhi, blo, l.ldN, M, K, N, dX, stream)) != BL_OK) return st;
+  }
+  if (dW) {   // dW [N, K] = dY^T [N, M] X [M, K]: A = dY^T [N, M], B = X^T [K, M]
+    float* ahi = reinterpret_cast<float*>(w);
+    float* alo = reinterpret_cast<float*>(w + l.dw_a);
+    float* bhi = reinterpret_cast<float*>(w + 2 * l.dw_a);
+    float* blo = reinterpret_cast<float*>(w + 2 * l.dw_a + l.dw_b);
+    split_tf32_kernel<true><<<grid_for(ceil_div(l.ldM, 32) * ceil_div(N, 32), 1), 256, 0, stream>>>(dY, M, N, N, ahi,
+                                                                                                   alo, l.ldM);
+    split_tf32_kernel<true><<<grid_for(ceil_div(l.ldM, 32) * ceil_div(K, 32), 1), 256, 0, stream>>>(X, M, K, K, bhi,
+                                                                                                   blo, l.ldM);
+    if ((st = launch_status()) != BL_OK) return st;
+    if ((st = run_tf32x3(ahi, alo, bhi, blo, l.ldM, N, K, M, dW, stream)) != BL_OK) return st;
+  }
+  if (db) {
+    colsum_kernel<<<grid_for(N, 256), 256, 0, stream>>>(dY, M, N, db);
+    if ((st = launch_status()) != BL_OK) return st;
+  }
+  return BL_OK;
 }
 
 // ---- deployed checkpoint ------------------------------------------------------

@@ -27,6 +27,10 @@ What it computes, and where the method is stated (page title, then section):
   the ternary weights at five per byte plus the float32 pieces (beta, biases),
   byte-exact; the file layout is read in ``oracle/checkpoint.py``.
 
+* ``backward.ste_backward`` -- part 2, section "autograd on a byte-graph, and
+  the straight-through lie": dL/dx = (dL/dy) W, dL/dW = (dL/dy)^T x,
+  dL/db = sum of dL/dy, on the float32 masters, in float64.
+
 Readings taken where the pages leave a step open:
 
 1. Precision.  The pages' arrays are numpy float32, so every quantizer step is
@@ -48,8 +52,14 @@ Readings taken where the pages leave a step open:
    byte-exactness): little-endian records of name, N, K, flags, beta bits,
    the packed rows without their 16-byte padding, then the bias.
 
-Every function here is pinned by ``tests/test_oracle_pins.py`` against hand-
-worked values, closed forms, invariants or brute force; none is unpinned.
+8. The straight-through backward uses the float32 master W and the float32
+   input x (the page: the quantizers and the per-row scale are treated as the
+   identity), not the dequantized beta W_q or s x_q.
+
+Every function here is pinned (``tests/test_oracle_pins.py``,
+``tests/test_oracle_checkpoint.py``, ``tests/test_oracle_backward.py``)
+against hand-worked values, closed forms, invariants or brute force; none is
+unpinned.
 """
 from .layer import (  # noqa: F401
     ACT_QMAX,

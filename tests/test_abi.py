@@ -241,3 +241,20 @@ def test_deployed_checkpoint_host_side(lib, tmp_path):
     assert lib.bl_save_deployed(str(empty).encode(), None, 0, None) == 0
     assert empty.read_bytes() == checkpoint.write_deployed([])
     assert lib.bl_save_deployed(str(tmp_path / "no_dir" / "x.blt").encode(), None, 0, None) == 8
+
+
+def test_backward_host_checks(lib):
+    assert lib.bl_linear_backward_workspace_size(0, 4, 4) == 0
+    # dX [M,K] splits: dY [M, ldN] and W^T [K, ldN] (hi and lo); dW: dY^T [N, ldM] and X^T [K, ldM]
+    M, N, K = 5, 6, 7
+    ldN, ldM = 8, 8
+    expect = max(2 * (_al(M * ldN * 4) + _al(K * ldN * 4)), 2 * (_al(N * ldM * 4) + _al(K * ldM * 4)))
+    assert lib.bl_linear_backward_workspace_size(M, N, K) == expect
+    assert lib.bl_linear_backward(NULL, 16, 16, 2, 3, 4, 16, 16, 16, 256, 1 << 20, NULL) == 1   # no dY
+    assert lib.bl_linear_backward(16, NULL, 16, 2, 3, 4, 16, 16, 16, 256, 1 << 20, NULL) == 1   # dW without X
+    assert lib.bl_linear_backward(16, 16, NULL, 2, 3, 4, 16, 16, 16, 256, 1 << 20, NULL) == 1   # dX without W
+    assert lib.bl_linear_backward(18, 16, 16, 2, 3, 4, 16, 16, 16, 256, 1 << 20, NULL) == 2
+    assert lib.bl_linear_backward(16, 16, 16, 2, 3, 4, 16, 16, 16, NULL, 0, NULL) == 4
+    assert lib.bl_linear_backward(16, 16, 16, 2, 3, 4, 16, 16, 16, 256, 8, NULL) == 4
+    assert lib.bl_linear_backward(NULL, NULL, NULL, 0, 3, 4, NULL, NULL, NULL, NULL, 0, NULL) == 0
+    assert lib.bl_linear_backward(16, 16, 16, 2, 0, 4, 16, 16, 16, 256, 1 << 20, NULL) == 1

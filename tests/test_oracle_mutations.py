@@ -112,6 +112,35 @@ MUTANTS = {
 }
 
 
+def _ste_dequantized(dY, X, W):
+    from oracle import backward as bw
+    import oracle as o
+    beta = o.absmean_beta(W, 1e-5)
+    Wd = o.ternarize(W, beta).astype(np.float32) * np.float32(beta)
+    return bw.__dict__["_orig"](dY, X, Wd)
+
+
+def _ste_transposed(dY, X, W):
+    dY, X, W = (np.asarray(a, np.float64) for a in (dY, X, W))
+    return dY @ W, X.T @ dY if X.shape[1] == dY.shape[1] else (dY.T @ X), dY.sum(0)
+
+
+def _ste_db_mean(dY, X, W):
+    dX, dW, db = __import__("oracle.backward", fromlist=["x"]).__dict__["_orig"](dY, X, W)
+    return dX, dW, db / np.asarray(dY).shape[0]
+
+
+@pytest.mark.parametrize("mutant", [_ste_dequantized, _ste_transposed, _ste_db_mean],
+                         ids=lambda f: f.__name__)
+def test_backward_pins_reject_mutant(mutant, monkeypatch):
+    from oracle import backward as bw
+    monkeypatch.setattr(bw, "_orig", bw.ste_backward, raising=False)
+    monkeypatch.setattr(bw, "ste_backward", mutant)
+    rc = pytest.main(["-q", "-x", "-p", "no:cacheprovider",
+                      __file__.replace("test_oracle_mutations.py", "test_oracle_backward.py")])
+    assert rc != 0
+
+
 def test_checkpoint_pins_reject_padded_rows(monkeypatch):
     from oracle import checkpoint as ck
     monkeypatch.setattr(ck, "write_deployed", _write_deployed_padded_rows)
