@@ -426,8 +426,8 @@ bl_status run_tc(const int8_t* Xq, int64_t ldx, int64_t M, int64_t K, const void
 // every row tile there).
 bl_status unpack_rows(const uint8_t* Wp, int64_t N, int64_t K, int64_t ldp, int8_t* Wq, int64_t ldk,
                       cudaStream_t st) {
-  const int64_t words = ceil_div(ceil_div(K, 5), 4);
-  unpack5_rows_kernel<<<grid_for(N * words, 256), 256, 0, st>>>(Wp, N, K, ldp, Wq, ldk);
+  if (ldk % 16 != 0 || ldk < K || ldp % 16 != 0 || !is_aligned(Wp, 16) || !is_aligned(Wq, 16)) return BL_ERR_ALIGNMENT;
+  unpack5_rows_kernel<<<grid_for(N * (ldp / 16), kUnpackThreads, 4), kUnpackThreads, 0, st>>>(Wp, N, ldp, Wq, ldk);
   return launch_status();
 }
 

@@ -87,7 +87,23 @@ struct TcArgs {
   int32_t* part;       // [split, M, N] int32 partial sums (split > 1)
 };
 
-// y (or acc) for 32 columns nb.. of row m from the 32 sums r.
+// Output tile t -> (row tile, column tile), grouped: consecutive tiles walk
+// kTcGroupM row tiles down one column of tiles before moving right, so the
+// CTAs running at one time share a few A row panels and B column panels and
+// the operands they re-read stay in L2.
+constexpr int kTcGroupM = 8;
+__device__ __forceinline__ void tc_tile_coords(const TcArgs& a, int t, int& tm, int& tn) {
+  const int per_group = kTcGroupM * a.tiles_n;
+  const int g = t / per_group, r = t - g * per_group;
+  const int first = g * kTcGroupM;
+  const int gm = min(kTcGroupM, a.tiles_m - first);
+  tm = first + r % gm;
+  tn = r / gm;
+}
+
+// y (or acc) for 32 columns nb.. of row m from the 32 sums r (streaming
+// stores: the output is not read again, so it should not push the operands
+// out of L2).
 template <bool kDequant>
 __device__ __forceinline__ void tc_store32(const TcArgs& a, const uint32_t (&r)[32], int64_t m, int64_t nb,
                                            float sbm, bool vec) {
@@ -102,7 +118,7 @@ __device__ __forceinline__ void tc_store32(const TcArgs& a, const uint32_t (&r)[
     if (vec && nb + 32 <= a.N) {
 #pragma unroll
       for (int j = 0; j < 32; j += 4)
-        *reinterpret_cast<float4*>(yr + j) = make_float4(y[j], y[j + 1], y[j + 2], y[j + 3]);
+        __stcs(reinterpret_cast<float4*>(yr + j), make_float4(y[j], y[j + 1], y[j + 2], y[j + 3]));
     } else {
       for (int j = 0; j < 32 && nb + j < a.N; ++j) yr[j] = y[j];
     }
@@ -111,7 +127,7 @@ __device__ __forceinline__ void tc_store32(const TcArgs& a, const uint32_t (&r)[
     if (vec && nb + 32 <= a.N) {
 #pragma unroll
       for (int j = 0; j < 32; j += 4)
-        *reinterpret_cast<int4*>(ar + j) = make_int4(int(r[j]), int(r[j + 1]), int(r[j + 2]), int(r[j + 3]));
+        __stcs(reinterpret_cast<int4*>(ar + j), make_int4(int(r[j]), int(r[j + 1]), int(r[j + 2]), int(r[j + 3])));
     } else {
       for (int j = 0; j < 32 && nb + j < a.N; ++j) ar[j] = int(r[j]);
     }
@@ -184,7 +200,8 @@ gemm_tc_kernel(const __grid_constant__ TcMaps maps, const TcArgs a) {
       for (int w = blockIdx.x; w < nwork && !*err; w += gridDim.x) {
         int t, j, kb0, kb1;
         work(w, t, j, kb0, kb1);
-        const int tm = t / a.tiles_n, tn = t - tm * a.tiles_n;
+        int tm, tn;
+        tc_tile_coords(a, t, tm, tn);
         for (int kb = kb0; kb < kb1; ++kb, ++it) {
           const int s = it % kStages;
           if (it >= kStages && !mbar_wait(&empty[s], uint32_t(it / kStages - 1) & 1u)) {
@@ -250,7 +267,8 @@ gemm_tc_kernel(const __grid_constant__ TcMaps maps, const TcArgs a) {
       for (int w = blockIdx.x; w < nwork && !*err; w += gridDim.x) {
         int t, j, kb0, kb1;
         work(w, t, j, kb0, kb1);
-        const int tn = t % a.tiles_n;
+        int tm, tn;
+        tc_tile_coords(a, t, tm, tn);
         for (int c = kb0 / kTcChunk; c * kTcChunk < kb1; ++c, ++pj) {
           const int p = pj % kPkStages;
           if (pj >= kPkStages && !mbar_wait(&pk_empty[p], uint32_t(pj / kPkStages - 1) & 1u)) {
@@ -367,7 +385,8 @@ gemm_tc_kernel(const __grid_constant__ TcMaps maps, const TcArgs a) {
       }
       if (*err) break;
       tc_fence_after();
-      const int tm = t / a.tiles_n, tn = t - tm * a.tiles_n;
+      int tm, tn;
+      tc_tile_coords(a, t, tm, tn);
       const int64_t m = int64_t(tm) * kTcBM + row;
       const int64_t n0 = int64_t(tn) * kBN;
       const uint32_t taddr = tmem + (uint32_t(q * 32) << 16) + uint32_t(b * kBN);
@@ -465,37 +484,62 @@ tc_reduce_kernel(const int32_t* __restrict__ part, int split, int64_t M, int64_t
   }
 }
 
-// W_q from the packed format into int8 rows [N, ldq] for the TMA loads: one
-// thread per 4 packed bytes (20 trits); trits at or past K are not written.
-__global__ void __launch_bounds__(256)
-unpack5_rows_kernel(const uint8_t* __restrict__ Wp, int64_t N, int64_t K, int64_t ldp,
-                    int8_t* __restrict__ Wq, int64_t ldq) {
-  const int64_t words = ceil_div(ceil_div(K, 5), 4);
-  const int64_t total = N * words;
+// W_q from the packed format into int8 rows [N, ldq] (ldq % 16 == 0) for the
+// tensor-core GEMM's TMA loads, at HBM speed: one thread per 16 packed bytes
+// (80 trits), one 16-byte load and five 16-byte stores (those below ldq), so
+// every warp reads 512 and writes 2560 contiguous bytes.  Trits t0..t3 of a
+// byte come from a table in shared memory with one copy per lane (word
+// 32 b + lane: no bank conflicts); t4 = floor(b/81) - 1 for four bytes at once
+// from b * 203 in 16-bit lanes (bits 14..15, exact for b <= 242); byte_perm
+// lays the 20 trits of four bytes out in order.  Row bytes from K to ldq hold
+// whatever the packed padding decodes to (121: zero trits); the GEMM's tensor
+// map ends at K, so it never reads them.
+constexpr int kUnpackThreads = 256;
+
+__global__ void __launch_bounds__(kUnpackThreads)
+unpack5_rows_kernel(const uint8_t* __restrict__ Wp, int64_t N, int64_t ldp, int8_t* __restrict__ Wq,
+                    int64_t ldq) {
+  __shared__ uint32_t lut[256 * 32];
+  for (int i = threadIdx.x; i < 256 * 32; i += kUnpackThreads) {
+    uint32_t b = uint32_t(i) >> 5, v = 0;
+    if (b > 242u) b = 121u;       // not a code: read as zero trits
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      v |= ((b % 3u + 255u) & 0xFFu) << (8 * k);
+      b /= 3u;
+    }
+    lut[i] = v;
+  }
+  __syncthreads();
+  const uint32_t* lut_l = lut + (threadIdx.x & 31);
+  const int64_t cpr = ldp / 16;                 // 16-byte chunks per packed row
+  const int64_t total = N * cpr;
   const bool small = total < (int64_t(1) << 32);
   for (int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
        i += int64_t(gridDim.x) * blockDim.x) {
-    int64_t row, g;
-    split_index(i, words, small, row, g);
-    const uint32_t w = *reinterpret_cast<const uint32_t*>(Wp + row * ldp + 4 * g);
-    uint32_t t[20];
+    int64_t row, c;
+    split_index(i, cpr, small, row, c);
+    const uint4 w4 = __ldg(reinterpret_cast<const uint4*>(Wp + row * ldp) + c);
+    const uint32_t wv[4] = {w4.x, w4.y, w4.z, w4.w};
+    uint32_t o[20];
 #pragma unroll
-    for (int b = 0; b < 4; ++b) {
-      int t5[5];
-      unpack5_byte((w >> (8 * b)) & 0xFFu, t5);
-#pragma unroll
-      for (int k = 0; k < 5; ++k) t[5 * b + k] = uint32_t(uint8_t(int8_t(t5[k])));
+    for (int q = 0; q < 4; ++q) {
+      const uint32_t four = wv[q];
+      const uint32_t L0 = lut_l[(four & 0xFFu) << 5], L1 = lut_l[((four >> 8) & 0xFFu) << 5];
+      const uint32_t L2 = lut_l[((four >> 16) & 0xFFu) << 5], L3 = lut_l[(four >> 24) << 5];
+      const uint32_t lo = (four & 0x00FF00FFu) * 203u, hi = ((four >> 8) & 0x00FF00FFu) * 203u;
+      const uint32_t T = (((__byte_perm(lo, hi, 0x7351) >> 6) & 0x03030303u) + 0x7F7F7F7Fu) ^ 0x80808080u;
+      o[5 * q + 0] = L0;
+      o[5 * q + 1] = __byte_perm(T, L1, 0x6540);
+      o[5 * q + 2] = __byte_perm(__byte_perm(L1, T, 0x0053), L2, 0x5410);
+      o[5 * q + 3] = __byte_perm(__byte_perm(L2, T, 0x0632), L3, 0x4210);
+      o[5 * q + 4] = __byte_perm(L3, T, 0x7321);
     }
-    int8_t* out = Wq + row * ldq + 20 * g;
-    const int64_t k0 = 20 * g;
-    if (k0 + 20 <= K) {
+    int8_t* dst = Wq + row * ldq + 80 * c;
 #pragma unroll
-      for (int v = 0; v < 5; ++v)
-        reinterpret_cast<uint32_t*>(out)[v] =
-            t[4 * v] | t[4 * v + 1] << 8 | t[4 * v + 2] << 16 | t[4 * v + 3] << 24;
-    } else {
-      for (int k = 0; k < 20 && k0 + k < K; ++k) out[k] = int8_t(t[k]);
-    }
+    for (int v = 0; v < 5; ++v)
+      if (80 * c + 16 * v + 16 <= ldq)
+        *reinterpret_cast<uint4*>(dst + 16 * v) = make_uint4(o[4 * v], o[4 * v + 1], o[4 * v + 2], o[4 * v + 3]);
   }
 }
 

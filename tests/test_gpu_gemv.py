@@ -82,11 +82,12 @@ def test_group_mixed_calls(bl):
         assert_y_exact(host(Y), ref)
 
 
-@pytest.mark.parametrize("M,K,N", [(1, 50000, 300), (2, 50000, 200), (2, 20000, 333), (4, 40000, 129),
+@pytest.mark.parametrize("M,K,N", [(1, 50000, 300), (2, 50000, 200), (2, 20000, 333), (4, 30000, 129),
                                    (3, 12345, 1000)])
 def test_gemv_long_rows(bl, M, K, N):
     """Rows of up to 10000 packed bytes: several 16-byte chunks per lane and up
-    to 16 warps per row slice."""
+    to 16 warps per row slice (M = 4 at K = 30000: 120 KB of decode-order codes
+    beside the 64 KB table)."""
     p = random_problem(M * 7 + K + N, M, K, N)
     Wd, beta = quantized(bl, p)
     assert bl.linear_plan(M, N, K, bl.PACK5)[0] == bl.PATH_GEMV
@@ -94,6 +95,18 @@ def test_gemv_long_rows(bl, M, K, N):
         Y = bl.linear(dev(p.X), Wd, bl.PACK5, N, K, beta, eps=p.eps, static_weights=static)
         assert bl.sync_status() == "BL_OK"
         assert_y_exact(host(Y), oracle.bitlinear(p.X, p.W, p.eps)["Y"])
+
+
+def test_gemv_declines_codes_beyond_shared_memory(bl):
+    """M = 4 at K = 40000 needs 160 KB of decode-order codes: the GEMV declines
+    and AUTO takes another path (the answer is the same)."""
+    assert bl.linear_plan(4, 129, 40000, bl.PACK5, bl.PATH_GEMV)[0] == -1
+    assert bl.linear_plan(4, 129, 40000, bl.PACK5)[0] == bl.PATH_SIMT
+    p = random_problem(77, 4, 40000, 129)
+    Wd, beta = quantized(bl, p)
+    Y = bl.linear(dev(p.X), Wd, bl.PACK5, 129, 40000, beta, eps=p.eps)
+    assert bl.sync_status() == "BL_OK"
+    assert_y_exact(host(Y), oracle.bitlinear(p.X, p.W, p.eps)["Y"])
 
 
 def test_chain_output_feeds_next_input(bl):
