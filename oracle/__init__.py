@@ -22,6 +22,10 @@ What it computes, and where the method is stated (page title, then section):
   ternary GPT" and "Layout" (5 ternary values per byte, ~1.6 bits/weight), and
   "a 1-bit llm, from scratch", tl;dr (1.6 bits each).  Byte = sum_k (t_k+1) 3^k.
 
+* ``rmsnorm`` and ``rmsnorm_act_quant`` -- part 2, section "attention, as graph
+  ops" (RMSNorm equation, learnable gain g), and the PyPI page's pre-norm block
+  "x = x + mha(norm1(x))": the normalized rows feed the BitLinear, so its
+  activation quantization follows the norm.
 * ``checkpoint.write_deployed`` / ``checkpoint.read_deployed`` -- "ultragraph-1bit
   0.12.0" (PyPI), section "A whole ternary GPT": the deployed checkpoint keeps
   the ternary weights at five per byte plus the float32 pieces (beta, biases),
@@ -56,6 +60,11 @@ Readings taken where the pages leave a step open:
    input x (the page: the quantizers and the per-row scale are treated as the
    identity), not the dequantized beta W_q or s x_q.
 
+9. RMSNorm's mean of squares is the exact sum of the float32 squares, rounded
+   once to float64, divided by d in float64 and rounded to float32 (the reading
+   of the mean in beta); + eps, sqrt, x / r and * g are float32 steps.  The
+   norm's eps is its own argument, separate from the quantizers'.
+
 Every function here is pinned (``tests/test_oracle_pins.py``,
 ``tests/test_oracle_checkpoint.py``, ``tests/test_oracle_backward.py``)
 against hand-worked values, closed forms, invariants or brute force; none is
@@ -72,6 +81,8 @@ from .layer import (  # noqa: F401
     dequant,
     pack5,
     pack5_ldp,
+    rmsnorm,
+    rmsnorm_act_quant,
     ternarize,
     unpack5,
 )

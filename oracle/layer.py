@@ -148,6 +148,38 @@ def dequant(acc: np.ndarray, s: np.ndarray, beta, bias: Optional[np.ndarray] = N
     return y.astype(_F32)
 
 
+def rmsnorm(X: np.ndarray, g: np.ndarray, eps_norm: float) -> np.ndarray:
+    """RMSNorm(x) = x / sqrt((1/d) sum_i x_i^2 + eps) * g over the last dimension
+    ("attention, as graph ops", RMSNorm equation; learnable gain g, float32).
+
+    Reading, as for beta: the sum of squares is the exact real sum (each float32
+    square is exact in float64), rounded once to float64 (``math.fsum``),
+    divided by d in float64 and rounded to float32; then, all in float32:
+    + eps, sqrt (correctly rounded), x / that, times g.
+    """
+    X = np.asarray(X, dtype=_F32)
+    g = np.asarray(g, dtype=_F32)
+    if X.ndim != 2 or g.shape != (X.shape[1],):
+        raise ValueError("X must be [M, d] and g [d]")
+    if not (np.all(np.isfinite(X)) and np.all(np.isfinite(g))):
+        raise ValueError("inputs must be finite")
+    M, d = X.shape
+    out = np.empty_like(X)
+    for m in range(M):
+        S = math.fsum(float(v) * float(v) for v in X[m].tolist())
+        ms = _F32(S / d)
+        r = np.sqrt(_F32(ms + _F32(eps_norm)))
+        out[m] = (X[m] / r) * g
+    return out
+
+
+def rmsnorm_act_quant(X: np.ndarray, g: np.ndarray, eps_norm: float, eps: float):
+    """The pre-norm block's input to a BitLinear: x_q, s = act_quant(RMSNorm(x))
+    (the PyPI page's block "x = x + mha(norm1(x))": the normalized rows are the
+    layer's activations)."""
+    return act_quant(rmsnorm(X, g, eps_norm), eps)
+
+
 def bitlinear(X: np.ndarray, W: np.ndarray, eps: float = 1e-5,
               bias: Optional[np.ndarray] = None) -> dict:
     """The whole layer from float32 W and X: every intermediate is returned."""

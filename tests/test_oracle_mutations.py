@@ -141,6 +141,45 @@ def test_backward_pins_reject_mutant(mutant, monkeypatch):
     assert rc != 0
 
 
+def _rms_sum_not_mean(X, g, eps):
+    X = np.asarray(X, F32)
+    out = np.empty_like(X)
+    for m in range(X.shape[0]):
+        S = math.fsum(float(v) * float(v) for v in X[m])
+        out[m] = (X[m] / np.sqrt(F32(F32(S) + F32(eps)))) * np.asarray(g, F32)
+    return out
+
+
+def _rms_float32_running_sum(X, g, eps):
+    X = np.asarray(X, F32)
+    out = np.empty_like(X)
+    for m in range(X.shape[0]):
+        S = F32(0)
+        for v in X[m]:
+            S = F32(S + F32(v * v))
+        out[m] = (X[m] / np.sqrt(F32(F32(S / F32(X.shape[1])) + F32(eps)))) * np.asarray(g, F32)
+    return out
+
+
+def _rms_eps_outside_sqrt(X, g, eps):
+    X = np.asarray(X, F32)
+    out = np.empty_like(X)
+    for m in range(X.shape[0]):
+        S = math.fsum(float(v) * float(v) for v in X[m])
+        out[m] = (X[m] / F32(np.sqrt(F32(S / X.shape[1])) + F32(eps))) * np.asarray(g, F32)
+    return out
+
+
+@pytest.mark.parametrize("mutant", [_rms_sum_not_mean, _rms_float32_running_sum, _rms_eps_outside_sqrt],
+                         ids=lambda f: f.__name__)
+def test_rmsnorm_pins_reject_mutant(mutant, monkeypatch):
+    monkeypatch.setattr(ob, "rmsnorm", mutant)
+    monkeypatch.setattr(oracle, "rmsnorm", mutant)
+    rc = pytest.main(["-q", "-x", "-p", "no:cacheprovider",
+                      __file__.replace("test_oracle_mutations.py", "test_oracle_rmsnorm.py")])
+    assert rc != 0
+
+
 def test_checkpoint_pins_reject_padded_rows(monkeypatch):
     from oracle import checkpoint as ck
     monkeypatch.setattr(ck, "write_deployed", _write_deployed_padded_rows)
