@@ -155,6 +155,21 @@ bl_status bl_unpack(const uint8_t* Wp, int64_t N, int64_t K, int64_t ldp, int8_t
 bl_status bl_quantize_act(const float* X, int64_t M, int64_t K, float eps, int8_t* Xq,
                           float* s, cudaStream_t stream);
 
+/* RMSNorm fused into the per-row activation quantization: the input of a
+ * BitLinear in a pre-norm block ("ultragraph-1bit 0.12.0" (PyPI): "x = x +
+ * mha(norm1(x))"), with RMSNorm(x) = x / sqrt((1/K) sum_k x_k^2 + eps_norm) * g
+ * ("ultragraph -- when the graph is the 1-bit LLM, part 2", section "attention,
+ * as graph ops"), then s and x_q of bl_quantize_act on the normalized row.
+ *   X [M, K] float32 contiguous, g [K] float32 (the gain), 1 <= K <= 49152.
+ *   eps_norm, eps: finite, > 0 (the norm's and the quantizer's).
+ *   Xq [M, K] int8, s [M] float32 (outputs).
+ * The mean of squares is exact: the sum of the float32 squares is formed
+ * exactly and rounded once to float64, divided by K in float64 and rounded to
+ * float32; + eps_norm, sqrt, x / r and * g are float32 IEEE steps.  One read of
+ * X; rows are independent. */
+bl_status bl_rmsnorm_quantize_act(const float* X, int64_t M, int64_t K, const float* g, float eps_norm, float eps,
+                                  int8_t* Xq, float* s, cudaStream_t stream);
+
 /* Bytes of `ws` that bl_linear needs for this shape and format (0 for shapes
  * that take the decode GEMV: ws may then be NULL). */
 size_t bl_linear_workspace_size(int64_t M, int64_t N, int64_t K, bl_wfmt f);

@@ -57,6 +57,7 @@ SIGNATURES = {
     "bl_pack": (_I, [_P, _I64, _I64, _P, _I64, _P]),
     "bl_unpack": (_I, [_P, _I64, _I64, _I64, _P, _P]),
     "bl_quantize_act": (_I, [_P, _I64, _I64, _F, _P, _P, _P]),
+    "bl_rmsnorm_quantize_act": (_I, [_P, _I64, _I64, _P, _F, _F, _P, _P, _P]),
     "bl_linear_workspace_size": (_SZ, [_I64, _I64, _I64, _I]),
     "bl_linear_ex_workspace_size": (_SZ, [_I64, _I64, _I64, _I, _I]),
     "bl_linear": (_I, [_P, _I64, _I64, _P, _I, _I64, _I64, _P, _P, _F, _P, _P, _SZ, _P]),
@@ -237,6 +238,19 @@ def quantize_act(X, eps: float = 1e-5) -> Tuple:
     s = torch.empty((M,), dtype=torch.float32, device=X.device)
     _check("bl_quantize_act", lib.bl_quantize_act(_ptr(X), M, K, eps, _ptr(Xq), _ptr(s),
                                                   _stream(torch, X)))
+    return Xq, s
+
+
+def rmsnorm_quantize_act(X, g, eps_norm: float = 1e-5, eps: float = 1e-5) -> Tuple:
+    """RMSNorm with gain g, then per-row int8 quantization: (Xq int8 [M,K], s float32 [M])."""
+    torch, lib = _torch(), load()
+    _dev(X, torch.float32)
+    _dev(g, torch.float32)
+    M, K = X.shape
+    Xq = torch.empty((M, K), dtype=torch.int8, device=X.device)
+    s = torch.empty((M,), dtype=torch.float32, device=X.device)
+    _check("bl_rmsnorm_quantize_act", lib.bl_rmsnorm_quantize_act(
+        _ptr(X), M, K, _ptr(g), eps_norm, eps, _ptr(Xq), _ptr(s), _stream(torch, X)))
     return Xq, s
 
 

@@ -22,6 +22,7 @@
 #include "gemm_tc.cuh"
 #include "deployed_io.cuh"
 #include "ste_backward.cuh"
+#include "rmsnorm_quant.cuh"
 
 namespace bl {
 namespace {
@@ -719,6 +720,19 @@ bl_status bl_quantize_act(const float* X, int64_t M, int64_t K, float eps, int8_
   if (!X || !Xq || !s || M > (int64_t(1) << 31) - 1) return BL_ERR_INVALID_ARG;
   if (!is_aligned(X, 4) || !is_aligned(s, 4)) return BL_ERR_ALIGNMENT;
   launch_act_quant(X, M, K, eps, Xq, K, s, stream);
+  return launch_status();
+}
+
+bl_status bl_rmsnorm_quantize_act(const float* X, int64_t M, int64_t K, const float* g, float eps_norm, float eps,
+                                  int8_t* Xq, float* s, cudaStream_t stream) {
+  if (M < 0 || K < 1 || K > kRnMaxK || !eps_ok(eps) || !eps_ok(eps_norm)) return BL_ERR_INVALID_ARG;
+  if (M == 0) return BL_OK;
+  if (!X || !g || !Xq || !s || M > (int64_t(1) << 31) - 1) return BL_ERR_INVALID_ARG;
+  if (!is_aligned(X, 4) || !is_aligned(g, 4) || !is_aligned(s, 4)) return BL_ERR_ALIGNMENT;
+  const int smem = int(K * 4);
+  if (cudaFuncSetAttribute(rmsnorm_quant_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+    return BL_ERR_CUDA;
+  rmsnorm_quant_kernel<<<unsigned(M), kRnThreads, smem, stream>>>(X, K, g, eps_norm, eps, Xq, K, s);
   return launch_status();
 }
 

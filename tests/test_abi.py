@@ -258,3 +258,12 @@ def test_backward_host_checks(lib):
     assert lib.bl_linear_backward(16, 16, 16, 2, 3, 4, 16, 16, 16, 256, 8, NULL) == 4
     assert lib.bl_linear_backward(NULL, NULL, NULL, 0, 3, 4, NULL, NULL, NULL, NULL, 0, NULL) == 0
     assert lib.bl_linear_backward(16, 16, 16, 2, 0, 4, 16, 16, 16, 256, 1 << 20, NULL) == 1
+
+
+def test_rmsnorm_quant_host_checks(lib):
+    assert lib.bl_rmsnorm_quantize_act(NULL, 0, 8, 16, 1e-5, 1e-5, NULL, NULL, NULL) == 0
+    assert lib.bl_rmsnorm_quantize_act(16, 2, 8, NULL, 1e-5, 1e-5, 16, 16, NULL) == 1
+    assert lib.bl_rmsnorm_quantize_act(16, 2, 8, 16, 0.0, 1e-5, 16, 16, NULL) == 1
+    assert lib.bl_rmsnorm_quantize_act(16, 2, 8, 16, 1e-5, float("inf"), 16, 16, NULL) == 1
+    assert lib.bl_rmsnorm_quantize_act(16, 2, 49153, 16, 1e-5, 1e-5, 16, 16, NULL) == 1
+    assert lib.bl_rmsnorm_quantize_act(18, 2, 8, 16, 1e-5, 1e-5, 16, 16, NULL) == 2
