@@ -520,6 +520,7 @@ bl_status run_gemv_group(int64_t M, const GemvCall* c, int n, bool prefetch, cud
     P.eps = c[i].eps;
     P.Y = c[i].Y;
     P.acc = c[i].acc;
+    if (!c[i].X || !is_aligned(c[i].X, 16)) P.xs_bytes = 0u;   // X read from global memory instead
     P.cta0 = cta;
     cta += int(ceil_div(c[i].N, int64_t(P.rows_per_cta)));   // every CTA has at least one row
     smem = P.smem > smem ? P.smem : smem;

@@ -13,9 +13,10 @@
 //
 // Per CTA (one per SM; two fit when the CTA's weights are small):
 //   * before the dependency wait (programmatic dependent launch): mbarriers,
-//     the decode table and -- when the caller declares the weights static --
-//     the bulk copies (TMA engine) of the CTA's whole block of packed rows
-//     into shared memory, so the weight stream overlaps the previous kernel;
+//     a bulk copy (TMA engine) of the decode table (a compile-time constant in
+//     global memory) and -- when the caller declares the weights static --
+//     the bulk copies of the CTA's whole block of packed rows into shared
+//     memory, so the weight stream overlaps the previous kernel;
 //   * griddepcontrol.wait, then launch_dependents (the next kernel may start
 //     its own prologue and weight copies while this one computes);
 //   * X: per-row absmax over the whole row (every CTA reads it, from L2), then
@@ -49,6 +50,7 @@ constexpr uint32_t kLutBytes = 256 * 256;      // a row for every byte value: no
 constexpr uint32_t kGemvMaxSmem = 232448 - 1024;  // 227 KB per CTA, less the static arrays
 constexpr uint32_t kGemvSegTarget = 12 * 1024;  // bytes per bulk copy (one mbarrier each)
 constexpr int kGemvMaxStages = 24;
+constexpr uint32_t kGemvXStageMax = 48 * 1024;  // float32 X rows staged in shared memory up to this
 
 struct GemvProb {
   const float* X;      // [M, K] float32 (activation quantization inside) or nullptr
@@ -65,7 +67,7 @@ struct GemvProb {
   int rows_per_cta;
   int S, G;            // warps per row slice, rows in flight
   int seg_rows, nstage;
-  uint32_t xc_off, part_off, bar_off, stage_off, smem;
+  uint32_t xc_off, xs_off, xs_bytes, part_off, bar_off, stage_off, smem;
 };
 
 struct GemvArgs {
@@ -102,13 +104,15 @@ inline bool gemv_plan_prob(int64_t M, int64_t N, int64_t K, int64_t ldp, int cta
   if (seg > P.rows_per_cta) seg = P.rows_per_cta;
   P.seg_rows = int(seg);
   P.xc_off = align_to(kLutBytes, 128);
-  P.part_off = align_to(P.xc_off + uint32_t(M * 5 * ldp), 16);
+  P.xs_off = align_to(P.xc_off + uint32_t(M * 5 * ldp), 16);
+  P.xs_bytes = (uint64_t(M * K * 4) <= kGemvXStageMax && K % 4 == 0) ? uint32_t(M * K * 4) : 0u;
+  P.part_off = align_to(P.xs_off + P.xs_bytes, 16);
   P.bar_off = align_to(P.part_off + uint32_t(M * P.rows_per_cta * 4), 16);
   const int64_t nseg = ceil_div(P.rows_per_cta, P.seg_rows);
   const uint32_t stage_bytes = uint32_t(P.seg_rows * ldp);
   int64_t ns = nseg < kGemvMaxStages ? nseg : kGemvMaxStages;
   for (; ns >= 1; --ns) {
-    P.stage_off = align_to(P.bar_off + uint32_t(8 * ns), 128);
+    P.stage_off = align_to(P.bar_off + uint32_t(8 * (ns + 2)), 128);
     if (int64_t(P.stage_off) + ns * stage_bytes <= kGemvMaxSmem) break;
   }
   if (ns < 1) return false;
@@ -129,6 +133,28 @@ inline bool gemv_feasible(int64_t M, int64_t N, int64_t K, int64_t ldp) {
   GemvProb P;
   return ch > 0 && gemv_plan_prob(M, N, K, ldp, int(N < kGemvCtas ? N : kGemvCtas), ch, P);
 }
+
+// The decode table as it sits in shared memory, built at compile time: word
+// b*64 + l (l < 32) holds trits t0..t3 of byte b as four int8 (lane l's copy;
+// words 32..63 of a row repeat them, so the row pitch is 256 bytes and one
+// byte_perm forms an address).  Bytes above 242 are not codes and read as 121
+// (five zero trits).  Each CTA copies it into shared memory with one bulk copy.
+struct TritLut {
+  uint32_t w[256 * 64];
+};
+constexpr TritLut make_trit_lut() {
+  TritLut t{};
+  for (uint32_t b = 0; b < 256; ++b) {
+    uint32_t x = b > 242u ? 121u : b, v = 0;
+    for (int k = 0; k < 4; ++k) {
+      v |= ((x % 3u + 255u) & 0xFFu) << (8 * k);
+      x /= 3u;
+    }
+    for (uint32_t l = 0; l < 64; ++l) t.w[b * 64 + l] = v;
+  }
+  return t;
+}
+__device__ __align__(128) const TritLut g_trit_lut = make_trit_lut();
 
 __device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void griddep_launch_dependents() {
@@ -181,54 +207,77 @@ __global__ void __launch_bounds__(kGemvThreads, kMinBlocks) gemv_pack5_kernel(co
   };
 
   // ---- prologue: nothing here reads what an earlier kernel may still write
+  // (the decode table is a constant of this library)
+  uint64_t* bar_lut = &bars[nstage];
+  uint64_t* bar_x = &bars[nstage + 1];
   if (tid == 0) {
-    for (int s = 0; s < nstage; ++s) mbar_init(&bars[s], 1);
+    for (int s = 0; s <= nstage + 1; ++s) mbar_init(&bars[s], 1);
     fence_mbar_init();
+    mbar_arrive_expect_tx(bar_lut, kLutBytes);
+    bulk_g2s(smem, &g_trit_lut, kLutBytes, bar_lut);
     if (a.prefetch)
       for (int sg = 0; sg < nseg && sg < nstage; ++sg) issue(sg);
     s_fail = 0;
   }
   if (tid < M) s_x4[tid] = 0;
   for (int i = tid; i < M * rpc; i += kGemvThreads) part[i] = 0;
-  // decode table: word b*64 + l holds trits t0..t3 of byte b as int8 (lane l's
-  // copy); bytes above 242 are not codes and read as 121 (five zero trits)
-  for (int i = tid; i < 256 * 32; i += kGemvThreads) {
-    uint32_t b = uint32_t(i) >> 5, v = 0;
-    if (b > 242u) b = 121u;
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      v |= ((b % 3u + 255u) & 0xFFu) << (8 * k);
-      b /= 3u;
-    }
-    reinterpret_cast<uint32_t*>(smem)[(uint32_t(i) >> 5) * 64u + uint32_t(i & 31)] = v;
-  }
 
   griddep_wait();                 // X (and W unless prefetched) may come from the previous kernel
   griddep_launch_dependents();
-  if (!a.prefetch && tid == 0)
-    for (int sg = 0; sg < nseg && sg < nstage; ++sg) issue(sg);
-  __syncthreads();
+  // float32 X into shared memory by one bulk copy (one latency for the whole row)
+  const bool staged = kFused && P.xs_bytes != 0u;
+  if (tid == 0) {
+    if (staged) {
+      mbar_arrive_expect_tx(bar_x, P.xs_bytes);
+      bulk_g2s(smem + P.xs_off, P.X, P.xs_bytes, bar_x);
+    }
+    if (!a.prefetch)
+      for (int sg = 0; sg < nseg && sg < nstage; ++sg) issue(sg);
+  }
+  if (!__syncthreads_and(staged ? mbar_wait(bar_x, 0u) : true)) {
+    if (tid == 0) {
+      raise_status(kDevTimeout);
+      (void)mbar_wait(bar_lut, 0u);
+      for (int sg = issued > nstage ? issued - nstage : 0; sg < issued; ++sg)
+        (void)mbar_wait(&bars[sg % nstage], uint32_t(sg / nstage) & 1u);
+    }
+    return;
+  }
 
   // ---- activations: codes in decode order, sum of the fifth-position codes
   const int kpad = int(5 * ldp);
   float scm[M];
+  const float* xsrc = staged ? reinterpret_cast<const float*>(smem + P.xs_off) : P.X;
+  // 16-byte loads of X: shared memory when staged, else the read-only path
+  // (four per thread issued together, so the latencies overlap)
+  auto ld4 = [&](const float* p) -> float4 {
+    return staged ? *reinterpret_cast<const float4*>(p) : __ldg(reinterpret_cast<const float4*>(p));
+  };
   if (kFused) {
-    const float* X = P.X;
-    const bool xvec = aligned(X, 16) && (K & 3) == 0;
+    const bool xvec = aligned(P.X, 16) && (K & 3) == 0;
     const int64_t K4 = xvec ? (K >> 2) : 0;
     bool bad = false;
 #pragma unroll
     for (int m = 0; m < M; ++m) {
       float amax = 0.f;
-      const float* xr = X + int64_t(m) * K;
-      for (int64_t i = tid; i < K4; i += kGemvThreads) {
-        const float4 v = __ldg(reinterpret_cast<const float4*>(xr) + i);
-        const float mx = fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w)));
-        bad |= !(mx <= 3.402823466e38f) | (v.x != v.x) | (v.y != v.y) | (v.z != v.z) | (v.w != v.w);
-        amax = fmaxf(amax, mx);
+      const float* xr = xsrc + int64_t(m) * K;
+      for (int64_t i0 = tid; i0 < K4; i0 += 4 * kGemvThreads) {
+        float4 v[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int64_t i = i0 + int64_t(u) * kGemvThreads;
+          v[u] = i < K4 ? ld4(xr + 4 * i) : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const float mx = fmaxf(fmaxf(fabsf(v[u].x), fabsf(v[u].y)), fmaxf(fabsf(v[u].z), fabsf(v[u].w)));
+          bad |= !(mx <= 3.402823466e38f) | (v[u].x != v[u].x) | (v[u].y != v[u].y) | (v[u].z != v[u].z) |
+                 (v[u].w != v[u].w);
+          amax = fmaxf(amax, mx);
+        }
       }
       for (int64_t i = (K4 << 2) + tid; i < K; i += kGemvThreads) {
-        const float v = fabsf(__ldg(xr + i));
+        const float v = fabsf(staged ? xr[i] : __ldg(xr + i));
         bad |= !(v <= 3.402823466e38f);
         amax = fmaxf(amax, v);
       }
@@ -247,7 +296,7 @@ __global__ void __launch_bounds__(kGemvThreads, kMinBlocks) gemv_pack5_kernel(co
   for (int m = 0; m < M; ++m) {
     int x4 = 0;
     unsigned char* xcm = xc + m * kpad;
-    const float* xr = kFused ? P.X + int64_t(m) * K : nullptr;
+    const float* xr = kFused ? xsrc + int64_t(m) * K : nullptr;
     const int8_t* xq = kFused ? nullptr : P.Xq + int64_t(m) * P.ldxq;
     const float sc = kFused ? scm[m] : 0.f, rc = kFused ? act_recip(sc) : 0.f;
     for (int i4 = tid; i4 < (kpad >> 2); i4 += kGemvThreads) {
@@ -256,14 +305,14 @@ __global__ void __launch_bounds__(kGemvThreads, kMinBlocks) gemv_pack5_kernel(co
       if (kFused) {
         bool tie = rc == 0.f;
         if (k + 4 <= K && aligned(xr + k, 16)) {
-          const float4 f = __ldg(reinterpret_cast<const float4*>(xr + k));
+          const float4 f = ld4(xr + k);
           c[0] = act_code_try(f.x, rc, tie);
           c[1] = act_code_try(f.y, rc, tie);
           c[2] = act_code_try(f.z, rc, tie);
           c[3] = act_code_try(f.w, rc, tie);
         } else {
 #pragma unroll
-          for (int e = 0; e < 4; ++e) c[e] = k + e < K ? act_code_try(__ldg(xr + k + e), rc, tie) : 0u;
+          for (int e = 0; e < 4; ++e) c[e] = k + e < K ? act_code_try(xr[k + e], rc, tie) : 0u;
         }
         if (tie)   // rare: a quotient near a half-integer; exact division
           for (int e = 0; e < 4 && k + e < K; ++e) c[e] = uint32_t(uint8_t(int8_t(act_code_slow(xr[k + e], sc))));
@@ -308,10 +357,11 @@ __global__ void __launch_bounds__(kGemvThreads, kMinBlocks) gemv_pack5_kernel(co
     }
   const uint32_t lanebase = uint32_t(lane) * 4u;
 
-  // ---- stream the segments
-  bool ok = true;
+  // ---- stream the segments (the table first; CTA-uniform, since the ring's
+  // loop below has barriers)
+  bool ok = __syncthreads_and(mbar_wait(bar_lut, 0u));
 #pragma unroll 1
-  for (int sg = 0; sg < nseg; ++sg) {
+  for (int sg = 0; sg < nseg && ok; ++sg) {
     const int buf = sg % nstage;
     if (!mbar_wait(&bars[buf], uint32_t(sg / nstage) & 1u)) {
       ok = false;
@@ -379,6 +429,7 @@ __global__ void __launch_bounds__(kGemvThreads, kMinBlocks) gemv_pack5_kernel(co
     // a copy never landed: let the ones still in flight finish, write nothing
     if (tid == 0) {
       raise_status(kDevTimeout);
+      (void)mbar_wait(bar_lut, 0u);
       for (int sg = issued > nstage ? issued - nstage : 0; sg < issued; ++sg)
         (void)mbar_wait(&bars[sg % nstage], uint32_t(sg / nstage) & 1u);
     }
