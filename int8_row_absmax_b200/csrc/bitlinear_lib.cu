@@ -20,6 +20,7 @@
 #include "linear_simt.cuh"
 #include "gemv_pack5.cuh"
 #include "gemm_tc.cuh"
+#include "gemm_swap.cuh"
 #include "deployed_io.cuh"
 #include "ste_backward.cuh"
 #include "rmsnorm_quant.cuh"
@@ -231,10 +232,20 @@ struct TcSplit {
   int split;
   size_t bytes;
 };
-TcSplit tc_split(int64_t M, int64_t N, int64_t K) {
+// Few-row packed layers (5 <= M <= 128) run the swapped GEMM: W rows are the
+// MMA's M side, X rows its N side (gemm_swap.cuh).
+bool tc_swap(int64_t M, bl_wfmt f) { return f == BL_W_PACK5 && M >= 1 && M <= kSwMaxNp; }
+
+TcSplit tc_split(int64_t M, int64_t N, int64_t K, bl_wfmt f) {
   TcSplit r;
-  r.tiles = ceil_div(M, int64_t(kTcBM)) * ceil_div(N, int64_t(kTcBN));
-  const int64_t nch = ceil_div(ceil_div(K, int64_t(kTcBK)), int64_t(kTcChunk));
+  int64_t nch;
+  if (tc_swap(M, f)) {   // 128-row W tiles, K blocks of 160 trits
+    r.tiles = ceil_div(N, int64_t(kSwBM));
+    nch = ceil_div(K, int64_t(kSwBK));
+  } else {
+    r.tiles = ceil_div(M, int64_t(kTcBM)) * ceil_div(N, int64_t(kTcBN));
+    nch = ceil_div(ceil_div(K, int64_t(kTcBK)), int64_t(kTcChunk));
+  }
   int64_t sp = kTcSplitSms / (r.tiles > 0 ? r.tiles : 1);
   if (sp > nch) sp = nch;
   if (sp > kTcMaxSplit) sp = kTcMaxSplit;
@@ -270,7 +281,7 @@ int resolve_path(int64_t M, int64_t N, int64_t K, bl_wfmt f, int path, int* laun
   } else if (p == BL_PATH_TC) {
     if (!tc_ok) return -1;
     // [act_quant,] [unpack,] GEMM [, K-split reduction]
-    n = (fused_quant ? 2 : 1) + (tc_unpack(M, f) ? 1 : 0) + (tc_split(M, N, K).split > 1 ? 1 : 0);
+    n = (fused_quant ? 2 : 1) + (tc_unpack(M, f) ? 1 : 0) + (tc_split(M, N, K, f).split > 1 ? 1 : 0);
   } else {
     return -1;
   }
@@ -389,7 +400,7 @@ bl_status run_tc(const int8_t* Xq, int64_t ldx, int64_t M, int64_t K, const void
   if (ldx % 16 != 0 || ldw % 16 != 0 || !is_aligned(Xq, 16) || !is_aligned(W, 16))
     return BL_ERR_ALIGNMENT;
   // no workspace (tcws null): no K split
-  TcSplit sp = tc_split(M, N, K);
+  TcSplit sp = tc_split(M, N, K, packed ? BL_W_PACK5 : BL_W_I8);
   if (!tcws) sp.split = 1;
   if (sp.tiles > (int64_t(1) << 28)) return BL_ERR_UNSUPPORTED;
   if (sp.split > 1 && (!is_aligned(tcws, kWsAlign) || tcws_bytes < sp.bytes)) return BL_ERR_WORKSPACE;
@@ -419,6 +430,88 @@ bl_status run_tc(const int8_t* Xq, int64_t ldx, int64_t M, int64_t K, const void
   else
     tc_reduce_kernel<false><<<grid_for(work, 256), 256, 0, st>>>(a.part, sp.split, M, N, nullptr, nullptr, nullptr,
                                                                 nullptr, acc);
+  return launch_status();
+}
+
+// X_q [M, ldx] int8 as boxes {inner, Np} with the given swizzle.
+bool make_map_xq(CUtensorMap* map, const void* base, int64_t K, int64_t M, int64_t ld, int inner, int rows,
+                 CUtensorMapSwizzle sw) {
+  EncodeTiledFn fn = encode_tiled();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {cuuint64_t(K), cuuint64_t(M)};
+  const cuuint64_t strides[1] = {cuuint64_t(ld)};
+  const cuuint32_t box[2] = {cuuint32_t(inner), cuuint32_t(rows)};
+  const cuuint32_t estr[2] = {1u, 1u};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Packed W [N, ldp] as boxes of {32 bytes, 128 rows}, no swizzle.
+bool make_map_wp32(CUtensorMap* map, const void* base, int64_t ldp, int64_t N) {
+  EncodeTiledFn fn = encode_tiled();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {cuuint64_t(ldp), cuuint64_t(N)};
+  const cuuint64_t strides[1] = {cuuint64_t(ldp)};
+  const cuuint32_t box[2] = {32u, cuuint32_t(kSwBM)};
+  const cuuint32_t estr[2] = {1u, 1u};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// The swapped GEMM for few-row packed layers (gemm_swap.cuh), then the K
+// split's reduction when there is one.
+bl_status run_swap(const int8_t* Xq, int64_t ldx, int64_t M, int64_t K, const void* W, int64_t ldw, int64_t N,
+                   const float* s, const float* beta, const float* bias, float* Y, int32_t* acc, void* tcws,
+                   size_t tcws_bytes, cudaStream_t st) {
+  if (ldx % 16 != 0 || ldw % 16 != 0 || !is_aligned(Xq, 16) || !is_aligned(W, 16)) return BL_ERR_ALIGNMENT;
+  if (M < 1 || M > kSwMaxNp) return BL_ERR_UNSUPPORTED;
+  TcSplit sp = tc_split(M, N, K, BL_W_PACK5);
+  if (!tcws) sp.split = 1;
+  if (sp.tiles > (int64_t(1) << 28)) return BL_ERR_UNSUPPORTED;
+  if (sp.split > 1 && (!is_aligned(tcws, kWsAlign) || tcws_bytes < sp.bytes)) return BL_ERR_WORKSPACE;
+  const int Np = int(round_up(M, 16));
+  SwMaps maps;
+  if (!make_map_xq(&maps.x128, Xq, K, M, ldx, 128, Np, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_map_xq(&maps.x32, Xq, K, M, ldx, 32, Np, CU_TENSOR_MAP_SWIZZLE_32B) ||
+      !make_map_wp32(&maps.wp, W, ldw, N))
+    return BL_ERR_CUDA;
+  SwArgs a;
+  a.M = M;
+  a.N = N;
+  a.K = K;
+  a.Np = Np;
+  a.s = s;
+  a.beta = beta;
+  a.bias = bias;
+  a.Y = Y;
+  a.acc = acc;
+  a.tiles = int(sp.tiles);
+  a.split = sp.split;
+  a.part = sp.split > 1 ? static_cast<int32_t*>(tcws) : nullptr;
+  const int64_t work = sp.tiles * sp.split;
+  const dim3 grid(unsigned(work < num_sms() ? work : num_sms()));
+  const bool dq = Y != nullptr;
+  if (dq) {
+    if (cudaFuncSetAttribute(gemm_swap_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, SwLayout::kSmem) !=
+        cudaSuccess)
+      return BL_ERR_CUDA;
+    gemm_swap_kernel<true><<<grid, kSwThreads, SwLayout::kSmem, st>>>(maps, a);
+  } else {
+    if (cudaFuncSetAttribute(gemm_swap_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             SwLayout::kSmem) != cudaSuccess)
+      return BL_ERR_CUDA;
+    gemm_swap_kernel<false><<<grid, kSwThreads, SwLayout::kSmem, st>>>(maps, a);
+  }
+  bl_status r = launch_status();
+  if (r != BL_OK || sp.split == 1) return r;
+  const int64_t rw = (N % 4 == 0 ? M * (N / 4) : M * N);
+  if (dq)
+    tc_reduce_kernel<true><<<grid_for(rw, 256), 256, 0, st>>>(a.part, sp.split, M, N, s, beta, bias, Y, nullptr);
+  else
+    tc_reduce_kernel<false><<<grid_for(rw, 256), 256, 0, st>>>(a.part, sp.split, M, N, nullptr, nullptr, nullptr,
+                                                              nullptr, acc);
   return launch_status();
 }
 
@@ -742,7 +835,7 @@ size_t bl_linear_ex_workspace_size(int64_t M, int64_t N, int64_t K, bl_wfmt f, i
   path &= kPathMask;
   const int p = resolve_path(M, N, K, f, path, nullptr);
   if (p == BL_PATH_GEMV) return 0;   // activation quantization inside the GEMV: no scratch
-  return lin_layout(M, K, N, p == BL_PATH_TC && tc_unpack(M, f), p == BL_PATH_TC ? tc_split(M, N, K).bytes : 0)
+  return lin_layout(M, K, N, p == BL_PATH_TC && tc_unpack(M, f), p == BL_PATH_TC ? tc_split(M, N, K, f).bytes : 0)
       .total;
 }
 
@@ -785,7 +878,7 @@ static bl_status linear_impl(const float* X, int64_t M, int64_t K, const void* W
   if (p < 0) return BL_ERR_UNSUPPORTED;
   if (p == BL_PATH_GEMV)   // needs no workspace
     return run_gemv(X, nullptr, 0, M, K, W, ldw, N, beta_dev, bias, eps, Y, nullptr, static_w, stream);
-  const size_t tcb = (p == BL_PATH_TC && allow_split) ? tc_split(M, N, K).bytes : 0;
+  const size_t tcb = (p == BL_PATH_TC && allow_split) ? tc_split(M, N, K, f).bytes : 0;
   const LinWs l = lin_layout(M, K, N, p == BL_PATH_TC && tc_unpack(M, f), tcb);
   if (!ws || !is_aligned(ws, kWsAlign) || ws_bytes < l.total) return BL_ERR_WORKSPACE;
   void* tcws = tcb ? static_cast<char*>(ws) + l.tc_off : nullptr;   // null: no K split
@@ -801,6 +894,8 @@ static bl_status linear_impl(const float* X, int64_t M, int64_t K, const void* W
       if (st != BL_OK) return st;
       return run_tc(Xq, l.ldx, M, K, scratch, l.ldk, false, N, s, beta_dev, bias, Y, nullptr, tcws, tcb, stream);
     }
+    if (tc_swap(M, f))
+      return run_swap(Xq, l.ldx, M, K, W, ldw, N, s, beta_dev, bias, Y, nullptr, tcws, tcb, stream);
     return run_tc(Xq, l.ldx, M, K, W, ldw, f == BL_W_PACK5, N, s, beta_dev, bias, Y, nullptr, tcws, tcb, stream);
   }
   return run_simt(Xq, l.ldx, M, K, W, f, ldw, N, s, beta_dev, bias, Y, nullptr, stream);
@@ -904,7 +999,7 @@ size_t bl_linear_acc_workspace_size(int64_t M, int64_t N, int64_t K, bl_wfmt f, 
   path &= kPathMask;
   const int p = resolve_path(M, N, K, f, path, nullptr, false);
   if (p != BL_PATH_TC) return 0;
-  return (tc_unpack(M, f) ? align_up(size_t(N) * size_t(round_up(K, 16))) : 0) + tc_split(M, N, K).bytes;
+  return (tc_unpack(M, f) ? align_up(size_t(N) * size_t(round_up(K, 16))) : 0) + tc_split(M, N, K, f).bytes;
 }
 
 // no_ws: bl_linear_acc, which takes no workspace: packed weights are then
@@ -936,7 +1031,7 @@ static bl_status linear_acc_impl(const int8_t* Xq, int64_t M, int64_t K, const v
   if (p == BL_PATH_TC) {
     const bool unp = !no_ws && tc_unpack(M, f);
     const size_t wq = unp ? align_up(size_t(N) * size_t(round_up(K, 16))) : 0;
-    const size_t need = no_ws ? 0 : wq + tc_split(M, N, K).bytes;
+    const size_t need = no_ws ? 0 : wq + tc_split(M, N, K, f).bytes;
     if (need && (!ws || !is_aligned(ws, kWsAlign) || ws_bytes < need)) return BL_ERR_WORKSPACE;
     void* tcws = need > wq ? static_cast<char*>(ws) + wq : nullptr;
     const size_t tcb = need > wq ? ws_bytes - wq : 0;
@@ -947,6 +1042,8 @@ static bl_status linear_acc_impl(const int8_t* Xq, int64_t M, int64_t K, const v
       return run_tc(Xq, K, M, K, scratch, round_up(K, 16), false, N, nullptr, nullptr, nullptr, nullptr, acc,
                     tcws, tcb, stream);
     }
+    if (tc_swap(M, f))
+      return run_swap(Xq, K, M, K, W, ldw, N, nullptr, nullptr, nullptr, nullptr, acc, tcws, tcb, stream);
     return run_tc(Xq, K, M, K, W, ldw, f == BL_W_PACK5, N, nullptr, nullptr, nullptr, nullptr, acc, tcws, tcb,
                   stream);
   }

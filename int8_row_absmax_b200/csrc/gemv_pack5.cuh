@@ -248,11 +248,10 @@ __global__ void __launch_bounds__(kGemvThreads, kMinBlocks) gemv_pack5_kernel(co
   const int kpad = int(5 * ldp);
   float scm[M];
   const float* xsrc = staged ? reinterpret_cast<const float*>(smem + P.xs_off) : P.X;
-  // 16-byte loads of X: shared memory when staged, else the read-only path
-  // (four per thread issued together, so the latencies overlap)
-  auto ld4 = [&](const float* p) -> float4 {
-    return staged ? *reinterpret_cast<const float4*>(p) : __ldg(reinterpret_cast<const float4*>(p));
-  };
+  // 16-byte loads of X through generic addresses, valid for the staged copy
+  // in shared memory and for global memory alike (four per thread issued
+  // together, so the latencies overlap); no global-only load form here
+  auto ld4 = [](const float* p) -> float4 { return *reinterpret_cast<const float4*>(p); };
   if (kFused) {
     const bool xvec = aligned(P.X, 16) && (K & 3) == 0;
     const int64_t K4 = xvec ? (K >> 2) : 0;
@@ -277,7 +276,7 @@ __global__ void __launch_bounds__(kGemvThreads, kMinBlocks) gemv_pack5_kernel(co
         }
       }
       for (int64_t i = (K4 << 2) + tid; i < K; i += kGemvThreads) {
-        const float v = fabsf(staged ? xr[i] : __ldg(xr + i));
+        const float v = fabsf(xr[i]);
         bad |= !(v <= 3.402823466e38f);
         amax = fmaxf(amax, v);
       }

@@ -127,11 +127,16 @@ def _al(v):
 def test_tensor_core_plan_and_workspace(lib, M, K, N):
     """The tensor-core plan, on the host: act_quant + GEMM, + the unpack of packed
     weights beyond 4 row tiles of 128, + the reduction of a K split, which is
-    taken when the 128 x 256 tiles are fewer than half of 148 SMs and K has at
-    least two 640-wide chunks (at most 8 splits).  The workspace holds X_q [M,
+    taken when the output tiles (128 x 256; for M <= 128 the swapped GEMM's 128
+    W rows) are fewer than half of 148 SMs and K has at least two K ranges
+    (640-wide chunks; 160-trit blocks when swapped), at most 8 splits.  The workspace holds X_q [M,
     ldx] and s, then the int8 copy of W_q, then the split's int32 partials."""
-    tiles = _cdiv(M, 128) * _cdiv(N, 256)
-    split = max(1, min(148 // tiles, _cdiv(_cdiv(K, 128), 5), 8))
+    if M <= 128:     # few rows, packed weights: the swapped GEMM (128 W rows per tile, 160-trit K blocks)
+        tiles = _cdiv(N, 128)
+        split = max(1, min(148 // tiles, _cdiv(K, 160), 8))
+    else:
+        tiles = _cdiv(M, 128) * _cdiv(N, 256)
+        split = max(1, min(148 // tiles, _cdiv(_cdiv(K, 128), 5), 8))
     n = ctypes.c_int(0)
     assert lib.bl_linear_plan(M, N, K, pkg.PACK5, pkg.PATH_TC, ctypes.byref(n)) == pkg.PATH_TC
     assert n.value == 2 + (M > 512) + (split > 1)
