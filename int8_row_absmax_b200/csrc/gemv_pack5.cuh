@@ -234,6 +234,7 @@ __global__ void __launch_bounds__(kGemvThreads, kMinBlocks) gemv_pack5_kernel(co
     if (!a.prefetch)
       for (int sg = 0; sg < nseg && sg < nstage; ++sg) issue(sg);
   }
+  __syncthreads();                // the mbarriers are initialized before any thread polls one
   if (!__syncthreads_and(staged ? mbar_wait(bar_x, 0u) : true)) {
     if (tid == 0) {
       raise_status(kDevTimeout);
