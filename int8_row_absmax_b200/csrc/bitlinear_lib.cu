@@ -490,19 +490,25 @@ bl_status run_swap(const int8_t* Xq, int64_t ldx, int64_t M, int64_t K, const vo
   a.tiles = int(sp.tiles);
   a.split = sp.split;
   a.part = sp.split > 1 ? static_cast<int32_t*>(tcws) : nullptr;
+  const SwLayout l = sw_layout(Np);
+  if (l.nst < 2) return BL_ERR_UNSUPPORTED;
+  a.nst = l.nst;
+  a.stage = l.stage;
+  a.pk_off = l.pk_off;
+  a.lut_off = l.lut_off;
   const int64_t work = sp.tiles * sp.split;
   const dim3 grid(unsigned(work < num_sms() ? work : num_sms()));
   const bool dq = Y != nullptr;
   if (dq) {
-    if (cudaFuncSetAttribute(gemm_swap_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, SwLayout::kSmem) !=
+    if (cudaFuncSetAttribute(gemm_swap_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSwSmemMax) !=
         cudaSuccess)
       return BL_ERR_CUDA;
-    gemm_swap_kernel<true><<<grid, kSwThreads, SwLayout::kSmem, st>>>(maps, a);
+    gemm_swap_kernel<true><<<grid, kSwThreads, l.smem, st>>>(maps, a);
   } else {
-    if (cudaFuncSetAttribute(gemm_swap_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             SwLayout::kSmem) != cudaSuccess)
+    if (cudaFuncSetAttribute(gemm_swap_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSwSmemMax) !=
+        cudaSuccess)
       return BL_ERR_CUDA;
-    gemm_swap_kernel<false><<<grid, kSwThreads, SwLayout::kSmem, st>>>(maps, a);
+    gemm_swap_kernel<false><<<grid, kSwThreads, l.smem, st>>>(maps, a);
   }
   bl_status r = launch_status();
   if (r != BL_OK || sp.split == 1) return r;

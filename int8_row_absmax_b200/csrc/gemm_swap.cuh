@@ -25,12 +25,13 @@
 //   * five tcgen05.mma.kind::i8 (M = 128, N = Np, K = 32) into a TMEM
 //     accumulator: A = W tile (interleave descriptor, chunk pair 2i, 2i+1),
 //     B = X_q tile (swizzled descriptors).
-// Roles: warp 0 issues the TMA loads, warp 1 the MMAs, warps 2..5 drain TMEM
-// (lane = W row, columns = X rows: y[m, n] for 32 consecutive n per store) with
-// the dequant fused, warps 6..21 decode (two groups of eight take the K blocks
-// in turn).  With fewer 128-row W tiles than SMs, K is split into ranges of
-// whole blocks whose int32 partials [split, M, N] tc_reduce_kernel adds up
-// (exact).  Every wait is bounded; on a timeout the kernel records kDevTimeout,
+// Roles: warp 0 issues the X_q loads into the stage ring, warp 22 the packed
+// tiles into a ring of their own (16 deep, so 64 KB of weights are in flight per
+// SM), warp 1 the MMAs, warps 2..5 drain TMEM (lane = W row, columns = X rows:
+// y[m, n] for 32 consecutive n per store) with the dequant fused, warps 6..21
+// decode (two groups of eight take the K blocks in turn).  With fewer 128-row
+// W tiles than SMs, K is split into ranges of whole blocks whose int32
+// partials [split, M, N] tc_reduce_kernel adds up (exact).  Every wait is bounded; on a timeout the kernel records kDevTimeout,
 // lets copies and MMAs in flight land and frees its TMEM.
 #pragma once
 
@@ -44,21 +45,33 @@ constexpr int kSwBK = 160;                 // trits per K block (5 MMAs of K = 3
 constexpr int kSwPkBytes = kSwBM * 32;     // packed tile: 4 KB
 constexpr int kSwATile = kSwBM * kSwBK;    // decoded W tile: 20 KB
 constexpr int kSwMaxNp = 128;              // X rows per MMA (N), multiple of 16
-constexpr int kSwStages = 4;
+constexpr int kSwMaxStages = 8;            // decoded-W / X stages (as many as fit)
+constexpr int kSwPkStages = 16;            // packed tiles in flight: 64 KB per SM
 constexpr int kSwDecWarps = 16, kSwDecGroups = 2;
 constexpr int kSwWpg = kSwDecWarps / kSwDecGroups;
-constexpr int kSwThreads = 192 + 32 * kSwDecWarps;
+constexpr int kSwPkWarp = 6 + kSwDecWarps;             // the packed tiles' producer
+constexpr int kSwThreads = 32 * (kSwPkWarp + 1);
 constexpr int kSwMaxSplit = 8;
 constexpr int kSwLutBytes = 256 * 128;     // word 32 b + lane
+constexpr int kSwSmemMax = 232448 - 2048;  // dynamic shared memory budget
 
-// Stage layout (bytes from the 1024-aligned base): X128 [Np x 128] (1024-aligned),
-// X32 [Np x 32] (256-aligned), packed [128 x 32], A [20 KB].
+// Shared memory (from the 1024-aligned base): `nst` stages of [X128: Np x 128
+// (1024-aligned) | A: 20 KB | X32: Np x 32 (256-aligned)], each rounded up to
+// 1024 bytes; then the packed ring (16 x 4 KB); then the decode table.
 struct SwLayout {
-  static constexpr int kX128 = kSwMaxNp * 128;   // 16 KB
-  static constexpr int kX32 = kSwMaxNp * 32;     // 4 KB
-  static constexpr int kStage = kX128 + kX32 + kSwPkBytes + kSwATile;   // 44 KB
-  static constexpr int kSmem = kSwStages * kStage + kSwLutBytes + 1024;
+  int stage, nst, pk_off, lut_off, smem;
 };
+inline SwLayout sw_layout(int Np) {
+  SwLayout l;
+  l.stage = int(round_up(int64_t(Np) * 128 + kSwATile + int64_t(Np) * 32, 1024));
+  const int fixed = kSwPkStages * kSwPkBytes + kSwLutBytes + 1024;
+  int n = (kSwSmemMax - fixed) / l.stage;
+  l.nst = n > kSwMaxStages ? kSwMaxStages : n;
+  l.pk_off = l.nst * l.stage;
+  l.lut_off = l.pk_off + kSwPkStages * kSwPkBytes;
+  l.smem = l.lut_off + kSwLutBytes + 1024;
+  return l;
+}
 
 struct alignas(64) SwMaps {
   CUtensorMap x128;   // X_q [M, ldx] int8, boxes {128, Np}, 128-byte swizzle
@@ -76,6 +89,7 @@ struct SwArgs {
   int32_t* acc;        // [M, N] int32 when Y is nullptr
   int tiles, split;
   int32_t* part;       // [split, M, N] int32 (split > 1)
+  int nst, stage, pk_off, lut_off;   // shared-memory layout (sw_layout)
 };
 
 // The table of trits t0..t3 per byte (word 32 b + lane), a compile-time constant.
@@ -131,7 +145,8 @@ template <bool kDequant>
 __global__ void __launch_bounds__(kSwThreads, 1)
 gemm_swap_kernel(const __grid_constant__ SwMaps maps, const SwArgs a) {
   extern __shared__ unsigned char smem_raw[];
-  __shared__ uint64_t ld_full[kSwStages], dec_full[kSwStages], empty[kSwStages];
+  __shared__ uint64_t ld_full[kSwMaxStages], dec_full[kSwMaxStages], empty[kSwMaxStages];
+  __shared__ uint64_t pk_full[kSwPkStages], pk_empty[kSwPkStages];
   __shared__ uint64_t acc_full[2], acc_empty[2], drain, lut_bar;
   __shared__ uint32_t s_tmem;
   __shared__ int s_err;
@@ -139,8 +154,8 @@ gemm_swap_kernel(const __grid_constant__ SwMaps maps, const SwArgs a) {
   volatile int* err = &s_err;
   const uint32_t base = (smem_u32(smem_raw) + 1023u) & ~1023u;
   unsigned char* smem = smem_raw + (base - smem_u32(smem_raw));
-  uint32_t* lut = reinterpret_cast<uint32_t*>(smem + kSwStages * SwLayout::kStage);
-  const int Np = a.Np;
+  uint32_t* lut = reinterpret_cast<uint32_t*>(smem + a.lut_off);
+  const int Np = a.Np, nst = a.nst;
   const int nkb = int(ceil_div(a.K, kSwBK));
   const int S = a.split;
   const int nwork = a.tiles * S;
@@ -150,18 +165,22 @@ gemm_swap_kernel(const __grid_constant__ SwMaps maps, const SwArgs a) {
     kb0 = j * nkb / S;
     kb1 = (j + 1) * nkb / S;
   };
-  auto stage_x128 = [&](int s) { return smem + s * SwLayout::kStage; };
-  auto stage_x32 = [&](int s) { return smem + s * SwLayout::kStage + SwLayout::kX128; };
-  auto stage_pk = [&](int s) { return smem + s * SwLayout::kStage + SwLayout::kX128 + SwLayout::kX32; };
-  auto stage_a = [&](int s) { return stage_pk(s) + kSwPkBytes; };
+  auto stage_x128 = [&](int s) { return smem + s * a.stage; };
+  auto stage_a = [&](int s) { return smem + s * a.stage + Np * 128; };
+  auto stage_x32 = [&](int s) { return smem + s * a.stage + Np * 128 + kSwATile; };
+  auto stage_pk = [&](int p) { return smem + a.pk_off + p * kSwPkBytes; };
   const uint32_t x_bytes = uint32_t(Np) * uint32_t(kSwBK);
 
   if (tid == 0) {
     s_err = 0;
-    for (int s = 0; s < kSwStages; ++s) {
+    for (int s = 0; s < nst; ++s) {
       mbar_init(&ld_full[s], 1);
       mbar_init(&dec_full[s], kSwWpg);
       mbar_init(&empty[s], 1);
+    }
+    for (int p = 0; p < kSwPkStages; ++p) {
+      mbar_init(&pk_full[p], 1);
+      mbar_init(&pk_empty[p], kSwWpg);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&acc_full[b], 1);
@@ -192,15 +211,14 @@ gemm_swap_kernel(const __grid_constant__ SwMaps maps, const SwArgs a) {
         int t, kb0, kb1, j;
         work(w, t, kb0, kb1, j);
         for (int kb = kb0; kb < kb1; ++kb, ++it) {
-          const int s = it % kSwStages;
-          if (it >= kSwStages && !mbar_wait(&empty[s], uint32_t(it / kSwStages - 1) & 1u)) {
+          const int s = it % nst;
+          if (it >= nst && !mbar_wait(&empty[s], uint32_t(it / nst - 1) & 1u)) {
             *err = 1;
             break;
           }
-          mbar_arrive_expect_tx(&ld_full[s], x_bytes + uint32_t(kSwPkBytes));
+          mbar_arrive_expect_tx(&ld_full[s], x_bytes);
           tma_load_2d(stage_x128(s), &maps.x128, kb * kSwBK, 0, &ld_full[s]);
           tma_load_2d(stage_x32(s), &maps.x32, kb * kSwBK + 128, 0, &ld_full[s]);
-          tma_load_2d(stage_pk(s), &maps.wp, kb * 32, t * kSwBM, &ld_full[s]);
         }
       }
     }
@@ -220,9 +238,9 @@ gemm_swap_kernel(const __grid_constant__ SwMaps maps, const SwArgs a) {
         const uint32_t d = tmem + uint32_t(b * kSwMaxNp);
         bool ok = true;
         for (int kb = kb0; kb < kb1; ++kb, ++it) {
-          const int s = it % kSwStages;
-          if (!mbar_wait(&ld_full[s], uint32_t(it / kSwStages) & 1u) ||
-              !mbar_wait(&dec_full[s], uint32_t(it / kSwStages) & 1u)) {
+          const int s = it % nst;
+          if (!mbar_wait(&ld_full[s], uint32_t(it / nst) & 1u) ||
+              !mbar_wait(&dec_full[s], uint32_t(it / nst) & 1u)) {
             ok = false;
             break;
           }
@@ -244,7 +262,7 @@ gemm_swap_kernel(const __grid_constant__ SwMaps maps, const SwArgs a) {
       }
       umma_commit(&drain);
     }
-  } else if (warp >= 6) {
+  } else if (warp >= 6 && warp < kSwPkWarp) {
     // decoder warps: group g decodes the blocks it % 2 == g; thread gt of the
     // group owns row gt / 2 and packed bytes 16 (gt % 2) .. +15 of the block
     constexpr int kGT = 32 * kSwWpg;                 // 256 threads: 128 rows x 2 halves
@@ -258,12 +276,13 @@ gemm_swap_kernel(const __grid_constant__ SwMaps maps, const SwArgs a) {
       work(w, t, kb0, kb1, j);
       for (int kb = kb0; kb < kb1; ++kb, ++it) {
         if (it % kSwDecGroups != g) continue;
-        const int s = it % kSwStages;
-        if (!mbar_wait(&ld_full[s], uint32_t(it / kSwStages) & 1u)) {
+        const int s = it % nst, pp = it % kSwPkStages;
+        if (!mbar_wait(&pk_full[pp], uint32_t(it / kSwPkStages) & 1u) ||
+            !mbar_wait(&ld_full[s], uint32_t(it / nst) & 1u)) {
           ok = false;
           break;
         }
-        const uint4 p = *reinterpret_cast<const uint4*>(stage_pk(s) + r * 32 + h * 16);
+        const uint4 p = *reinterpret_cast<const uint4*>(stage_pk(pp) + r * 32 + h * 16);
         const uint32_t pw[4] = {p.x, p.y, p.z, p.w};
         uint32_t o[20];
 #pragma unroll
@@ -285,11 +304,35 @@ gemm_swap_kernel(const __grid_constant__ SwMaps maps, const SwArgs a) {
           *reinterpret_cast<uint4*>(dst + v * 2048) = make_uint4(o[4 * v], o[4 * v + 1], o[4 * v + 2], o[4 * v + 3]);
         fence_proxy_async_smem();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&dec_full[s]);
+        if (lane == 0) {
+          mbar_arrive(&dec_full[s]);
+          mbar_arrive(&pk_empty[pp]);
+        }
       }
     }
     if (!ok) *err = 1;
-  } else if (warp >= 2) {
+  } else if (warp == kSwPkWarp) {
+    // packed producer: up to 16 packed tiles ahead of the decoders
+    if (lane == 0) {
+      int it = 0;
+      for (int w = blockIdx.x; w < nwork && !*err; w += gridDim.x) {
+        int t, kb0, kb1, j;
+        work(w, t, kb0, kb1, j);
+        for (int kb = kb0; kb < kb1; ++kb, ++it) {
+          const int pp = it % kSwPkStages;
+          if (it >= kSwPkStages && !mbar_wait(&pk_empty[pp], uint32_t(it / kSwPkStages - 1) & 1u)) {
+            *err = 1;
+            break;
+          }
+          mbar_arrive_expect_tx(&pk_full[pp], uint32_t(kSwPkBytes));
+          tma_load_2d(stage_pk(pp), &maps.wp, kb * 32, t * kSwBM, &pk_full[pp]);
+        }
+      }
+      // copies still in flight (after an error) land before the CTA exits
+      for (int q = it > kSwPkStages ? it - kSwPkStages : 0; q < it; ++q)
+        (void)mbar_wait(&pk_full[q % kSwPkStages], uint32_t(q / kSwPkStages) & 1u);
+    }
+  } else if (warp >= 2 && warp < 6) {
     // epilogue warps 2..5: TMEM lane = W row of the tile, columns = X rows
     const int q = warp & 3;
     const int rl = q * 32 + lane;

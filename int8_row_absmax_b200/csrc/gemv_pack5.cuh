@@ -372,45 +372,59 @@ __global__ void __launch_bounds__(kGemvThreads, kMinBlocks) gemv_pack5_kernel(co
     const int r0 = sg * seg_rows;
     const int nr = min(seg_rows, rows - r0);
     if (grp < G) {
+      // two rows per pass (rl, rl + G) and two accumulators per row and x row
+      // (even and odd words): independent dp4a and table-lookup chains
 #pragma unroll 1
-      for (int rl = grp; rl < nr; rl += G) {
-        const unsigned char* rowp = sbuf + int64_t(rl) * ldp;
-        int am[M], a4[M];
+      for (int rl = grp; rl < nr; rl += 2 * G) {
+        const bool two = rl + G < nr;
+        const unsigned char* rowp0 = sbuf + int64_t(rl) * ldp;
+        const unsigned char* rowp1 = two ? rowp0 + int64_t(G) * ldp : rowp0;
+        int am[2][M][2], a4[2][M];
 #pragma unroll
-        for (int m = 0; m < M; ++m) am[m] = a4[m] = 0;
+        for (int rr = 0; rr < 2; ++rr)
+#pragma unroll
+          for (int m = 0; m < M; ++m) am[rr][m][0] = am[rr][m][1] = a4[rr][m] = 0;
 #pragma unroll
         for (int i = 0; i < CH; ++i) {
           const int64_t c = c0 + lane + 32 * i;
           if (c < c1) {
-            const uint4 w4 = *reinterpret_cast<const uint4*>(rowp + 16 * c);
-            const uint32_t wv[4] = {w4.x, w4.y, w4.z, w4.w};
+            const uint4 w40 = *reinterpret_cast<const uint4*>(rowp0 + 16 * c);
+            const uint4 w41 = *reinterpret_cast<const uint4*>(rowp1 + 16 * c);
+            const uint32_t wv[2][4] = {{w40.x, w40.y, w40.z, w40.w}, {w41.x, w41.y, w41.z, w41.w}};
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
-              const uint32_t w = wv[q];
-              uint32_t t[4];
 #pragma unroll
-              for (int bb = 0; bb < 4; ++bb)
-                t[bb] = *reinterpret_cast<const uint32_t*>(smem + __byte_perm(w, lanebase, 0x5504u | (bb << 4)));
-              const uint32_t E = __byte_perm(w, 0u, 0x4240u) * 203u;
-              const uint32_t O = __byte_perm(w, 0u, 0x4341u) * 203u;
-              const uint32_t D = __byte_perm(E, O, 0x7351u) & 0xC0C0C0C0u;
+              for (int rr = 0; rr < 2; ++rr) {
+                const uint32_t w = wv[rr][q];
+                uint32_t t[4];
 #pragma unroll
-              for (int m = 0; m < M; ++m) {
-                int acc = am[m];
+                for (int bb = 0; bb < 4; ++bb)
+                  t[bb] = *reinterpret_cast<const uint32_t*>(smem + __byte_perm(w, lanebase, 0x5504u | (bb << 4)));
+                const uint32_t E = __byte_perm(w, 0u, 0x4240u) * 203u;
+                const uint32_t O = __byte_perm(w, 0u, 0x4341u) * 203u;
+                const uint32_t D = __byte_perm(E, O, 0x7351u) & 0xC0C0C0C0u;
 #pragma unroll
-                for (int bb = 0; bb < 4; ++bb) acc = __dp4a(int(t[bb]), int(xr[m][i][5 * q + bb]), acc);
-                am[m] = acc;
-                a4[m] = dp4a_us(D, xr[m][i][5 * q + 4], a4[m]);
+                for (int m = 0; m < M; ++m) {
+                  int acc = am[rr][m][q & 1];
+#pragma unroll
+                  for (int bb = 0; bb < 4; ++bb) acc = __dp4a(int(t[bb]), int(xr[m][i][5 * q + bb]), acc);
+                  am[rr][m][q & 1] = acc;
+                  a4[rr][m] = dp4a_us(D, xr[m][i][5 * q + 4], a4[rr][m]);
+                }
               }
             }
           }
         }
 #pragma unroll
-        for (int m = 0; m < M; ++m) {
-          const int tot = __reduce_add_sync(0xffffffffu, am[m] + (a4[m] >> 6));
-          if (lane == 0) {
-            if (S == 1) part[m * rpc + r0 + rl] = tot;
-            else atomicAdd(&part[m * rpc + r0 + rl], tot);
+        for (int rr = 0; rr < 2; ++rr) {
+#pragma unroll
+          for (int m = 0; m < M; ++m) {
+            const int tot = __reduce_add_sync(0xffffffffu, am[rr][m][0] + am[rr][m][1] + (a4[rr][m] >> 6));
+            if (lane == 0 && (rr == 0 || two)) {
+              const int row = r0 + rl + rr * G;
+              if (S == 1) part[m * rpc + row] = tot;
+              else atomicAdd(&part[m * rpc + row], tot);
+            }
           }
         }
       }
