@@ -573,6 +573,7 @@ bl_status launch_gemv_f(int M, int ch, const GemvArgs& a, int grid, uint32_t sme
   switch (M * 8 + ch) {
     case 1 * 8 + 1: return launch_gemv_inst<1, 1, F>(a, grid, smem, st);
     case 1 * 8 + 2: return launch_gemv_inst<1, 2, F>(a, grid, smem, st);
+    case 1 * 8 + 3: return launch_gemv_inst<1, 3, F>(a, grid, smem, st);
     case 1 * 8 + 4: return launch_gemv_inst<1, 4, F>(a, grid, smem, st);
     case 2 * 8 + 1: return launch_gemv_inst<2, 1, F>(a, grid, smem, st);
     case 2 * 8 + 2: return launch_gemv_inst<2, 2, F>(a, grid, smem, st);

@@ -48,7 +48,7 @@ constexpr int kGemvThreads = kGemvWarps * 32;
 constexpr int kGemvMaxProbs = 4;
 constexpr uint32_t kLutBytes = 256 * 256;      // a row for every byte value: no read leaves the table
 constexpr uint32_t kGemvMaxSmem = 232448 - 1024;  // 227 KB per CTA, less the static arrays
-constexpr uint32_t kGemvSegTarget = 12 * 1024;  // bytes per bulk copy (one mbarrier each)
+constexpr uint32_t kGemvSegTarget = 32 * 1024;  // bytes per bulk copy (one mbarrier each): few, large copies
 constexpr int kGemvMaxStages = 24;
 constexpr uint32_t kGemvXStageMax = 48 * 1024;  // float32 X rows staged in shared memory up to this
 
@@ -78,14 +78,15 @@ struct GemvArgs {
 
 inline uint32_t align_to(uint32_t v, uint32_t a) { return (v + a - 1) / a * a; }
 
-// Chunks of 16 packed bytes per lane, for M rows and a row of ldp bytes
-// (x codes in registers: 20 words per chunk and row, at most 80 in all).
+// Chunks of 16 packed bytes per lane, for M rows and a row of ldp bytes: as
+// many as it takes for one warp to cover a row (independent work per lane),
+// up to 4 / M (x codes in registers: 20 words per chunk and row, at most 80).
 inline int gemv_chunks_per_lane(int64_t M, int64_t ldp) {
   const int64_t nch = ldp / 16;
-  const int chmax = int(4 / M);
-  for (int ch = 1; ch <= chmax; ch *= 2)
-    if (ceil_div(nch, int64_t(32) * ch) <= kGemvWarps) return ch;
-  return 0;
+  const int64_t chmax = 4 / M;
+  const int64_t ch = ceil_div(nch, int64_t(32)) < chmax ? ceil_div(nch, int64_t(32)) : chmax;
+  if (ch < 1 || ceil_div(nch, int64_t(32) * ch) > kGemvWarps) return 0;
+  return int(ch);
 }
 
 // Geometry of one problem on `ctas` CTAs: warps per slice, row groups, the
@@ -99,8 +100,8 @@ inline bool gemv_plan_prob(int64_t M, int64_t N, int64_t K, int64_t ldp, int cta
   P.S = int(S);
   P.G = kGemvWarps / P.S;
   P.rows_per_cta = int(ceil_div(N, int64_t(ctas)));
-  int64_t seg = P.G * (int64_t(kGemvSegTarget) / (int64_t(P.G) * ldp));
-  if (seg < P.G) seg = P.G;
+  int64_t per = int64_t(kGemvSegTarget) / (int64_t(P.G) * ldp);   // rows per warp group and segment
+  int64_t seg = P.G * (per < 2 ? 2 : per);
   if (seg > P.rows_per_cta) seg = P.rows_per_cta;
   P.seg_rows = int(seg);
   P.xc_off = align_to(kLutBytes, 128);
@@ -292,6 +293,10 @@ __global__ void __launch_bounds__(kGemvThreads, kMinBlocks) gemv_pack5_kernel(co
       if (tid == 0) s_scale[m] = scm[m];
     }
   }
+  // codes in decode order, one packed word's 20 activations per thread: five
+  // 16-byte loads, twenty codes, five 32-bit stores (x[5j..5j+3] for the four
+  // j, then the four x[5j+4])
+  const int ngrp = int(ldp / 4);
 #pragma unroll
   for (int m = 0; m < M; ++m) {
     int x4 = 0;
@@ -299,33 +304,38 @@ __global__ void __launch_bounds__(kGemvThreads, kMinBlocks) gemv_pack5_kernel(co
     const float* xr = kFused ? xsrc + int64_t(m) * K : nullptr;
     const int8_t* xq = kFused ? nullptr : P.Xq + int64_t(m) * P.ldxq;
     const float sc = kFused ? scm[m] : 0.f, rc = kFused ? act_recip(sc) : 0.f;
-    for (int i4 = tid; i4 < (kpad >> 2); i4 += kGemvThreads) {
-      const int k = 4 * i4;
-      uint32_t c[4];
+    for (int gi = tid; gi < ngrp; gi += kGemvThreads) {
+      const int k0 = 20 * gi;
+      uint32_t c[20];
       if (kFused) {
         bool tie = rc == 0.f;
-        if (k + 4 <= K && aligned(xr + k, 16)) {
-          const float4 f = ld4(xr + k);
-          c[0] = act_code_try(f.x, rc, tie);
-          c[1] = act_code_try(f.y, rc, tie);
-          c[2] = act_code_try(f.z, rc, tie);
-          c[3] = act_code_try(f.w, rc, tie);
+        if (k0 + 20 <= K && aligned(xr + k0, 16)) {
+#pragma unroll
+          for (int v = 0; v < 5; ++v) {
+            const float4 f = ld4(xr + k0 + 4 * v);
+            c[4 * v + 0] = act_code_try(f.x, rc, tie);
+            c[4 * v + 1] = act_code_try(f.y, rc, tie);
+            c[4 * v + 2] = act_code_try(f.z, rc, tie);
+            c[4 * v + 3] = act_code_try(f.w, rc, tie);
+          }
         } else {
 #pragma unroll
-          for (int e = 0; e < 4; ++e) c[e] = k + e < K ? act_code_try(xr[k + e], rc, tie) : 0u;
+          for (int e = 0; e < 20; ++e) c[e] = k0 + e < K ? act_code_try(xr[k0 + e], rc, tie) : 0u;
         }
         if (tie)   // rare: a quotient near a half-integer; exact division
-          for (int e = 0; e < 4 && k + e < K; ++e) c[e] = uint32_t(uint8_t(int8_t(act_code_slow(xr[k + e], sc))));
+          for (int e = 0; e < 20; ++e)
+            if (k0 + e < K) c[e] = uint32_t(uint8_t(int8_t(act_code_slow(xr[k0 + e], sc))));
       } else {
 #pragma unroll
-        for (int e = 0; e < 4; ++e) c[e] = k + e < K ? uint32_t(uint8_t(xq[k + e])) : 0u;
+        for (int e = 0; e < 20; ++e) c[e] = k0 + e < K ? uint32_t(uint8_t(xq[k0 + e])) : 0u;
       }
+      uint32_t* dst = reinterpret_cast<uint32_t*>(xcm + 20 * gi);
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const uint32_t kk = uint32_t(k + e);
-        xcm[gemv_xpos(kk)] = uint8_t(c[e]);
-        if (kk % 5u == 4u) x4 += int(int8_t(uint8_t(c[e])));
-      }
+      for (int i = 0; i < 4; ++i)
+        dst[i] = c[5 * i] | (c[5 * i + 1] << 8) | (c[5 * i + 2] << 16) | (c[5 * i + 3] << 24);
+      dst[4] = c[4] | (c[9] << 8) | (c[14] << 16) | (c[19] << 24);
+      x4 += int(int8_t(uint8_t(c[4]))) + int(int8_t(uint8_t(c[9]))) + int(int8_t(uint8_t(c[14]))) +
+            int(int8_t(uint8_t(c[19])));
     }
     x4 = __reduce_add_sync(0xffffffffu, x4);
     if (lane == 0 && x4) atomicAdd(&s_x4[m], x4);
@@ -372,29 +382,37 @@ __global__ void __launch_bounds__(kGemvThreads, kMinBlocks) gemv_pack5_kernel(co
     const int r0 = sg * seg_rows;
     const int nr = min(seg_rows, rows - r0);
     if (grp < G) {
-      // two rows per pass (rl, rl + G) and two accumulators per row and x row
-      // (even and odd words): independent dp4a and table-lookup chains
+      // kRows rows per pass (rl, rl + G) and two accumulators per row and x row
+      // (even and odd words): independent dp4a and table-lookup chains; with
+      // several chunks per lane one row at a time already has them
+      constexpr int kRows = (M * CH <= 2) ? 2 : 1;
 #pragma unroll 1
-      for (int rl = grp; rl < nr; rl += 2 * G) {
-        const bool two = rl + G < nr;
+      for (int rl = grp; rl < nr; rl += kRows * G) {
+        const bool two = kRows == 2 && rl + G < nr;
         const unsigned char* rowp0 = sbuf + int64_t(rl) * ldp;
         const unsigned char* rowp1 = two ? rowp0 + int64_t(G) * ldp : rowp0;
-        int am[2][M][2], a4[2][M];
+        int am[kRows][M][2], a4[kRows][M];
 #pragma unroll
-        for (int rr = 0; rr < 2; ++rr)
+        for (int rr = 0; rr < kRows; ++rr)
 #pragma unroll
           for (int m = 0; m < M; ++m) am[rr][m][0] = am[rr][m][1] = a4[rr][m] = 0;
 #pragma unroll
         for (int i = 0; i < CH; ++i) {
           const int64_t c = c0 + lane + 32 * i;
           if (c < c1) {
-            const uint4 w40 = *reinterpret_cast<const uint4*>(rowp0 + 16 * c);
-            const uint4 w41 = *reinterpret_cast<const uint4*>(rowp1 + 16 * c);
-            const uint32_t wv[2][4] = {{w40.x, w40.y, w40.z, w40.w}, {w41.x, w41.y, w41.z, w41.w}};
+            uint32_t wv[kRows][4];
+#pragma unroll
+            for (int rr = 0; rr < kRows; ++rr) {
+              const uint4 w4 = *reinterpret_cast<const uint4*>((rr ? rowp1 : rowp0) + 16 * c);
+              wv[rr][0] = w4.x;
+              wv[rr][1] = w4.y;
+              wv[rr][2] = w4.z;
+              wv[rr][3] = w4.w;
+            }
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
 #pragma unroll
-              for (int rr = 0; rr < 2; ++rr) {
+              for (int rr = 0; rr < kRows; ++rr) {
                 const uint32_t w = wv[rr][q];
                 uint32_t t[4];
 #pragma unroll
@@ -416,7 +434,7 @@ __global__ void __launch_bounds__(kGemvThreads, kMinBlocks) gemv_pack5_kernel(co
           }
         }
 #pragma unroll
-        for (int rr = 0; rr < 2; ++rr) {
+        for (int rr = 0; rr < kRows; ++rr) {
 #pragma unroll
           for (int m = 0; m < M; ++m) {
             const int tot = __reduce_add_sync(0xffffffffu, am[rr][m][0] + am[rr][m][1] + (a4[rr][m] >> 6));
