@@ -15,8 +15,9 @@
 //   * before the dependency wait (programmatic dependent launch): mbarriers,
 //     a bulk copy (TMA engine) of the decode table (a compile-time constant in
 //     global memory) and -- when the caller declares the weights static --
-//     the bulk copies of the CTA's whole block of packed rows into shared
-//     memory, so the weight stream overlaps the previous kernel;
+//     the bulk copy of the CTA's first segment of packed rows, so the weight
+//     stream starts while the previous kernel finishes; the other segments
+//     follow the copy of X, which is on the critical path;
 //   * griddepcontrol.wait, then launch_dependents (the next kernel may start
 //     its own prologue and weight copies while this one computes);
 //   * X: per-row absmax over the whole row (every CTA reads it, from L2), then
@@ -216,8 +217,7 @@ __global__ void __launch_bounds__(kGemvThreads, kMinBlocks) gemv_pack5_kernel(co
     fence_mbar_init();
     mbar_arrive_expect_tx(bar_lut, kLutBytes);
     bulk_g2s(smem, &g_trit_lut, kLutBytes, bar_lut);
-    if (a.prefetch)
-      for (int sg = 0; sg < nseg && sg < nstage; ++sg) issue(sg);
+    if (a.prefetch && nseg > 0) issue(0);   // the rest after X: X is on the critical path
     s_fail = 0;
   }
   if (tid < M) s_x4[tid] = 0;
@@ -232,8 +232,7 @@ __global__ void __launch_bounds__(kGemvThreads, kMinBlocks) gemv_pack5_kernel(co
       mbar_arrive_expect_tx(bar_x, P.xs_bytes);
       bulk_g2s(smem + P.xs_off, P.X, P.xs_bytes, bar_x);
     }
-    if (!a.prefetch)
-      for (int sg = 0; sg < nseg && sg < nstage; ++sg) issue(sg);
+    for (int sg = a.prefetch ? 1 : 0; sg < nseg && sg < nstage; ++sg) issue(sg);
   }
   __syncthreads();                // the mbarriers are initialized before any thread polls one
   if (!__syncthreads_and(staged ? mbar_wait(bar_x, 0u) : true)) {
