@@ -79,16 +79,19 @@ struct GemvArgs {
 
 inline uint32_t align_to(uint32_t v, uint32_t a) { return (v + a - 1) / a * a; }
 
-// Chunks of 16 packed bytes per lane, for M rows and a row of ldp bytes: as
-// many as it takes for one warp to cover a row (independent work per lane),
-// up to 4 / M (x codes in registers: 20 words per chunk and row, at most 80).
+// Chunks of 16 packed bytes per lane, for M rows and a row of ldp bytes: the
+// fewest that let at most 16 warps cover a row (every warp keeps the codes of
+// its own chunks in registers, and all of them are read from shared memory
+// once per warp), up to 4 / M (20 code words per chunk and row, at most 80).
 inline int gemv_chunks_per_lane(int64_t M, int64_t ldp) {
   const int64_t nch = ldp / 16;
-  const int64_t chmax = 4 / M;
-  const int64_t ch = ceil_div(nch, int64_t(32)) < chmax ? ceil_div(nch, int64_t(32)) : chmax;
-  if (ch < 1 || ceil_div(nch, int64_t(32) * ch) > kGemvWarps) return 0;
-  return int(ch);
+  for (int64_t ch = 1; ch <= 4 / M; ++ch)
+    if (ceil_div(nch, int64_t(32) * ch) <= kGemvWarps) return int(ch);
+  return 0;
 }
+
+// Rows a warp works on at once (independent chains of loads and dp4a).
+__host__ __device__ constexpr int gemv_rows_per_pass(int M, int CH) { return M * CH >= 4 ? 1 : 4 / (M * CH); }
 
 // Geometry of one problem on `ctas` CTAs: warps per slice, row groups, the
 // segment ring and the shared-memory layout.  False if the GEMV cannot take it.
@@ -101,8 +104,11 @@ inline bool gemv_plan_prob(int64_t M, int64_t N, int64_t K, int64_t ldp, int cta
   P.S = int(S);
   P.G = kGemvWarps / P.S;
   P.rows_per_cta = int(ceil_div(N, int64_t(ctas)));
-  int64_t per = int64_t(kGemvSegTarget) / (int64_t(P.G) * ldp);   // rows per warp group and segment
-  int64_t seg = P.G * (per < 2 ? 2 : per);
+  // rows per warp group and segment: at least one pass of gemv_rows_per_pass rows
+  const int64_t rpp = gemv_rows_per_pass(int(M), ch);
+  int64_t per = int64_t(kGemvSegTarget) / (int64_t(P.G) * ldp);
+  per = per < rpp ? rpp : per / rpp * rpp;
+  int64_t seg = P.G * per;
   if (seg > P.rows_per_cta) seg = P.rows_per_cta;
   P.seg_rows = int(seg);
   P.xc_off = align_to(kLutBytes, 128);
@@ -381,15 +387,15 @@ __global__ void __launch_bounds__(kGemvThreads, kMinBlocks) gemv_pack5_kernel(co
     const int r0 = sg * seg_rows;
     const int nr = min(seg_rows, rows - r0);
     if (grp < G) {
-      // kRows rows per pass (rl, rl + G) and two accumulators per row and x row
-      // (even and odd words): independent dp4a and table-lookup chains; with
-      // several chunks per lane one row at a time already has them
-      constexpr int kRows = (M * CH <= 2) ? 2 : 1;
+      // kRows rows per pass (rl, rl + G, ...) and two accumulators per row and x
+      // row (even and odd words): independent chains of table loads and dp4a
+      constexpr int kRows = gemv_rows_per_pass(M, CH);
 #pragma unroll 1
       for (int rl = grp; rl < nr; rl += kRows * G) {
-        const bool two = kRows == 2 && rl + G < nr;
-        const unsigned char* rowp0 = sbuf + int64_t(rl) * ldp;
-        const unsigned char* rowp1 = two ? rowp0 + int64_t(G) * ldp : rowp0;
+        const unsigned char* rowp[kRows];
+#pragma unroll
+        for (int rr = 0; rr < kRows; ++rr)
+          rowp[rr] = sbuf + int64_t(rl + rr * G < nr ? rl + rr * G : rl) * ldp;
         int am[kRows][M][2], a4[kRows][M];
 #pragma unroll
         for (int rr = 0; rr < kRows; ++rr)
@@ -402,7 +408,7 @@ __global__ void __launch_bounds__(kGemvThreads, kMinBlocks) gemv_pack5_kernel(co
             uint32_t wv[kRows][4];
 #pragma unroll
             for (int rr = 0; rr < kRows; ++rr) {
-              const uint4 w4 = *reinterpret_cast<const uint4*>((rr ? rowp1 : rowp0) + 16 * c);
+              const uint4 w4 = *reinterpret_cast<const uint4*>(rowp[rr] + 16 * c);
               wv[rr][0] = w4.x;
               wv[rr][1] = w4.y;
               wv[rr][2] = w4.z;
@@ -434,13 +440,13 @@ __global__ void __launch_bounds__(kGemvThreads, kMinBlocks) gemv_pack5_kernel(co
         }
 #pragma unroll
         for (int rr = 0; rr < kRows; ++rr) {
+          const int row_l = rl + rr * G;
 #pragma unroll
           for (int m = 0; m < M; ++m) {
             const int tot = __reduce_add_sync(0xffffffffu, am[rr][m][0] + am[rr][m][1] + (a4[rr][m] >> 6));
-            if (lane == 0 && (rr == 0 || two)) {
-              const int row = r0 + rl + rr * G;
-              if (S == 1) part[m * rpc + row] = tot;
-              else atomicAdd(&part[m * rpc + row], tot);
+            if (lane == 0 && row_l < nr) {
+              if (S == 1) part[m * rpc + r0 + row_l] = tot;
+              else atomicAdd(&part[m * rpc + r0 + row_l], tot);
             }
           }
         }
