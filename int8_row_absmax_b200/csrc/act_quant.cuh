@@ -8,6 +8,8 @@
 #pragma once
 
 #include "common.cuh"
+#include "ptx.cuh"
+#include "trit_table.cuh"
 
 namespace bl {
 
@@ -163,6 +165,105 @@ act_quant_reg_kernel(const float* __restrict__ X, int64_t K, float eps, int8_t* 
     if (i < K4) reinterpret_cast<uint32_t*>(qr)[i] = act_codes4(v[u], s, r);
   }
   for (int64_t i = K + threadIdx.x; i < ldq; i += kActThreads) qr[i] = 0;
+}
+
+// The same codes, written in the decode order of trit_table.cuh (positions
+// dorder_pos(k); bytes [K, ldq) of the order's row are 0), for the swapped
+// tensor-core GEMM.  One CTA of 512 threads per row; each thread of the second
+// pass writes one packed word's five code words.  It lets the next kernel on
+// the stream begin its prologue at once (programmatic dependent launch).
+constexpr int kActDoThreads = 512;
+__global__ void __launch_bounds__(kActDoThreads)
+act_quant_dorder_kernel(const float* __restrict__ X, int64_t K, float eps, int8_t* __restrict__ Xq,
+                        int64_t ldq, float* __restrict__ s_out) {
+  __shared__ float s_red[kActDoThreads / 32];
+  __shared__ float s_scale;
+  griddep_wait();
+  griddep_launch_dependents();
+  const int tid = threadIdx.x;
+  const int64_t m = blockIdx.x;
+  const float* xr = X + m * K;
+  uint32_t* qw = reinterpret_cast<uint32_t*>(Xq + m * ldq);
+  const bool vec = aligned(xr, 16) && (K & 3) == 0;
+  const int64_t K4 = vec ? (K >> 2) : 0;
+  float amax = 0.f;
+  bool bad = false;
+  for (int64_t i = tid; i < K4; i += kActDoThreads) {
+    const float4 v = reinterpret_cast<const float4*>(xr)[i];
+    const float a = fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w)));
+    bad |= !(a <= 3.402823466e38f) | (v.x != v.x) | (v.y != v.y) | (v.z != v.z) | (v.w != v.w);
+    amax = fmaxf(amax, a);
+  }
+  for (int64_t i = (K4 << 2) + tid; i < K; i += kActDoThreads) {
+    const float a = fabsf(xr[i]);
+    bad |= !(a <= 3.402823466e38f);
+    amax = fmaxf(amax, a);
+  }
+  amax = warp_max(amax);
+  if ((tid & 31) == 0) s_red[tid >> 5] = amax;
+  if (__syncthreads_or(bad) && tid == 0) raise_status(kDevNonFinite);
+  if (tid < 32) {
+    float w = tid < kActDoThreads / 32 ? s_red[tid] : 0.f;
+    w = warp_max(w);
+    if (tid == 0) {
+      const float s = __fadd_rn(__fdiv_rn(w, float(kActQmax)), eps);
+      s_scale = s;
+      s_out[m] = s;
+    }
+  }
+  __syncthreads();
+  const float s = s_scale;
+  const float rc = act_recip(s);
+  const int64_t ngrp = (K + 19) / 20;
+  for (int64_t gi = tid; gi < ngrp; gi += kActDoThreads) {
+    const int64_t k0 = 20 * gi;
+    uint32_t c[20];
+    bool tie = rc == 0.f;
+    if (vec && k0 + 20 <= K) {
+#pragma unroll
+      for (int v = 0; v < 5; ++v) {
+        const float4 f = reinterpret_cast<const float4*>(xr + k0)[v];
+        c[4 * v + 0] = act_code_try(f.x, rc, tie);
+        c[4 * v + 1] = act_code_try(f.y, rc, tie);
+        c[4 * v + 2] = act_code_try(f.z, rc, tie);
+        c[4 * v + 3] = act_code_try(f.w, rc, tie);
+      }
+    } else {
+#pragma unroll
+      for (int e = 0; e < 20; ++e) c[e] = k0 + e < K ? act_code_try(xr[k0 + e], rc, tie) : 0u;
+    }
+    if (tie)   // rare: a quotient near a half-integer; exact division
+      for (int e = 0; e < 20; ++e)
+        if (k0 + e < K) c[e] = uint32_t(uint8_t(int8_t(act_code_slow(xr[k0 + e], s))));
+    uint32_t* dst = qw + 5 * gi;
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+      dst[i] = c[5 * i] | (c[5 * i + 1] << 8) | (c[5 * i + 2] << 16) | (c[5 * i + 3] << 24);
+    dst[4] = c[4] | (c[9] << 8) | (c[14] << 16) | (c[19] << 24);
+  }
+  for (int64_t i = 5 * ngrp + tid; i < (ldq >> 2); i += kActDoThreads) qw[i] = 0u;
+}
+
+// Given codes [M, ldx] in natural order -> the decode order [M, ldd] (ldd % 4
+// == 0, ldd >= dorder_len(K)); one thread per output word.
+__global__ void xq_dorder_kernel(const int8_t* __restrict__ Xq, int64_t ldx, int64_t M, int64_t K,
+                                 int8_t* __restrict__ Xd, int64_t ldd) {
+  griddep_wait();
+  griddep_launch_dependents();
+  const int64_t wpr = ldd >> 2;
+  for (int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; i < M * wpr;
+       i += int64_t(gridDim.x) * blockDim.x) {
+    const int64_t m = i / wpr, wi = i - m * wpr;
+    const int64_t g = wi / 5, q = wi - 5 * g;
+    const int8_t* xr = Xq + m * ldx;
+    uint32_t v = 0;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int64_t k = q < 4 ? 5 * (4 * g + q) + e : 5 * (4 * g + e) + 4;
+      if (k < K) v |= uint32_t(uint8_t(xr[k])) << (8 * e);
+    }
+    reinterpret_cast<uint32_t*>(Xd + m * ldd)[wi] = v;
+  }
 }
 
 }  // namespace bl

@@ -174,16 +174,21 @@ bl_status check_ws(const void* ws, size_t ws_bytes, size_t need) {
 }
 
 // ---- linear --------------------------------------------------------------
+// Row stride of the swapped GEMM's decode-order codes: whole 128-byte atoms.
+int64_t swap_ldx(int64_t K) { return round_up(dorder_len(K), 128); }
+
 struct LinWs {
   int64_t ldx, ldk;
   size_t xq_off, s_off, wq_off, tc_off, total;
 };
 // X_q [M, ldx] and s [M]; with `unpacked_w`, an int8 copy of the packed weights
 // [N, ldk] for the tensor-core path; then `tc_bytes` for the tensor-core GEMM's
-// K-split partials.
-LinWs lin_layout(int64_t M, int64_t K, int64_t N = 0, bool unpacked_w = false, size_t tc_bytes = 0) {
+// K-split partials.  With `dorder`, X_q rows are in the decode order of the
+// swapped GEMM (whole packed words: dorder_len(K) bytes).
+LinWs lin_layout(int64_t M, int64_t K, int64_t N = 0, bool unpacked_w = false, size_t tc_bytes = 0,
+                 bool dorder = false) {
   LinWs l;
-  l.ldx = round_up(K, 16);
+  l.ldx = dorder ? swap_ldx(K) : round_up(K, 16);
   l.ldk = round_up(K, 16);
   l.xq_off = 0;
   l.s_off = align_up(size_t(M) * size_t(l.ldx));
@@ -239,9 +244,9 @@ bool tc_swap(int64_t M, bl_wfmt f) { return f == BL_W_PACK5 && M >= 1 && M <= kS
 TcSplit tc_split(int64_t M, int64_t N, int64_t K, bl_wfmt f) {
   TcSplit r;
   int64_t nch;
-  if (tc_swap(M, f)) {   // 128-row W tiles, K blocks of 160 trits
+  if (tc_swap(M, f)) {   // 128-row W tiles, K chunks of four 160-trit blocks
     r.tiles = ceil_div(N, int64_t(kSwBM));
-    nch = ceil_div(K, int64_t(kSwBK));
+    nch = ceil_div(K, int64_t(kSwBoxKb * kSwBK));
   } else {
     r.tiles = ceil_div(M, int64_t(kTcBM)) * ceil_div(N, int64_t(kTcBN));
     nch = ceil_div(ceil_div(K, int64_t(kTcBK)), int64_t(kTcChunk));
@@ -447,25 +452,61 @@ bool make_map_xq(CUtensorMap* map, const void* base, int64_t K, int64_t M, int64
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// Packed W [N, ldp] as boxes of {32 bytes, 128 rows}, no swizzle.
-bool make_map_wp32(CUtensorMap* map, const void* base, int64_t ldp, int64_t N) {
+// Packed W [N, ldp] as boxes of {128 bytes, 128 rows}, 128-byte swizzle.
+bool make_map_wp128(CUtensorMap* map, const void* base, int64_t ldp, int64_t N) {
   EncodeTiledFn fn = encode_tiled();
   if (!fn) return false;
   const cuuint64_t dims[2] = {cuuint64_t(ldp), cuuint64_t(N)};
   const cuuint64_t strides[1] = {cuuint64_t(ldp)};
-  const cuuint32_t box[2] = {32u, cuuint32_t(kSwBM)};
+  const cuuint32_t box[2] = {128u, cuuint32_t(kSwBM)};
   const cuuint32_t estr[2] = {1u, 1u};
   return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// A launch that may begin while the previous kernel on the stream finishes
+// (programmatic dependent launch); the kernel waits (griddepcontrol.wait)
+// before it touches what that kernel writes.
+template <typename... KArgs, typename... Args>
+bl_status launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                     Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, args...) == cudaSuccess ? launch_status() : BL_ERR_CUDA;
+}
+
+// X_q in decode order [M, ldx] (ldx % 128 == 0) as a 3-D tensor {128 bytes, M
+// rows, ldx / 128 atoms}, boxes {128, Np, 5} (one chunk of four K blocks),
+// 128-byte swizzle.
+bool make_map_x3d(CUtensorMap* map, const void* base, int64_t ldx, int64_t M, int Np) {
+  EncodeTiledFn fn = encode_tiled();
+  if (!fn) return false;
+  const cuuint64_t dims[3] = {128u, cuuint64_t(M), cuuint64_t(ldx / 128)};
+  const cuuint64_t strides[2] = {cuuint64_t(ldx), 128u};
+  const cuuint32_t box[3] = {128u, cuuint32_t(Np), 5u};
+  const cuuint32_t estr[3] = {1u, 1u, 1u};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 // The swapped GEMM for few-row packed layers (gemm_swap.cuh), then the K
-// split's reduction when there is one.
-bl_status run_swap(const int8_t* Xq, int64_t ldx, int64_t M, int64_t K, const void* W, int64_t ldw, int64_t N,
+// split's reduction when there is one.  Xd: the codes in decode order [M, ldx]
+// (ldx = swap_ldx(K), bytes beyond dorder_len(K) 0).
+bl_status run_swap(const int8_t* Xd, int64_t ldx, int64_t M, int64_t K, const void* W, int64_t ldw, int64_t N,
                    const float* s, const float* beta, const float* bias, float* Y, int32_t* acc, void* tcws,
-                   size_t tcws_bytes, cudaStream_t st) {
-  if (ldx % 16 != 0 || ldw % 16 != 0 || !is_aligned(Xq, 16) || !is_aligned(W, 16)) return BL_ERR_ALIGNMENT;
+                   size_t tcws_bytes, bool static_w, cudaStream_t st) {
+  if (ldx % 128 != 0 || ldx < dorder_len(K) || ldw % 16 != 0 || !is_aligned(Xd, 16) || !is_aligned(W, 16))
+    return BL_ERR_ALIGNMENT;
   if (M < 1 || M > kSwMaxNp) return BL_ERR_UNSUPPORTED;
   TcSplit sp = tc_split(M, N, K, BL_W_PACK5);
   if (!tcws) sp.split = 1;
@@ -473,9 +514,7 @@ bl_status run_swap(const int8_t* Xq, int64_t ldx, int64_t M, int64_t K, const vo
   if (sp.split > 1 && (!is_aligned(tcws, kWsAlign) || tcws_bytes < sp.bytes)) return BL_ERR_WORKSPACE;
   const int Np = int(round_up(M, 16));
   SwMaps maps;
-  if (!make_map_xq(&maps.x128, Xq, K, M, ldx, 128, Np, CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !make_map_xq(&maps.x32, Xq, K, M, ldx, 32, Np, CU_TENSOR_MAP_SWIZZLE_32B) ||
-      !make_map_wp32(&maps.wp, W, ldw, N))
+  if (!make_map_x3d(&maps.x, Xd, ldx, M, Np) || !make_map_wp128(&maps.wp, W, ldw, N))
     return BL_ERR_CUDA;
   SwArgs a;
   a.M = M;
@@ -491,34 +530,29 @@ bl_status run_swap(const int8_t* Xq, int64_t ldx, int64_t M, int64_t K, const vo
   a.split = sp.split;
   a.part = sp.split > 1 ? static_cast<int32_t*>(tcws) : nullptr;
   const SwLayout l = sw_layout(Np);
-  if (l.nst < 2) return BL_ERR_UNSUPPORTED;
+  if (l.nst < 1) return BL_ERR_UNSUPPORTED;
   a.nst = l.nst;
-  a.stage = l.stage;
-  a.pk_off = l.pk_off;
+  a.xst = l.xst;
   a.lut_off = l.lut_off;
+  a.x_off = l.x_off;
+  a.static_w = static_w ? 1 : 0;
+  a.mma_warps = sw_mma_warps(Np);
   const int64_t work = sp.tiles * sp.split;
   const dim3 grid(unsigned(work < num_sms() ? work : num_sms()));
   const bool dq = Y != nullptr;
-  if (dq) {
-    if (cudaFuncSetAttribute(gemm_swap_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSwSmemMax) !=
-        cudaSuccess)
-      return BL_ERR_CUDA;
-    gemm_swap_kernel<true><<<grid, kSwThreads, l.smem, st>>>(maps, a);
-  } else {
-    if (cudaFuncSetAttribute(gemm_swap_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSwSmemMax) !=
-        cudaSuccess)
-      return BL_ERR_CUDA;
-    gemm_swap_kernel<false><<<grid, kSwThreads, l.smem, st>>>(maps, a);
-  }
-  bl_status r = launch_status();
+  auto kern = dq ? gemm_swap_kernel<true> : gemm_swap_kernel<false>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSwSmemMax) != cudaSuccess)
+    return BL_ERR_CUDA;
+  bl_status r = launch_pdl(kern, grid, dim3(kSwThreads), size_t(l.smem), st, maps, a);
   if (r != BL_OK || sp.split == 1) return r;
   const int64_t rw = (N % 4 == 0 ? M * (N / 4) : M * N);
+  const dim3 rg(unsigned(grid_for(rw, 256)));
   if (dq)
-    tc_reduce_kernel<true><<<grid_for(rw, 256), 256, 0, st>>>(a.part, sp.split, M, N, s, beta, bias, Y, nullptr);
-  else
-    tc_reduce_kernel<false><<<grid_for(rw, 256), 256, 0, st>>>(a.part, sp.split, M, N, nullptr, nullptr, nullptr,
-                                                              nullptr, acc);
-  return launch_status();
+    return launch_pdl(tc_reduce_kernel<true>, rg, dim3(256), 0, st, static_cast<const int32_t*>(a.part), sp.split,
+                      M, N, s, beta, bias, Y, static_cast<int32_t*>(nullptr));
+  return launch_pdl(tc_reduce_kernel<false>, rg, dim3(256), 0, st, static_cast<const int32_t*>(a.part), sp.split,
+                    M, N, static_cast<const float*>(nullptr), static_cast<const float*>(nullptr),
+                    static_cast<const float*>(nullptr), static_cast<float*>(nullptr), acc);
 }
 
 // Packed weights -> int8 rows in the workspace, for tensor-core GEMMs with more
@@ -842,7 +876,8 @@ size_t bl_linear_ex_workspace_size(int64_t M, int64_t N, int64_t K, bl_wfmt f, i
   path &= kPathMask;
   const int p = resolve_path(M, N, K, f, path, nullptr);
   if (p == BL_PATH_GEMV) return 0;   // activation quantization inside the GEMV: no scratch
-  return lin_layout(M, K, N, p == BL_PATH_TC && tc_unpack(M, f), p == BL_PATH_TC ? tc_split(M, N, K, f).bytes : 0)
+  return lin_layout(M, K, N, p == BL_PATH_TC && tc_unpack(M, f), p == BL_PATH_TC ? tc_split(M, N, K, f).bytes : 0,
+                    p == BL_PATH_TC && tc_swap(M, f))
       .total;
 }
 
@@ -850,7 +885,7 @@ size_t bl_linear_ex_workspace_size(int64_t M, int64_t N, int64_t K, bl_wfmt f, i
 static size_t linear_ws_nosplit(int64_t M, int64_t N, int64_t K, bl_wfmt f) {
   const int p = resolve_path(M, N, K, f, BL_PATH_AUTO, nullptr);
   if (p == BL_PATH_GEMV) return 0;
-  return lin_layout(M, K, N, p == BL_PATH_TC && tc_unpack(M, f), 0).total;
+  return lin_layout(M, K, N, p == BL_PATH_TC && tc_unpack(M, f), 0, p == BL_PATH_TC && tc_swap(M, f)).total;
 }
 
 size_t bl_linear_workspace_size(int64_t M, int64_t N, int64_t K, bl_wfmt f) {
@@ -886,12 +921,16 @@ static bl_status linear_impl(const float* X, int64_t M, int64_t K, const void* W
   if (p == BL_PATH_GEMV)   // needs no workspace
     return run_gemv(X, nullptr, 0, M, K, W, ldw, N, beta_dev, bias, eps, Y, nullptr, static_w, stream);
   const size_t tcb = (p == BL_PATH_TC && allow_split) ? tc_split(M, N, K, f).bytes : 0;
-  const LinWs l = lin_layout(M, K, N, p == BL_PATH_TC && tc_unpack(M, f), tcb);
+  const bool swap = p == BL_PATH_TC && tc_swap(M, f);
+  const LinWs l = lin_layout(M, K, N, p == BL_PATH_TC && tc_unpack(M, f), tcb, swap);
   if (!ws || !is_aligned(ws, kWsAlign) || ws_bytes < l.total) return BL_ERR_WORKSPACE;
   void* tcws = tcb ? static_cast<char*>(ws) + l.tc_off : nullptr;   // null: no K split
   int8_t* Xq = reinterpret_cast<int8_t*>(static_cast<char*>(ws) + l.xq_off);
   float* s = reinterpret_cast<float*>(static_cast<char*>(ws) + l.s_off);
-  launch_act_quant(X, M, K, eps, Xq, l.ldx, s, stream);
+  if (swap)   // codes in the swapped GEMM's decode order
+    act_quant_dorder_kernel<<<unsigned(M), kActDoThreads, 0, stream>>>(X, K, eps, Xq, l.ldx, s);
+  else
+    launch_act_quant(X, M, K, eps, Xq, l.ldx, s, stream);
   st = launch_status();
   if (st != BL_OK) return st;
   if (p == BL_PATH_TC) {
@@ -901,8 +940,8 @@ static bl_status linear_impl(const float* X, int64_t M, int64_t K, const void* W
       if (st != BL_OK) return st;
       return run_tc(Xq, l.ldx, M, K, scratch, l.ldk, false, N, s, beta_dev, bias, Y, nullptr, tcws, tcb, stream);
     }
-    if (tc_swap(M, f))
-      return run_swap(Xq, l.ldx, M, K, W, ldw, N, s, beta_dev, bias, Y, nullptr, tcws, tcb, stream);
+    if (swap)
+      return run_swap(Xq, l.ldx, M, K, W, ldw, N, s, beta_dev, bias, Y, nullptr, tcws, tcb, static_w, stream);
     return run_tc(Xq, l.ldx, M, K, W, ldw, f == BL_W_PACK5, N, s, beta_dev, bias, Y, nullptr, tcws, tcb, stream);
   }
   return run_simt(Xq, l.ldx, M, K, W, f, ldw, N, s, beta_dev, bias, Y, nullptr, stream);
@@ -1006,11 +1045,14 @@ size_t bl_linear_acc_workspace_size(int64_t M, int64_t N, int64_t K, bl_wfmt f, 
   path &= kPathMask;
   const int p = resolve_path(M, N, K, f, path, nullptr, false);
   if (p != BL_PATH_TC) return 0;
+  if (tc_swap(M, f))   // the split's partials, then the codes in decode order
+    return tc_split(M, N, K, f).bytes + align_up(size_t(M) * size_t(swap_ldx(K)));
   return (tc_unpack(M, f) ? align_up(size_t(N) * size_t(round_up(K, 16))) : 0) + tc_split(M, N, K, f).bytes;
 }
 
 // no_ws: bl_linear_acc, which takes no workspace: packed weights are then
-// decoded inside the tensor-core GEMM at any M, and K is not split.
+// decoded inside the un-swapped tensor-core GEMM at any M, and K is not split
+// (the swapped GEMM needs the codes in decode order, a copy in the workspace).
 static bl_status linear_acc_impl(const int8_t* Xq, int64_t M, int64_t K, const void* W, bl_wfmt f, int64_t N,
                           int64_t ldw, int32_t* acc, void* ws, size_t ws_bytes, int path, bool no_ws,
                           cudaStream_t stream) {
@@ -1026,8 +1068,10 @@ static bl_status linear_acc_impl(const int8_t* Xq, int64_t M, int64_t K, const v
   if (!Xq || !acc) return BL_ERR_INVALID_ARG;
   if (!is_aligned(acc, 4)) return BL_ERR_ALIGNMENT;
   int p = resolve_path(M, N, K, f, path, nullptr, false, ldw, W);
-  // X_q given by the caller: the tensor cores need a TMA-able [M, K] int8 matrix
-  const bool tc_x_ok = K % 16 == 0 && is_aligned(Xq, 16);
+  const bool swap = p == BL_PATH_TC && tc_swap(M, f) && !no_ws;
+  // X_q given by the caller: the un-swapped tensor-core GEMM needs a TMA-able
+  // [M, K] int8 matrix (the swapped one reads a decode-order copy)
+  const bool tc_x_ok = swap || (K % 16 == 0 && is_aligned(Xq, 16));
   if (p == BL_PATH_TC && !tc_x_ok) {
     if (path == BL_PATH_TC) return BL_ERR_UNSUPPORTED;
     p = resolve_path(M, N, K, f, BL_PATH_GEMV, nullptr, false) >= 0 ? BL_PATH_GEMV : BL_PATH_SIMT;
@@ -1035,6 +1079,18 @@ static bl_status linear_acc_impl(const int8_t* Xq, int64_t M, int64_t K, const v
   if (p < 0) return BL_ERR_UNSUPPORTED;
   if (p == BL_PATH_GEMV)
     return run_gemv(nullptr, Xq, K, M, K, W, ldw, N, nullptr, nullptr, 0.f, nullptr, acc, static_w, stream);
+  if (p == BL_PATH_TC && swap) {
+    const int64_t ldd = swap_ldx(K);
+    const TcSplit sp = tc_split(M, N, K, f);
+    const size_t need = sp.bytes + align_up(size_t(M) * size_t(ldd));
+    if (!ws || !is_aligned(ws, kWsAlign) || ws_bytes < need) return BL_ERR_WORKSPACE;
+    int8_t* Xd = static_cast<int8_t*>(ws) + sp.bytes;
+    bl_status st2 = launch_pdl(xq_dorder_kernel, dim3(unsigned(grid_for(M * (ldd / 4), 256))), dim3(256), 0,
+                               stream, Xq, K, M, K, Xd, ldd);
+    if (st2 != BL_OK) return st2;
+    return run_swap(Xd, ldd, M, K, W, ldw, N, nullptr, nullptr, nullptr, nullptr, acc, sp.bytes ? ws : nullptr,
+                    sp.bytes, static_w, stream);
+  }
   if (p == BL_PATH_TC) {
     const bool unp = !no_ws && tc_unpack(M, f);
     const size_t wq = unp ? align_up(size_t(N) * size_t(round_up(K, 16))) : 0;
@@ -1049,8 +1105,6 @@ static bl_status linear_acc_impl(const int8_t* Xq, int64_t M, int64_t K, const v
       return run_tc(Xq, K, M, K, scratch, round_up(K, 16), false, N, nullptr, nullptr, nullptr, nullptr, acc,
                     tcws, tcb, stream);
     }
-    if (tc_swap(M, f))
-      return run_swap(Xq, K, M, K, W, ldw, N, nullptr, nullptr, nullptr, nullptr, acc, tcws, tcb, stream);
     return run_tc(Xq, K, M, K, W, ldw, f == BL_W_PACK5, N, nullptr, nullptr, nullptr, nullptr, acc, tcws, tcb,
                   stream);
   }

@@ -437,6 +437,7 @@ template <bool kDequant>
 __global__ void __launch_bounds__(256)
 tc_reduce_kernel(const int32_t* __restrict__ part, int split, int64_t M, int64_t N, const float* s,
                  const float* beta, const float* bias, float* Y, int32_t* acc) {
+  griddep_wait();   // launched as a dependent of the GEMM: its partials are complete
   const bool v4 = (N & 3) == 0 && (kDequant ? aligned(Y, 16) : aligned(acc, 16));
   const int64_t per_row = v4 ? N / 4 : N;
   const int64_t total = M * per_row;

@@ -40,6 +40,7 @@
 #include "act_quant.cuh"
 #include "common.cuh"
 #include "ptx.cuh"
+#include "trit_table.cuh"
 
 namespace bl {
 
@@ -47,7 +48,6 @@ constexpr int kGemvMaxM = 4;
 constexpr int kGemvWarps = 16;
 constexpr int kGemvThreads = kGemvWarps * 32;
 constexpr int kGemvMaxProbs = 4;
-constexpr uint32_t kLutBytes = 256 * 256;      // a row for every byte value: no read leaves the table
 constexpr uint32_t kGemvMaxSmem = 232448 - 1024;  // 227 KB per CTA, less the static arrays
 constexpr uint32_t kGemvSegTarget = 32 * 1024;  // bytes per bulk copy (one mbarrier each): few, large copies
 constexpr int kGemvMaxStages = 24;
@@ -140,40 +140,6 @@ inline bool gemv_feasible(int64_t M, int64_t N, int64_t K, int64_t ldp) {
   const int ch = gemv_chunks_per_lane(M, ldp);
   GemvProb P;
   return ch > 0 && gemv_plan_prob(M, N, K, ldp, int(N < kGemvCtas ? N : kGemvCtas), ch, P);
-}
-
-// The decode table as it sits in shared memory, built at compile time: word
-// b*64 + l (l < 32) holds trits t0..t3 of byte b as four int8 (lane l's copy;
-// words 32..63 of a row repeat them, so the row pitch is 256 bytes and one
-// byte_perm forms an address).  Bytes above 242 are not codes and read as 121
-// (five zero trits).  Each CTA copies it into shared memory with one bulk copy.
-struct TritLut {
-  uint32_t w[256 * 64];
-};
-constexpr TritLut make_trit_lut() {
-  TritLut t{};
-  for (uint32_t b = 0; b < 256; ++b) {
-    uint32_t x = b > 242u ? 121u : b, v = 0;
-    for (int k = 0; k < 4; ++k) {
-      v |= ((x % 3u + 255u) & 0xFFu) << (8 * k);
-      x /= 3u;
-    }
-    for (uint32_t l = 0; l < 64; ++l) t.w[b * 64 + l] = v;
-  }
-  return t;
-}
-__device__ __align__(128) const TritLut g_trit_lut = make_trit_lut();
-
-__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
-__device__ __forceinline__ void griddep_launch_dependents() {
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-}
-
-// Byte offset of activation element k in the decode-order code row.
-__device__ __forceinline__ uint32_t gemv_xpos(uint32_t k) {
-  const uint32_t j = __umulhi(k, 0xCCCCCCCDu) >> 2;   // k / 5
-  const uint32_t r = k - 5u * j;
-  return 20u * (j >> 2) + (r < 4u ? 4u * (j & 3u) + r : 16u + (j & 3u));
 }
 
 template <int M, int CH, bool kFused, int kMinBlocks>
@@ -421,11 +387,8 @@ __global__ void __launch_bounds__(kGemvThreads, kMinBlocks) gemv_pack5_kernel(co
                 const uint32_t w = wv[rr][q];
                 uint32_t t[4];
 #pragma unroll
-                for (int bb = 0; bb < 4; ++bb)
-                  t[bb] = *reinterpret_cast<const uint32_t*>(smem + __byte_perm(w, lanebase, 0x5504u | (bb << 4)));
-                const uint32_t E = __byte_perm(w, 0u, 0x4240u) * 203u;
-                const uint32_t O = __byte_perm(w, 0u, 0x4341u) * 203u;
-                const uint32_t D = __byte_perm(E, O, 0x7351u) & 0xC0C0C0C0u;
+                for (int bb = 0; bb < 4; ++bb) t[bb] = lut_t0123(smem, w, lanebase, bb);
+                const uint32_t D = d4x64(w);
 #pragma unroll
                 for (int m = 0; m < M; ++m) {
                   int acc = am[rr][m][q & 1];

@@ -129,21 +129,25 @@ def test_tensor_core_plan_and_workspace(lib, M, K, N):
     weights beyond 4 row tiles of 128, + the reduction of a K split, which is
     taken when the output tiles (128 x 256; for M <= 128 the swapped GEMM's 128
     W rows) are fewer than half of 148 SMs and K has at least two K ranges
-    (640-wide chunks; 160-trit blocks when swapped), at most 8 splits.  The workspace holds X_q [M,
+    (640-wide chunks; 640-trit chunks of four blocks when swapped), at most 8 splits.  The workspace holds X_q [M,
     ldx] and s, then the int8 copy of W_q, then the split's int32 partials."""
-    if M <= 128:     # few rows, packed weights: the swapped GEMM (128 W rows per tile, 160-trit K blocks)
+    if M <= 128:     # few rows, packed weights: the swapped GEMM (128 W rows per tile, K in chunks of 640 trits)
         tiles = _cdiv(N, 128)
-        split = max(1, min(148 // tiles, _cdiv(K, 160), 8))
+        split = max(1, min(148 // tiles, _cdiv(K, 640), 8))
     else:
         tiles = _cdiv(M, 128) * _cdiv(N, 256)
         split = max(1, min(148 // tiles, _cdiv(_cdiv(K, 128), 5), 8))
     n = ctypes.c_int(0)
     assert lib.bl_linear_plan(M, N, K, pkg.PACK5, pkg.PATH_TC, ctypes.byref(n)) == pkg.PATH_TC
     assert n.value == 2 + (M > 512) + (split > 1)
-    ldx = _cdiv(K, 16) * 16
-    extra = (_al(N * ldx) if M > 512 else 0) + (_al(split * M * N * 4) if split > 1 else 0)
+    # the swapped GEMM reads X_q in decode order: rows of whole packed words (20
+    # trits), padded to whole 128-byte swizzle atoms
+    ldx = _cdiv(20 * _cdiv(K, 20), 128) * 128 if M <= 128 else _cdiv(K, 16) * 16
+    extra = (_al(N * _cdiv(K, 16) * 16) if M > 512 else 0) + (_al(split * M * N * 4) if split > 1 else 0)
     assert lib.bl_linear_ex_workspace_size(M, N, K, pkg.PACK5, pkg.PATH_TC) == _al(M * ldx) + _al(M * 4 + 4) + extra
-    assert lib.bl_linear_acc_workspace_size(M, N, K, pkg.PACK5, pkg.PATH_TC) == extra
+    # bl_linear_acc_ex: the split's partials, and for the swapped GEMM the decode-order copy of X_q
+    acc_extra = extra + (_al(M * ldx) if M <= 128 else 0)
+    assert lib.bl_linear_acc_workspace_size(M, N, K, pkg.PACK5, pkg.PATH_TC) == acc_extra
 
 
 def test_decode_gemv_needs_no_workspace(lib):

@@ -551,8 +551,11 @@ def test_linear_bias(bl):
 
 def acc_supported(bl, M, N, K, f, path):
     """Whether bl_linear_acc_ex takes the pinned path with contiguous X_q [M, K]."""
-    if path == bl.PATH_TC:     # X_q rows of K bytes must be TMA-aligned
-        return K >= 128 and K % 16 == 0 and bl.linear_plan(M, N, K, f, path)[0] == path
+    if path == bl.PATH_TC:
+        # the swapped GEMM (packed weights, M <= 128) reads a decode-order copy of
+        # X_q in the workspace; otherwise X_q rows of K bytes must be TMA-aligned
+        swapped = f == bl.PACK5 and M <= 128
+        return K >= 128 and (swapped or K % 16 == 0) and bl.linear_plan(M, N, K, f, path)[0] == path
     return bl.linear_plan(M, N, K, f, path)[0] == path or path == bl.PATH_AUTO
 
 
