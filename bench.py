@@ -191,8 +191,10 @@ def tensor_roofline(macs, ms, peaks, burst=True):
 KERNEL_SOURCES = {
     "wquant_kernel": (("weight_fused.cuh", "weight_quant.cuh", "act_quant.cuh", "common.cuh", "ptx.cuh"),
                       ("wquant", "kFu", "fused")),
-    "gemv_pack5_kernel": (("gemv_pack5.cuh", "act_quant.cuh", "common.cuh", "ptx.cuh"),
+    "gemv_pack5_kernel": (("gemv_pack5.cuh", "trit_table.cuh", "act_quant.cuh", "common.cuh", "ptx.cuh"),
                           ("gemv", "Gemv")),
+    "gemm_swap_kernel": (("gemm_swap.cuh", "trit_table.cuh", "common.cuh", "ptx.cuh"),
+                         ("swap", "Swap", "run_swap", "sw_")),
 }
 
 
