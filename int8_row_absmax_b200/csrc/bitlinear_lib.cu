@@ -537,6 +537,8 @@ bl_status run_swap(const int8_t* Xd, int64_t ldx, int64_t M, int64_t K, const vo
   a.x_off = l.x_off;
   a.static_w = static_w ? 1 : 0;
   a.mma_warps = sw_mma_warps(Np);
+  a.a_col0 = sw_a_col0(Np);
+  a.nsa = sw_a_stages(Np);
   const int64_t work = sp.tiles * sp.split;
   const dim3 grid(unsigned(work < num_sms() ? work : num_sms()));
   const bool dq = Y != nullptr;

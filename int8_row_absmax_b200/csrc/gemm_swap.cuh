@@ -27,15 +27,18 @@
 //   * per block, five tcgen05.mma.kind::i8 (M = 128, N = Np, K = 32): A from
 //     TMEM columns 8i.., B at position 160 h + 32 i of the chunk (atom and
 //     offset of the 128-byte swizzle).
-// Roles: warp 0 issues the X_q loads, warp 22 the packed boxes, warp 1 the
-// MMAs, warps 2..5 drain TMEM (lane = W row, columns = X rows) with the dequant
-// fused, warps 6..21 decode.  With fewer 128-row W tiles than SMs, K is split
-// into ranges of whole chunks whose int32 partials [split, M, N]
-// tc_reduce_kernel adds up (exact).  The launch is a programmatic dependent
-// one: barriers, TMEM, the table copy and (for static weights) the first packed
-// boxes are set up while the previous kernel finishes.  Every wait is bounded;
-// on a timeout the kernel records kDevTimeout, lets copies and MMAs in flight
-// land and frees its TMEM.
+// Roles: warp 0 issues the X_q loads, warp 22 the packed boxes, warp 1 holds
+// the TMEM allocation, warps 6..21 decode, warps 2..5 issue the MMAs (one
+// thread issues a tcgen05.mma only every 60-110 ns, and issuers in several
+// warps overlap) into an accumulator each, then drain TMEM (lane = W row,
+// columns = X rows), add the accumulators and fuse the dequant into the
+// stores.  With fewer 128-row W tiles than SMs, K is split into ranges of
+// whole chunks whose int32 partials [split, M, N] tc_reduce_kernel adds up
+// (exact).  The launch is a programmatic dependent one: barriers, TMEM, the
+// decode table (written into shared memory by the CTA) and (for static
+// weights) the first packed boxes are set up while the previous kernel
+// finishes.  Every wait is bounded; on a timeout the kernel records
+// kDevTimeout, lets copies and MMAs in flight land and frees its TMEM.
 #pragma once
 
 #include "common.cuh"
@@ -52,10 +55,9 @@ constexpr int kSwPkSlots = 4;              // packed boxes in flight: 64 KB per 
 constexpr int kSwMaxNp = 128;              // X rows per MMA (N), multiple of 16
 constexpr int kSwChunkX = 5 * 128;         // X_q bytes per row and chunk (640 trits)
 constexpr int kSwMaxXStages = 16;          // X chunks in flight (as many as fit)
-constexpr int kSwAStages = 4;              // decoded W blocks in flight (TMEM)
-constexpr int kSwAccCols = 256;            // TMEM columns 0..255: one accumulator per MMA issuer
-constexpr int kSwACol0 = kSwAccCols;       // then the A stages
-constexpr int kSwAStride = 64;             // TMEM columns per A stage (40 used)
+constexpr int kSwMaxAStages = 8;           // decoded W blocks in flight (TMEM), as many as fit
+constexpr int kSwAccCols = 256;            // at most 256 TMEM columns of accumulators (one per MMA issuer)
+constexpr int kSwAStride = 64;             // TMEM columns per A stage (40 used), 64-column aligned
 constexpr int kSwTmemCols = 512;
 constexpr int kSwDecGroups = 4, kSwDecWarps = 4 * kSwDecGroups;
 constexpr int kSwPkWarp = 6 + kSwDecWarps;             // the packed boxes' producer
@@ -63,7 +65,7 @@ constexpr int kSwThreads = 32 * (kSwPkWarp + 1);
 constexpr int kSwMaxSplit = 8;
 constexpr int kSwSmemMax = 232448 - 1024;  // dynamic shared memory budget
 
-static_assert(kSwACol0 + kSwAStages * kSwAStride <= kSwTmemCols, "TMEM columns");
+static_assert(kSwAccCols + 4 * kSwAStride <= kSwTmemCols, "TMEM columns");
 
 // Shared memory (from the 1024-aligned base): the packed ring (4 x 16 KB), the
 // decode table (64 KB), then `nst` X chunks of [5 atoms][Np rows][128 B].  X has
@@ -87,6 +89,14 @@ inline SwLayout sw_layout(int Np) {
 // accumulator columns of TMEM, else two (a divisor of the four A stages, so
 // that every stage is always released by the same issuer, in order).
 inline int sw_mma_warps(int Np) { return Np <= kSwAccCols / 4 ? 4 : 2; }
+// TMEM: the accumulators (issuers x Np columns) from column 0, then the A
+// stages from the next multiple of 64 columns, as many as fit (up to 8), so
+// that a decoder group fills its next stage while the MMAs read the last one.
+inline int sw_a_col0(int Np) { return int(round_up(int64_t(sw_mma_warps(Np)) * Np, kSwAStride)); }
+inline int sw_a_stages(int Np) {
+  const int n = (kSwTmemCols - sw_a_col0(Np)) / kSwAStride;
+  return n > kSwMaxAStages ? kSwMaxAStages : n;
+}
 
 struct alignas(64) SwMaps {
   CUtensorMap x;      // X_q in decode order as {128 B, M rows, ldx/128 atoms}, boxes {128, Np, 5}, 128-byte swizzle
@@ -106,6 +116,7 @@ struct SwArgs {
   int nst, xst, lut_off, x_off;   // shared-memory layout (sw_layout); nst X stages
   int static_w;        // 1: W is not written by earlier kernels (copied before the dependency wait)
   int mma_warps;       // MMA issuers, one accumulator each (sw_mma_warps)
+  int a_col0, nsa;     // TMEM column of the first A stage, number of A stages
 };
 
 // The TMEM load of 16 consecutive 32-bit columns of this thread's lane.
@@ -135,9 +146,9 @@ template <bool kDequant>
 __global__ void __launch_bounds__(kSwThreads, 1)
 gemm_swap_kernel(const __grid_constant__ SwMaps maps, const SwArgs a) {
   extern __shared__ unsigned char smem_raw[];
-  __shared__ uint64_t ld_full[kSwMaxXStages], x_empty[kSwMaxXStages], dec_full[kSwAStages], a_empty[kSwAStages];
+  __shared__ uint64_t ld_full[kSwMaxXStages], x_empty[kSwMaxXStages], dec_full[kSwMaxAStages], a_empty[kSwMaxAStages];
   __shared__ uint64_t pk_full[kSwPkSlots], pk_empty[kSwPkSlots];
-  __shared__ uint64_t acc_full, acc_empty, drain, lut_bar;
+  __shared__ uint64_t acc_full, acc_empty, drain;
   __shared__ uint32_t s_tmem;
   __shared__ int s_err;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -145,7 +156,7 @@ gemm_swap_kernel(const __grid_constant__ SwMaps maps, const SwArgs a) {
   const uint32_t base = (smem_u32(smem_raw) + 1023u) & ~1023u;
   unsigned char* smem = smem_raw + (base - smem_u32(smem_raw));
   const unsigned char* lut = smem + a.lut_off;
-  const int Np = a.Np, nst = a.nst;
+  const int Np = a.Np, nst = a.nst, nsa = a.nsa;
   const int nkb = int(ceil_div(a.K, kSwBK));
   const int nch = (nkb + kSwBoxKb - 1) / kSwBoxKb;   // chunks of four K blocks
   const int S = a.split;
@@ -168,7 +179,7 @@ gemm_swap_kernel(const __grid_constant__ SwMaps maps, const SwArgs a) {
       mbar_init(&ld_full[s], 1);
       mbar_init(&x_empty[s], a.mma_warps);  // every issuer, once per chunk
     }
-    for (int s = 0; s < kSwAStages; ++s) {
+    for (int s = 0; s < a.nsa; ++s) {
       mbar_init(&dec_full[s], 4);            // the four warps of a decoder group
       mbar_init(&a_empty[s], 1);
     }
@@ -179,13 +190,11 @@ gemm_swap_kernel(const __grid_constant__ SwMaps maps, const SwArgs a) {
     mbar_init(&acc_full, a.mma_warps);
     mbar_init(&acc_empty, 4);
     mbar_init(&drain, a.mma_warps);
-    mbar_init(&lut_bar, 1);
     fence_mbar_init();
     prefetch_tmap(&maps.x);
     prefetch_tmap(&maps.wp);
-    mbar_arrive_expect_tx(&lut_bar, kLutBytes);
-    bulk_g2s(smem + a.lut_off, &g_trit_lut, kLutBytes, &lut_bar);
   }
+  build_trit_lut(smem + a.lut_off, tid, kSwThreads);   // visible after the barrier below
   if (warp == 1) {
     tmem_alloc(&s_tmem, kSwTmemCols);
     tmem_relinquish();
@@ -265,7 +274,7 @@ gemm_swap_kernel(const __grid_constant__ SwMaps maps, const SwArgs a) {
     const uint32_t tlane = tmem + (uint32_t(qd * 32) << 16);
     // 16-byte chunks 2g, 2g + 1 of the row's 128 bytes, at their swizzled places
     const int c0 = (2 * g) ^ (r & 7), c1 = (2 * g + 1) ^ (r & 7);
-    bool ok = __all_sync(0xffffffffu, mbar_wait(&lut_bar, 0u));
+    bool ok = true;
     int it = 0, bi = 0;
     for (int w = blockIdx.x; w < nwork && ok && !*err; w += gridDim.x) {
       int t, kb0, kb1, j;
@@ -280,9 +289,8 @@ gemm_swap_kernel(const __grid_constant__ SwMaps maps, const SwArgs a) {
         }
         const int l = kSwBoxKb * b + g;
         if (l < nl) {
-          const int itb = it + l, s = itb % kSwAStages;
-          if (itb >= kSwAStages &&
-              !__all_sync(0xffffffffu, mbar_wait(&a_empty[s], uint32_t(itb / kSwAStages - 1) & 1u))) {
+          const int itb = it + l, s = itb % nsa;
+          if (itb >= nsa && !__all_sync(0xffffffffu, mbar_wait(&a_empty[s], uint32_t(itb / nsa - 1) & 1u))) {
             ok = false;
             break;
           }
@@ -292,7 +300,7 @@ gemm_swap_kernel(const __grid_constant__ SwMaps maps, const SwArgs a) {
           uint32_t o[40];
           sw_decode_block(lut, lanebase, p0, p1, o);
           tc_fence_after();            // the MMAs that read this stage before are complete
-          const uint32_t ta = tlane + uint32_t(kSwACol0 + s * kSwAStride);
+          const uint32_t ta = tlane + uint32_t(a.a_col0 + s * kSwAStride);
           tmem_st32(ta, o);
           tmem_st8(ta + 32u, o + 32);
           tmem_st_wait();
@@ -337,9 +345,9 @@ gemm_swap_kernel(const __grid_constant__ SwMaps maps, const SwArgs a) {
           const int s = ci % nst;
           const int hend = min(kSwBoxKb, nl - l0);
           for (int h = mw; h < hend; h += nmw) {
-            const int itb = it + l0 + h, sa = itb % kSwAStages;
+            const int itb = it + l0 + h, sa = itb % nsa;
             const bool got = mbar_wait(&ld_full[s], uint32_t(ci / nst) & 1u) &&
-                             mbar_wait(&dec_full[sa], uint32_t(itb / kSwAStages) & 1u);
+                             mbar_wait(&dec_full[sa], uint32_t(itb / nsa) & 1u);
             if (!__all_sync(0xffffffffu, got)) {
               ok = false;
               break;
@@ -347,7 +355,7 @@ gemm_swap_kernel(const __grid_constant__ SwMaps maps, const SwArgs a) {
             tc_fence_after();
             if (lane == 0) {
               const uint32_t xa = smem_u32(stage_x(s));
-              const uint32_t acol = tmem + uint32_t(kSwACol0 + sa * kSwAStride);
+              const uint32_t acol = tmem + uint32_t(a.a_col0 + sa * kSwAStride);
 #pragma unroll
               for (int i = 0; i < 5; ++i) {
                 const uint32_t pos = uint32_t(kSwBK * h + 32 * i);   // position in the chunk
@@ -428,7 +436,6 @@ gemm_swap_kernel(const __grid_constant__ SwMaps maps, const SwArgs a) {
     tc_fence_after();
     tmem_dealloc(tmem, kSwTmemCols);
   }
-  if (tid == 0) (void)mbar_wait(&lut_bar, 0u);   // the table copy has landed before the CTA exits
 }
 
 }  // namespace bl

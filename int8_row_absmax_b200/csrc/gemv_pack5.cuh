@@ -13,9 +13,9 @@
 //
 // Per CTA (one per SM; two fit when the CTA's weights are small):
 //   * before the dependency wait (programmatic dependent launch): mbarriers,
-//     a bulk copy (TMA engine) of the decode table (a compile-time constant in
-//     global memory) and -- when the caller declares the weights static --
-//     the bulk copy of the CTA's first segment of packed rows, so the weight
+//     the decode table written into shared memory by the CTA's threads and --
+//     when the caller declares the weights static -- the bulk copy (TMA
+//     engine) of the CTA's first segment of packed rows, so the weight
 //     stream starts while the previous kernel finishes; the other segments
 //     follow the copy of X, which is on the critical path;
 //   * griddepcontrol.wait, then launch_dependents (the next kernel may start
@@ -120,7 +120,7 @@ inline bool gemv_plan_prob(int64_t M, int64_t N, int64_t K, int64_t ldp, int cta
   const uint32_t stage_bytes = uint32_t(P.seg_rows * ldp);
   int64_t ns = nseg < kGemvMaxStages ? nseg : kGemvMaxStages;
   for (; ns >= 1; --ns) {
-    P.stage_off = align_to(P.bar_off + uint32_t(8 * (ns + 2)), 128);
+    P.stage_off = align_to(P.bar_off + uint32_t(8 * (ns + 1)), 128);
     if (int64_t(P.stage_off) + ns * stage_bytes <= kGemvMaxSmem) break;
   }
   if (ns < 1) return false;
@@ -181,19 +181,16 @@ __global__ void __launch_bounds__(kGemvThreads, kMinBlocks) gemv_pack5_kernel(co
   };
 
   // ---- prologue: nothing here reads what an earlier kernel may still write
-  // (the decode table is a constant of this library)
-  uint64_t* bar_lut = &bars[nstage];
-  uint64_t* bar_x = &bars[nstage + 1];
+  uint64_t* bar_x = &bars[nstage];
   if (tid == 0) {
-    for (int s = 0; s <= nstage + 1; ++s) mbar_init(&bars[s], 1);
+    for (int s = 0; s <= nstage; ++s) mbar_init(&bars[s], 1);
     fence_mbar_init();
-    mbar_arrive_expect_tx(bar_lut, kLutBytes);
-    bulk_g2s(smem, &g_trit_lut, kLutBytes, bar_lut);
     if (a.prefetch && nseg > 0) issue(0);   // the rest after X: X is on the critical path
     s_fail = 0;
   }
   if (tid < M) s_x4[tid] = 0;
   for (int i = tid; i < M * rpc; i += kGemvThreads) part[i] = 0;
+  build_trit_lut(smem, tid, kGemvThreads);   // visible after the barriers below
 
   griddep_wait();                 // X (and W unless prefetched) may come from the previous kernel
   griddep_launch_dependents();
@@ -210,7 +207,6 @@ __global__ void __launch_bounds__(kGemvThreads, kMinBlocks) gemv_pack5_kernel(co
   if (!__syncthreads_and(staged ? mbar_wait(bar_x, 0u) : true)) {
     if (tid == 0) {
       raise_status(kDevTimeout);
-      (void)mbar_wait(bar_lut, 0u);
       for (int sg = issued > nstage ? issued - nstage : 0; sg < issued; ++sg)
         (void)mbar_wait(&bars[sg % nstage], uint32_t(sg / nstage) & 1u);
     }
@@ -338,9 +334,8 @@ __global__ void __launch_bounds__(kGemvThreads, kMinBlocks) gemv_pack5_kernel(co
     }
   const uint32_t lanebase = uint32_t(lane) * 4u;
 
-  // ---- stream the segments (the table first; CTA-uniform, since the ring's
-  // loop below has barriers)
-  bool ok = __syncthreads_and(mbar_wait(bar_lut, 0u));
+  // ---- stream the segments (ok is CTA-uniform: the ring's loop has barriers)
+  bool ok = true;
 #pragma unroll 1
   for (int sg = 0; sg < nseg && ok; ++sg) {
     const int buf = sg % nstage;
@@ -429,7 +424,6 @@ __global__ void __launch_bounds__(kGemvThreads, kMinBlocks) gemv_pack5_kernel(co
     // a copy never landed: let the ones still in flight finish, write nothing
     if (tid == 0) {
       raise_status(kDevTimeout);
-      (void)mbar_wait(bar_lut, 0u);
       for (int sg = issued > nstage ? issued - nstage : 0; sg < issued; ++sg)
         (void)mbar_wait(&bars[sg % nstage], uint32_t(sg / nstage) & 1u);
     }

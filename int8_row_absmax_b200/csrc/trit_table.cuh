@@ -22,27 +22,29 @@ namespace bl {
 
 constexpr uint32_t kLutBytes = 256 * 256;   // a row for every byte value: no read leaves the table
 
-// The table as it sits in shared memory, built at compile time: word b*64 + l
-// (l < 32) holds trits t0..t3 of byte b as four int8 (lane l's copy; words
-// 32..63 of a row repeat them, so the row pitch is 256 bytes and one byte_perm
-// forms an address).  Bytes above 242 read as 121 (four zero trits).  Each CTA
-// copies it into shared memory with one bulk copy.
-struct TritLut {
-  uint32_t w[256 * 64];
-};
-constexpr TritLut make_trit_lut() {
-  TritLut t{};
-  for (uint32_t b = 0; b < 256; ++b) {
-    uint32_t x = b > 242u ? 121u : b, v = 0;
-    for (int k = 0; k < 4; ++k) {
-      v |= ((x % 3u + 255u) & 0xFFu) << (8 * k);
-      x /= 3u;
-    }
-    for (uint32_t l = 0; l < 64; ++l) t.w[b * 64 + l] = v;
+// The table as it sits in shared memory: word b*64 + l (l < 32) holds trits
+// t0..t3 of byte b as four int8 (lane l's copy; words 32..63 of a row repeat
+// them, so the row pitch is 256 bytes and one byte_perm forms an address).
+// Bytes above 242 read as 121 (four zero trits).  Each CTA writes it with 16
+// stores of 16 bytes per 256-byte row (no global traffic).
+__device__ __forceinline__ uint32_t trit_word(uint32_t b) {
+  uint32_t x = b > 242u ? 121u : b, v = 0u;
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const uint32_t q = x / 3u;
+    v |= ((x - 3u * q + 255u) & 0xFFu) << (8 * k);
+    x = q;
   }
-  return t;
+  return v;
 }
-__device__ __align__(128) const TritLut g_trit_lut = make_trit_lut();
+// Threads tid = 0 .. nthreads-1 of the CTA write the table at `lut` (kLutBytes,
+// 16-byte aligned); the caller's next CTA barrier makes it visible.
+__device__ __forceinline__ void build_trit_lut(unsigned char* lut, int tid, int nthreads) {
+  for (int i = tid; i < 256 * 16; i += nthreads) {
+    const uint32_t v = trit_word(uint32_t(i) >> 4);
+    *reinterpret_cast<uint4*>(lut + 16 * i) = make_uint4(v, v, v, v);
+  }
+}
 
 // Trits t0..t3 of byte `bb` (0..3) of packed word w, from the table at `lut`
 // (shared memory); lanebase = 4 * lane.
