@@ -258,7 +258,11 @@ TcSplit tc_split(int64_t M, int64_t N, int64_t K, bl_wfmt f) {
   r.bytes = r.split > 1 ? align_up(size_t(r.split) * size_t(M) * size_t(N) * 4) : 0;
   return r;
 }
-constexpr int64_t kTcMinM = 5;     // AUTO: tensor cores above the GEMV's M <= 4 (measured faster than dp4a from M = 5)
+// AUTO: the swapped tensor-core GEMM from M = 4 for packed weights (measured
+// faster than the dp4a GEMV there at K = 2560 .. 8192), the tensor cores from
+// M = 5 for one trit per byte.
+constexpr int64_t kSwMinM = 4;
+constexpr int64_t kTcMinM = 5;
 
 // Whether the tensor-core path can take the shape: K at least one 128-byte K
 // block, and for one-trit-per-byte weights a TMA-able row stride.
@@ -276,7 +280,7 @@ int resolve_path(int64_t M, int64_t N, int64_t K, bl_wfmt f, int path, int* laun
   const bool tc_ok = tc_feasible(M, N, K, f, ldw, W);
   int p = path;
   if (p == BL_PATH_AUTO)
-    p = (M >= kTcMinM && tc_ok) ? BL_PATH_TC : (gemv_ok ? BL_PATH_GEMV : BL_PATH_SIMT);
+    p = (M >= (f == BL_W_PACK5 ? kSwMinM : kTcMinM) && tc_ok) ? BL_PATH_TC : (gemv_ok ? BL_PATH_GEMV : BL_PATH_SIMT);
   int n = 0;
   if (p == BL_PATH_SIMT) {
     n = fused_quant ? 2 : 1;  // act_quant + contraction

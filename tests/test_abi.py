@@ -131,7 +131,8 @@ def test_tensor_core_plan_and_workspace(lib, M, K, N):
     W rows) are fewer than half of 148 SMs and K has at least two K ranges
     (640-wide chunks; 640-trit chunks of four blocks when swapped), at most 8 splits.  The workspace holds X_q [M,
     ldx] and s, then the int8 copy of W_q, then the split's int32 partials."""
-    if M <= 128:     # few rows, packed weights: the swapped GEMM (128 W rows per tile, K in chunks of 640 trits)
+    swapped = M <= 128
+    if swapped:      # few rows, packed weights: the swapped GEMM (128 W rows per tile, K in chunks of 640 trits)
         tiles = _cdiv(N, 128)
         split = max(1, min(148 // tiles, _cdiv(K, 640), 8))
     else:
@@ -152,19 +153,23 @@ def test_tensor_core_plan_and_workspace(lib, M, K, N):
 
 def test_decode_gemv_needs_no_workspace(lib):
     for M in (1, 2, 3, 4):
-        assert lib.bl_linear_workspace_size(M, 6912, 2560, pkg.PACK5) == 0
         assert lib.bl_linear_ex_workspace_size(M, 6912, 2560, pkg.PACK5, pkg.PATH_GEMV) == 0
-    assert lib.bl_linear_workspace_size(5, 6912, 2560, pkg.PACK5) > 0
+    for M in (1, 2, 3):
+        assert lib.bl_linear_workspace_size(M, 6912, 2560, pkg.PACK5) == 0
+    assert lib.bl_linear_workspace_size(4, 6912, 2560, pkg.PACK5) > 0      # the swapped GEMM from M = 4
     assert lib.bl_linear_workspace_size(1, 6912, 2560, pkg.I8) > 0      # one trit per byte: not the GEMV
 
 
 def test_auto_path_crossover(lib):
-    """AUTO: the decode GEMV for M <= 4 (packed weights), the tensor cores from M = 5."""
+    """AUTO: the decode GEMV for M <= 3 with packed weights and the tensor cores
+    (the swapped GEMM up to M = 128) from M = 4; one trit per byte: from M = 5."""
     n = ctypes.c_int(0)
-    for M in (1, 2, 3, 4):
+    for M in (1, 2, 3):
         assert lib.bl_linear_plan(M, 4096, 4096, pkg.PACK5, pkg.PATH_AUTO, ctypes.byref(n)) == pkg.PATH_GEMV
-    for M in (5, 8, 100, 4096):
+    for M in (4, 5, 8, 100, 4096):
         assert lib.bl_linear_plan(M, 4096, 4096, pkg.PACK5, pkg.PATH_AUTO, ctypes.byref(n)) == pkg.PATH_TC
+    assert lib.bl_linear_plan(4, 4096, 4096, pkg.I8, pkg.PATH_AUTO, ctypes.byref(n)) != pkg.PATH_TC
+    assert lib.bl_linear_plan(5, 4096, 4096, pkg.I8, pkg.PATH_AUTO, ctypes.byref(n)) == pkg.PATH_TC
 
 
 def test_linear_call_struct_layout_matches_the_header(tmp_path):

@@ -90,9 +90,9 @@ def test_gemv_long_rows(bl, M, K, N):
     beside the 64 KB table)."""
     p = random_problem(M * 7 + K + N, M, K, N)
     Wd, beta = quantized(bl, p)
-    assert bl.linear_plan(M, N, K, bl.PACK5)[0] == bl.PATH_GEMV
+    assert bl.linear_plan(M, N, K, bl.PACK5, bl.PATH_GEMV)[0] == bl.PATH_GEMV
     for static in (False, True):
-        Y = bl.linear(dev(p.X), Wd, bl.PACK5, N, K, beta, eps=p.eps, static_weights=static)
+        Y = bl.linear(dev(p.X), Wd, bl.PACK5, N, K, beta, eps=p.eps, path=bl.PATH_GEMV, static_weights=static)
         assert bl.sync_status() == "BL_OK"
         assert_y_exact(host(Y), oracle.bitlinear(p.X, p.W, p.eps)["Y"])
 
@@ -101,7 +101,7 @@ def test_gemv_declines_codes_beyond_shared_memory(bl):
     """M = 4 at K = 40000 needs 160 KB of decode-order codes: the GEMV declines
     and AUTO takes another path (the answer is the same)."""
     assert bl.linear_plan(4, 129, 40000, bl.PACK5, bl.PATH_GEMV)[0] == -1
-    assert bl.linear_plan(4, 129, 40000, bl.PACK5)[0] == bl.PATH_SIMT
+    assert bl.linear_plan(4, 129, 40000, bl.PACK5)[0] == bl.PATH_TC
     p = random_problem(77, 4, 40000, 129)
     Wd, beta = quantized(bl, p)
     Y = bl.linear(dev(p.X), Wd, bl.PACK5, 129, 40000, beta, eps=p.eps)
