@@ -169,10 +169,24 @@ act_quant_reg_kernel(const float* __restrict__ X, int64_t K, float eps, int8_t* 
 
 // The same codes, written in the decode order of trit_table.cuh (positions
 // dorder_pos(k); bytes [K, ldq) of the order's row are 0), for the swapped
-// tensor-core GEMM.  One CTA of 512 threads per row; each thread of the second
-// pass writes one packed word's five code words.  It lets the next kernel on
-// the stream begin its prologue at once (programmatic dependent launch).
+// tensor-core GEMM.  One CTA of 512 threads per row.  With G > 0 the row fits
+// in registers (at most G packed words of 20 activations per thread): each
+// thread issues all its loads at once, takes the max, and after the CTA's
+// reduction turns the same registers into its words' five code words each, so
+// X is read once.  G = 0: two passes over the row (max, then codes).  It lets
+// the next kernel on the stream begin its prologue at once (programmatic
+// dependent launch).
 constexpr int kActDoThreads = 512;
+
+// Codes of one packed word's 20 activations (c[e] = code of x[e]) as the five
+// decode-order words at dst.
+__device__ __forceinline__ void store_dorder_word(uint32_t* dst, const uint32_t* c) {
+#pragma unroll
+  for (int i = 0; i < 4; ++i) dst[i] = c[5 * i] | (c[5 * i + 1] << 8) | (c[5 * i + 2] << 16) | (c[5 * i + 3] << 24);
+  dst[4] = c[4] | (c[9] << 8) | (c[14] << 16) | (c[19] << 24);
+}
+
+template <int G>
 __global__ void __launch_bounds__(kActDoThreads)
 act_quant_dorder_kernel(const float* __restrict__ X, int64_t K, float eps, int8_t* __restrict__ Xq,
                         int64_t ldq, float* __restrict__ s_out) {
@@ -185,19 +199,49 @@ act_quant_dorder_kernel(const float* __restrict__ X, int64_t K, float eps, int8_
   const float* xr = X + m * K;
   uint32_t* qw = reinterpret_cast<uint32_t*>(Xq + m * ldq);
   const bool vec = aligned(xr, 16) && (K & 3) == 0;
-  const int64_t K4 = vec ? (K >> 2) : 0;
+  const int64_t ngrp = (K + 19) / 20;
   float amax = 0.f;
   bool bad = false;
-  for (int64_t i = tid; i < K4; i += kActDoThreads) {
-    const float4 v = reinterpret_cast<const float4*>(xr)[i];
-    const float a = fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w)));
-    bad |= !(a <= 3.402823466e38f) | (v.x != v.x) | (v.y != v.y) | (v.z != v.z) | (v.w != v.w);
-    amax = fmaxf(amax, a);
-  }
-  for (int64_t i = (K4 << 2) + tid; i < K; i += kActDoThreads) {
-    const float a = fabsf(xr[i]);
-    bad |= !(a <= 3.402823466e38f);
-    amax = fmaxf(amax, a);
+  float v[G > 0 ? G : 1][20];
+  if constexpr (G > 0) {
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+      const int64_t k0 = 20 * (int64_t(tid) + int64_t(g) * kActDoThreads);
+      if (vec && k0 + 20 <= K) {
+#pragma unroll
+        for (int q = 0; q < 5; ++q) {
+          const float4 f = reinterpret_cast<const float4*>(xr + k0)[q];
+          v[g][4 * q] = f.x;
+          v[g][4 * q + 1] = f.y;
+          v[g][4 * q + 2] = f.z;
+          v[g][4 * q + 3] = f.w;
+        }
+      } else {
+#pragma unroll
+        for (int e = 0; e < 20; ++e) v[g][e] = k0 + e < K ? xr[k0 + e] : 0.f;
+      }
+    }
+#pragma unroll
+    for (int g = 0; g < G; ++g)
+#pragma unroll
+      for (int e = 0; e < 20; ++e) {
+        const float a = fabsf(v[g][e]);
+        bad |= !(a <= 3.402823466e38f);
+        amax = fmaxf(amax, a);
+      }
+  } else {
+    const int64_t K4 = vec ? (K >> 2) : 0;
+    for (int64_t i = tid; i < K4; i += kActDoThreads) {
+      const float4 f = reinterpret_cast<const float4*>(xr)[i];
+      const float a = fmaxf(fmaxf(fabsf(f.x), fabsf(f.y)), fmaxf(fabsf(f.z), fabsf(f.w)));
+      bad |= !(a <= 3.402823466e38f) | (f.x != f.x) | (f.y != f.y) | (f.z != f.z) | (f.w != f.w);
+      amax = fmaxf(amax, a);
+    }
+    for (int64_t i = (K4 << 2) + tid; i < K; i += kActDoThreads) {
+      const float a = fabsf(xr[i]);
+      bad |= !(a <= 3.402823466e38f);
+      amax = fmaxf(amax, a);
+    }
   }
   amax = warp_max(amax);
   if ((tid & 31) == 0) s_red[tid >> 5] = amax;
@@ -206,42 +250,66 @@ act_quant_dorder_kernel(const float* __restrict__ X, int64_t K, float eps, int8_
     float w = tid < kActDoThreads / 32 ? s_red[tid] : 0.f;
     w = warp_max(w);
     if (tid == 0) {
-      const float s = __fadd_rn(__fdiv_rn(w, float(kActQmax)), eps);
-      s_scale = s;
-      s_out[m] = s;
+      const float sc = __fadd_rn(__fdiv_rn(w, float(kActQmax)), eps);
+      s_scale = sc;
+      s_out[m] = sc;
     }
   }
   __syncthreads();
   const float s = s_scale;
   const float rc = act_recip(s);
-  const int64_t ngrp = (K + 19) / 20;
-  for (int64_t gi = tid; gi < ngrp; gi += kActDoThreads) {
-    const int64_t k0 = 20 * gi;
-    uint32_t c[20];
-    bool tie = rc == 0.f;
-    if (vec && k0 + 20 <= K) {
+  if constexpr (G > 0) {
 #pragma unroll
-      for (int v = 0; v < 5; ++v) {
-        const float4 f = reinterpret_cast<const float4*>(xr + k0)[v];
-        c[4 * v + 0] = act_code_try(f.x, rc, tie);
-        c[4 * v + 1] = act_code_try(f.y, rc, tie);
-        c[4 * v + 2] = act_code_try(f.z, rc, tie);
-        c[4 * v + 3] = act_code_try(f.w, rc, tie);
-      }
-    } else {
+    for (int g = 0; g < G; ++g) {
+      const int64_t gi = int64_t(tid) + int64_t(g) * kActDoThreads;
+      if (gi >= ngrp) break;
+      const int64_t k0 = 20 * gi;
+      uint32_t c[20];
+      bool tie = rc == 0.f;
 #pragma unroll
-      for (int e = 0; e < 20; ++e) c[e] = k0 + e < K ? act_code_try(xr[k0 + e], rc, tie) : 0u;
-    }
-    if (tie)   // rare: a quotient near a half-integer; exact division
+      for (int e = 0; e < 20; ++e) c[e] = act_code_try(v[g][e], rc, tie);
+      if (tie)   // rare: a quotient near a half-integer; exact division
+        for (int e = 0; e < 20; ++e) c[e] = uint32_t(uint8_t(int8_t(act_code_slow(v[g][e], s))));
+#pragma unroll
       for (int e = 0; e < 20; ++e)
-        if (k0 + e < K) c[e] = uint32_t(uint8_t(int8_t(act_code_slow(xr[k0 + e], s))));
-    uint32_t* dst = qw + 5 * gi;
+        if (k0 + e >= K) c[e] = 0u;
+      store_dorder_word(qw + 5 * gi, c);
+    }
+  } else {
+    for (int64_t gi = tid; gi < ngrp; gi += kActDoThreads) {
+      const int64_t k0 = 20 * gi;
+      uint32_t c[20];
+      bool tie = rc == 0.f;
+      if (vec && k0 + 20 <= K) {
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
-      dst[i] = c[5 * i] | (c[5 * i + 1] << 8) | (c[5 * i + 2] << 16) | (c[5 * i + 3] << 24);
-    dst[4] = c[4] | (c[9] << 8) | (c[14] << 16) | (c[19] << 24);
+        for (int q = 0; q < 5; ++q) {
+          const float4 f = reinterpret_cast<const float4*>(xr + k0)[q];
+          c[4 * q + 0] = act_code_try(f.x, rc, tie);
+          c[4 * q + 1] = act_code_try(f.y, rc, tie);
+          c[4 * q + 2] = act_code_try(f.z, rc, tie);
+          c[4 * q + 3] = act_code_try(f.w, rc, tie);
+        }
+      } else {
+#pragma unroll
+        for (int e = 0; e < 20; ++e) c[e] = k0 + e < K ? act_code_try(xr[k0 + e], rc, tie) : 0u;
+      }
+      if (tie)   // rare: a quotient near a half-integer; exact division
+        for (int e = 0; e < 20; ++e)
+          if (k0 + e < K) c[e] = uint32_t(uint8_t(int8_t(act_code_slow(xr[k0 + e], s))));
+      store_dorder_word(qw + 5 * gi, c);
+    }
   }
   for (int64_t i = 5 * ngrp + tid; i < (ldq >> 2); i += kActDoThreads) qw[i] = 0u;
+}
+
+// The decode-order quantizer for M rows of K (the register form when the row fits).
+inline void launch_act_quant_dorder(const float* X, int64_t M, int64_t K, float eps, int8_t* Xq, int64_t ldq,
+                                    float* s, cudaStream_t st) {
+  const int64_t ngrp = (K + 19) / 20;
+  const unsigned g = unsigned(M);
+  if (ngrp <= kActDoThreads) act_quant_dorder_kernel<1><<<g, kActDoThreads, 0, st>>>(X, K, eps, Xq, ldq, s);
+  else if (ngrp <= 2 * kActDoThreads) act_quant_dorder_kernel<2><<<g, kActDoThreads, 0, st>>>(X, K, eps, Xq, ldq, s);
+  else act_quant_dorder_kernel<0><<<g, kActDoThreads, 0, st>>>(X, K, eps, Xq, ldq, s);
 }
 
 // Given codes [M, ldx] in natural order -> the decode order [M, ldd] (ldd % 4

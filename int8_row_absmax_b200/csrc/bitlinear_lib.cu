@@ -934,7 +934,7 @@ static bl_status linear_impl(const float* X, int64_t M, int64_t K, const void* W
   int8_t* Xq = reinterpret_cast<int8_t*>(static_cast<char*>(ws) + l.xq_off);
   float* s = reinterpret_cast<float*>(static_cast<char*>(ws) + l.s_off);
   if (swap)   // codes in the swapped GEMM's decode order
-    act_quant_dorder_kernel<<<unsigned(M), kActDoThreads, 0, stream>>>(X, K, eps, Xq, l.ldx, s);
+    launch_act_quant_dorder(X, M, K, eps, Xq, l.ldx, s, stream);
   else
     launch_act_quant(X, M, K, eps, Xq, l.ldx, s, stream);
   st = launch_status();
