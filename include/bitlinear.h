@@ -380,6 +380,14 @@ bl_status bl_load_deployed_layer(const char* path, int index, uint8_t* Wp, int64
  * if the stream reports an error, else BL_OK. */
 bl_status bl_sync_status(cudaStream_t stream);
 
+/* Self-test of the device timeout path: one thread waits, with the bounded
+ * wait every kernel of this library uses, on an mbarrier phase that nothing
+ * completes, and gives up after `limit_ns` nanoseconds of %globaltimer
+ * (1000 <= limit_ns <= 10^9, else BL_ERR_INVALID_ARG); it records the timeout
+ * in the status word as any kernel does, so the next bl_sync_status returns
+ * BL_ERR_DEVICE_TIMEOUT (and clears it).  Nothing faults or hangs. */
+bl_status bl_selftest_wait_timeout(int64_t limit_ns, cudaStream_t stream);
+
 /* A static, human-readable name for a status code. */
 const char* bl_status_string(bl_status s);
 

@@ -78,6 +78,7 @@ SIGNATURES = {
     "bl_deployed_layer_info": (_I, [ctypes.c_char_p, _I, ctypes.POINTER(_I64), ctypes.POINTER(_I64),
                                     ctypes.POINTER(ctypes.c_int), ctypes.c_char_p, _SZ]),
     "bl_load_deployed_layer": (_I, [ctypes.c_char_p, _I, _P, _I64, _P, _P, _P]),
+    "bl_selftest_wait_timeout": (_I, [_I64, _P]),
     "bl_sync_status": (_I, [_P]),
     "bl_status_string": (ctypes.c_char_p, [_I]),
 }
@@ -426,6 +427,14 @@ def load_deployed(path: str, device=None):
             path.encode(), i, _ptr(Wp), Wp.shape[1], _ptr(beta), _ptr(bias), _stream(torch, Wp)))
         out.append({"name": name.value.decode(), "N": N.value, "K": K.value, "Wp": Wp, "beta": beta, "bias": bias})
     return out
+
+
+def selftest_wait_timeout(limit_ns: int = 2_000_000):
+    """bl_selftest_wait_timeout on the current stream: a bounded wait that runs out
+    and records BL_ERR_DEVICE_TIMEOUT for the next sync_status()."""
+    torch, lib = _torch(), load()
+    _check("bl_selftest_wait_timeout",
+           lib.bl_selftest_wait_timeout(int(limit_ns), ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)))
 
 
 def sync_status(device=None) -> str:

@@ -588,7 +588,7 @@ struct GemvCall {
 
 template <int M, int CH, bool F>
 bl_status launch_gemv_inst(const GemvArgs& a, int grid, uint32_t smem, cudaStream_t st) {
-  constexpr int kMinBlocks = (M * CH == 1) ? 2 : 1;    // two CTAs per SM when their data fit
+  constexpr int kMinBlocks = 1;   // the table and the staged rows hold one CTA per SM: registers are free
   auto kern = gemv_pack5_kernel<M, CH, F, kMinBlocks>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kGemvMaxSmem)) != cudaSuccess)
     return BL_ERR_CUDA;
@@ -1378,6 +1378,20 @@ bl_status bl_load_deployed_layer(const char* path, int index, uint8_t* Wp, int64
   }
   free(buf);
   return st;
+}
+
+// One thread waits on a phase that nothing completes, with a short limit.
+__global__ void selftest_timeout_kernel(uint64_t limit_ns) {
+  __shared__ uint64_t bar;
+  mbar_init(&bar, 1);
+  fence_mbar_init();
+  if (!mbar_wait(&bar, 0u, limit_ns)) raise_status(kDevTimeout);
+}
+
+bl_status bl_selftest_wait_timeout(int64_t limit_ns, cudaStream_t stream) {
+  if (limit_ns < 1000 || limit_ns > int64_t(kWaitLimitNs)) return BL_ERR_INVALID_ARG;
+  selftest_timeout_kernel<<<1, 1, 0, stream>>>(uint64_t(limit_ns));
+  return launch_status();
 }
 
 bl_status bl_sync_status(cudaStream_t stream) {

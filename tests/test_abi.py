@@ -281,3 +281,9 @@ def test_rmsnorm_quant_host_checks(lib):
     assert lib.bl_rmsnorm_quantize_act(16, 2, 8, 16, 1e-5, float("inf"), 16, 16, NULL) == 1
     assert lib.bl_rmsnorm_quantize_act(16, 2, 49153, 16, 1e-5, 1e-5, 16, 16, NULL) == 1
     assert lib.bl_rmsnorm_quantize_act(18, 2, 8, 16, 1e-5, 1e-5, 16, 16, NULL) == 2
+
+
+def test_selftest_timeout_host_checks(lib):
+    """The timeout self-test's limit is checked on the host before any launch."""
+    for limit in (0, 999, 10 ** 9 + 1):
+        assert lib.bl_selftest_wait_timeout(limit, None) == 1     # BL_ERR_INVALID_ARG
