@@ -11,15 +11,16 @@
 // that read different activations (for instance the projections that share
 // one input) stream their weights in one grid.
 //
-// Per CTA (one per SM; two fit when the CTA's weights are small):
-//   * before the dependency wait (programmatic dependent launch): mbarriers,
-//     the decode table written into shared memory by the CTA's threads and --
-//     when the caller declares the weights static -- the bulk copy (TMA
+// Per CTA (one per SM):
+//   * before the dependency wait (programmatic dependent launch): mbarriers
+//     and -- when the caller declares the weights static -- the bulk copy (TMA
 //     engine) of the CTA's first segment of packed rows, so the weight
 //     stream starts while the previous kernel finishes; the other segments
 //     follow the copy of X, which is on the critical path;
 //   * griddepcontrol.wait, then launch_dependents (the next kernel may start
-//     its own prologue and weight copies while this one computes);
+//     its own prologue and weight copies while this one computes); thread 0
+//     issues the copy of X and the other segments, and while X is in flight the
+//     CTA writes the decode table into shared memory;
 //   * X: per-row absmax over the whole row (every CTA reads it, from L2), then
 //     exactly the codes of bl_quantize_act, stored in shared memory in decode
 //     order: for packed word g (bytes 4g..4g+3, trits 20g..20g+19) five words,
@@ -67,6 +68,7 @@ struct GemvProb {
   int cta0;            // first CTA of this problem
   int rows_per_cta;
   int S, G;            // warps per row slice, rows in flight
+  int slice;           // 16-byte chunks per row slice: ceil(ldp / 16 / S)
   int seg_rows, nstage;
   uint32_t xc_off, xs_off, xs_bytes, part_off, bar_off, stage_off, smem;
 };
@@ -103,6 +105,7 @@ inline bool gemv_plan_prob(int64_t M, int64_t N, int64_t K, int64_t ldp, int cta
   if (S > kGemvWarps) return false;
   P.S = int(S);
   P.G = kGemvWarps / P.S;
+  P.slice = int(ceil_div(nch, S));
   P.rows_per_cta = int(ceil_div(N, int64_t(ctas)));
   // rows per warp group and segment: at least one pass of gemv_rows_per_pass rows
   const int64_t rpp = gemv_rows_per_pass(int(M), ch);
@@ -189,8 +192,6 @@ __global__ void __launch_bounds__(kGemvThreads, kMinBlocks) gemv_pack5_kernel(co
     s_fail = 0;
   }
   if (tid < M) s_x4[tid] = 0;
-  for (int i = tid; i < M * rpc; i += kGemvThreads) part[i] = 0;
-  build_trit_lut(smem, tid, kGemvThreads);   // visible after the barriers below
 
   griddep_wait();                 // X (and W unless prefetched) may come from the previous kernel
   griddep_launch_dependents();
@@ -203,6 +204,9 @@ __global__ void __launch_bounds__(kGemvThreads, kMinBlocks) gemv_pack5_kernel(co
     }
     for (int sg = a.prefetch ? 1 : 0; sg < nseg && sg < nstage; ++sg) issue(sg);
   }
+  // while X is in flight: the decode table and the zeroed row sums
+  for (int i = tid; i < M * rpc; i += kGemvThreads) part[i] = 0;
+  build_trit_lut(smem, tid, kGemvThreads);
   __syncthreads();                // the mbarriers are initialized before any thread polls one
   if (!__syncthreads_and(staged ? mbar_wait(bar_x, 0u) : true)) {
     if (tid == 0) {
@@ -311,18 +315,17 @@ __global__ void __launch_bounds__(kGemvThreads, kMinBlocks) gemv_pack5_kernel(co
 
   // ---- this lane's x registers: chunks c0 + lane + 32 i of its K slice
   const int S = P.S, G = P.G;
-  const int sl = warp % S, grp = warp / S;
-  const int64_t nch = ldp / 16;
-  const int64_t slice = (nch + S - 1) / S;
-  const int64_t c0 = int64_t(sl) * slice;
-  const int64_t c1 = min(nch, c0 + slice);
+  const int grp = warp / S, sl = warp - grp * S;
+  const int nch = int(ldp >> 4);
+  const int c0 = sl * P.slice;
+  const int c1 = min(nch, c0 + P.slice);
   uint32_t xr[M][CH][20];
 #pragma unroll
   for (int m = 0; m < M; ++m)
 #pragma unroll
     for (int i = 0; i < CH; ++i) {
-      const int64_t c = c0 + lane + 32 * i;
-      const uint4* src = reinterpret_cast<const uint4*>(xc + int64_t(m) * kpad + 80 * c);
+      const int c = c0 + lane + 32 * i;
+      const uint4* src = reinterpret_cast<const uint4*>(xc + m * kpad + 80 * c);
 #pragma unroll
       for (int v = 0; v < 5; ++v) {
         const uint4 u = (c < c1) ? src[v] : make_uint4(0u, 0u, 0u, 0u);
@@ -364,7 +367,7 @@ __global__ void __launch_bounds__(kGemvThreads, kMinBlocks) gemv_pack5_kernel(co
           for (int m = 0; m < M; ++m) am[rr][m][0] = am[rr][m][1] = a4[rr][m] = 0;
 #pragma unroll
         for (int i = 0; i < CH; ++i) {
-          const int64_t c = c0 + lane + 32 * i;
+          const int c = c0 + lane + 32 * i;
           if (c < c1) {
             uint32_t wv[kRows][4];
 #pragma unroll
