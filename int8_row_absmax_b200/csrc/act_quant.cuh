@@ -60,6 +60,16 @@ __device__ __forceinline__ uint32_t act_code_try(float x, float r, bool& tie) {
   tie |= fabsf(fabsf(d) - 0.5f) < 3.0517578125e-05f;
   return __float_as_uint(t) & 0xFFu;
 }
+// Whether act_code_try's code for x may differ from act_code: the product
+// within 2^-15 of a half-integer, or no usable reciprocal (r == 0).  A group
+// whose `tie` came back set redoes only these elements with the exact division.
+__device__ __forceinline__ bool act_near_tie(float x, float r) {
+  if (r == 0.f) return true;
+  const float y = fminf(fmaxf(__fmul_rn(x, r), -float(kActQmax)), float(kActQmax));
+  const float t = __fadd_rn(y, 12582912.0f);
+  const float d = __fsub_rn(y, __fsub_rn(t, 12582912.0f));
+  return fabsf(fabsf(d) - 0.5f) < 3.0517578125e-05f;
+}
 // Four codes packed little-endian into one word.
 __device__ __forceinline__ uint32_t act_codes4(float4 v, float s, float r) {
   return __byte_perm(__byte_perm(act_code_bits(v.x, s, r), act_code_bits(v.y, s, r), 0x0040),
@@ -268,8 +278,9 @@ act_quant_dorder_kernel(const float* __restrict__ X, int64_t K, float eps, int8_
       bool tie = rc == 0.f;
 #pragma unroll
       for (int e = 0; e < 20; ++e) c[e] = act_code_try(v[g][e], rc, tie);
-      if (tie)   // rare: a quotient near a half-integer; exact division
-        for (int e = 0; e < 20; ++e) c[e] = uint32_t(uint8_t(int8_t(act_code_slow(v[g][e], s))));
+      if (tie)   // rare: a quotient near a half-integer; exact division for those elements
+        for (int e = 0; e < 20; ++e)
+          if (act_near_tie(v[g][e], rc)) c[e] = uint32_t(uint8_t(int8_t(act_code_slow(v[g][e], s))));
 #pragma unroll
       for (int e = 0; e < 20; ++e)
         if (k0 + e >= K) c[e] = 0u;
@@ -293,9 +304,10 @@ act_quant_dorder_kernel(const float* __restrict__ X, int64_t K, float eps, int8_
 #pragma unroll
         for (int e = 0; e < 20; ++e) c[e] = k0 + e < K ? act_code_try(xr[k0 + e], rc, tie) : 0u;
       }
-      if (tie)   // rare: a quotient near a half-integer; exact division
+      if (tie)   // rare: a quotient near a half-integer; exact division for those elements
         for (int e = 0; e < 20; ++e)
-          if (k0 + e < K) c[e] = uint32_t(uint8_t(int8_t(act_code_slow(xr[k0 + e], s))));
+          if (k0 + e < K && act_near_tie(xr[k0 + e], rc))
+            c[e] = uint32_t(uint8_t(int8_t(act_code_slow(xr[k0 + e], s))));
       store_dorder_word(qw + 5 * gi, c);
     }
   }

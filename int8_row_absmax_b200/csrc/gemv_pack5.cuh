@@ -293,9 +293,10 @@ __global__ void __launch_bounds__(kGemvThreads, kMinBlocks) gemv_pack5_kernel(co
 #pragma unroll
           for (int e = 0; e < 20; ++e) c[e] = k0 + e < K ? act_code_try(xr[k0 + e], rc, tie) : 0u;
         }
-        if (tie)   // rare: a quotient near a half-integer; exact division
+        if (tie)   // rare: a quotient near a half-integer; exact division for those elements
           for (int e = 0; e < 20; ++e)
-            if (k0 + e < K) c[e] = uint32_t(uint8_t(int8_t(act_code_slow(xr[k0 + e], sc))));
+            if (k0 + e < K && act_near_tie(xr[k0 + e], rc))
+              c[e] = uint32_t(uint8_t(int8_t(act_code_slow(xr[k0 + e], sc))));
       } else {
 #pragma unroll
         for (int e = 0; e < 20; ++e) c[e] = k0 + e < K ? uint32_t(uint8_t(xq[k0 + e])) : 0u;

@@ -441,11 +441,11 @@ wquant_kernel(const __grid_constant__ WqArgs a) {
           q.y = act_codef_try(v.y, rc, tie);
           q.z = act_codef_try(v.z, rc, tie);
           q.w = act_codef_try(v.w, rc, tie);
-          if (tie) {   // rare: a quotient near a half-integer; exact division
-            q.x = float(act_code_slow(v.x, sc));
-            q.y = float(act_code_slow(v.y, sc));
-            q.z = float(act_code_slow(v.z, sc));
-            q.w = float(act_code_slow(v.w, sc));
+          if (tie) {   // rare: a quotient near a half-integer; exact division for those elements
+            if (act_near_tie(v.x, rc)) q.x = float(act_code_slow(v.x, sc));
+            if (act_near_tie(v.y, rc)) q.y = float(act_code_slow(v.y, sc));
+            if (act_near_tie(v.z, rc)) q.z = float(act_code_slow(v.z, sc));
+            if (act_near_tie(v.w, rc)) q.w = float(act_code_slow(v.w, sc));
           }
           xo[i] = q;
         }
