@@ -70,6 +70,44 @@ __device__ __forceinline__ bool act_near_tie(float x, float r) {
   const float d = __fsub_rn(y, __fsub_rn(t, 12582912.0f));
   return fabsf(fabsf(d) - 0.5f) < 3.0517578125e-05f;
 }
+// Codes of 20 activations x[0..19] (elements from `valid` on are not part of
+// the row: code 0).  The fast path of act_code_try, and on the hot path one
+// exact division per call, for the group's one near-tie element if it has
+// one (element 0 otherwise); only a group with two
+// or more near-tie elements, or no usable reciprocal, takes the out-of-line
+// exact division per element.  (A rarely executed branch costs its
+// instruction fetches each launch, which a per-CTA quantization of the same
+// row would pay in every CTA.)
+__device__ __forceinline__ void act_codes20(const float* x, int valid, float s, float rc, uint32_t* c) {
+  int te = 0, nt = 0;
+#pragma unroll
+  for (int e = 0; e < 20; ++e) {
+    bool nr = false;
+    c[e] = act_code_try(x[e], rc, nr);
+    if (nr && e < valid) {
+      te = e;
+      ++nt;
+    }
+  }
+  float xt = x[0];
+#pragma unroll
+  for (int e = 1; e < 20; ++e)
+    if (e == te) xt = x[e];
+  const uint32_t ce = uint32_t(uint8_t(int8_t(act_code(xt, s))));
+  if (rc == 0.f || nt > 1) {
+#pragma unroll
+    for (int e = 0; e < 20; ++e)
+      if (e < valid && (rc == 0.f || act_near_tie(x[e], rc))) c[e] = uint32_t(uint8_t(int8_t(act_code_slow(x[e], s))));
+  } else if (nt == 1) {
+#pragma unroll
+    for (int e = 0; e < 20; ++e)
+      if (e == te) c[e] = ce;
+  }
+#pragma unroll
+  for (int e = 0; e < 20; ++e)
+    if (e >= valid) c[e] = 0u;
+}
+
 // Four codes packed little-endian into one word.
 __device__ __forceinline__ uint32_t act_codes4(float4 v, float s, float r) {
   return __byte_perm(__byte_perm(act_code_bits(v.x, s, r), act_code_bits(v.y, s, r), 0x0040),
@@ -275,39 +313,28 @@ act_quant_dorder_kernel(const float* __restrict__ X, int64_t K, float eps, int8_
       if (gi >= ngrp) break;
       const int64_t k0 = 20 * gi;
       uint32_t c[20];
-      bool tie = rc == 0.f;
-#pragma unroll
-      for (int e = 0; e < 20; ++e) c[e] = act_code_try(v[g][e], rc, tie);
-      if (tie)   // rare: a quotient near a half-integer; exact division for those elements
-        for (int e = 0; e < 20; ++e)
-          if (act_near_tie(v[g][e], rc)) c[e] = uint32_t(uint8_t(int8_t(act_code_slow(v[g][e], s))));
-#pragma unroll
-      for (int e = 0; e < 20; ++e)
-        if (k0 + e >= K) c[e] = 0u;
+      act_codes20(v[g], int(min(int64_t(20), K - k0)), s, rc, c);
       store_dorder_word(qw + 5 * gi, c);
     }
   } else {
     for (int64_t gi = tid; gi < ngrp; gi += kActDoThreads) {
       const int64_t k0 = 20 * gi;
-      uint32_t c[20];
-      bool tie = rc == 0.f;
+      float xv[20];
       if (vec && k0 + 20 <= K) {
 #pragma unroll
         for (int q = 0; q < 5; ++q) {
           const float4 f = reinterpret_cast<const float4*>(xr + k0)[q];
-          c[4 * q + 0] = act_code_try(f.x, rc, tie);
-          c[4 * q + 1] = act_code_try(f.y, rc, tie);
-          c[4 * q + 2] = act_code_try(f.z, rc, tie);
-          c[4 * q + 3] = act_code_try(f.w, rc, tie);
+          xv[4 * q] = f.x;
+          xv[4 * q + 1] = f.y;
+          xv[4 * q + 2] = f.z;
+          xv[4 * q + 3] = f.w;
         }
       } else {
 #pragma unroll
-        for (int e = 0; e < 20; ++e) c[e] = k0 + e < K ? act_code_try(xr[k0 + e], rc, tie) : 0u;
+        for (int e = 0; e < 20; ++e) xv[e] = k0 + e < K ? xr[k0 + e] : 0.f;
       }
-      if (tie)   // rare: a quotient near a half-integer; exact division for those elements
-        for (int e = 0; e < 20; ++e)
-          if (k0 + e < K && act_near_tie(xr[k0 + e], rc))
-            c[e] = uint32_t(uint8_t(int8_t(act_code_slow(xr[k0 + e], s))));
+      uint32_t c[20];
+      act_codes20(xv, int(min(int64_t(20), K - k0)), s, rc, c);
       store_dorder_word(qw + 5 * gi, c);
     }
   }

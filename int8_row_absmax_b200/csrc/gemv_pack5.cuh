@@ -279,24 +279,21 @@ __global__ void __launch_bounds__(kGemvThreads, kMinBlocks) gemv_pack5_kernel(co
       const int k0 = 20 * gi;
       uint32_t c[20];
       if (kFused) {
-        bool tie = rc == 0.f;
+        float xv[20];
         if (k0 + 20 <= K && aligned(xr + k0, 16)) {
 #pragma unroll
           for (int v = 0; v < 5; ++v) {
             const float4 f = ld4(xr + k0 + 4 * v);
-            c[4 * v + 0] = act_code_try(f.x, rc, tie);
-            c[4 * v + 1] = act_code_try(f.y, rc, tie);
-            c[4 * v + 2] = act_code_try(f.z, rc, tie);
-            c[4 * v + 3] = act_code_try(f.w, rc, tie);
+            xv[4 * v] = f.x;
+            xv[4 * v + 1] = f.y;
+            xv[4 * v + 2] = f.z;
+            xv[4 * v + 3] = f.w;
           }
         } else {
 #pragma unroll
-          for (int e = 0; e < 20; ++e) c[e] = k0 + e < K ? act_code_try(xr[k0 + e], rc, tie) : 0u;
+          for (int e = 0; e < 20; ++e) xv[e] = k0 + e < K ? xr[k0 + e] : 0.f;
         }
-        if (tie)   // rare: a quotient near a half-integer; exact division for those elements
-          for (int e = 0; e < 20; ++e)
-            if (k0 + e < K && act_near_tie(xr[k0 + e], rc))
-              c[e] = uint32_t(uint8_t(int8_t(act_code_slow(xr[k0 + e], sc))));
+        act_codes20(xv, int(min(int64_t(20), K - int64_t(k0))), sc, rc, c);
       } else {
 #pragma unroll
         for (int e = 0; e < 20; ++e) c[e] = k0 + e < K ? uint32_t(uint8_t(xq[k0 + e])) : 0u;

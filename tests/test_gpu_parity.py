@@ -402,6 +402,34 @@ def test_quantize_act_ties_and_zero_rows(bl):
     check_ok(bl)
 
 
+@pytest.mark.parametrize("M", [1, 3, 4, 9])
+def test_near_tie_groups_in_fused_quantization(bl, M):
+    """Quotients within the fast path's 2^-15 window of a half-integer, placed in
+    the 20-activation groups that the GEMV (M <= 3) and the swapped GEMM's
+    quantizer (M >= 4) code together: one such element in a group (the single
+    exact division on the hot path), two in a group, and one in the ragged last
+    group.  Codes, scales and Y must equal the oracle's."""
+    rng = np.random.default_rng(21)
+    K, N = 413, 96
+    X = rng.standard_normal((M, K)).astype(F32)
+    X[:, 0] = 100.0                                    # fixes max|x| per row
+    eps = F32(1e-5)
+    s = (F32(100.0) / F32(127)).astype(F32) + eps      # the scale every row gets
+    for m in range(M):
+        for k, h in ((3, 2.5), (25, -7.5), (31, 11.5), (410, 0.5)):   # group 0: one; group 1: two; last group
+            X[m, k] = F32(h) * s
+    p = random_problem(5, M, K, N)
+    Wd, beta = bl.quantize_weights_pack5(dev(p.W), p.eps)
+    ref = oracle.bitlinear(X, p.W, eps)["Y"]
+    rq, _ = oracle.act_quant(X, eps)
+    assert any(abs(float(X[0, k]) / float(s) - h) < 2.0 ** -15 for k, h in ((3, 2.5),))
+    Y = bl.linear(dev(X), Wd, bl.PACK5, N, K, beta, eps=float(eps))
+    check_ok(bl)
+    assert_y_close(host(Y), ref)
+    Xq, _ = bl.quantize_act(dev(X), float(eps))
+    np.testing.assert_array_equal(host(Xq), rq)
+
+
 def test_nonfinite_activation_is_reported(bl):
     X = np.ones((3, 10), F32)
     X[1, 4] = np.nan
