@@ -85,12 +85,15 @@ typedef enum {
  *
  * BL_FLAG_STATIC_WEIGHTS: the caller guarantees that W is not written by any
  * kernel that may still be running when the call is issued (for instance
- * weights quantized once and only read while decoding).  The decode GEMV is
- * launched with programmatic dependent launch in every case, so its prologue
- * overlaps the previous kernel on the stream; with this flag it also starts
- * copying W into shared memory before that kernel has finished, and waits for
- * it only before reading X and writing Y.  Results are identical with and
- * without the flag; a call that breaks the guarantee may read stale weights. */
+ * weights quantized once and only read while decoding).  The GEMV and the
+ * swapped tensor-core GEMM are launched with programmatic dependent launch in
+ * every case, so their prologue overlaps the previous kernel on the stream;
+ * with this flag the swapped GEMM also starts copying W before that kernel has
+ * finished (its weights have a producer of their own), and waits for it only
+ * before reading X and writing Y.  The decode GEMV copies X first either way
+ * (a weight copy issued ahead of X was measured to delay it).  Results are
+ * identical with and without the flag; a call that breaks the guarantee may
+ * read stale weights. */
 #define BL_FLAG_STATIC_WEIGHTS 0x100
 
 /* Packed row stride in bytes: ceil(K/5) rounded up to a multiple of 16. */

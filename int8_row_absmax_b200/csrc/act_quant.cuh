@@ -70,18 +70,18 @@ __device__ __forceinline__ bool act_near_tie(float x, float r) {
   const float d = __fsub_rn(y, __fsub_rn(t, 12582912.0f));
   return fabsf(fabsf(d) - 0.5f) < 3.0517578125e-05f;
 }
-// Codes of 20 activations x[0..19] (elements from `valid` on are not part of
-// the row: code 0).  The fast path of act_code_try, and on the hot path one
-// exact division per call, for the group's one near-tie element if it has
-// one (element 0 otherwise); only a group with two
-// or more near-tie elements, or no usable reciprocal, takes the out-of-line
-// exact division per element.  (A rarely executed branch costs its
-// instruction fetches each launch, which a per-CTA quantization of the same
-// row would pay in every CTA.)
-__device__ __forceinline__ void act_codes20(const float* x, int valid, float s, float rc, uint32_t* c) {
+// Codes of N activations x[0..N-1] (elements from `valid` on are not part of
+// the row: code 0).  The fast path of act_code_try, plus on the hot path one
+// exact division per call, for the unit's one near-tie element if it has one
+// (element 0 otherwise); only a unit with two or more near-tie elements, or no
+// usable reciprocal, takes the out-of-line exact division per element.  (A
+// rarely executed branch costs its instruction fetches in every launch that
+// takes it, and a per-CTA quantization of the same row takes it in every CTA.)
+template <int N>
+__device__ __forceinline__ void act_codes_n(const float* x, int valid, float s, float rc, uint32_t* c) {
   int te = 0, nt = 0;
 #pragma unroll
-  for (int e = 0; e < 20; ++e) {
+  for (int e = 0; e < N; ++e) {
     bool nr = false;
     c[e] = act_code_try(x[e], rc, nr);
     if (nr && e < valid) {
@@ -91,20 +91,20 @@ __device__ __forceinline__ void act_codes20(const float* x, int valid, float s, 
   }
   float xt = x[0];
 #pragma unroll
-  for (int e = 1; e < 20; ++e)
+  for (int e = 1; e < N; ++e)
     if (e == te) xt = x[e];
   const uint32_t ce = uint32_t(uint8_t(int8_t(act_code(xt, s))));
   if (rc == 0.f || nt > 1) {
 #pragma unroll
-    for (int e = 0; e < 20; ++e)
+    for (int e = 0; e < N; ++e)
       if (e < valid && (rc == 0.f || act_near_tie(x[e], rc))) c[e] = uint32_t(uint8_t(int8_t(act_code_slow(x[e], s))));
   } else if (nt == 1) {
 #pragma unroll
-    for (int e = 0; e < 20; ++e)
+    for (int e = 0; e < N; ++e)
       if (e == te) c[e] = ce;
   }
 #pragma unroll
-  for (int e = 0; e < 20; ++e)
+  for (int e = 0; e < N; ++e)
     if (e >= valid) c[e] = 0u;
 }
 
@@ -313,7 +313,7 @@ act_quant_dorder_kernel(const float* __restrict__ X, int64_t K, float eps, int8_
       if (gi >= ngrp) break;
       const int64_t k0 = 20 * gi;
       uint32_t c[20];
-      act_codes20(v[g], int(min(int64_t(20), K - k0)), s, rc, c);
+      act_codes_n<20>(v[g], int(min(int64_t(20), K - k0)), s, rc, c);
       store_dorder_word(qw + 5 * gi, c);
     }
   } else {
@@ -334,7 +334,7 @@ act_quant_dorder_kernel(const float* __restrict__ X, int64_t K, float eps, int8_
         for (int e = 0; e < 20; ++e) xv[e] = k0 + e < K ? xr[k0 + e] : 0.f;
       }
       uint32_t c[20];
-      act_codes20(xv, int(min(int64_t(20), K - k0)), s, rc, c);
+      act_codes_n<20>(xv, int(min(int64_t(20), K - k0)), s, rc, c);
       store_dorder_word(qw + 5 * gi, c);
     }
   }

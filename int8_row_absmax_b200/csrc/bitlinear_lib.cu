@@ -639,7 +639,7 @@ bl_status run_gemv_group(int64_t M, const GemvCall* c, int n, bool prefetch, cud
   }
   GemvArgs a = {};
   a.nprob = n;
-  a.prefetch = prefetch ? 1 : 0;
+  (void)prefetch;   // the GEMV copies X before its weights either way
   int cta = 0;
   uint32_t smem = 0;
   for (int i = 0; i < n; ++i) {

@@ -12,15 +12,14 @@
 // one input) stream their weights in one grid.
 //
 // Per CTA (one per SM):
-//   * before the dependency wait (programmatic dependent launch): mbarriers
-//     and -- when the caller declares the weights static -- the bulk copy (TMA
-//     engine) of the CTA's first segment of packed rows, so the weight
-//     stream starts while the previous kernel finishes; the other segments
-//     follow the copy of X, which is on the critical path;
+//   * before the dependency wait (programmatic dependent launch): mbarriers;
 //   * griddepcontrol.wait, then launch_dependents (the next kernel may start
-//     its own prologue and weight copies while this one computes); thread 0
-//     issues the copy of X and the other segments, and while X is in flight the
-//     CTA writes the decode table into shared memory;
+//     its own prologue while this one computes); thread 0 issues the copy of X
+//     first (X is on the critical path, and every copy issued ahead of it --
+//     weights included, even with static weights -- was measured to delay it),
+//     then the segments of packed rows (bulk copies into shared memory) and,
+//     last, a bulk copy of the decode table (a compile-time constant in global
+//     memory), which is needed only once the activation codes are ready;
 //   * X: per-row absmax over the whole row (every CTA reads it, from L2), then
 //     exactly the codes of bl_quantize_act, stored in shared memory in decode
 //     order: for packed word g (bytes 4g..4g+3, trits 20g..20g+19) five words,
@@ -76,7 +75,6 @@ struct GemvProb {
 struct GemvArgs {
   GemvProb p[kGemvMaxProbs];
   int nprob;
-  int prefetch;        // 1: stream W before the dependency wait
 };
 
 inline uint32_t align_to(uint32_t v, uint32_t a) { return (v + a - 1) / a * a; }
@@ -123,7 +121,7 @@ inline bool gemv_plan_prob(int64_t M, int64_t N, int64_t K, int64_t ldp, int cta
   const uint32_t stage_bytes = uint32_t(P.seg_rows * ldp);
   int64_t ns = nseg < kGemvMaxStages ? nseg : kGemvMaxStages;
   for (; ns >= 1; --ns) {
-    P.stage_off = align_to(P.bar_off + uint32_t(8 * (ns + 1)), 128);
+    P.stage_off = align_to(P.bar_off + uint32_t(8 * (ns + 2)), 128);
     if (int64_t(P.stage_off) + ns * stage_bytes <= kGemvMaxSmem) break;
   }
   if (ns < 1) return false;
@@ -185,15 +183,15 @@ __global__ void __launch_bounds__(kGemvThreads, kMinBlocks) gemv_pack5_kernel(co
 
   // ---- prologue: nothing here reads what an earlier kernel may still write
   uint64_t* bar_x = &bars[nstage];
+  uint64_t* bar_lut = &bars[nstage + 1];
   if (tid == 0) {
-    for (int s = 0; s <= nstage; ++s) mbar_init(&bars[s], 1);
+    for (int s = 0; s <= nstage + 1; ++s) mbar_init(&bars[s], 1);
     fence_mbar_init();
-    if (a.prefetch && nseg > 0) issue(0);   // the rest after X: X is on the critical path
     s_fail = 0;
   }
   if (tid < M) s_x4[tid] = 0;
 
-  griddep_wait();                 // X (and W unless prefetched) may come from the previous kernel
+  griddep_wait();                 // X and W may come from the previous kernel
   griddep_launch_dependents();
   // float32 X into shared memory by one bulk copy (one latency for the whole row)
   const bool staged = kFused && P.xs_bytes != 0u;
@@ -202,15 +200,17 @@ __global__ void __launch_bounds__(kGemvThreads, kMinBlocks) gemv_pack5_kernel(co
       mbar_arrive_expect_tx(bar_x, P.xs_bytes);
       bulk_g2s(smem + P.xs_off, P.X, P.xs_bytes, bar_x);
     }
-    for (int sg = a.prefetch ? 1 : 0; sg < nseg && sg < nstage; ++sg) issue(sg);
+    for (int sg = 0; sg < nseg && sg < nstage; ++sg) issue(sg);
+    // the decode table last: it is needed only once the codes are ready
+    mbar_arrive_expect_tx(bar_lut, kLutBytes);
+    bulk_g2s(smem, &g_trit_lut, kLutBytes, bar_lut);
   }
-  // while X is in flight: the decode table and the zeroed row sums
   for (int i = tid; i < M * rpc; i += kGemvThreads) part[i] = 0;
-  build_trit_lut(smem, tid, kGemvThreads);
   __syncthreads();                // the mbarriers are initialized before any thread polls one
   if (!__syncthreads_and(staged ? mbar_wait(bar_x, 0u) : true)) {
     if (tid == 0) {
       raise_status(kDevTimeout);
+      (void)mbar_wait(bar_lut, 0u);
       for (int sg = issued > nstage ? issued - nstage : 0; sg < issued; ++sg)
         (void)mbar_wait(&bars[sg % nstage], uint32_t(sg / nstage) & 1u);
     }
@@ -293,7 +293,7 @@ __global__ void __launch_bounds__(kGemvThreads, kMinBlocks) gemv_pack5_kernel(co
 #pragma unroll
           for (int e = 0; e < 20; ++e) xv[e] = k0 + e < K ? xr[k0 + e] : 0.f;
         }
-        act_codes20(xv, int(min(int64_t(20), K - int64_t(k0))), sc, rc, c);
+        act_codes_n<20>(xv, int(min(int64_t(20), K - int64_t(k0))), sc, rc, c);
       } else {
 #pragma unroll
         for (int e = 0; e < 20; ++e) c[e] = k0 + e < K ? uint32_t(uint8_t(xq[k0 + e])) : 0u;
@@ -335,8 +335,9 @@ __global__ void __launch_bounds__(kGemvThreads, kMinBlocks) gemv_pack5_kernel(co
     }
   const uint32_t lanebase = uint32_t(lane) * 4u;
 
-  // ---- stream the segments (ok is CTA-uniform: the ring's loop has barriers)
-  bool ok = true;
+  // ---- stream the segments (the table first; ok is CTA-uniform: the ring's
+  // loop has barriers)
+  bool ok = __syncthreads_and(mbar_wait(bar_lut, 0u));
 #pragma unroll 1
   for (int sg = 0; sg < nseg && ok; ++sg) {
     const int buf = sg % nstage;
@@ -425,6 +426,7 @@ __global__ void __launch_bounds__(kGemvThreads, kMinBlocks) gemv_pack5_kernel(co
     // a copy never landed: let the ones still in flight finish, write nothing
     if (tid == 0) {
       raise_status(kDevTimeout);
+      (void)mbar_wait(bar_lut, 0u);
       for (int sg = issued > nstage ? issued - nstage : 0; sg < issued; ++sg)
         (void)mbar_wait(&bars[sg % nstage], uint32_t(sg / nstage) & 1u);
     }

@@ -37,6 +37,25 @@ __device__ __forceinline__ uint32_t trit_word(uint32_t b) {
   }
   return v;
 }
+// The same table as a compile-time constant in global memory, for CTAs that
+// copy it (one bulk copy) instead of writing it.
+struct TritLut {
+  uint32_t w[256 * 64];
+};
+constexpr TritLut make_trit_lut() {
+  TritLut t{};
+  for (uint32_t b = 0; b < 256; ++b) {
+    uint32_t x = b > 242u ? 121u : b, v = 0;
+    for (int k = 0; k < 4; ++k) {
+      v |= ((x % 3u + 255u) & 0xFFu) << (8 * k);
+      x /= 3u;
+    }
+    for (uint32_t l = 0; l < 64; ++l) t.w[b * 64 + l] = v;
+  }
+  return t;
+}
+__device__ __align__(128) const TritLut g_trit_lut = make_trit_lut();
+
 // Threads tid = 0 .. nthreads-1 of the CTA write the table at `lut` (kLutBytes,
 // 16-byte aligned); the caller's next CTA barrier makes it visible.
 __device__ __forceinline__ void build_trit_lut(unsigned char* lut, int tid, int nthreads) {
