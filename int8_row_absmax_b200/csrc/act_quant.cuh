@@ -70,11 +70,38 @@ __device__ __forceinline__ bool act_near_tie(float x, float r) {
   const float d = __fsub_rn(y, __fsub_rn(t, 12582912.0f));
   return fabsf(fabsf(d) - 0.5f) < 3.0517578125e-05f;
 }
+// The exact code of x for a product x * r within 2^-15 of a half-integer
+// (r = act_recip(s) != 0), with no division.  Let a = |x|, n = floor(RN(a r))
+// and h = n + 1/2; the exact quotient a / s lies within 2^-15 + 1.5 ulp of h,
+// so RN(a / s) is h, a float below h (code n) or a float above h (code n + 1).
+// For h <= 127.5 the last significand bit of h is 0, so the two midpoints
+// h -+ ulp(h)/2 round to h: RN(a / s) = h exactly when s (h - u/2) <= a <=
+// s (h + u/2), u = ulp(h).  Those bounds are products of a 24-bit and a 25-bit
+// significand, exact in float64, so two comparisons decide; RN(a / s) = h then
+// rounds half to even.  (For h = 1/2 the float below h is only ulp(h)/2 away,
+// but every quotient at or below h then has code 0 either way.)  The code of
+// -x is minus that of x.
+__device__ __forceinline__ uint32_t act_code_tie_exact(float x, float s, float r) {
+  const float a = fabsf(x);
+  const float yq = fminf(__fmul_rn(a, r), float(kActQmax));
+  const float n = floorf(yq);
+  const float h = __fadd_rn(n, 0.5f);
+  const int eh = (int((__float_as_uint(h) >> 23) & 0xFFu)) - 127;   // h >= 0.5: normal
+  const double hu = __longlong_as_double(int64_t(1023 + eh - 24) << 52);   // ulp(h) / 2 = 2^(eh-24)
+  const double ds = double(s), da = double(a);
+  const double lo = ds * (double(h) - hu), hi = ds * (double(h) + hu);
+  const int ni = int(n);
+  int q = da < lo ? ni : (da > hi ? ni + 1 : ni + (ni & 1));
+  q = q > kActQmax ? kActQmax : q;
+  return uint32_t(uint8_t(int8_t(x < 0.f ? -q : q)));
+}
+
 // Codes of N activations x[0..N-1] (elements from `valid` on are not part of
-// the row: code 0).  The fast path of act_code_try, plus on the hot path one
-// exact division per call, for the unit's one near-tie element if it has one
-// (element 0 otherwise); only a unit with two or more near-tie elements, or no
-// usable reciprocal, takes the out-of-line exact division per element.  (A
+// the row: code 0).  The fast path of act_code_try, plus on the hot path the
+// division-free exact code of act_code_tie_exact for the unit's one near-tie
+// element if it has one (element 0 otherwise); only a unit with two or more
+// near-tie elements, or no usable reciprocal, takes the out-of-line exact
+// division per element.  (A
 // rarely executed branch costs its instruction fetches in every launch that
 // takes it, and a per-CTA quantization of the same row takes it in every CTA.)
 template <int N>
@@ -93,7 +120,7 @@ __device__ __forceinline__ void act_codes_n(const float* x, int valid, float s, 
 #pragma unroll
   for (int e = 1; e < N; ++e)
     if (e == te) xt = x[e];
-  const uint32_t ce = uint32_t(uint8_t(int8_t(act_code(xt, s))));
+  const uint32_t ce = rc == 0.f ? 0u : act_code_tie_exact(xt, s, rc);
   if (rc == 0.f || nt > 1) {
 #pragma unroll
     for (int e = 0; e < N; ++e)

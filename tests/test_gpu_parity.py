@@ -430,6 +430,34 @@ def test_near_tie_groups_in_fused_quantization(bl, M):
     np.testing.assert_array_equal(host(Xq), rq)
 
 
+@pytest.mark.parametrize("M", [1, 2, 5])
+def test_many_near_ties_in_fused_quantization(bl, M):
+    """Every 5-activation unit (a quarter of a 20-activation group) holds one
+    product within the fast path's window
+    of a half-integer (quotients a few ulps either side of n + 1/2,
+    n = 0..125, both signs), every seventh unit a second one: the division-free exact code
+    and the per-element fallback against the oracle's float32 division."""
+    rng = np.random.default_rng(22)
+    K, N = 2000, 64
+    X = rng.standard_normal((M, K)).astype(F32)
+    X[:, 0] = 127.0
+    eps = F32(2.0 ** -12)
+    s = (F32(127.0) / F32(127)).astype(F32) + eps
+    for m in range(M):
+        for u in range(1, K // 5):
+            for k in ([5 * u + 1] + ([5 * u + 3] if u % 7 == 0 else [])):
+                h = F32(int(rng.integers(0, 126)) + 0.5)     # |x| stays below the row max 127
+                x = F32(h * s)
+                for _ in range(int(rng.integers(0, 6))):
+                    x = np.nextafter(x, F32(np.inf) if rng.integers(0, 2) else F32(-np.inf)).astype(F32)
+                X[m, k] = x if rng.integers(0, 2) else -x
+    p = random_problem(6, M, K, N)
+    Wd, beta = bl.quantize_weights_pack5(dev(p.W), float(eps))      # the oracle uses one eps for both
+    Y = bl.linear(dev(X), Wd, bl.PACK5, N, K, beta, eps=float(eps))
+    check_ok(bl)
+    assert_y_close(host(Y), oracle.bitlinear(X, p.W, eps)["Y"])
+
+
 def test_nonfinite_activation_is_reported(bl):
     X = np.ones((3, 10), F32)
     X[1, 4] = np.nan
