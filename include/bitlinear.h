@@ -13,8 +13,9 @@
  *
  * Conventions shared by every entry point
  *   - Matrices are row-major.  W is [N, K] (out x in), X is [M, K], Y is [M, N].
- *   - Every pointer argument is a DEVICE pointer owned by the caller; the library
- *     allocates no memory.  Scratch memory is passed in as `ws` (device, 256-byte
+ *   - Every pointer argument is a DEVICE pointer owned by the caller (except the
+ *     host buffers of bl_linear_group_host and the checkpoint paths); the library
+ *     allocates no device memory.  Scratch memory is passed in as `ws` (device, 256-byte
  *     aligned) with a size from the matching *_workspace_size function.
  *   - Calls are asynchronous on `stream` (NULL = the legacy default stream).  A
  *     validation error returns at once and launches nothing.  A failed launch
@@ -276,6 +277,40 @@ size_t bl_linear_group_workspace_size(const bl_linear_call* calls, int count);
  * errors as for bl_linear. */
 bl_status bl_linear_group(const bl_linear_call* calls, int count, int flags, void* ws, size_t ws_bytes,
                           cudaStream_t stream);
+
+/* The host buffers of one call of bl_linear_group_host. */
+typedef struct {
+  const float* X_host;   /* [M, K] float32 rows in host memory, contiguous */
+  float* Y_host;         /* [M, N] float32 in host memory, contiguous */
+} bl_host_io;
+
+/* bl_linear_group with the activations read from, and the results written to,
+ * host memory (same equation and results as bl_linear_group).  Enqueued on
+ * `stream`, in this order, with no host synchronization:
+ *   1. io[i].X_host (M*K floats) is moved into calls[i].X, which serves as the
+ *      call's device staging buffer (the library overwrites it);
+ *   2. the calls run as bl_linear_group(calls, count, flags, ws, ws_bytes);
+ *   3. the results (M*N floats per call) land in io[i].Y_host.
+ * The caller synchronizes `stream` before it reads Y_host or reuses X_host.
+ * How the bytes move:
+ *   - Host memory that is page-locked and mapped into the device's address space
+ *     (cudaHostAlloc / cudaMallocHost, or cudaHostRegister'd memory, on a system
+ *     with unified addressing): the activations, up to 4 MiB per call of this
+ *     function, are read over the bus by a kernel of the library (no copy-engine
+ *     hand-off between kernels), and a call on the decode GEMV stores its results
+ *     straight into Y_host (its calls[i].Y is then left unwritten).
+ *   - Otherwise (pageable memory, larger inputs, other paths): copies on
+ *     `stream`; those of consecutive calls whose host ranges and device ranges
+ *     both follow one another end to end are merged into one transfer.  From
+ *     pageable memory the CUDA runtime stages the copies and they may return
+ *     only once done.
+ * Ownership: all buffers stay the caller's.
+ * Errors: as bl_linear_group; BL_ERR_INVALID_ARG also for a NULL `io` (count >
+ * 0) or a NULL host pointer of a call with M > 0.  Every call is validated
+ * before anything is enqueued; BL_ERR_CUDA if a copy or launch cannot be
+ * enqueued (work enqueued before it stays enqueued). */
+bl_status bl_linear_group_host(const bl_linear_call* calls, const bl_host_io* io, int count, int flags,
+                               void* ws, size_t ws_bytes, cudaStream_t stream);
 
 /* Size of the scratch array built into the library for bl_linear_noalloc. */
 #define BL_LINEAR_NOALLOC_SCRATCH_BYTES ((size_t)16 << 20)

@@ -39,6 +39,14 @@ class LinearCall(ctypes.Structure):
 _CALLS = ctypes.POINTER(LinearCall)
 
 
+class HostIO(ctypes.Structure):
+    """bl_host_io: the host buffers of one call of bl_linear_group_host (as in the header)."""
+    _fields_ = [("X_host", _P), ("Y_host", _P)]
+
+
+_IOS = ctypes.POINTER(HostIO)
+
+
 class DeployedLayer(ctypes.Structure):
     """bl_deployed_layer: one layer for bl_save_deployed (as in the header)."""
     _fields_ = [("name", ctypes.c_char_p), ("N", _I64), ("K", _I64), ("Wp", _P), ("ldp", _I64),
@@ -64,6 +72,7 @@ SIGNATURES = {
     "bl_linear_ex": (_I, [_P, _I64, _I64, _P, _I, _I64, _I64, _P, _P, _F, _P, _P, _SZ, _I, _P]),
     "bl_linear_group_workspace_size": (_SZ, [_CALLS, _I]),
     "bl_linear_group": (_I, [_CALLS, _I, _I, _P, _SZ, _P]),
+    "bl_linear_group_host": (_I, [_CALLS, _IOS, _I, _I, _P, _SZ, _P]),
     "bl_linear_noalloc": (_I, [_P, _I64, _I64, _P, _I, _I64, _I64, _P, _P, _F, _P, _P]),
     "bl_bitlinear_forward_workspace_size": (_SZ, [_I64, _I64, _I64, _I]),
     "bl_bitlinear_forward": (_I, [_P, _I64, _I64, _P, _I, _I64, _F, _P, _I64, _P, _P, _P, _P, _SZ, _P]),
@@ -319,6 +328,59 @@ def linear_group(calls, static_weights: bool = False, ws=None, outs=None):
         arr, len(calls), FLAG_STATIC_WEIGHTS if static_weights else 0, _ptr(ws),
         0 if ws is None else ws.numel(), stream))
     return Ys
+
+
+def _host(t, shape):
+    torch = _torch()
+    if t.is_cuda:
+        raise ValueError("host tensor expected")
+    if not t.is_contiguous() or t.dtype != torch.float32 or tuple(t.shape) != tuple(shape):
+        raise ValueError(f"expected a contiguous float32 host tensor of shape {tuple(shape)}")
+    return t
+
+
+class LinearGroupHost:
+    """bl_linear_group_host with its arguments marshalled once: calling the object
+    enqueues, on the stream current at construction, the copies of every host X
+    into its device staging tensor, the group, and the copies of every Y back to
+    its host tensor (no host synchronization; synchronize the stream before
+    reading the host Y).  calls = [(X_dev, W, fmt, N, K, beta, bias, eps)] as for
+    linear_group; hX[i] [M_i, K_i] and hY[i] [M_i, N_i] float32 host tensors
+    (page-locked for asynchronous copies).  The tensors stay referenced by the
+    object."""
+
+    def __init__(self, calls, hX, hY, static_weights: bool = False, ws=None, outs=None):
+        torch, self._lib = _torch(), load()
+        if not (len(calls) == len(hX) == len(hY)):
+            raise ValueError("calls, hX and hY differ in length")
+        self._calls, self._ys = _call_array(calls, outs)
+        self._io = (HostIO * max(1, len(calls)))()
+        for i, (c, x, y) in enumerate(zip(calls, hX, hY)):
+            _host(x, c[0].shape)
+            _host(y, (c[0].shape[0], c[3]))
+            self._io[i] = HostIO(x.data_ptr(), y.data_ptr())
+        need = self._lib.bl_linear_group_workspace_size(self._calls, len(calls))
+        if ws is None and need:
+            ws = workspace(need, calls[0][0].device)
+        self._keep = (calls, hX, hY, ws, outs)
+        self._args = (self._calls, self._io, len(calls), FLAG_STATIC_WEIGHTS if static_weights else 0,
+                      _ptr(ws), 0 if ws is None else ws.numel(),
+                      _stream(torch, calls[0][0]) if calls else None)
+
+    @property
+    def device_outputs(self):
+        return self._ys
+
+    def __call__(self):
+        _check("bl_linear_group_host", self._lib.bl_linear_group_host(*self._args))
+
+
+def linear_group_host(calls, hX, hY, static_weights: bool = False, ws=None, outs=None):
+    """bl_linear_group_host once: enqueue host X -> device, the group, Y -> host hY;
+    returns the device Y list.  Synchronize the stream before reading hY."""
+    g = LinearGroupHost(calls, hX, hY, static_weights, ws, outs)
+    g()
+    return g.device_outputs
 
 
 def bitlinear_forward(X, W, fmt: int = PACK5, bias=None, eps: float = 1e-5, ws=None, w_out=None,

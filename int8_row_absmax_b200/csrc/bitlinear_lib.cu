@@ -4,10 +4,12 @@
 // step of the computation runs in the kernels included below; there is no CPU
 // fallback.  One translation unit, so the per-device status word is a single
 // symbol without relocatable device code.
+#include <algorithm>
 #include <cmath>
 #include <cstdint>
 #include <cstring>
 #include <mutex>
+#include <vector>
 
 #include <cuda_runtime.h>
 
@@ -24,6 +26,7 @@
 #include "deployed_io.cuh"
 #include "ste_backward.cuh"
 #include "rmsnorm_quant.cuh"
+#include "host_io.cuh"
 
 namespace bl {
 namespace {
@@ -1027,6 +1030,130 @@ bl_status bl_linear_group(const bl_linear_call* calls, int count, int flags, voi
     off += align_up(wsz);
   }
   return BL_OK;
+}
+
+// One copy of bl_linear_group_host: `bytes` from src to dst.
+struct CopySpan {
+  char* dst;
+  const char* src;
+  size_t bytes;
+};
+
+// Enqueues the spans in order, one cudaMemcpyAsync per run of spans that follow
+// one another end to end on both sides (empty spans are skipped).
+static bl_status enqueue_copy_runs(const std::vector<CopySpan>& s, cudaMemcpyKind kind, cudaStream_t stream) {
+  size_t i = 0;
+  while (i < s.size()) {
+    if (s[i].bytes == 0) {
+      ++i;
+      continue;
+    }
+    CopySpan run = s[i];
+    size_t j = i + 1;
+    for (; j < s.size(); ++j) {
+      if (s[j].bytes == 0) continue;
+      if (s[j].dst != run.dst + run.bytes || s[j].src != run.src + run.bytes) break;
+      run.bytes += s[j].bytes;
+    }
+    if (cudaMemcpyAsync(run.dst, run.src, run.bytes, kind, stream) != cudaSuccess) return BL_ERR_CUDA;
+    i = j;
+  }
+  return BL_OK;
+}
+
+// The device address through which kernels reach host memory at p (page-locked
+// and mapped into the device's address space), else nullptr (pageable memory,
+// device memory, or an unknown pointer).
+static void* host_alias(const void* p) {
+  cudaPointerAttributes at;
+  if (cudaPointerGetAttributes(&at, p) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return nullptr;
+  }
+  return at.type == cudaMemoryTypeHost ? at.devicePointer : nullptr;
+}
+
+// Mapped host rows moved by span_copy_kernel rather than the copy engine, up to
+// this many bytes per call (beyond it the copy engine's bandwidth wins).
+constexpr size_t kSpanKernelMaxBytes = size_t(4) << 20;
+
+// Copies the runs of `s` (host-mapped sources, device destinations) with
+// span_copy_kernel, kSpanMax spans per launch, programmatic dependent launch.
+static bl_status enqueue_span_kernels(const std::vector<CopySpan>& s, cudaStream_t stream) {
+  std::vector<CopySpan> runs;
+  for (const CopySpan& c : s) {
+    if (c.bytes == 0) continue;
+    if (!runs.empty() && runs.back().dst + runs.back().bytes == c.dst && runs.back().src + runs.back().bytes == c.src)
+      runs.back().bytes += c.bytes;
+    else
+      runs.push_back(c);
+  }
+  for (size_t i0 = 0; i0 < runs.size(); i0 += kSpanMax) {
+    const int n = int(std::min(runs.size() - i0, size_t(kSpanMax)));
+    bool v16 = true;
+    for (int j = 0; j < n; ++j) {
+      const CopySpan& c = runs[i0 + j];
+      v16 = v16 && is_aligned(c.dst, 16) && is_aligned(c.src, 16) && c.bytes % 16 == 0;
+    }
+    const int unit = v16 ? 16 : 4;
+    SpanCopy a = {};
+    a.n = n;
+    a.first[0] = 0;
+    for (int j = 0; j < n; ++j) {
+      a.dst[j] = runs[i0 + j].dst;
+      a.src[j] = runs[i0 + j].src;
+      a.first[j + 1] = a.first[j] + int64_t(runs[i0 + j].bytes / unit);
+    }
+    for (int j = n; j < kSpanMax; ++j) a.first[j + 1] = a.first[n];
+    const int64_t blocks = std::min<int64_t>(ceil_div(a.first[n], int64_t(kSpanThreads) * kSpanPre), 8 * 148);
+    const bl_status st = v16 ? launch_pdl(span_copy_kernel<16>, dim3(unsigned(blocks)), dim3(kSpanThreads), 0, stream, a)
+                             : launch_pdl(span_copy_kernel<4>, dim3(unsigned(blocks)), dim3(kSpanThreads), 0, stream, a);
+    if (st != BL_OK) return st;
+  }
+  return BL_OK;
+}
+
+bl_status bl_linear_group_host(const bl_linear_call* calls, const bl_host_io* io, int count, int flags,
+                               void* ws, size_t ws_bytes, cudaStream_t stream) {
+  if (count < 0 || (count > 0 && (!calls || !io))) return BL_ERR_INVALID_ARG;
+  if (flags & ~BL_FLAG_STATIC_WEIGHTS) return BL_ERR_INVALID_ARG;
+  for (int i = 0; i < count; ++i) {
+    const bl_linear_call& c = calls[i];
+    const bl_status st = check_linear(c.X, c.M, c.K, c.W, c.f, c.N, c.ldw, c.beta_dev, c.bias, c.eps, c.Y);
+    if (st != BL_OK) return st;
+    if (c.M > 0 && (!io[i].X_host || !io[i].Y_host)) return BL_ERR_INVALID_ARG;
+  }
+  const size_t need = bl_linear_group_workspace_size(calls, count);
+  if (need && (!ws || !is_aligned(ws, kWsAlign) || ws_bytes < need)) return BL_ERR_WORKSPACE;
+  // inputs: mapped host rows by span_copy_kernel (up to kSpanKernelMaxBytes),
+  // the rest by the copy engine; results: a decode-GEMV call whose Y_host is
+  // mapped gets it as its Y (plain stores over the bus), the rest are copied back
+  std::vector<bl_linear_call> run(calls, calls + count);
+  std::vector<CopySpan> in_k, in_c, out_c;
+  size_t kbytes = 0;
+  for (int i = 0; i < count; ++i) {
+    const bl_linear_call& c = calls[i];
+    if (c.M == 0) continue;
+    char* xd = reinterpret_cast<char*>(const_cast<float*>(c.X));
+    const size_t xb = size_t(c.M) * size_t(c.K) * 4, yb = size_t(c.M) * size_t(c.N) * 4;
+    const void* xa = host_alias(io[i].X_host);
+    if (xa && kbytes + xb <= kSpanKernelMaxBytes) {
+      in_k.push_back(CopySpan{xd, static_cast<const char*>(xa), xb});
+      kbytes += xb;
+    } else {
+      in_c.push_back(CopySpan{xd, reinterpret_cast<const char*>(io[i].X_host), xb});
+    }
+    void* ya = group_gemv(c) ? host_alias(io[i].Y_host) : nullptr;
+    if (ya)
+      run[size_t(i)].Y = static_cast<float*>(ya);
+    else
+      out_c.push_back(CopySpan{reinterpret_cast<char*>(io[i].Y_host), reinterpret_cast<const char*>(c.Y), yb});
+  }
+  bl_status st = enqueue_copy_runs(in_c, cudaMemcpyHostToDevice, stream);
+  if (st == BL_OK) st = enqueue_span_kernels(in_k, stream);
+  if (st == BL_OK) st = bl_linear_group(run.data(), count, flags, ws, ws_bytes, stream);
+  if (st == BL_OK) st = enqueue_copy_runs(out_c, cudaMemcpyDeviceToHost, stream);
+  return st;
 }
 
 bl_status bl_linear_noalloc(const float* X, int64_t M, int64_t K, const void* W, bl_wfmt f,

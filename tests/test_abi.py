@@ -172,21 +172,22 @@ def test_auto_path_crossover(lib):
     assert lib.bl_linear_plan(5, 4096, 4096, pkg.I8, pkg.PATH_AUTO, ctypes.byref(n)) == pkg.PATH_TC
 
 
-def test_linear_call_struct_layout_matches_the_header(tmp_path):
-    """The binding's bl_linear_call mirrors the C struct: size and every field's
-    offset, as a C compiler lays them out from the header."""
-    fields = [f for f, _ in pkg.LinearCall._fields_]
+@pytest.mark.parametrize("struct,cls", [("bl_linear_call", pkg.LinearCall), ("bl_host_io", pkg.HostIO)])
+def test_call_struct_layout_matches_the_header(tmp_path, struct, cls):
+    """The binding's bl_linear_call and bl_host_io mirror the C structs: size and
+    every field's offset, as a C compiler lays them out from the header."""
+    fields = [f for f, _ in cls._fields_]
     src = tmp_path / "layout.c"
     src.write_text("#include <stdio.h>\n#include <stddef.h>\n#include \"bitlinear.h\"\nint main(void){\n"
-                   "printf(\"%zu\\n\", sizeof(bl_linear_call));\n" +
-                   "".join(f"printf(\"%zu\\n\", offsetof(bl_linear_call, {f}));\n" for f in fields) +
+                   f"printf(\"%zu\\n\", sizeof({struct}));\n" +
+                   "".join(f"printf(\"%zu\\n\", offsetof({struct}, {f}));\n" for f in fields) +
                    "return 0;}\n")
     exe = tmp_path / "layout"
     subprocess.run(["gcc", "-I", os.path.join(ROOT, "include"), "-I", "/usr/local/cuda/include",
                     str(src), "-o", str(exe)], check=True)
     out = [int(v) for v in subprocess.run([str(exe)], capture_output=True, text=True, check=True).stdout.split()]
-    assert out[0] == ctypes.sizeof(pkg.LinearCall)
-    assert out[1:] == [getattr(pkg.LinearCall, f).offset for f in fields]
+    assert out[0] == ctypes.sizeof(cls)
+    assert out[1:] == [getattr(cls, f).offset for f in fields]
 
 
 def test_linear_group_host_checks(lib):
@@ -206,6 +207,30 @@ def test_linear_group_host_checks(lib):
     assert lib.bl_linear_group(bad, 2, 0, None, 0, None) == 2              # unaligned packed W
     neg = (C * 1)(C(16, 1, 2560, 16, 6912, 512, pkg.PACK5, 0.0, 16, None, 16))
     assert lib.bl_linear_group(neg, 1, 0, None, 0, None) == 1              # eps <= 0
+
+
+def test_linear_group_host_buffers_checks(lib):
+    """The host-buffer group validates every call and its host pointers before
+    it enqueues anything: an empty group is a no-op, a NULL io array or host
+    pointer and unknown flags are invalid arguments, a missing workspace and a
+    misaligned weight pointer are reported as for bl_linear_group."""
+    C, H = pkg.LinearCall, pkg.HostIO
+    gemv = C(16, 1, 2560, 16, 6912, 512, pkg.PACK5, 1e-5, 16, None, 16)
+    tc = C(16, 64, 2560, 16, 6912, 512, pkg.PACK5, 1e-5, 16, None, 16)
+    empty = C(16, 0, 2560, 16, 6912, 512, pkg.PACK5, 1e-5, 16, None, 16)
+    arr = (C * 2)(gemv, tc)
+    io = (H * 2)(H(64, 64), H(64, 64))
+    f = lib.bl_linear_group_host
+    assert f(arr, io, 0, 0, None, 0, None) == 0
+    assert f(arr, None, 0, 0, None, 0, None) == 0
+    assert f(arr, None, 1, 0, None, 0, None) == 1                          # io missing
+    assert f(arr, (H * 1)(H(None, 64)), 1, 0, None, 0, None) == 1          # X_host missing
+    assert f(arr, (H * 1)(H(64, None)), 1, 0, None, 0, None) == 1          # Y_host missing
+    assert f((C * 1)(empty), (H * 1)(H(None, None)), 1, 0, None, 0, None) == 0   # M = 0: nothing to copy
+    assert f(arr, io, 1, 0x1, None, 0, None) == 1                          # unknown flag
+    assert f(arr, io, 2, 0, None, 0, None) == 4                            # workspace missing
+    bad = (C * 2)(gemv, C(16, 1, 2560, 17, 6912, 512, pkg.PACK5, 1e-5, 16, None, 16))
+    assert f(bad, io, 2, 0, None, 0, None) == 2                            # unaligned packed W
 
 
 def test_static_weights_flag_is_a_flag(lib):

@@ -159,3 +159,76 @@ def test_integer_product_with_static_weights(bl):
         acc = bl.linear_acc(dev(Xq), bl.pack(dev(Wq)), bl.PACK5, N, K, path=bl.PATH_GEMV, static_weights=True)
         assert bl.sync_status() == "BL_OK"
         np.testing.assert_array_equal(host(acc), oracle.contract(Xq, Wq))
+
+
+def _pinned(a):
+    import torch
+    return torch.from_numpy(np.ascontiguousarray(a)).pin_memory()
+
+
+def test_group_host_buffers_back_to_back(bl):
+    """bl_linear_group_host on the decode workload with both layers' rows back
+    to back in one page-locked host buffer and one device buffer (each copy
+    direction merged into one transfer): every output against the oracle, twice
+    through the same marshalled call with new activations written in between."""
+    import torch
+    ps = list(problems(2))
+    Ws = [quantized(bl, p) for p in ps]
+    Kt = sum(p.K for p in ps)
+    Nt = sum(p.N for p in ps)
+    hx = torch.empty(Kt, dtype=torch.float32).pin_memory()
+    hy = torch.full((Nt,), np.nan, dtype=torch.float32).pin_memory()
+    dx = torch.empty(Kt, dtype=torch.float32, device="cuda")
+    dy = torch.empty(Nt, dtype=torch.float32, device="cuda")
+    calls, hX, hY, outs, k0, n0 = [], [], [], [], 0, 0
+    for p, (Wd, beta) in zip(ps, Ws):
+        calls.append((dx[k0:k0 + p.K].view(1, p.K), Wd, bl.PACK5, p.N, p.K, beta, None, p.eps))
+        hX.append(hx[k0:k0 + p.K].view(1, p.K))
+        hY.append(hy[n0:n0 + p.N].view(1, p.N))
+        outs.append(dy[n0:n0 + p.N].view(1, p.N))
+        k0, n0 = k0 + p.K, n0 + p.N
+    g = bl.LinearGroupHost(calls, hX, hY, static_weights=True, outs=outs)
+    for rep in range(2):
+        Xs = [p.X if rep == 0 else np.random.default_rng(70 + i).standard_normal(p.X.shape).astype(F32) * 3
+              for i, p in enumerate(ps)]
+        for x, h in zip(Xs, hX):
+            h.copy_(torch.from_numpy(x))
+        g()
+        torch.cuda.current_stream().synchronize()
+        assert bl.sync_status() == "BL_OK"
+        for x, p, h in zip(Xs, ps, hY):
+            assert_y_exact(h.numpy(), oracle.bitlinear(x, p.W, p.eps)["Y"])
+
+
+def test_group_host_buffers_mixed_calls(bl):
+    """bl_linear_group_host over decode-GEMV, swapped tensor-core, unswapped
+    tensor-core and one-trit-per-byte calls with separate host buffers: mapped
+    page-locked rows read by the library's kernel (4-byte units, since one row
+    block is not a whole number of 16-byte units), rows beyond the kernel's byte
+    budget and a pageable pair moved by copies; decode results stored straight
+    into host memory, the others copied back.  Every result equals the oracle's
+    and bl_linear_group's."""
+    import torch
+    specs = [(1, 2560, 700), (1, 999, 1500), (2, 3000, 500), (64, 1040, 300), (3, 77, 90), (9, 640, 129),
+             (300, 4000, 260), (1, 4096, 333)]
+    calls, hX, hY, refs = [], [], [], []
+    for i, (M, K, N) in enumerate(specs):
+        p = random_problem(950 + i, M, K, N)
+        fmt = bl.I8 if i == 4 else bl.PACK5
+        Wd, beta = quantized(bl, p, fmt)
+        bias = (np.random.default_rng(i).standard_normal(N) * 0.1).astype(F32) if i % 2 else None
+        calls.append((torch.empty((M, K), dtype=torch.float32, device="cuda"), Wd, fmt, N, K, beta,
+                      None if bias is None else dev(bias), p.eps))
+        pageable = i == 1
+        hX.append(torch.from_numpy(p.X.copy()) if pageable else _pinned(p.X))
+        hY.append(torch.full((M, N), np.nan, dtype=torch.float32) if pageable
+                  else torch.full((M, N), np.nan, dtype=torch.float32).pin_memory())
+        refs.append(oracle.bitlinear(p.X, p.W, p.eps, bias)["Y"])
+    assert sum(x.numel() * 4 for x in hX[:7]) > 4 << 20      # the last rows exceed the kernel's budget
+    bl.linear_group_host(calls, hX, hY)
+    torch.cuda.current_stream().synchronize()
+    assert bl.sync_status() == "BL_OK"
+    again = bl.linear_group(calls)
+    for h, Y2, ref in zip(hY, again, refs):
+        assert_y_exact(h.numpy(), ref)
+        np.testing.assert_array_equal(host(Y2), h.numpy())
