@@ -96,36 +96,41 @@ __device__ __forceinline__ uint32_t act_code_tie_exact(float x, float s, float r
   return uint32_t(uint8_t(int8_t(x < 0.f ? -q : q)));
 }
 
-// Codes of N activations x[0..N-1] (elements from `valid` on are not part of
-// the row: code 0).  The fast path of act_code_try, plus on the hot path the
-// division-free exact code of act_code_tie_exact for the unit's one near-tie
-// element if it has one (element 0 otherwise); only a unit with two or more
-// near-tie elements, or no usable reciprocal, takes the out-of-line exact
-// division per element.  (A
-// rarely executed branch costs its instruction fetches in every launch that
-// takes it, and a per-CTA quantization of the same row takes it in every CTA.)
+// Codes of N activations x[0..N-1] of a row whose scale s came from that row's
+// own max|x| (so |x| <= max|x| <= 127 s, and the product x RN(1/s) stays below
+// 127.5: no clamp is needed before rounding); elements from `valid` on are not
+// part of the row (code 0).  Returned in the low byte of c[e].  Per element:
+// one multiply, the round-to-nearest-even of act_code_try and its near-tie
+// test, collected in a bit mask.  A unit with one near-tie element takes the
+// division-free exact code of act_code_tie_exact for it (inline: per-CTA
+// quantizations of the same row take the same branches in every CTA, and an
+// out-of-line routine costs its instruction fetches each time); two or more,
+// or no usable reciprocal (rc == 0), take the exact division per element.
 template <int N>
 __device__ __forceinline__ void act_codes_n(const float* x, int valid, float s, float rc, uint32_t* c) {
-  int te = 0, nt = 0;
+  uint32_t near = 0u;
 #pragma unroll
   for (int e = 0; e < N; ++e) {
-    bool nr = false;
-    c[e] = act_code_try(x[e], rc, nr);
-    if (nr && e < valid) {
-      te = e;
-      ++nt;
-    }
+    const float y = __fmul_rn(x[e], rc);
+    const float t = __fadd_rn(y, 12582912.0f);
+    const float d = __fsub_rn(y, __fsub_rn(t, 12582912.0f));
+    near |= uint32_t(fabsf(fabsf(d) - 0.5f) < 3.0517578125e-05f) << e;
+    c[e] = __float_as_uint(t) & 0xFFu;
   }
-  float xt = x[0];
-#pragma unroll
-  for (int e = 1; e < N; ++e)
-    if (e == te) xt = x[e];
-  const uint32_t ce = rc == 0.f ? 0u : act_code_tie_exact(xt, s, rc);
-  if (rc == 0.f || nt > 1) {
+  const uint32_t vmask = valid >= N ? 0xFFFFFFFFu : (valid <= 0 ? 0u : (1u << valid) - 1u);
+  near &= vmask;
+  if (rc == 0.f || (near & (near - 1u)) != 0u) {
 #pragma unroll
     for (int e = 0; e < N; ++e)
-      if (e < valid && (rc == 0.f || act_near_tie(x[e], rc))) c[e] = uint32_t(uint8_t(int8_t(act_code_slow(x[e], s))));
-  } else if (nt == 1) {
+      if (((vmask >> e) & 1u) && (rc == 0.f || ((near >> e) & 1u)))
+        c[e] = uint32_t(uint8_t(int8_t(act_code_slow(x[e], s))));
+  } else if (near) {
+    const int te = __ffs(int(near)) - 1;
+    float xt = x[0];
+#pragma unroll
+    for (int e = 1; e < N; ++e)
+      if (e == te) xt = x[e];
+    const uint32_t ce = act_code_tie_exact(xt, s, rc);
 #pragma unroll
     for (int e = 0; e < N; ++e)
       if (e == te) c[e] = ce;

@@ -49,7 +49,8 @@ constexpr int kGemvWarps = 16;
 constexpr int kGemvThreads = kGemvWarps * 32;
 constexpr int kGemvMaxProbs = 4;
 constexpr uint32_t kGemvMaxSmem = 232448 - 1024;  // 227 KB per CTA, less the static arrays
-constexpr uint32_t kGemvSegTarget = 32 * 1024;  // bytes per bulk copy (one mbarrier each): few, large copies
+constexpr uint32_t kGemvSegTarget = 128 * 1024;  // bytes per bulk copy (one mbarrier each): few, large copies
+constexpr uint32_t kGemvSegMin = 4 * 1024;
 constexpr int kGemvMaxStages = 24;
 constexpr uint32_t kGemvXStageMax = 48 * 1024;  // float32 X rows staged in shared memory up to this
 
@@ -105,29 +106,40 @@ inline bool gemv_plan_prob(int64_t M, int64_t N, int64_t K, int64_t ldp, int cta
   P.G = kGemvWarps / P.S;
   P.slice = int(ceil_div(nch, S));
   P.rows_per_cta = int(ceil_div(N, int64_t(ctas)));
-  // rows per warp group and segment: at least one pass of gemv_rows_per_pass rows
-  const int64_t rpp = gemv_rows_per_pass(int(M), ch);
-  int64_t per = int64_t(kGemvSegTarget) / (int64_t(P.G) * ldp);
-  per = per < rpp ? rpp : per / rpp * rpp;
-  int64_t seg = P.G * per;
-  if (seg > P.rows_per_cta) seg = P.rows_per_cta;
-  P.seg_rows = int(seg);
   P.xc_off = align_to(kLutBytes, 128);
   P.xs_off = align_to(P.xc_off + uint32_t(M * 5 * ldp), 16);
   P.xs_bytes = (uint64_t(M * K * 4) <= kGemvXStageMax && K % 4 == 0) ? uint32_t(M * K * 4) : 0u;
   P.part_off = align_to(P.xs_off + P.xs_bytes, 16);
   P.bar_off = align_to(P.part_off + uint32_t(M * P.rows_per_cta * 4), 16);
-  const int64_t nseg = ceil_div(P.rows_per_cta, P.seg_rows);
-  const uint32_t stage_bytes = uint32_t(P.seg_rows * ldp);
-  int64_t ns = nseg < kGemvMaxStages ? nseg : kGemvMaxStages;
-  for (; ns >= 1; --ns) {
-    P.stage_off = align_to(P.bar_off + uint32_t(8 * (ns + 2)), 128);
-    if (int64_t(P.stage_off) + ns * stage_bytes <= kGemvMaxSmem) break;
+  // rows per warp group and segment: at least one pass of gemv_rows_per_pass
+  // rows.  Fewer, larger copies were measured faster (each costs its issuing
+  // thread time), so the largest segment target that either holds all of the
+  // CTA's rows at once or still gives a ring of three stages; failing both, the
+  // smallest target that fits at all.
+  const int64_t rpp = gemv_rows_per_pass(int(M), ch);
+  bool found = false;
+  for (uint32_t target = kGemvSegTarget; target >= kGemvSegMin; target /= 2) {
+    int64_t per = int64_t(target) / (int64_t(P.G) * ldp);
+    per = per < rpp ? rpp : per / rpp * rpp;
+    int64_t seg = P.G * per;
+    if (seg > P.rows_per_cta) seg = P.rows_per_cta;
+    const int64_t nseg = ceil_div(P.rows_per_cta, seg);
+    const uint32_t stage_bytes = uint32_t(seg * ldp);
+    int64_t ns = nseg < kGemvMaxStages ? nseg : kGemvMaxStages;
+    uint32_t stage_off = 0;
+    for (; ns >= 1; --ns) {
+      stage_off = align_to(P.bar_off + uint32_t(8 * (ns + 2)), 128);
+      if (int64_t(stage_off) + ns * stage_bytes <= kGemvMaxSmem) break;
+    }
+    if (ns < 1) continue;
+    P.stage_off = stage_off;
+    P.seg_rows = int(seg);
+    P.nstage = int(ns);
+    P.smem = uint32_t(stage_off + ns * stage_bytes);
+    found = true;
+    if (ns >= nseg || ns >= 3) break;
   }
-  if (ns < 1) return false;
-  P.nstage = int(ns);
-  P.smem = uint32_t(P.stage_off + ns * stage_bytes);
-  return true;
+  return found;
 }
 
 // CTAs of one GEMV launch, split over its problems in proportion to their
@@ -264,10 +276,11 @@ __global__ void __launch_bounds__(kGemvThreads, kMinBlocks) gemv_pack5_kernel(co
       if (tid == 0) s_scale[m] = scm[m];
     }
   }
-  // codes in decode order, one packed word's 20 activations per thread: five
-  // 16-byte loads, twenty codes, five 32-bit stores (x[5j..5j+3] for the four
-  // j, then the four x[5j+4])
-  const int ngrp = int(ldp / 4);
+  // codes in decode order, one packed byte's five activations per thread (the
+  // most threads the row allows): byte j = 4 g + i of packed word g puts its
+  // first four codes in word i of the word's five (xc + 20 g + 4 i) and its
+  // fifth code in byte i of the fifth word
+  const int nbyte = int(ldp);
 #pragma unroll
   for (int m = 0; m < M; ++m) {
     int x4 = 0;
@@ -275,36 +288,22 @@ __global__ void __launch_bounds__(kGemvThreads, kMinBlocks) gemv_pack5_kernel(co
     const float* xr = kFused ? xsrc + int64_t(m) * K : nullptr;
     const int8_t* xq = kFused ? nullptr : P.Xq + int64_t(m) * P.ldxq;
     const float sc = kFused ? scm[m] : 0.f, rc = kFused ? act_recip(sc) : 0.f;
-    for (int gi = tid; gi < ngrp; gi += kGemvThreads) {
-      const int k0 = 20 * gi;
-      uint32_t c[20];
+    for (int j = tid; j < nbyte; j += kGemvThreads) {
+      const int k0 = 5 * j;
+      uint32_t c[5];
       if (kFused) {
-        float xv[20];
-        if (k0 + 20 <= K && aligned(xr + k0, 16)) {
+        float xv[5];
 #pragma unroll
-          for (int v = 0; v < 5; ++v) {
-            const float4 f = ld4(xr + k0 + 4 * v);
-            xv[4 * v] = f.x;
-            xv[4 * v + 1] = f.y;
-            xv[4 * v + 2] = f.z;
-            xv[4 * v + 3] = f.w;
-          }
-        } else {
-#pragma unroll
-          for (int e = 0; e < 20; ++e) xv[e] = k0 + e < K ? xr[k0 + e] : 0.f;
-        }
-        act_codes_n<20>(xv, int(min(int64_t(20), K - int64_t(k0))), sc, rc, c);
+        for (int e = 0; e < 5; ++e) xv[e] = k0 + e < K ? xr[k0 + e] : 0.f;
+        act_codes_n<5>(xv, int(min(int64_t(5), K - int64_t(k0))), sc, rc, c);
       } else {
 #pragma unroll
-        for (int e = 0; e < 20; ++e) c[e] = k0 + e < K ? uint32_t(uint8_t(xq[k0 + e])) : 0u;
+        for (int e = 0; e < 5; ++e) c[e] = k0 + e < K ? uint32_t(uint8_t(xq[k0 + e])) : 0u;
       }
-      uint32_t* dst = reinterpret_cast<uint32_t*>(xcm + 20 * gi);
-#pragma unroll
-      for (int i = 0; i < 4; ++i)
-        dst[i] = c[5 * i] | (c[5 * i + 1] << 8) | (c[5 * i + 2] << 16) | (c[5 * i + 3] << 24);
-      dst[4] = c[4] | (c[9] << 8) | (c[14] << 16) | (c[19] << 24);
-      x4 += int(int8_t(uint8_t(c[4]))) + int(int8_t(uint8_t(c[9]))) + int(int8_t(uint8_t(c[14]))) +
-            int(int8_t(uint8_t(c[19])));
+      unsigned char* dst = xcm + 20 * (j >> 2);
+      *reinterpret_cast<uint32_t*>(dst + 4 * (j & 3)) = c[0] | (c[1] << 8) | (c[2] << 16) | (c[3] << 24);
+      dst[16 + (j & 3)] = uint8_t(c[4]);
+      x4 += int(int8_t(uint8_t(c[4])));
     }
     x4 = __reduce_add_sync(0xffffffffu, x4);
     if (lane == 0 && x4) atomicAdd(&s_x4[m], x4);

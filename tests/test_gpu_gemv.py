@@ -109,6 +109,27 @@ def test_gemv_declines_codes_beyond_shared_memory(bl):
     assert_y_exact(host(Y), oracle.bitlinear(p.X, p.W, p.eps)["Y"])
 
 
+@pytest.mark.parametrize("M", [1, 2])
+def test_gemv_segment_ring(bl, M):
+    """K = 6912, N = 16000: each CTA's 109 rows of packed weights (152 KB) do not
+    fit its shared memory at once, so they stream through a ring of segments
+    reused as the CTA computes.  Every output against the oracle (weights
+    ternarized and contracted in row blocks to bound host memory)."""
+    K, N, eps = 6912, 16000, 1e-5
+    rng = np.random.default_rng(31 + M)
+    W = rng.standard_normal((N, K), dtype=np.float32) * F32(0.02)
+    X = rng.standard_normal((M, K), dtype=np.float32)
+    Wd, beta = quantized(bl, _P(W))
+    Y = host(bl.linear(dev(X), Wd, bl.PACK5, N, K, beta, eps=eps, path=bl.PATH_GEMV))
+    assert bl.sync_status() == "BL_OK"
+    b = oracle.absmean_beta(W, eps)
+    assert float(host(beta)[0]) == float(b)
+    Xq, sc = oracle.act_quant(X, eps)
+    for r0 in range(0, N, 4000):
+        acc = oracle.contract(Xq, oracle.ternarize(W[r0:r0 + 4000], b))
+        assert_y_exact(Y[:, r0:r0 + 4000], oracle.dequant(acc, sc, b))
+
+
 def test_chain_output_feeds_next_input(bl):
     """Twelve GEMVs back to back on one stream, each reading the previous one's
     Y as its X (K = N), with static weights: the dependency wait must order
