@@ -99,45 +99,59 @@ __device__ __forceinline__ uint32_t act_code_tie_exact(float x, float s, float r
 // Codes of N activations x[0..N-1] of a row whose scale s came from that row's
 // own max|x| (so |x| <= max|x| <= 127 s, and the product x RN(1/s) stays below
 // 127.5: no clamp is needed before rounding); elements from `valid` on are not
-// part of the row (code 0).  Returned in the low byte of c[e].  Per element:
-// one multiply, the round-to-nearest-even of act_code_try and its near-tie
-// test, collected in a bit mask.  A unit with one near-tie element takes the
-// division-free exact code of act_code_tie_exact for it (inline: per-CTA
-// quantizations of the same row take the same branches in every CTA, and an
-// out-of-line routine costs its instruction fetches each time); two or more,
-// or no usable reciprocal (rc == 0), take the exact division per element.
+// part of the row (code 0; the caller passes them as 0).  Each code is returned
+// in the LOW BYTE of c[e] (the upper bytes are not cleared: pack with
+// byte_perm).  Per element: one multiply, the round-to-nearest-even of
+// act_code_try and the distance of the product from the nearest half-integer,
+// of which the unit keeps only the minimum.  A unit whose minimum lies within
+// 2^-15 finds its near-tie elements: one takes the division-free exact code of
+// act_code_tie_exact (inline: per-CTA quantizations of the same row take the
+// same branches in every CTA, and an out-of-line routine costs its instruction
+// fetches each time); two or more, or no usable reciprocal (rc == 0), take the
+// exact division per element.
 template <int N>
 __device__ __forceinline__ void act_codes_n(const float* x, int valid, float s, float rc, uint32_t* c) {
-  uint32_t near = 0u;
+  float dmin = 1.0f;
 #pragma unroll
   for (int e = 0; e < N; ++e) {
     const float y = __fmul_rn(x[e], rc);
     const float t = __fadd_rn(y, 12582912.0f);
     const float d = __fsub_rn(y, __fsub_rn(t, 12582912.0f));
-    near |= uint32_t(fabsf(fabsf(d) - 0.5f) < 3.0517578125e-05f) << e;
-    c[e] = __float_as_uint(t) & 0xFFu;
+    dmin = fminf(dmin, fabsf(__fsub_rn(fabsf(d), 0.5f)));
+    c[e] = __float_as_uint(t);
   }
-  const uint32_t vmask = valid >= N ? 0xFFFFFFFFu : (valid <= 0 ? 0u : (1u << valid) - 1u);
-  near &= vmask;
-  if (rc == 0.f || (near & (near - 1u)) != 0u) {
+  if (rc == 0.f || dmin < 3.0517578125e-05f) {
+    uint32_t near = 0u;
 #pragma unroll
     for (int e = 0; e < N; ++e)
-      if (((vmask >> e) & 1u) && (rc == 0.f || ((near >> e) & 1u)))
-        c[e] = uint32_t(uint8_t(int8_t(act_code_slow(x[e], s))));
-  } else if (near) {
-    const int te = __ffs(int(near)) - 1;
-    float xt = x[0];
+      if (e < valid && act_near_tie(x[e], rc)) near |= 1u << e;
+    if (rc == 0.f || (near & (near - 1u)) != 0u) {
 #pragma unroll
-    for (int e = 1; e < N; ++e)
-      if (e == te) xt = x[e];
-    const uint32_t ce = act_code_tie_exact(xt, s, rc);
+      for (int e = 0; e < N; ++e)
+        if (e < valid && (rc == 0.f || ((near >> e) & 1u)))
+          c[e] = uint32_t(uint8_t(int8_t(act_code_slow(x[e], s))));
+    } else if (near) {
+      const int te = __ffs(int(near)) - 1;
+      float xt = x[0];
+#pragma unroll
+      for (int e = 1; e < N; ++e)
+        if (e == te) xt = x[e];
+      const uint32_t ce = act_code_tie_exact(xt, s, rc);
+#pragma unroll
+      for (int e = 0; e < N; ++e)
+        if (e == te) c[e] = ce;
+    }
+  }
+  if (valid < N) {
 #pragma unroll
     for (int e = 0; e < N; ++e)
-      if (e == te) c[e] = ce;
+      if (e >= valid) c[e] = 0u;
   }
-#pragma unroll
-  for (int e = 0; e < N; ++e)
-    if (e >= valid) c[e] = 0u;
+}
+
+// The low bytes of four code words, little-endian, in one word.
+__device__ __forceinline__ uint32_t pack_code_bytes(uint32_t c0, uint32_t c1, uint32_t c2, uint32_t c3) {
+  return __byte_perm(__byte_perm(c0, c1, 0x0040), __byte_perm(c2, c3, 0x0040), 0x5410);
 }
 
 // Four codes packed little-endian into one word.
@@ -262,8 +276,8 @@ constexpr int kActDoThreads = 512;
 // decode-order words at dst.
 __device__ __forceinline__ void store_dorder_word(uint32_t* dst, const uint32_t* c) {
 #pragma unroll
-  for (int i = 0; i < 4; ++i) dst[i] = c[5 * i] | (c[5 * i + 1] << 8) | (c[5 * i + 2] << 16) | (c[5 * i + 3] << 24);
-  dst[4] = c[4] | (c[9] << 8) | (c[14] << 16) | (c[19] << 24);
+  for (int i = 0; i < 4; ++i) dst[i] = pack_code_bytes(c[5 * i], c[5 * i + 1], c[5 * i + 2], c[5 * i + 3]);
+  dst[4] = pack_code_bytes(c[4], c[9], c[14], c[19]);
 }
 
 template <int G>

@@ -301,7 +301,7 @@ __global__ void __launch_bounds__(kGemvThreads, kMinBlocks) gemv_pack5_kernel(co
         for (int e = 0; e < 5; ++e) c[e] = k0 + e < K ? uint32_t(uint8_t(xq[k0 + e])) : 0u;
       }
       unsigned char* dst = xcm + 20 * (j >> 2);
-      *reinterpret_cast<uint32_t*>(dst + 4 * (j & 3)) = c[0] | (c[1] << 8) | (c[2] << 16) | (c[3] << 24);
+      *reinterpret_cast<uint32_t*>(dst + 4 * (j & 3)) = pack_code_bytes(c[0], c[1], c[2], c[3]);
       dst[16 + (j & 3)] = uint8_t(c[4]);
       x4 += int(int8_t(uint8_t(c[4])));
     }
