@@ -43,6 +43,7 @@
 
 #include "common.cuh"
 #include "ptx.cuh"
+#include "trit_table.cuh"
 
 namespace bl {
 
@@ -500,16 +501,15 @@ constexpr int kUnpackThreads = 256;
 __global__ void __launch_bounds__(kUnpackThreads)
 unpack5_rows_kernel(const uint8_t* __restrict__ Wp, int64_t N, int64_t ldp, int8_t* __restrict__ Wq,
                     int64_t ldq) {
-  __shared__ uint32_t lut[256 * 32];
-  for (int i = threadIdx.x; i < 256 * 32; i += kUnpackThreads) {
-    uint32_t b = uint32_t(i) >> 5, v = 0;
-    if (b > 242u) b = 121u;       // not a code: read as zero trits
+  __shared__ __align__(16) uint32_t lut[256 * 32];
+  static_assert(kUnpackThreads == 256, "one table row per thread");
+  {
+    // thread b writes the 32 lane copies of byte b's word (bytes above 242
+    // are not codes: trit_word reads them as zero trits)
+    const uint32_t v = trit_word(uint32_t(threadIdx.x));
+    uint4* row = reinterpret_cast<uint4*>(lut + 32 * threadIdx.x);
 #pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      v |= ((b % 3u + 255u) & 0xFFu) << (8 * k);
-      b /= 3u;
-    }
-    lut[i] = v;
+    for (int j = 0; j < 8; ++j) row[(j + threadIdx.x) & 7] = make_uint4(v, v, v, v);
   }
   __syncthreads();
   const uint32_t* lut_l = lut + (threadIdx.x & 31);

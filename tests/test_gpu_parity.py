@@ -364,7 +364,8 @@ def test_pack_all_patterns(bl):
 
 
 # ------------------------------------------------------------ activations ---
-@pytest.mark.parametrize("M,K", [(8, 128), (1, 2560), (3, 7), (5, 1), (17, 6912), (2, 11008), (70, 333)])
+@pytest.mark.parametrize("M,K", [(8, 128), (1, 2560), (3, 7), (5, 1), (17, 6912), (2, 11008), (70, 333),
+                                 (9, 8192), (3, 12288), (4, 16384), (3, 30000), (2, 32768), (2, 40000)])
 def test_quantize_act(bl, M, K):
     p = random_problem(M * 3 + K, M, K, 1)
     X = p.X * np.linspace(0.01, 100, M, dtype=F32)[:, None]
