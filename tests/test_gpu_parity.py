@@ -376,10 +376,12 @@ def test_quantize_act(bl, M, K):
     np.testing.assert_array_equal(host(Xq), rq)
 
 
-@pytest.mark.parametrize("M,K", [(600, 4096), (700, 1000), (320, 12288), (1000, 12)])
+@pytest.mark.parametrize("M,K", [(600, 4096), (700, 1000), (320, 12288), (1000, 12), (297, 16384), (4096, 4),
+                                 (1203, 11008), (400, 16388)])
 def test_quantize_act_many_rows(bl, M, K):
-    """Many rows take the persistent bulk-copy kernel (rows streamed through a
-    ring of shared-memory stages); codes and scales as the oracle's."""
+    """Many rows, one CTA per row (the register kernel up to K = 16384, the
+    two-pass kernel beyond, and for rows that are not whole float4s); codes and
+    scales as the oracle's."""
     rng = np.random.default_rng(M + K)
     X = rng.standard_normal((M, K)).astype(F32)
     X[::17] *= F32(40.0)
