@@ -445,20 +445,6 @@ bl_status run_tc(const int8_t* Xq, int64_t ldx, int64_t M, int64_t K, const void
   return launch_status();
 }
 
-// X_q [M, ldx] int8 as boxes {inner, Np} with the given swizzle.
-bool make_map_xq(CUtensorMap* map, const void* base, int64_t K, int64_t M, int64_t ld, int inner, int rows,
-                 CUtensorMapSwizzle sw) {
-  EncodeTiledFn fn = encode_tiled();
-  if (!fn) return false;
-  const cuuint64_t dims[2] = {cuuint64_t(K), cuuint64_t(M)};
-  const cuuint64_t strides[1] = {cuuint64_t(ld)};
-  const cuuint32_t box[2] = {cuuint32_t(inner), cuuint32_t(rows)};
-  const cuuint32_t estr[2] = {1u, 1u};
-  return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 // Packed W [N, ldp] as boxes of {128 bytes, 128 rows}, 128-byte swizzle.
 bool make_map_wp128(CUtensorMap* map, const void* base, int64_t ldp, int64_t N) {
   EncodeTiledFn fn = encode_tiled();
