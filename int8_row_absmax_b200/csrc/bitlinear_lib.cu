@@ -614,6 +614,52 @@ bl_status launch_gemv_f(int M, int ch, const GemvArgs& a, int grid, uint32_t sme
 
 // Up to kGemvMaxProbs problems with the same M in one launch; every call
 // either quantizes float32 X (fused) or reads given X_q (not fused).
+// CTAs of one GEMV launch per problem.  A CTA's time is modelled as a part
+// that grows with K (every CTA copies and quantizes the whole X row: about as
+// long as decoding four packed bytes per activation; one byte when the codes
+// are given) plus its share of the packed bytes; the split evens out those
+// times (water-filling: T with sum_i B_i / (T - r_i) = kGemvCtas, r_i the K
+// part, B_i the packed bytes), rounded to whole CTAs, at least one per problem
+// and at most one per row.
+void gemv_split_ctas(const GemvCall* c, int n, bool fused, int64_t* want) {
+  double r[kGemvMaxProbs], B[kGemvMaxProbs], rmax = 0.0, btot = 0.0;
+  for (int i = 0; i < n; ++i) {
+    r[i] = double(c[i].K) * (fused ? 4.0 : 1.0);
+    B[i] = double(c[i].N) * double(c[i].ldw);
+    rmax = r[i] > rmax ? r[i] : rmax;
+    btot += B[i];
+  }
+  if (n == 1) {
+    want[0] = std::min<int64_t>(kGemvCtas, c[0].N);
+    return;
+  }
+  double lo = rmax, hi = rmax + btot;   // sum_i B_i / (T - r_i) falls from +inf to <= 1 over (lo, hi]
+  for (int it = 0; it < 100; ++it) {
+    const double T = 0.5 * (lo + hi);
+    double s = 0.0;
+    for (int i = 0; i < n; ++i) s += B[i] / (T - r[i]);
+    (s > double(kGemvCtas) ? lo : hi) = T;
+  }
+  double frac[kGemvMaxProbs];
+  int64_t used = 0;
+  for (int i = 0; i < n; ++i) {
+    const double x = B[i] / (hi - r[i]);
+    want[i] = std::max<int64_t>(1, int64_t(x));
+    frac[i] = x - double(want[i]);
+    used += want[i];
+  }
+  while (used < kGemvCtas) {   // the remainder to the largest fractions
+    int best = -1;
+    for (int i = 0; i < n; ++i)
+      if (want[i] < c[i].N && (best < 0 || frac[i] > frac[best])) best = i;
+    if (best < 0) break;
+    ++want[best];
+    frac[best] -= 1.0;
+    ++used;
+  }
+  for (int i = 0; i < n; ++i) want[i] = std::min<int64_t>(want[i], c[i].N);
+}
+
 bl_status run_gemv_group(int64_t M, const GemvCall* c, int n, bool prefetch, cudaStream_t st) {
   if (n < 1 || n > kGemvMaxProbs || M < 1 || M > kGemvMaxM) return BL_ERR_UNSUPPORTED;
   const bool fused = c[0].X != nullptr;
@@ -629,12 +675,13 @@ bl_status run_gemv_group(int64_t M, const GemvCall* c, int n, bool prefetch, cud
   GemvArgs a = {};
   a.nprob = n;
   (void)prefetch;   // the GEMV copies X before its weights either way
+  (void)total;
+  int64_t wants[kGemvMaxProbs];
+  gemv_split_ctas(c, n, fused, wants);
   int cta = 0;
   uint32_t smem = 0;
   for (int i = 0; i < n; ++i) {
-    int64_t want = int64_t(double(kGemvCtas) * double(c[i].N) * double(c[i].ldw) / total + 0.5);
-    if (want < 1) want = 1;
-    if (want > c[i].N) want = c[i].N;
+    const int64_t want = wants[i];
     GemvProb& P = a.p[i];
     if (!gemv_plan_prob(M, c[i].N, c[i].K, c[i].ldw, int(want), ch, P)) return BL_ERR_UNSUPPORTED;
     P.X = c[i].X;
