@@ -91,8 +91,10 @@ inline int gemv_chunks_per_lane(int64_t M, int64_t ldp) {
   return 0;
 }
 
-// Rows a warp works on at once (independent chains of loads and dp4a).
-__host__ __device__ constexpr int gemv_rows_per_pass(int M, int CH) { return M * CH >= 4 ? 1 : 4 / (M * CH); }
+// Rows a warp works on at once (independent chains of loads and dp4a): three
+// for one row of X and one chunk per lane (measured: 6.30 us for the decode step
+// against 6.34 with two and 6.77 with four).
+__host__ __device__ constexpr int gemv_rows_per_pass(int M, int CH) { return M * CH == 1 ? 3 : (M * CH >= 4 ? 1 : 4 / (M * CH)); }
 
 // Geometry of one problem on `ctas` CTAs: warps per slice, row groups, the
 // segment ring and the shared-memory layout.  False if the GEMV cannot take it.
