@@ -52,7 +52,7 @@ constexpr uint32_t kGemvMaxSmem = 232448 - 1024;  // 227 KB per CTA, less the st
 constexpr uint32_t kGemvSegTarget = 128 * 1024;  // bytes per bulk copy (one mbarrier each): few, large copies
 constexpr uint32_t kGemvSegMin = 4 * 1024;
 constexpr int kGemvMaxStages = 24;
-constexpr uint32_t kGemvXStageMax = 48 * 1024;  // float32 X rows staged in shared memory up to this
+constexpr uint32_t kGemvXStageMax = 64 * 1024;  // float32 X rows staged in shared memory up to this
 
 struct GemvProb {
   const float* X;      // [M, K] float32 (activation quantization inside) or nullptr
@@ -96,28 +96,15 @@ inline int gemv_chunks_per_lane(int64_t M, int64_t ldp) {
 // against 6.34 with two and 6.77 with four).
 __host__ __device__ constexpr int gemv_rows_per_pass(int M, int CH) { return M * CH == 1 ? 3 : (M * CH >= 4 ? 1 : 4 / (M * CH)); }
 
-// Geometry of one problem on `ctas` CTAs: warps per slice, row groups, the
-// segment ring and the shared-memory layout.  False if the GEMV cannot take it.
-inline bool gemv_plan_prob(int64_t M, int64_t N, int64_t K, int64_t ldp, int ctas, int ch,
-                           GemvProb& P) {
-  if (M < 1 || M > kGemvMaxM || N < 1 || K < 1 || ldp % 16 != 0 || ldp * 5 < K || ctas < 1) return false;
-  const int64_t nch = ldp / 16;
-  const int64_t S = ceil_div(nch, int64_t(32) * ch);
-  if (S > kGemvWarps) return false;
-  P.S = int(S);
-  P.G = kGemvWarps / P.S;
-  P.slice = int(ceil_div(nch, S));
-  P.rows_per_cta = int(ceil_div(N, int64_t(ctas)));
-  P.xc_off = align_to(kLutBytes, 128);
-  P.xs_off = align_to(P.xc_off + uint32_t(M * 5 * ldp), 16);
-  P.xs_bytes = (uint64_t(M * K * 4) <= kGemvXStageMax && K % 4 == 0) ? uint32_t(M * K * 4) : 0u;
+// The weights' segment ring of a problem whose other offsets are set: rows per
+// warp group and segment are at least one pass of gemv_rows_per_pass rows.
+// Fewer, larger copies were measured faster (each costs its issuing thread
+// time), so the largest segment target that either holds all of the CTA's rows
+// at once or still gives a ring of three stages; failing both, the smallest
+// target that fits at all.  False if no ring fits.
+inline bool gemv_plan_ring(int64_t M, int64_t ldp, int ch, GemvProb& P) {
   P.part_off = align_to(P.xs_off + P.xs_bytes, 16);
   P.bar_off = align_to(P.part_off + uint32_t(M * P.rows_per_cta * 4), 16);
-  // rows per warp group and segment: at least one pass of gemv_rows_per_pass
-  // rows.  Fewer, larger copies were measured faster (each costs its issuing
-  // thread time), so the largest segment target that either holds all of the
-  // CTA's rows at once or still gives a ring of three stages; failing both, the
-  // smallest target that fits at all.
   const int64_t rpp = gemv_rows_per_pass(int(M), ch);
   bool found = false;
   for (uint32_t target = kGemvSegTarget; target >= kGemvSegMin; target /= 2) {
@@ -144,8 +131,32 @@ inline bool gemv_plan_prob(int64_t M, int64_t N, int64_t K, int64_t ldp, int cta
   return found;
 }
 
-// CTAs of one GEMV launch, split over its problems in proportion to their
-// packed bytes.  Planned for B200's 148 SMs (a fixed figure, so that plans and
+// Geometry of one problem on `ctas` CTAs: warps per slice, row groups, the
+// segment ring and the shared-memory layout.  False if the GEMV cannot take it.
+inline bool gemv_plan_prob(int64_t M, int64_t N, int64_t K, int64_t ldp, int ctas, int ch,
+                           GemvProb& P) {
+  if (M < 1 || M > kGemvMaxM || N < 1 || K < 1 || ldp % 16 != 0 || ldp * 5 < K || ctas < 1) return false;
+  const int64_t nch = ldp / 16;
+  const int64_t S = ceil_div(nch, int64_t(32) * ch);
+  if (S > kGemvWarps) return false;
+  P.S = int(S);
+  P.G = kGemvWarps / P.S;
+  P.slice = int(ceil_div(nch, S));
+  P.rows_per_cta = int(ceil_div(N, int64_t(ctas)));
+  P.xc_off = align_to(kLutBytes, 128);
+  P.xs_off = align_to(P.xc_off + uint32_t(M * 5 * ldp), 16);
+  // X staged in shared memory when it fits (and the weights' ring still does),
+  // else read from global memory
+  const bool stage_x = uint64_t(M * K * 4) <= kGemvXStageMax && K % 4 == 0;
+  for (int attempt = stage_x ? 0 : 1; attempt < 2; ++attempt) {
+    P.xs_bytes = attempt == 0 ? uint32_t(M * K * 4) : 0u;
+    if (gemv_plan_ring(M, ldp, ch, P)) return true;
+  }
+  return false;
+}
+
+// CTAs of one GEMV launch (split over its problems by the launch's time
+// model).  Planned for B200's 148 SMs (a fixed figure, so that plans and
 // the feasibility test need no device query; on a smaller device the extra
 // CTAs simply queue, since GEMV CTAs never wait on one another).
 constexpr int kGemvCtas = 148;
