@@ -664,18 +664,15 @@ bl_status run_gemv_group(int64_t M, const GemvCall* c, int n, bool prefetch, cud
   if (n < 1 || n > kGemvMaxProbs || M < 1 || M > kGemvMaxM) return BL_ERR_UNSUPPORTED;
   const bool fused = c[0].X != nullptr;
   int ch = 1;
-  double total = 0.0;
   for (int i = 0; i < n; ++i) {
     if ((c[i].X != nullptr) != fused) return BL_ERR_UNSUPPORTED;
     const int chi = gemv_chunks_per_lane(M, c[i].ldw);
     if (chi == 0) return BL_ERR_UNSUPPORTED;
     ch = chi > ch ? chi : ch;
-    total += double(c[i].N) * double(c[i].ldw);
   }
   GemvArgs a = {};
   a.nprob = n;
   (void)prefetch;   // the GEMV copies X before its weights either way
-  (void)total;
   int64_t wants[kGemvMaxProbs];
   gemv_split_ctas(c, n, fused, wants);
   int cta = 0;
