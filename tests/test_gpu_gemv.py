@@ -253,3 +253,27 @@ def test_group_host_buffers_mixed_calls(bl):
     for h, Y2, ref in zip(hY, again, refs):
         assert_y_exact(h.numpy(), ref)
         np.testing.assert_array_equal(host(Y2), h.numpy())
+
+
+def test_group_host_buffers_with_an_empty_call(bl):
+    """An M = 0 call inside a host-buffer group moves and computes nothing; the
+    calls around it are exact (each host Y written, the empty one untouched)."""
+    import torch
+    specs = [(1, 2560, 300), (0, 640, 200), (2, 999, 129)]
+    calls, hX, hY, refs = [], [], [], []
+    for i, (M, K, N) in enumerate(specs):
+        p = random_problem(990 + i, max(M, 1), K, N)
+        Wd, beta = quantized(bl, p)
+        X = p.X[:M]
+        calls.append((torch.empty((M, K), dtype=torch.float32, device="cuda"), Wd, bl.PACK5, N, K, beta, None, p.eps))
+        hX.append(_pinned(X))
+        hY.append(torch.full((M, N), np.nan, dtype=torch.float32).pin_memory())
+        refs.append(oracle.bitlinear(X, p.W, p.eps)["Y"] if M else None)
+    bl.linear_group_host(calls, hX, hY, static_weights=True)
+    torch.cuda.current_stream().synchronize()
+    assert bl.sync_status() == "BL_OK"
+    for h, ref in zip(hY, refs):
+        if ref is not None:
+            assert_y_exact(h.numpy(), ref)
+        else:
+            assert h.numel() == 0
